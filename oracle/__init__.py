@@ -1,0 +1,35 @@
+"""CPU oracle for the DeepSeek-Sparse-Attention hot path (TEST INFRASTRUCTURE ONLY).
+
+This package is a plain, slow, fp64 restatement of what the hot path computes:
+the lightning indexer, the per-query top-k selection and absorbed MLA attention
+over the selected rows, plus two independent cross-checks (dense causal MLA and
+explicit per-head MLA).  It exists to prove the CUDA library right.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+reference arm of ``bench.py`` may import it.  The CUDA library under
+``sparse_attention_16_b200`` never imports it, shares no code with it, and
+fails loudly instead of falling back to it.
+
+Parity status per function (what pins it, see tests/test_oracle_pins.py):
+  index_scores      pinned: closed forms (one-hot head / unit query), the odd-part
+                    identity relu(x) - relu(-x) = x, positive homogeneity,
+                    hand-worked integer example, causal/sequence-offset checks.
+  topk_select       pinned: brute force by repeated argmax on tiny inputs with
+                    forced ties, order/padding invariants, closed forms for
+                    monotone and all-equal rows.
+  sparse_mla        pinned: equals dense_causal_mla when every candidate is
+                    selected; equals explicit_mla (random W_UK / W_UV); single
+                    row and zero-multiplier closed forms; permutation invariance.
+  dense_causal_mla  pinned through the same equalities (independent code path).
+  explicit_mla      pinned through the same equality (independent code path).
+  forward           composition of the above; no separate pin needed.
+"""
+
+from .dsa_oracle import (  # noqa: F401
+    index_scores,
+    topk_select,
+    sparse_mla,
+    dense_causal_mla,
+    explicit_mla,
+    forward,
+)

@@ -1,0 +1,80 @@
+"""Plant plausible mistakes in a copy of the CPU oracle and check that the pins
+in test_oracle_pins.py catch every one.  Runs on the CPU only: the mistakes
+live in a throw-away module built from the oracle's source text."""
+
+import importlib.util
+import inspect
+import os
+import types
+
+import pytest
+
+import oracle.dsa_oracle as real
+import tests.test_oracle_pins as pins
+
+SRC = inspect.getsource(real)
+
+MUTATIONS = {
+    "indexer_drops_relu": ("np.maximum(dots, 0.0) @ wt[t]", "dots @ wt[t]"),
+    "indexer_relu_after_weighting": ("np.maximum(dots, 0.0) @ wt[t]", "np.maximum(dots @ wt[t], 0.0)"),
+    "indexer_ignores_weights": ("np.maximum(dots, 0.0) @ wt[t]", "np.maximum(dots, 0.0).sum(1)"),
+    "indexer_excludes_own_position": (
+        "        n = int(q_pos[t]) + 1\n        if n <= 0:\n            continue\n        base = int(seq_row_start[int(q_seq[t])])\n        k_rows",
+        "        n = int(q_pos[t])\n        if n <= 0:\n            continue\n        base = int(seq_row_start[int(q_seq[t])])\n        k_rows"),
+    "indexer_ignores_sequence_offset": (
+        "        k_rows = _f64(keys[base:base + n])", "        k_rows = _f64(keys[0:n])"),
+    "topk_ties_to_higher_position": ("np.lexsort((pos, -cand))", "np.lexsort((-pos, -cand))"),
+    "topk_ascending_scores": ("np.lexsort((pos, -cand))", "np.lexsort((pos, cand))"),
+    "topk_unsorted_output": ("chosen = np.sort(order[:keff])", "chosen = order[:keff]"),
+    "topk_count_not_clamped": ("count[t] = keff", "count[t] = int(k)"),
+    "attn_drops_multiplier": ("z = z * scale * mult[:, None]", "z = z * scale"),
+    "attn_drops_scale": ("z = z * scale * mult[:, None]", "z = z * mult[:, None]"),
+    "attn_drops_rotary_term": ("z = z + qp @ rows[:, d_c:d_c + qp.shape[1]].T", "z = z"),
+    "attn_rotary_reads_latent": ("z = z + qp @ rows[:, d_c:d_c + qp.shape[1]].T",
+                                 "z = z + qp @ rows[:, :qp.shape[1]].T"),
+    "attn_lse_without_max": ("lse = zmax[:, 0] + np.log(", "lse = np.log("),
+    "attn_values_shifted_window": ("return p @ rows[:, :d_c], lse", "return p @ rows[:, -d_c:], lse"),
+}
+
+
+def _mutant(name):
+    old, new = MUTATIONS[name]
+    assert SRC.count(old) >= 1, name
+    mod = types.ModuleType("oracle_mutant_" + name)
+    exec(compile(SRC.replace(old, new, 1), mod.__name__, "exec"), mod.__dict__)
+    return mod
+
+
+def _run_pins(mod, golden_dir, monkeypatch):
+    for fn in ("index_scores", "topk_select", "sparse_mla", "dense_causal_mla", "explicit_mla",
+               "forward"):
+        monkeypatch.setattr(pins, fn, getattr(mod, fn))
+    failures = 0
+    for tname, test in inspect.getmembers(pins, inspect.isfunction):
+        if not tname.startswith("test_"):
+            continue
+        params = inspect.signature(test).parameters
+        variants = [{}]
+        if "trial" in params:
+            variants = [{"trial": i} for i in range(40)]
+        if "d_r" in params:
+            variants = [{"d_r": 64}, {"d_r": 0}]
+        for kw in variants:
+            if "golden_dir" in params:
+                kw = dict(kw, golden_dir=golden_dir)
+            try:
+                test(**kw)
+            except Exception:
+                failures += 1
+    return failures
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, golden_dir, monkeypatch):
+    assert _run_pins(_mutant(name), golden_dir, monkeypatch) > 0, name
+
+
+def test_unmutated_oracle_passes_every_pin(golden_dir, monkeypatch):
+    mod = types.ModuleType("oracle_copy")
+    exec(compile(SRC, mod.__name__, "exec"), mod.__dict__)
+    assert _run_pins(mod, golden_dir, monkeypatch) == 0

@@ -1,0 +1,356 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix,
+never against a retyped copy of the oracle's own formulas.
+
+Each test names the property it relies on.  A plausible mistake in the oracle
+(dropped ReLU, wrong sign, transposed operand, wrong tie rule, missing scale or
+multiplier, off-by-one in the causal range, wrong sequence offset) fails at
+least one of them.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import (dense_causal_mla, explicit_mla, forward, index_scores,
+                    sparse_mla, topk_select)
+
+RNG = np.random.default_rng(1234)
+
+
+def _bf16ish(x):
+    """Round float64 values to bf16-representable float32 (truncate-to-nearest via float32 bits)."""
+    f = np.asarray(x, dtype=np.float32)
+    b = f.view(np.uint32).astype(np.uint64)
+    b = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16) << 16
+    return b.astype(np.uint32).view(np.float32)
+
+
+def _toy(golden_dir):
+    with open(os.path.join(golden_dir, "toy_examples.json")) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------- indexer
+
+def test_indexer_hand_worked_example(golden_dir):
+    g = _toy(golden_dir)["indexer"]
+    s = index_scores(np.array(g["q_idx"], float), np.array(g["w"]), np.array(g["k_idx"], float),
+                     np.array(g["seq_row_start"]), np.array(g["q_seq"]), np.array(g["q_pos"]),
+                     g["ld"])
+    want = np.array([[float(v) for v in row] for row in g["scores"]])
+    assert np.array_equal(s, want)
+
+
+def _rand_index_case(T=3, lens=(40, 75, 9), H=32, D=128):
+    rows = sum(lens)
+    starts = np.cumsum([0] + list(lens[:-1]))
+    q = _bf16ish(RNG.standard_normal((T, H, D)))
+    w = (RNG.standard_normal((T, H)) / math.sqrt(H)).astype(np.float32).astype(np.float64)
+    k = _bf16ish(RNG.standard_normal((rows, D)))
+    q_seq = np.arange(T) % len(lens)
+    q_pos = np.array([lens[b] - 1 for b in q_seq])
+    return q, w, k, starts, q_seq, q_pos, max(lens)
+
+
+def test_indexer_single_head_unit_query_closed_form():
+    # w = a * e_j and q[t, j] = beta * e_d  =>  I[t, s] = a * beta * max(0, k[s, d]).
+    q, w, k, starts, q_seq, q_pos, ld = _rand_index_case()
+    j, d, a, beta = 5, 17, -1.75, 2.5
+    w[:] = 0.0
+    w[:, j] = a
+    q[:, j, :] = 0.0
+    q[:, j, d] = beta
+    s = index_scores(q, w, k, starts, q_seq, q_pos, ld)
+    for t in range(len(q_seq)):
+        n = q_pos[t] + 1
+        rows = k[starts[q_seq[t]]:starts[q_seq[t]] + n, d].astype(np.float64)
+        np.testing.assert_allclose(s[t, :n], a * beta * np.maximum(rows, 0.0), rtol=0, atol=0)
+
+
+def test_indexer_odd_part_identity():
+    # relu(x) - relu(-x) = x, so I(k) - I(-k) = (sum_j w_j q_j) . k: linear in k,
+    # with the head weights applied once and the ReLU present.
+    q, w, k, starts, q_seq, q_pos, ld = _rand_index_case()
+    sp = index_scores(q, w, k, starts, q_seq, q_pos, ld)
+    sm = index_scores(q, w, -k, starts, q_seq, q_pos, ld)
+    for t in range(len(q_seq)):
+        n = q_pos[t] + 1
+        d = (w[t].astype(np.float64)[:, None] * q[t].astype(np.float64)).sum(0)
+        rows = k[starts[q_seq[t]]:starts[q_seq[t]] + n].astype(np.float64)
+        np.testing.assert_allclose(sp[t, :n] - sm[t, :n], rows @ d, rtol=1e-10, atol=1e-9)
+        # and both parts are genuinely non-linear: I(k) + I(-k) = sum_j w_j |q_j . k|
+        assert not np.allclose(sp[t, :n] + sm[t, :n], 0.0)
+
+
+def test_indexer_homogeneity_and_sign_of_w():
+    q, w, k, starts, q_seq, q_pos, ld = _rand_index_case()
+    base = index_scores(q, w, k, starts, q_seq, q_pos, ld)
+    fin = np.isfinite(base)
+    # positive scaling of q or k passes through the ReLU; w enters linearly.
+    np.testing.assert_allclose(index_scores(2 * q, w, k, starts, q_seq, q_pos, ld)[fin],
+                               2 * base[fin], rtol=1e-12)
+    np.testing.assert_allclose(index_scores(q, w, 0.5 * k, starts, q_seq, q_pos, ld)[fin],
+                               0.5 * base[fin], rtol=1e-12)
+    np.testing.assert_allclose(index_scores(q, -3 * w, k, starts, q_seq, q_pos, ld)[fin],
+                               -3 * base[fin], rtol=1e-12)
+    # with every weight positive, every score is non-negative (ReLU before weighting)
+    assert (index_scores(q, np.abs(w), k, starts, q_seq, q_pos, ld)[fin] >= 0).all()
+
+
+def test_indexer_causal_range_and_sequence_offsets():
+    q, w, k, starts, q_seq, q_pos, ld = _rand_index_case(T=3, lens=(40, 75, 9))
+    s = index_scores(q, w, k, starts, q_seq, q_pos, ld)
+    for t in range(3):
+        n = q_pos[t] + 1
+        assert np.isfinite(s[t, :n]).all()            # own position included
+        assert np.isneginf(s[t, n:]).all()            # later positions masked
+    # changing another sequence's keys, or keys beyond q_pos, changes nothing
+    k2 = k.copy()
+    k2[starts[1]:starts[1] + 75] = 0.0
+    s2 = index_scores(q, w, k2, starts, q_seq, q_pos, ld)
+    np.testing.assert_allclose(s2[[0, 2]], s[[0, 2]], rtol=1e-12, atol=1e-12)
+    assert np.all(s2[1, :75] == 0.0)
+    # moving the query earlier only truncates its row
+    q_pos3 = q_pos.copy()
+    q_pos3[1] = 30
+    s3 = index_scores(q, w, k, starts, q_seq, q_pos3, ld)
+    np.testing.assert_allclose(s3[1, :31], s[1, :31], rtol=1e-12, atol=1e-12)
+    assert np.isneginf(s3[1, 31:]).all()
+
+
+# --------------------------------------------------------------------------- top-k
+
+def test_topk_hand_worked_example(golden_dir):
+    g = _toy(golden_dir)["indexer"]
+    scores = np.array([[float(v) for v in row] for row in g["scores"]])
+    for key, kk in (("k1", 1), ("k2", 2), ("k4", 4)):
+        idx, cnt = topk_select(scores, np.array(g["q_pos"]), kk)
+        assert idx.tolist() == g["topk"][key]["idx"]
+        assert cnt.tolist() == g["topk"][key]["count"]
+
+
+def _select_by_repeated_argmax(row, k):
+    """Brute force: repeatedly take the best remaining score, lower position first on ties."""
+    vals = [(-math.inf if math.isnan(v) else v) for v in row]
+    left = list(range(len(vals)))
+    chosen = []
+    for _ in range(min(k, len(vals))):
+        best = left[0]
+        for i in left[1:]:
+            if vals[i] > vals[best]:
+                best = i
+        chosen.append(best)
+        left.remove(best)
+    return sorted(chosen)
+
+
+@pytest.mark.parametrize("trial", range(40))
+def test_topk_brute_force_tiny_with_ties(trial):
+    rng = np.random.default_rng(100 + trial)
+    T, ld = 3, int(rng.integers(1, 24))
+    k = int(rng.integers(1, 12))
+    scores = rng.integers(-3, 4, size=(T, ld)).astype(np.float64)   # many ties
+    if trial % 5 == 0:
+        scores[:, ::3] = -0.0
+    q_pos = rng.integers(0, ld, size=T)
+    idx, cnt = topk_select(scores, q_pos, k)
+    for t in range(T):
+        want = _select_by_repeated_argmax(list(scores[t, :q_pos[t] + 1]), k)
+        assert cnt[t] == len(want)
+        assert idx[t, :cnt[t]].tolist() == want
+        assert (idx[t, cnt[t]:] == -1).all()
+
+
+def test_topk_signed_zero_and_nan():
+    scores = np.array([[0.0, -0.0, np.nan, 0.0, -1.0, np.nan]])
+    idx, cnt = topk_select(scores, np.array([5]), 3)
+    assert idx.tolist() == [[0, 1, 3]]      # -0 == +0, ties to lower positions
+    idx, cnt = topk_select(scores, np.array([5]), 5)
+    assert idx.tolist() == [[0, 1, 2, 3, 4]]  # NaN ranks as -inf, below -1.0, lower NaN first
+
+
+def test_topk_closed_forms():
+    n, k = 300, 37
+    q_pos = np.array([n - 1])
+    idx, _ = topk_select(np.full((1, n), 2.5), q_pos, k)
+    assert idx[0].tolist() == list(range(k))                 # all equal -> lowest positions
+    idx, _ = topk_select(-np.arange(n, dtype=float)[None], q_pos, k)
+    assert idx[0].tolist() == list(range(k))                 # decreasing
+    idx, _ = topk_select(np.arange(n, dtype=float)[None], q_pos, k)
+    assert idx[0].tolist() == list(range(n - k, n))          # increasing
+    idx, cnt = topk_select(np.arange(n, dtype=float)[None], q_pos, 2048)
+    assert cnt[0] == n and idx[0, :n].tolist() == list(range(n)) and (idx[0, n:] == -1).all()
+
+
+def test_topk_invariants_random():
+    rng = np.random.default_rng(7)
+    T, ld, k = 4, 5000, 2048
+    scores = rng.standard_normal((T, ld)).astype(np.float32).astype(np.float64)
+    scores[:, 100:140] = scores[0, 3]   # a block of exact ties
+    q_pos = np.array([4999, 3000, 2047, 10])
+    idx, cnt = topk_select(scores, q_pos, k)
+    for t in range(T):
+        n = q_pos[t] + 1
+        sel = idx[t, :cnt[t]]
+        assert cnt[t] == min(k, n)
+        assert np.all(np.diff(sel) > 0)
+        rest = np.setdiff1d(np.arange(n), sel)
+        if rest.size:
+            lo = scores[t, sel].min()
+            assert lo >= scores[t, rest].max()
+            tied_out = rest[scores[t, rest] == lo]
+            tied_in = sel[scores[t, sel] == lo]
+            if tied_out.size:
+                assert tied_in.max() < tied_out.min()
+
+
+# --------------------------------------------------------------------------- attention
+
+def test_attention_hand_worked_example(golden_dir):
+    g = _toy(golden_dir)["attention"]
+    cache = np.array(g["cache"], float)
+    for c in g["cases"]:
+        o, lse = sparse_mla(np.array([[c["q_nope"]]]), np.array([[c["q_pe"]]]), np.ones((1, 1)),
+                            g["scale"], cache, g["d_rope"], np.array([0]), np.array([0]),
+                            np.array([[0, 1]]), np.array([2]))
+        np.testing.assert_allclose(o[0, 0], c["o"], rtol=1e-12)
+        np.testing.assert_allclose(lse[0, 0], c["lse"], rtol=1e-12)
+
+
+def _rand_attn_case(T=2, lens=(33, 50), H=64, d_c=512, d_r=64, std=1.0 / math.sqrt(192)):
+    rows = sum(lens)
+    starts = np.cumsum([0] + list(lens[:-1]))
+    cache = _bf16ish(RNG.standard_normal((rows, d_c + d_r)))
+    qn = _bf16ish(RNG.standard_normal((T, H, d_c)) * std)
+    qp = _bf16ish(RNG.standard_normal((T, H, d_r)) * std) if d_r else None
+    m = (RNG.random((T, H)) + 0.5).astype(np.float32)
+    q_seq = np.arange(T) % len(lens)
+    q_pos = np.array([lens[b] - 1 for b in q_seq])
+    return qn, qp, m, cache, starts, q_seq, q_pos
+
+
+@pytest.mark.parametrize("d_r", [64, 0])
+def test_sparse_equals_dense_when_everything_is_selected(d_r):
+    qn, qp, m, cache, starts, q_seq, q_pos = _rand_attn_case(d_r=d_r, std=1.0)
+    scale = 1.0 / math.sqrt(192)
+    n_max = q_pos.max() + 1
+    idx = np.full((len(q_seq), 2048), -1, np.int32)
+    cnt = np.zeros(len(q_seq), np.int32)
+    for t in range(len(q_seq)):
+        n = q_pos[t] + 1
+        idx[t, :n] = RNG.permutation(n)          # any order of the full set
+        cnt[t] = n
+    o_s, l_s = sparse_mla(qn, qp, m, scale, cache, d_r, starts, q_seq, idx, cnt)
+    o_d, l_d = dense_causal_mla(qn, qp, m, scale, cache, d_r, starts, q_seq, q_pos)
+    assert n_max <= 2048
+    np.testing.assert_allclose(o_s, o_d, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(l_s, l_d, rtol=1e-12)
+
+
+def test_absorbed_equals_explicit_per_head_mla():
+    # q_nope_h = W_UK_h^T q_h  and  out_h = W_UV_h o_h  (absorption of the up-projections).
+    H, d_c, d_r, d_h = 64, 512, 64, 128
+    qn_unused, qp, m, cache, starts, q_seq, q_pos = _rand_attn_case(T=2, H=H, d_c=d_c, d_r=d_r)
+    W_UK = RNG.standard_normal((H, d_h, d_c)) / math.sqrt(d_c)
+    W_UV = RNG.standard_normal((H, d_h, d_c)) / math.sqrt(d_c)
+    q_head = RNG.standard_normal((2, H, d_h))
+    q_nope = np.einsum("hdc,thd->thc", W_UK, q_head)
+    idx = np.full((2, 2048), -1, np.int32)
+    cnt = np.array([20, 41], np.int32)
+    idx[0, :20] = np.sort(RNG.choice(33, 20, replace=False))
+    idx[1, :41] = np.sort(RNG.choice(50, 41, replace=False))
+    scale = 1.0 / math.sqrt(192)
+    o_abs, _ = sparse_mla(q_nope, qp, m, scale, cache, d_r, starts, q_seq, idx, cnt)
+    out = explicit_mla(q_head, qp, W_UK, W_UV, m, scale, cache, d_r, starts, q_seq, idx, cnt)
+    np.testing.assert_allclose(np.einsum("hdc,thc->thd", W_UV, o_abs), out, rtol=1e-9, atol=1e-12)
+
+
+def test_single_row_and_uniform_closed_forms():
+    qn, qp, m, cache, starts, q_seq, q_pos = _rand_attn_case(T=1, lens=(60,))
+    scale = 0.3
+    idx = np.full((1, 2048), -1, np.int32)
+    idx[0, 0] = 17
+    o, lse = sparse_mla(qn, qp, m, scale, cache, 64, starts, q_seq, idx, np.array([1]))
+    np.testing.assert_allclose(o[0], np.broadcast_to(cache[17, :512], (64, 512)), rtol=1e-15)
+    z = ((qn[0].astype(float) @ cache[17, :512]) + qp[0].astype(float) @ cache[17, 512:]) * scale * m[0]
+    np.testing.assert_allclose(lse[0], z, rtol=1e-12)
+    # zero multiplier: uniform weights -> mean of the selected rows, lse = ln n
+    sel = np.array([3, 9, 10, 44, 59])
+    idx[0, :5] = sel
+    o, lse = sparse_mla(qn, qp, np.zeros_like(m), scale, cache, 64, starts, q_seq, idx, np.array([5]))
+    np.testing.assert_allclose(o[0], np.broadcast_to(cache[sel, :512].astype(np.float64).mean(0), (64, 512)), rtol=1e-12)
+    np.testing.assert_allclose(lse[0], math.log(5), rtol=1e-12)
+
+
+def test_softmax_normalises_and_rows_weighted():
+    # For a tiny head the logits are computed by loops here; the oracle's lse must
+    # normalise them and o must be the corresponding weighted sum of rows.
+    H, d_c, d_r = 2, 3, 2
+    cache = np.array([[1, -2, 0.5, 1, 0], [0, 1, 2, -1, 3], [2, 2, -1, 0.5, 0.5]], float)
+    qn = np.array([[[0.3, -0.1, 0.7], [1.0, 0.0, -0.5]]])
+    qp = np.array([[[0.2, 0.1], [-0.3, 0.4]]])
+    m = np.array([[1.5, 0.5]])
+    idx = np.array([[0, 2, 1]])
+    o, lse = sparse_mla(qn, qp, m, 0.9, cache, d_r, np.array([0]), np.array([0]), idx, np.array([3]))
+    for h in range(H):
+        z = []
+        for s in (0, 2, 1):
+            acc = 0.0
+            for d in range(d_c):
+                acc += qn[0, h, d] * cache[s, d]
+            for r in range(d_r):
+                acc += qp[0, h, r] * cache[s, d_c + r]
+            z.append(acc * 0.9 * m[0, h])
+        p = [math.exp(v - lse[0, h]) for v in z]
+        assert abs(sum(p) - 1.0) < 1e-12
+        want = [sum(p[i] * cache[s, d] for i, s in enumerate((0, 2, 1))) for d in range(d_c)]
+        np.testing.assert_allclose(o[0, h], want, rtol=1e-12)
+
+
+def test_permutation_and_padding_invariance():
+    qn, qp, m, cache, starts, q_seq, q_pos = _rand_attn_case(T=1, lens=(80,))
+    sel = np.sort(RNG.choice(80, 30, replace=False))
+    idx = np.full((1, 2048), -1, np.int32)
+    idx[0, :30] = sel
+    o1, l1 = sparse_mla(qn, qp, m, 0.1, cache, 64, starts, q_seq, idx, np.array([30]))
+    idx[0, :30] = sel[::-1]
+    o2, l2 = sparse_mla(qn, qp, m, 0.1, cache, 64, starts, q_seq, idx, np.array([30]))
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(l1, l2, rtol=1e-12)
+
+
+def test_nope_layer_equals_rope_layer_with_zero_rotary_query():
+    qn, qp, m, cache, starts, q_seq, q_pos = _rand_attn_case(T=1, lens=(40,))
+    idx = np.full((1, 2048), -1, np.int32)
+    idx[0, :25] = np.arange(25)
+    o_r, l_r = sparse_mla(qn, np.zeros_like(qp), m, 0.2, cache, 64, starts, q_seq, idx, np.array([25]))
+    o_n, l_n = sparse_mla(qn, None, m, 0.2, np.ascontiguousarray(cache[:, :512]), 0, starts, q_seq,
+                          idx, np.array([25]))
+    np.testing.assert_allclose(o_r, o_n, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(l_r, l_n, rtol=1e-12)
+
+
+def test_empty_selection():
+    qn, qp, m, cache, starts, q_seq, q_pos = _rand_attn_case(T=1, lens=(10,))
+    idx = np.full((1, 2048), -1, np.int32)
+    o, lse = sparse_mla(qn, qp, m, 0.2, cache, 64, starts, q_seq, idx, np.array([0]))
+    assert np.all(o == 0) and np.all(np.isneginf(lse))
+
+
+# --------------------------------------------------------------------------- composition
+
+def test_forward_shares_one_selection_across_layers():
+    q, w, k, starts, q_seq, q_pos, ld = _rand_index_case(T=2, lens=(300, 120))
+    qn, qp, m, cache, _, _, _ = _rand_attn_case(T=2, lens=(300, 120))
+    layers = [dict(q_nope=qn, q_pe=qp, qmul=m, cache=cache, d_rope=64),
+              dict(q_nope=qn, q_pe=None, qmul=m, cache=np.ascontiguousarray(cache[:, :512]),
+                   d_rope=0)]
+    idx, cnt, outs = forward(q, w, k, starts, q_seq, q_pos, layers, 0.1, k=64)
+    assert cnt.tolist() == [64, 64]
+    for lay, (o, lse) in zip(layers, outs):
+        o2, _ = sparse_mla(lay["q_nope"], lay["q_pe"], lay["qmul"], 0.1, lay["cache"],
+                           lay["d_rope"], starts, q_seq, idx, cnt)
+        np.testing.assert_array_equal(o, o2)
