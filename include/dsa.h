@@ -1,0 +1,205 @@
+/*
+ * dsa.h - C ABI of the B200 (sm_100a) DeepSeek-Sparse-Attention hot path:
+ *         lightning indexer -> per-query top-k -> absorbed sparse MLA.
+ *
+ * What the calls compute (sources: the "Mistral Large 4" concept page,
+ * liminalml.com/concepts/mistral-large-4, paragraphs "What to keep",
+ * "Where to look", "Cache", "Sparse attention", "Query scaling"; and the
+ * DSA paragraph of the reading of the technical report at
+ * avisoori1x.github.io/mistral_large_4):
+ *
+ *   indexer     I[t,s] = sum_{j<32} w[t,j] * max(0, q[t,j,:] . k[s,:])      (128-dim heads)
+ *   selection   the k best positions s <= q_pos[t] (ties to the lower position)
+ *   attention   z[h,i] = (q_nope[t,h,:] . c_{s_i} + q_pe[t,h,:] . kR_{s_i}) * scale * m[t,h]
+ *               o[t,h,:] = sum_i softmax_i(z[h,:]) c_{s_i}       (64 heads, 512-value latent)
+ *
+ * Conventions shared by every call
+ *   - Every tensor argument is a DEVICE pointer owned by the caller (allocated
+ *     by PyTorch or cudaMalloc); the library allocates nothing on the hot path
+ *     and keeps no state between calls except a per-device error word read by
+ *     dsa_check_errors().  Scratch memory is passed in as `workspace`.
+ *   - All calls are asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  They only enqueue work; outputs are valid once
+ *     the stream reaches that point.
+ *   - bf16 tensors are row-major with the innermost dimension contiguous and
+ *     every pointer 16-byte aligned.  Row strides are given in elements.
+ *   - Sequence description: rows of sequence b occupy
+ *     [seq_row_start[b], seq_row_start[b] + length) of EVERY cache buffer
+ *     (index keys and latent caches alike); query t belongs to sequence
+ *     q_seq[t] and sits at absolute position q_pos[t]; its candidates are the
+ *     positions 0..q_pos[t] (its own position included).  Decode: q_pos = L-1.
+ *     Prefill chunk: q_pos = P + i.
+ *   - T == 0 is a no-op returning DSA_OK.
+ *   - Errors: argument problems visible on the host return DSA_ERR_INVALID_ARG
+ *     (nothing is launched); a failed launch returns DSA_ERR_CUDA.  Problems
+ *     only visible on the device (an index or sequence id out of range, a
+ *     query group that mixes sequences, a pipeline wait that gave up) do not
+ *     fault: the kernel skips the bad element, sets a bit in the device error
+ *     word and finishes; dsa_check_errors() reports and clears it.
+ *     dsa_last_error() returns a text for the last failure on this thread.
+ *   - Thread safety: calls may be issued from several host threads; calls
+ *     that overlap on the GPU only share the device error word.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dsa_status {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size or stride          */
+  DSA_ERR_UNSUPPORTED = 2,   /* a shape this build does not implement                  */
+  DSA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed                   */
+  DSA_ERR_DEVICE_CHECK = 4,  /* device-side check failed (see dsa_check_errors)        */
+  DSA_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up                     */
+  DSA_ERR_WORKSPACE = 6      /* workspace too small or misaligned                      */
+} dsa_status_t;
+
+/* Device error word bits (returned through dsa_check_errors' out argument). */
+#define DSA_DEVERR_BAD_INDEX    0x1u  /* a selected position outside its sequence's rows */
+#define DSA_DEVERR_BAD_SEQ      0x2u  /* q_seq out of range or q_pos >= ld               */
+#define DSA_DEVERR_MIXED_GROUP  0x4u  /* q_group > 1 but a group spans several sequences */
+#define DSA_DEVERR_TIMEOUT      0x8u  /* a pipeline barrier wait hit its iteration limit */
+
+/* Fixed dimensions of this build (one Mistral Large 4 attention layer). */
+#define DSA_IDX_HEADS 32   /* indexer heads                        */
+#define DSA_IDX_DIM   128  /* indexer head dimension               */
+#define DSA_HEADS     64   /* attention heads                      */
+#define DSA_LATENT    512  /* latent c_s per position              */
+#define DSA_ROPE      64   /* rotary key kR_s per position (RoPE)  */
+
+/*
+ * dsa_index_scores - lightning-indexer scores.
+ * Concept page, "Where to look" and "Sparse attention": a scorer with 32 small
+ * heads rates every earlier position, 32 x 128 multiply-adds each.
+ *
+ *   q_idx   bf16 [T, 32, 128]   indexer queries
+ *   w       f32  [T, 32]        per-head weights
+ *   k_idx   bf16 [n_rows, 128]  index keys, rows located by seq_row_start
+ *   seq_row_start int64 [B], q_seq int32 [T], q_pos int32 [T]  (device); B >= 1
+ *   q_group 1: no assumption.  8: the caller guarantees that queries
+ *           [8g, 8g+8) share one sequence (chunked prefill); they are then
+ *           scored together, 8 queries x 32 heads per tensor-core tile.
+ *   scores  f32 [T, ld]: I[t,s] for s <= q_pos[t], -inf for q_pos[t] < s < ld.
+ *           ld >= max(q_pos) + 1 and ld % 4 == 0.
+ * Returns DSA_ERR_INVALID_ARG for null/misaligned pointers, T < 0, n_rows < 1,
+ * n_rows >= 2^31 - 256, ld < 4 or ld % 4, q_group not 1 or 8.
+ */
+dsa_status_t dsa_index_scores(const void* q_idx, const float* w, const void* k_idx,
+                              int64_t n_rows, const int64_t* seq_row_start, int32_t B,
+                              const int32_t* q_seq, const int32_t* q_pos, int32_t T,
+                              int32_t q_group, float* scores, int64_t ld, void* stream);
+
+/*
+ * dsa_topk - per-query top-k of a score array.
+ * Concept page, "Sparse attention" (keeps the top 2,048) and the report's DSA
+ * paragraph (chosen per query).  Candidates of query t are columns
+ * 0..q_pos[t] of scores[t, :].  Ranking: higher score first; equal scores go to
+ * the lower position; -0.0 == +0.0; NaN ranks as -inf.  Writes the best
+ * k_eff = min(k, q_pos[t] + 1) positions to idx[t, 0:k_eff] in ascending order,
+ * -1 in idx[t, k_eff:k], and k_eff to count[t].  Bit-exact and deterministic.
+ *
+ *   scores f32 [T, ld] (ld % 4 == 0, 16-byte aligned), q_pos int32 [T],
+ *   idx int32 [T, k] (out), count int32 [T] (out), 1 <= k <= 16384.
+ *   workspace: dsa_topk_workspace_size() bytes (currently 0; may be NULL).
+ */
+size_t dsa_topk_workspace_size(int32_t T, int64_t ld, int32_t k);
+dsa_status_t dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, int32_t T,
+                      int32_t k, int32_t* idx, int32_t* count, void* workspace,
+                      size_t ws_bytes, void* stream);
+
+/*
+ * sparse_mla_attend - absorbed MLA over the selected rows of a latent cache.
+ * Concept page, "What to keep" (512-value latent + 64-value rotary key per
+ * position shared by all 64 heads), "Sparse attention" (attention normalizes
+ * over the selected positions alone, 64 x (512 + 64 + 512) multiply-adds per
+ * attended position) and "Query scaling" (a per-head query multiplier).
+ *
+ *   q_nope bf16 [T, 64, 512]   absorbed no-rope queries (W_UK already applied)
+ *   q_pe   bf16 [T, 64, 64]    rotary queries; NULL iff d_rope == 0 (NoPE layer)
+ *   qmul   f32  [T, 64]        per-(t, head) query multiplier m[t,h]
+ *   softmax_scale              e.g. 1/sqrt(192)
+ *   cache  bf16 [n_rows, ld_c] rows [c_s (512) | kR_s (d_rope)]; ld_c >= 512 + d_rope,
+ *                              ld_c % 8 == 0;  d_rope in {0, 64}
+ *   seq_row_start int64 [B], q_seq int32 [T]; B >= 1
+ *   idx    int32 [T, k] positions (ascending or not; -1 entries are skipped),
+ *   count  int32 [T]    number of leading idx entries to use (<= k)
+ *   out    bf16 [T, 64, 512]   o[t,h] = sum_i p_i c_{s_i}   (round to nearest even)
+ *   lse    f32  [T, 64] or NULL: natural-log log-sum-exp of the logits
+ *   count == 0 gives out = 0 and lse = -inf.
+ *   workspace: sparse_mla_workspace_size(T, k) bytes, 256-byte aligned.
+ */
+size_t sparse_mla_workspace_size(int32_t T, int32_t k);
+dsa_status_t sparse_mla_attend(const void* q_nope, const void* q_pe, const float* qmul,
+                               float softmax_scale, const void* cache, int64_t n_rows,
+                               int32_t ld_c, int32_t d_rope, const int64_t* seq_row_start,
+                               int32_t B, const int32_t* q_seq, const int32_t* idx,
+                               const int32_t* count,
+                               int32_t T, int32_t k, void* out, float* lse, void* workspace,
+                               size_t ws_bytes, void* stream);
+
+/* One attention layer fed by a shared selection (fields as in sparse_mla_attend). */
+typedef struct dsa_layer_args {
+  const void* q_nope;   /* bf16 [T, 64, 512]                      */
+  const void* q_pe;     /* bf16 [T, 64, 64] or NULL (NoPE)        */
+  const float* qmul;    /* f32 [T, 64]                            */
+  const void* cache;    /* bf16 [n_rows, ld_c]                    */
+  int32_t ld_c;
+  int32_t d_rope;       /* 64 or 0                                */
+  void* out;            /* bf16 [T, 64, 512]                      */
+  float* lse;           /* f32 [T, 64] or NULL                    */
+} dsa_layer_args;
+
+/*
+ * dsa_sparse_mla_forward - one selection reused by several layers.
+ * Concept page bullet "28 layers reuse the selection made by the most recent
+ * layer that ran its indexer": the indexer and top-k run once, then every
+ * layer in `layers` (host array of n_layers entries, device pointers inside)
+ * attends over that selection.  Queries are processed in chunks so that the
+ * fp32 score rows fit the workspace (chunked prefill).
+ *
+ *   idx_out / count_out: optional [T, k] / [T] copies of the selection (NULL = not needed).
+ *   workspace: at least dsa_forward_workspace_size(T, ld, k, q_group) bytes for
+ *   one pass over all queries; a smaller workspace (>= the size for q_group
+ *   queries) makes the call process queries in chunks.
+ */
+size_t dsa_forward_workspace_size(int32_t T, int64_t ld, int32_t k, int32_t q_group);
+dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const void* k_idx,
+                                    int64_t n_rows, const int64_t* seq_row_start, int32_t B,
+                                    const int32_t* q_seq, const int32_t* q_pos, int32_t T,
+                                    int32_t q_group, int64_t ld, int32_t n_layers,
+                                    const dsa_layer_args* layers, float softmax_scale,
+                                    int32_t k, int32_t* idx_out, int32_t* count_out,
+                                    void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * dsa_check_errors - synchronizes `stream`, returns DSA_ERR_DEVICE_CHECK (or
+ * DSA_ERR_TIMEOUT if that bit is set) when any kernel on the current device
+ * set a bit of the device error word since the last check, stores the word in
+ * *bits (if non-NULL) and clears it.  DSA_OK otherwise.
+ */
+dsa_status_t dsa_check_errors(void* stream, uint32_t* bits);
+
+/*
+ * dsa_launch_count - number of kernels this library has launched in this
+ * process so far (all devices, all threads).  Callers difference two readings
+ * to count the launches of a region of work.
+ */
+uint64_t dsa_launch_count(void);
+
+/* Text of the last failure reported on the calling thread ("" if none). */
+const char* dsa_last_error(void);
+
+/* ABI version of this library (major * 100 + minor). */
+int32_t dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

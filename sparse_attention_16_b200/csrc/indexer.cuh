@@ -1,0 +1,330 @@
+// indexer.cuh - the DSA lightning indexer on sm_100a tensor cores.
+//
+// Computes I[t,s] = sum_{j<32} w[t,j] * max(0, q[t,j,:] . k[s,:]) (the concept
+// page's "Where to look" / "Sparse attention": 32 small heads, 32 x 128
+// multiply-adds per scored position).
+//
+// One tile = 128 consecutive key rows of one sequence x QG queries (QG = 1 for
+// decode, 8 for chunked prefill).  The 128 x 128 bf16 key tile and the
+// (32*QG) x 128 query block are brought into shared memory by TMA with the
+// 128-byte swizzle; one tcgen05.mma chain (M = 128 keys, N = 32*QG, K = 128)
+// leaves, in TMEM lane r, the 32 head dot products of key r for every query in
+// the group.  The epilogue applies ReLU, the head weights and the head sum in
+// registers, so each key row costs one TMEM row read and a 32-term FMA chain.
+//
+// Warp roles (persistent CTA, one per SM, contiguous range of tiles):
+//   warp 0        TMA producer (key tiles ring, query block buffers)
+//   warp 1        TMEM owner + single-thread MMA issuer
+//   warps 2..     epilogue (4 or 8 warps), two TMEM accumulators in flight
+#pragma once
+
+#include <cuda.h>
+
+#include "ptx.cuh"
+
+namespace dsa {
+
+constexpr int kIdxHeads = 32;
+constexpr int kIdxDim = 128;
+constexpr int kKeyTile = 128;
+
+template <int QG>
+struct IdxCfg {
+  static constexpr int N = 32 * QG;                     // MMA N: heads x queries
+  static constexpr int STAGES = (QG == 1) ? 6 : 4;      // key tiles in flight
+  static constexpr int QBUFS = (QG == 1) ? 2 : 1;       // query blocks in flight
+  static constexpr int KHALF = kKeyTile * 128;          // bytes of one 64-column half
+  static constexpr int KT_BYTES = 2 * KHALF;            // 32 KB per key tile
+  static constexpr int QHALF = N * 128;
+  static constexpr int Q_BYTES = 2 * QHALF;
+  static constexpr int EPI_WARPS = (QG == 1) ? 4 : 8;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int TMEM_COLS = (2 * N < 32) ? 32 : 2 * N;
+  static constexpr int SMEM_TILES = STAGES * KT_BYTES + QBUFS * Q_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024 + EPI_WARPS * ((QG == 1) ? 1 : 4) * kIdxHeads * 4;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(128, N, 0, 0);
+};
+
+struct IndexerParams {
+  const float* w;                 // [T, 32]
+  const int64_t* seq_row_start;   // [B]
+  const int32_t* q_seq;           // [T]
+  const int32_t* q_pos;           // [T]
+  float* scores;                  // [T, ld]
+  int64_t ld;
+  int64_t n_rows;
+  int64_t n_units;                // n_groups * n_kt
+  int32_t T;
+  int32_t B;
+  int32_t n_kt;                   // ceil(ld / 128)
+};
+
+struct GroupInfo {
+  int64_t row_base;   // first key row of the sequence
+  int32_t maxpos;     // largest candidate position over the group (-1: none)
+};
+
+template <int QG>
+__device__ __forceinline__ GroupInfo load_group(const IndexerParams& p, int g, bool report) {
+  GroupInfo gi{0, -1};
+  const int t0 = g * QG;
+  const int b = p.q_seq[t0];
+  if (b < 0 || b >= p.B) {
+    if (report) raise_error(kErrBadSeq);
+    return gi;
+  }
+  gi.row_base = p.seq_row_start[b];
+  int mx = -1;
+#pragma unroll
+  for (int i = 0; i < QG; ++i) {
+    const int t = t0 + i;
+    if (t < p.T) {
+      if (QG > 1 && p.q_seq[t] != b && report) raise_error(kErrMixedGroup);
+      int qp = p.q_pos[t];
+      if (qp >= p.ld) {
+        if (report) raise_error(kErrBadSeq);
+        qp = (int)p.ld - 1;
+      }
+      mx = max(mx, qp);
+    }
+  }
+  if (mx >= 0 && gi.row_base + mx >= p.n_rows) {
+    if (report) raise_error(kErrBadSeq);
+  }
+  gi.maxpos = mx;
+  return gi;
+}
+
+struct Ring {
+  int idx;
+  uint32_t phase;
+  __device__ __forceinline__ void next(int n) {
+    if (++idx == n) {
+      idx = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+template <int QG>
+__global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                   const IndexerParams p) {
+  using C = IdxCfg<QG>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* ktiles = smem;
+  uint8_t* qbufs = smem + C::STAGES * C::KT_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_TILES);
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = k_full + C::STAGES;
+  uint64_t* q_full = k_empty + C::STAGES;
+  uint64_t* q_empty = q_full + C::QBUFS;
+  uint64_t* acc_full = q_empty + C::QBUFS;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* mma_done = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* w_s = reinterpret_cast<float*>(smem + C::SMEM_TILES + 1024);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < C::QBUFS; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], C::EPI_WARPS);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int64_t u_begin = (int64_t)blockIdx.x * p.n_units / gridDim.x;
+  const int64_t u_end = (int64_t)(blockIdx.x + 1) * p.n_units / gridDim.x;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tmap(&kmap);
+      prefetch_tmap(&qmap);
+      Ring ks{0, 0}, qs{C::QBUFS - 1, 1u};
+      int cur_g = -1;
+      GroupInfo gi{0, -1};
+      bool kused[C::STAGES] = {};
+      uint32_t klast[C::STAGES] = {};
+      bool qused[C::QBUFS] = {};
+      uint32_t qlast[C::QBUFS] = {};
+      bool ok = true;
+      for (int64_t u = u_begin; u < u_end && ok; ++u) {
+        const int g = (int)(u / p.n_kt);
+        const int kt = (int)(u % p.n_kt);
+        if (g != cur_g) {
+          gi = load_group<QG>(p, g, true);
+          cur_g = g;
+          qs.next(C::QBUFS);
+          if (!mbar_wait(&q_empty[qs.idx], qs.phase ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&q_full[qs.idx], C::Q_BYTES);
+          uint8_t* qb = qbufs + qs.idx * C::Q_BYTES;
+          tma_load_2d(qb, &qmap, 0, g * C::N, &q_full[qs.idx]);
+          tma_load_2d(qb + C::QHALF, &qmap, 64, g * C::N, &q_full[qs.idx]);
+          qused[qs.idx] = true;
+          qlast[qs.idx] = qs.phase;
+        }
+        if (kt * kKeyTile > gi.maxpos) continue;   // nothing to score in this tile
+        if (!mbar_wait(&k_empty[ks.idx], ks.phase ^ 1u, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&k_full[ks.idx], C::KT_BYTES);
+        uint8_t* kb = ktiles + ks.idx * C::KT_BYTES;
+        const int32_t row0 = (int32_t)(gi.row_base + (int64_t)kt * kKeyTile);
+        tma_load_2d(kb, &kmap, 0, row0, &k_full[ks.idx]);
+        tma_load_2d(kb + C::KHALF, &kmap, 64, row0, &k_full[ks.idx]);
+        kused[ks.idx] = true;
+        klast[ks.idx] = ks.phase;
+        ks.next(C::STAGES);
+      }
+      if (!ok) *abort_flag = 1;
+      // Never leave the CTA with TMA writes still landing in its shared memory.
+      for (int i = 0; i < C::STAGES; ++i)
+        if (kused[i]) mbar_wait(&k_full[i], klast[i], nullptr);
+      for (int i = 0; i < C::QBUFS; ++i)
+        if (qused[i]) mbar_wait(&q_full[i], qlast[i], nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      Ring ks{0, 0}, qs{C::QBUFS - 1, 1u}, as{0, 0};
+      int cur_g = -1;
+      GroupInfo gi{0, -1};
+      bool ok = true;
+      for (int64_t u = u_begin; u < u_end && ok; ++u) {
+        if (*abort_flag) { ok = false; break; }
+        const int g = (int)(u / p.n_kt);
+        const int kt = (int)(u % p.n_kt);
+        if (g != cur_g) {
+          gi = load_group<QG>(p, g, false);
+          if (cur_g >= 0) mma_commit(&q_empty[qs.idx]);   // old query block free once drained
+          cur_g = g;
+          qs.next(C::QBUFS);
+          if (!mbar_wait(&q_full[qs.idx], qs.phase, abort_flag)) { ok = false; break; }
+        }
+        if (kt * kKeyTile > gi.maxpos) continue;
+        if (!mbar_wait(&acc_empty[as.idx], as.phase ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&k_full[ks.idx], ks.phase, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kaddr = smem_u32(ktiles + ks.idx * C::KT_BYTES);
+        const uint32_t qaddr = smem_u32(qbufs + qs.idx * C::Q_BYTES);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(as.idx * C::N);
+#pragma unroll
+        for (int kk = 0; kk < kIdxDim / 16; ++kk) {
+          const uint32_t off = (uint32_t)((kk & 3) * 32);
+          const uint64_t ad = sdesc_sw128(kaddr + (kk >> 2) * C::KHALF + off, 16, 1024);
+          const uint64_t bd = sdesc_sw128(qaddr + (kk >> 2) * C::QHALF + off, 16, 1024);
+          mma_bf16_ss(d_tmem, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&k_empty[ks.idx]);
+        mma_commit(&acc_full[as.idx]);
+        ks.next(C::STAGES);
+        as.next(2);
+      }
+      if (!ok) *abort_flag = 1;
+      // Drain: every MMA issued by this thread has finished before TMEM is freed.
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int epi = warp - 2;                     // 0 .. EPI_WARPS-1
+    const int quarter = warp & 3;                 // TMEM lanes this warp may read
+    const int row = quarter * 32 + lane;          // key row within the tile
+    constexpr int QPW = (QG == 1) ? 1 : 4;        // queries per epilogue warp
+    const int qbase = (QG == 1) ? 0 : (epi >> 2) * 4;
+    float* w_my = w_s + epi * (QPW * kIdxHeads);
+    Ring as{0, 0};
+    int cur_g = -1;
+    GroupInfo gi{0, -1};
+    int qpos_q[QPW];
+    for (int64_t u = u_begin; u < u_end; ++u) {
+      if (*abort_flag) break;
+      const int g = (int)(u / p.n_kt);
+      const int kt = (int)(u % p.n_kt);
+      if (g != cur_g) {
+        gi = load_group<QG>(p, g, false);
+        cur_g = g;
+        // Weights of this warp's queries, in a warp-private slice of shared memory.
+        __syncwarp();
+#pragma unroll
+        for (int qi = 0; qi < QPW; ++qi) {
+          const int t = g * QG + qbase + qi;
+          w_my[qi * kIdxHeads + lane] = (t < p.T) ? p.w[(int64_t)t * kIdxHeads + lane] : 0.f;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int qi = 0; qi < QPW; ++qi) {
+          const int t = g * QG + qbase + qi;
+          int qp = (t < p.T) ? p.q_pos[t] : -1;
+          qpos_q[qi] = (qp >= p.ld) ? (int)p.ld - 1 : qp;
+          if (gi.maxpos < 0) qpos_q[qi] = -1;     // bad sequence id: nothing valid
+        }
+      }
+      const int64_t pos = (int64_t)kt * kKeyTile + row;
+      float res[QPW];
+      if (kt * kKeyTile <= gi.maxpos) {
+        if (!mbar_wait(&acc_full[as.idx], as.phase, abort_flag)) { *abort_flag = 1; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int qi = 0; qi < QPW; ++qi) {
+          uint32_t v[32];
+          const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                                 (uint32_t)(as.idx * C::N + (qbase + qi) * 32);
+          tmem_ld32(taddr, v);
+          tmem_wait_ld();
+          const float* wq = w_my + qi * kIdxHeads;
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) s = fmaf(wq[j], fmaxf(__uint_as_float(v[j]), 0.f), s);
+          res[qi] = s;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[as.idx]);
+        as.next(2);
+      } else {
+#pragma unroll
+        for (int qi = 0; qi < QPW; ++qi) res[qi] = -INFINITY;
+      }
+      if (pos < p.ld) {
+#pragma unroll
+        for (int qi = 0; qi < QPW; ++qi) {
+          const int t = g * QG + qbase + qi;
+          if (t < p.T) p.scores[(int64_t)t * p.ld + pos] = (pos <= qpos_q[qi]) ? res[qi] : -INFINITY;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace dsa

@@ -1,0 +1,291 @@
+// topk.cuh - per-query top-k over fp32 scores (radix select, exact tie rule).
+//
+// Selection rule (concept page "Sparse attention": keep the best 2,048 earlier
+// positions per query; readings: ties go to the lower position, -0 == +0, NaN
+// ranks as -inf): candidates of query t are columns 0..q_pos[t].
+//
+// Scores are mapped to order-preserving 32-bit keys.  Three histogram passes
+// (11 + 11 + 10 bits) find the k-th largest key tau and how many keys equal to
+// tau must be taken (need_eq).  A final ordered pass writes the positions of
+// keys > tau and of the first need_eq keys == tau, in ascending position order
+// (output slot of a kept element = #(> tau before it) + min(#(== tau before it),
+// need_eq)), so the result is unique and deterministic.
+//
+// One query is processed by a cluster of CL CTAs (CL in {1, 2, 4, 8}); each CTA
+// owns a contiguous slice of the candidates, stages its keys in shared memory
+// when they fit, and the per-CTA histograms and counts are combined through
+// distributed shared memory with cluster barriers (hardware barriers: every
+// CTA of a cluster is co-resident, so no software spin is involved).
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "ptx.cuh"
+
+namespace dsa {
+
+namespace cg = cooperative_groups;
+
+constexpr int kTopkThreads = 1024;
+constexpr int kTopkBins = 2048;                 // passes 1 and 2 (11 bits); pass 3 uses 1024
+constexpr int kTopkStashCap = 49152;            // keys staged in shared memory per CTA
+constexpr int kTopkSmemBytes = 2 * kTopkBins * 4 + 1024 + kTopkStashCap * 4;
+
+struct TopkParams {
+  const float* scores;   // [T, ld]
+  const int32_t* q_pos;  // [T]
+  int32_t* idx;          // [T, k]
+  int32_t* count;        // [T]
+  int64_t ld;
+  int32_t T;
+  int32_t k;
+};
+
+__device__ __forceinline__ uint32_t score_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) u = 0xFF800000u;  // NaN ranks as -inf
+  if (u == 0x80000000u) u = 0u;                           // -0 == +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive scan of one uint32 per thread over the whole 1024-thread block.
+// `tmp` needs 33 words of shared memory; returns the block total in *total.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = tmp[lane];
+    uint32_t s = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    tmp[lane] = s - w;          // exclusive prefix of warp totals
+    if (lane == 31) tmp[32] = s;
+  }
+  __syncthreads();
+  const uint32_t r = tmp[warp] + x - v;
+  *total = tmp[32];
+  __syncthreads();
+  return r;
+}
+
+// Finds bin b (scanning from the top) with above(b) < need <= above(b) + h[b],
+// where above(b) counts elements in bins above b.  Writes (b, above(b)) to res.
+template <int NB>
+__device__ __forceinline__ void find_threshold_bin(const uint32_t* h, uint32_t need, uint32_t* tmp,
+                                                   uint32_t* res) {
+  constexpr int PER = NB / kTopkThreads;  // 2 or 1 bins per thread, descending
+  uint32_t mine = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) mine += h[NB - 1 - (threadIdx.x * PER + i)];
+  uint32_t total;
+  uint32_t above = block_excl_scan(mine, tmp, &total);
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int b = NB - 1 - (threadIdx.x * PER + i);
+    const uint32_t c = h[b];
+    if (above < need && need <= above + c) {
+      res[0] = (uint32_t)b;
+      res[1] = above;
+    }
+    above += c;
+  }
+  __syncthreads();
+}
+
+template <int CL>
+__device__ __forceinline__ void cluster_barrier() {
+  if constexpr (CL > 1) {
+    cg::this_cluster().sync();
+  } else {
+    __syncthreads();
+  }
+}
+
+// Sums the NB-bin histograms of all CTAs in the cluster into `tot`.
+template <int CL, int NB>
+__device__ __forceinline__ void cluster_sum_hist(uint32_t* hist, uint32_t* tot) {
+  cluster_barrier<CL>();
+  if constexpr (CL > 1) {
+    cg::cluster_group cl = cg::this_cluster();
+    for (int b = threadIdx.x; b < NB; b += kTopkThreads) {
+      uint32_t s = 0;
+#pragma unroll
+      for (int r = 0; r < CL; ++r) s += cl.map_shared_rank(hist, r)[b];
+      tot[b] = s;
+    }
+  } else {
+    for (int b = threadIdx.x; b < NB; b += kTopkThreads) tot[b] = hist[b];
+  }
+  cluster_barrier<CL>();  // peers are done reading `hist` before it is reused
+}
+
+template <int CL>
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
+  uint32_t* tot = hist + kTopkBins;
+  uint32_t* tmp = tot + kTopkBins;           // 33 words of scan scratch
+  uint32_t* res = tmp + 40;                  // threshold results
+  uint32_t* cnt = res + 8;                   // this CTA's (#gt, #eq), read by peers
+  uint32_t* stash = reinterpret_cast<uint32_t*>(smem_raw + 2 * kTopkBins * 4 + 1024);
+
+  const int t = blockIdx.x / CL;
+  int rank = 0;
+  if constexpr (CL > 1) rank = (int)cg::this_cluster().block_rank();
+  if (t >= p.T) return;  // whole clusters only: T * CL blocks are launched
+
+  int qp = p.q_pos[t];
+  if (qp >= p.ld) {
+    if (threadIdx.x == 0 && rank == 0) raise_error(kErrBadSeq);
+    qp = (int)p.ld - 1;
+  }
+  const int64_t n = (qp < 0) ? 0 : (int64_t)qp + 1;
+  int32_t* out = p.idx + (int64_t)t * p.k;
+
+  if (n <= p.k) {  // every candidate is kept
+    for (int64_t i = (int64_t)rank * kTopkThreads + threadIdx.x; i < p.k; i += (int64_t)CL * kTopkThreads)
+      out[i] = (i < n) ? (int32_t)i : -1;
+    if (rank == 0 && threadIdx.x == 0) p.count[t] = (int32_t)n;
+    return;
+  }
+
+  const float* row = p.scores + (int64_t)t * p.ld;
+  const int64_t lo = ((int64_t)rank * n / CL) & ~int64_t(3);
+  const int64_t hi = (rank == CL - 1) ? n : (((int64_t)(rank + 1) * n / CL) & ~int64_t(3));
+  const int64_t len = hi - lo;
+  const bool staged = len <= kTopkStashCap;
+
+  // ---- pass 1: top 11 bits
+  for (int b = threadIdx.x; b < kTopkBins; b += kTopkThreads) hist[b] = 0;
+  __syncthreads();
+  {
+    const int64_t n4 = len >> 2;
+    const float4* row4 = reinterpret_cast<const float4*>(row + lo);
+    for (int64_t i = threadIdx.x; i < n4; i += kTopkThreads) {
+      const float4 f = row4[i];
+      const uint32_t k0 = score_key(f.x), k1 = score_key(f.y), k2 = score_key(f.z), k3 = score_key(f.w);
+      atomicAdd(&hist[k0 >> 21], 1u);
+      atomicAdd(&hist[k1 >> 21], 1u);
+      atomicAdd(&hist[k2 >> 21], 1u);
+      atomicAdd(&hist[k3 >> 21], 1u);
+      if (staged) reinterpret_cast<uint4*>(stash)[i] = make_uint4(k0, k1, k2, k3);
+    }
+    for (int64_t i = (n4 << 2) + threadIdx.x; i < len; i += kTopkThreads) {
+      const uint32_t kk = score_key(row[lo + i]);
+      atomicAdd(&hist[kk >> 21], 1u);
+      if (staged) stash[i] = kk;
+    }
+  }
+  __syncthreads();
+  cluster_sum_hist<CL, kTopkBins>(hist, tot);
+  find_threshold_bin<kTopkBins>(tot, (uint32_t)p.k, tmp, res);
+  const uint32_t b1 = res[0];
+  uint32_t above = res[1];
+  uint32_t need = (uint32_t)p.k - above;
+
+  auto key_at = [&](int64_t i) -> uint32_t { return staged ? stash[i] : score_key(row[lo + i]); };
+
+  // ---- pass 2: next 11 bits of keys in bin b1
+  for (int b = threadIdx.x; b < kTopkBins; b += kTopkThreads) hist[b] = 0;
+  __syncthreads();
+  for (int64_t i = threadIdx.x; i < len; i += kTopkThreads) {
+    const uint32_t kk = key_at(i);
+    if ((kk >> 21) == b1) atomicAdd(&hist[(kk >> 10) & 0x7FFu], 1u);
+  }
+  __syncthreads();
+  cluster_sum_hist<CL, kTopkBins>(hist, tot);
+  find_threshold_bin<kTopkBins>(tot, need, tmp, res);
+  const uint32_t pre2 = (b1 << 11) | res[0];
+  above += res[1];
+  need -= res[1];
+
+  // ---- pass 3: last 10 bits of keys with prefix pre2
+  for (int b = threadIdx.x; b < 1024; b += kTopkThreads) hist[b] = 0;
+  __syncthreads();
+  for (int64_t i = threadIdx.x; i < len; i += kTopkThreads) {
+    const uint32_t kk = key_at(i);
+    if ((kk >> 10) == pre2) atomicAdd(&hist[kk & 0x3FFu], 1u);
+  }
+  __syncthreads();
+  cluster_sum_hist<CL, 1024>(hist, tot);
+  find_threshold_bin<1024>(tot, need, tmp, res);
+  const uint32_t tau = (pre2 << 10) | res[0];
+  need -= res[1];                 // keys == tau still to take (>= 1)
+  const uint32_t need_eq = need;
+
+  // ---- counts of this slice, exchanged so each CTA knows what precedes it
+  uint32_t my_gt = 0, my_eq = 0;
+  for (int64_t i = threadIdx.x; i < len; i += kTopkThreads) {
+    const uint32_t kk = key_at(i);
+    my_gt += (kk > tau);
+    my_eq += (kk == tau);
+  }
+  {
+    uint32_t tt;
+    const uint32_t g_total_dummy = block_excl_scan(my_gt, tmp, &tt);
+    (void)g_total_dummy;
+    my_gt = tt;
+    block_excl_scan(my_eq, tmp, &tt);
+    my_eq = tt;
+  }
+  if (threadIdx.x == 0) {
+    cnt[0] = my_gt;
+    cnt[1] = my_eq;
+  }
+  cluster_barrier<CL>();
+  uint32_t base_gt = 0, base_eq = 0;
+  if constexpr (CL > 1) {
+    cg::cluster_group cl = cg::this_cluster();
+    for (int r = 0; r < rank; ++r) {
+      const uint32_t* pc = cl.map_shared_rank(cnt, r);
+      base_gt += pc[0];
+      base_eq += pc[1];
+    }
+  }
+  cluster_barrier<CL>();  // peers finished reading cnt (the CTA may exit after this)
+
+  // ---- ordered compaction: 4 consecutive candidates per thread per round
+  for (int64_t r0 = 0; r0 < len; r0 += 4 * kTopkThreads) {
+    const int64_t i0 = r0 + 4 * (int64_t)threadIdx.x;
+    uint32_t kk[4];
+    uint32_t c_gt = 0, c_eq = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      kk[e] = (i0 + e < len) ? key_at(i0 + e) : 0u;
+      c_gt += (i0 + e < len) && (kk[e] > tau);
+      c_eq += (i0 + e < len) && (kk[e] == tau);
+    }
+    uint32_t total;
+    const uint32_t ex = block_excl_scan((c_gt << 16) | c_eq, tmp, &total);
+    uint32_t g = base_gt + (ex >> 16), q = base_eq + (ex & 0xFFFFu);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (i0 + e < len) {
+        if (kk[e] > tau) {
+          const uint32_t slot = g + min(q, need_eq);
+          if (slot < (uint32_t)p.k) out[slot] = (int32_t)(lo + i0 + e);
+          ++g;
+        } else if (kk[e] == tau) {
+          if (q < need_eq && g + q < (uint32_t)p.k) out[g + q] = (int32_t)(lo + i0 + e);
+          ++q;
+        }
+      }
+    }
+    base_gt += total >> 16;
+    base_eq += total & 0xFFFFu;
+  }
+  if (rank == 0 && threadIdx.x == 0) p.count[t] = p.k;
+  (void)above;
+}
+
+}  // namespace dsa

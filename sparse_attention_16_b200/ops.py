@@ -1,0 +1,222 @@
+"""ctypes binding of libdsa.so (include/dsa.h), argument marshalling only.
+
+Each function takes torch tensors (device memory owned by the caller), checks
+dtypes/shapes, and passes raw pointers and sizes to the C ABI on the current
+torch stream.  All computation happens in the library's CUDA kernels; if the
+library is missing or fails to load, every call raises - there is no CPU path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdsa.so")
+
+DSA_OK = 0
+STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_CUDA",
+          4: "DSA_ERR_DEVICE_CHECK", 5: "DSA_ERR_TIMEOUT", 6: "DSA_ERR_WORKSPACE"}
+DEVERR_BAD_INDEX, DEVERR_BAD_SEQ, DEVERR_MIXED_GROUP, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+
+SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
+
+# Every symbol include/dsa.h declares, with (restype, argtypes).
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_F = ctypes.c_float
+
+
+class LayerArgs(ctypes.Structure):
+    """Mirror of ``dsa_layer_args``."""
+
+    _fields_ = [("q_nope", _P), ("q_pe", _P), ("qmul", _P), ("cache", _P), ("ld_c", _I32),
+                ("d_rope", _I32), ("out", _P), ("lse", _P)]
+
+
+SIGNATURES = {
+    "dsa_index_scores": (_I32, [_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _P, _I64, _P]),
+    "dsa_topk_workspace_size": (_SZ, [_I32, _I64, _I32]),
+    "dsa_topk": (_I32, [_P, _I64, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
+    "sparse_mla_workspace_size": (_SZ, [_I32, _I32]),
+    "sparse_mla_attend": (_I32, [_P, _P, _P, _F, _P, _I64, _I32, _I32, _P, _I32, _P, _P, _P, _I32,
+                                 _I32, _P, _P, _P, _SZ, _P]),
+    "dsa_forward_workspace_size": (_SZ, [_I32, _I64, _I32, _I32]),
+    "dsa_sparse_mla_forward": (_I32, [_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I64, _I32,
+                                      ctypes.POINTER(LayerArgs), _F, _I32, _P, _P, _P, _SZ, _P]),
+    "dsa_check_errors": (_I32, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "dsa_launch_count": (ctypes.c_uint64, []),
+    "dsa_last_error": (ctypes.c_char_p, []),
+    "dsa_version": (_I32, []),
+}
+
+_lib = None
+
+
+class DSAError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads libdsa.so once and declares every exported function."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m sparse_attention_16_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status):
+    if status != DSA_OK:
+        raise DSAError(status, load_library().dsa_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, dtype, shape, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+# ----------------------------------------------------------------- calls
+
+def index_scores(q_idx, w, k_idx, seq_row_start, q_seq, q_pos, scores, q_group=1, stream=None):
+    """I[t, s] into ``scores`` [T, ld] (see dsa_index_scores)."""
+    T = q_idx.shape[0]
+    _need(q_idx, torch.bfloat16, (T, 32, 128), "q_idx")
+    _need(w, torch.float32, (T, 32), "w")
+    _need(k_idx, torch.bfloat16, None, "k_idx")
+    _need(seq_row_start, torch.int64, None, "seq_row_start")
+    _need(q_seq, torch.int32, (T,), "q_seq")
+    _need(q_pos, torch.int32, (T,), "q_pos")
+    _need(scores, torch.float32, None, "scores")
+    lib = load_library()
+    _check(lib.dsa_index_scores(_ptr(q_idx), _ptr(w), _ptr(k_idx), k_idx.shape[0], _ptr(seq_row_start),
+                                seq_row_start.shape[0], _ptr(q_seq), _ptr(q_pos), T, q_group,
+                                _ptr(scores), scores.shape[1], _stream(stream)))
+    return scores
+
+
+def topk(scores, q_pos, k, idx, count, stream=None):
+    """Top-k positions per query into ``idx`` [T, k] and ``count`` [T] (see dsa_topk)."""
+    T = scores.shape[0]
+    _need(scores, torch.float32, None, "scores")
+    _need(q_pos, torch.int32, (T,), "q_pos")
+    _need(idx, torch.int32, (T, k), "idx")
+    _need(count, torch.int32, (T,), "count")
+    lib = load_library()
+    _check(lib.dsa_topk(_ptr(scores), scores.shape[1], _ptr(q_pos), T, k, _ptr(idx), _ptr(count),
+                        None, 0, _stream(stream)))
+    return idx, count
+
+
+def attend_workspace_bytes(T, k):
+    return int(load_library().sparse_mla_workspace_size(T, k))
+
+
+def forward_workspace_bytes(T, ld, k, q_group=1):
+    return int(load_library().dsa_forward_workspace_size(T, ld, k, q_group))
+
+
+def workspace(nbytes, device):
+    """A 256-byte aligned uint8 device buffer (torch allocations are 512-byte aligned)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def sparse_mla_attend(q_nope, q_pe, qmul, cache, d_rope, seq_row_start, q_seq, idx, count, out,
+                      lse=None, softmax_scale=SOFTMAX_SCALE, ws=None, stream=None):
+    """Absorbed sparse MLA into ``out`` [T, 64, 512] bf16 (see sparse_mla_attend)."""
+    T = q_nope.shape[0]
+    k = idx.shape[1]
+    _need(q_nope, torch.bfloat16, (T, 64, 512), "q_nope")
+    if d_rope:
+        _need(q_pe, torch.bfloat16, (T, 64, d_rope), "q_pe")
+    _need(qmul, torch.float32, (T, 64), "qmul")
+    _need(cache, torch.bfloat16, None, "cache")
+    _need(idx, torch.int32, (T, k), "idx")
+    _need(count, torch.int32, (T,), "count")
+    _need(out, torch.bfloat16, (T, 64, 512), "out")
+    if lse is not None:
+        _need(lse, torch.float32, (T, 64), "lse")
+    lib = load_library()
+    need = attend_workspace_bytes(T, k)
+    if ws is None and need > 0:
+        ws = workspace(need, q_nope.device)
+    _check(lib.sparse_mla_attend(_ptr(q_nope), _ptr(q_pe) if d_rope else None, _ptr(qmul),
+                                 float(softmax_scale), _ptr(cache), cache.shape[0], cache.shape[1],
+                                 d_rope, _ptr(seq_row_start), seq_row_start.shape[0], _ptr(q_seq),
+                                 _ptr(idx), _ptr(count), T, k, _ptr(out), _ptr(lse), _ptr(ws),
+                                 0 if ws is None else ws.numel(), _stream(stream)))
+    return out, lse
+
+
+def sparse_mla_forward(q_idx, w, k_idx, seq_row_start, q_seq, q_pos, layers, ld, k=2048, q_group=1,
+                       idx_out=None, count_out=None, softmax_scale=SOFTMAX_SCALE, ws=None,
+                       stream=None):
+    """Indexer + top-k once, then attention for every layer (see dsa_sparse_mla_forward).
+
+    ``layers``: list of dicts with q_nope, q_pe (or None), qmul, cache, d_rope, out, lse (or None).
+    """
+    T = q_idx.shape[0]
+    _need(q_idx, torch.bfloat16, (T, 32, 128), "q_idx")
+    _need(w, torch.float32, (T, 32), "w")
+    arr = (LayerArgs * max(1, len(layers)))()
+    for i, L in enumerate(layers):
+        _need(L["q_nope"], torch.bfloat16, (T, 64, 512), f"layers[{i}].q_nope")
+        _need(L["out"], torch.bfloat16, (T, 64, 512), f"layers[{i}].out")
+        arr[i] = LayerArgs(L["q_nope"].data_ptr(),
+                           L["q_pe"].data_ptr() if L.get("q_pe") is not None else None,
+                           L["qmul"].data_ptr(), L["cache"].data_ptr(), L["cache"].shape[1],
+                           L["d_rope"], L["out"].data_ptr(),
+                           L["lse"].data_ptr() if L.get("lse") is not None else None)
+    lib = load_library()
+    if ws is None:
+        ws = workspace(forward_workspace_bytes(T, ld, k, q_group), q_idx.device)
+    _check(lib.dsa_sparse_mla_forward(_ptr(q_idx), _ptr(w), _ptr(k_idx), k_idx.shape[0],
+                                      _ptr(seq_row_start), seq_row_start.shape[0], _ptr(q_seq),
+                                      _ptr(q_pos), T, q_group, ld, len(layers), arr,
+                                      float(softmax_scale), k, _ptr(idx_out), _ptr(count_out),
+                                      _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def launch_count():
+    """Kernels launched by the library in this process so far."""
+    return int(load_library().dsa_launch_count())
+
+
+def check_errors(stream=None):
+    """Synchronizes and returns the device error word (raises DSAError if set)."""
+    lib = load_library()
+    bits = ctypes.c_uint32(0)
+    st = lib.dsa_check_errors(_stream(stream), ctypes.byref(bits))
+    if st != DSA_OK:
+        raise DSAError(st, lib.dsa_last_error().decode() + f" (bits=0x{bits.value:x})")
+    return bits.value

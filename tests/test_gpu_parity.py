@@ -1,0 +1,278 @@
+"""GPU parity: every C-ABI call against the fp64 oracle on seeded inputs.
+
+Sizes span several tiles and ragged tails while the oracle still finishes in
+seconds; the full-size configurations are checked on sampled queries in
+test_gpu_fullsize.py.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_16_b200 import ops
+from sparse_attention_16_b200.workloads import (CONFIGS, SOFTMAX_SCALE, make_workload, small_case,
+                                                to_numpy)
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    ops.load_library()
+    yield
+    assert ops.check_errors() == 0
+
+
+# ------------------------------------------------------------------ indexer
+
+INDEX_CASES = [
+    small_case("ragged_decode", (4096, 4096, 1500, 37, 129, 128, 1), seed=11),
+    small_case("one_long", (20000,), seed=12),
+    small_case("many_short", tuple(range(1, 400, 23)), seed=13),
+]
+
+
+@pytest.mark.parametrize("case", INDEX_CASES, ids=lambda c: c.name)
+def test_indexer_matches_oracle_decode(case):
+    wl = make_workload(case, DEV)
+    s = pu.gpu_scores(wl)
+    ts = list(range(wl.T))
+    ref = pu.oracle_scores(wl, ts, case.ld)
+    pu.assert_scores_close(to_numpy(s), ref, to_numpy(wl.q_pos))
+
+
+@pytest.mark.parametrize("new", [45, 64, 8, 3])
+def test_indexer_matches_oracle_prefill_groups(new):
+    case = small_case(f"prefill_{new}", kind="prefill", cached=700, new=new, seed=14)
+    wl = make_workload(case, DEV)
+    for qg in (8, 1):
+        s = pu.gpu_scores(wl, q_group=qg)
+        ref = pu.oracle_scores(wl, list(range(wl.T)), case.ld)
+        pu.assert_scores_close(to_numpy(s), ref, to_numpy(wl.q_pos))
+
+
+def test_indexer_integer_inputs_are_bit_exact():
+    # Small-integer q, k and dyadic w make every product and partial sum exact in fp32.
+    case = small_case("int_exact", (3000, 700, 130), seed=15)
+    wl = make_workload(case, DEV)
+    g = torch.Generator(device=DEV).manual_seed(5)
+    wl.q_idx = torch.randint(-3, 4, wl.q_idx.shape, generator=g, device=DEV).to(torch.bfloat16)
+    wl.k_idx = torch.randint(-3, 4, wl.k_idx.shape, generator=g, device=DEV).to(torch.bfloat16)
+    wl.w = torch.randint(-8, 9, wl.w.shape, generator=g, device=DEV).float() / 4.0
+    s = to_numpy(pu.gpu_scores(wl))
+    ref = pu.oracle_scores(wl, list(range(wl.T)), case.ld)
+    qp = to_numpy(wl.q_pos)
+    for t in range(wl.T):
+        n = qp[t] + 1
+        np.testing.assert_array_equal(s[t, :n].astype(np.float64), ref[t, :n])
+
+
+# ------------------------------------------------------------------ top-k
+
+@pytest.mark.parametrize("k", [2048, 1, 7, 4096])
+def test_topk_bit_exact_on_gpu_scores(k):
+    case = small_case("topk_src", (4096, 9000, 1500, 37, 2049, 2048), seed=16)
+    wl = make_workload(case, DEV)
+    s = pu.gpu_scores(wl)
+    idx, cnt = pu.gpu_topk(s, wl.q_pos, k)
+    pu.assert_topk_exact(to_numpy(idx), to_numpy(cnt), to_numpy(s).astype(np.float64),
+                         to_numpy(wl.q_pos), k)
+
+
+@pytest.mark.parametrize("T,ld", [(1, 100_000), (1, 500_000), (200, 40_000), (100, 5_000), (3, 131_072)])
+def test_topk_cluster_sizes_and_ties(T, ld):
+    # Integer-valued scores: heavy ties everywhere, including at the threshold.
+    g = torch.Generator(device=DEV).manual_seed(T * 7 + ld)
+    scores = torch.randint(-40, 41, (T, ld), generator=g, device=DEV).float()
+    scores[:, ::5] = -0.0
+    q_pos = torch.randint(ld // 2, ld, (T,), generator=g, device=DEV, dtype=torch.int32)
+    q_pos[0] = ld - 1
+    idx, cnt = pu.gpu_topk(scores, q_pos, 2048)
+    pu.assert_topk_exact(to_numpy(idx), to_numpy(cnt), to_numpy(scores).astype(np.float64),
+                         to_numpy(q_pos), 2048)
+
+
+def test_topk_special_values_and_short_rows():
+    ld = 6000
+    s = torch.randn((6, ld), device=DEV)
+    s[0, :] = 1.0                        # all equal: lowest positions win
+    s[1, 100:3000] = float("nan")        # NaN ranks as -inf
+    s[2, :] = -0.0
+    s[2, ::2] = 0.0                      # signed zeros are equal
+    s[3, 500:700] = float("inf")
+    q_pos = torch.tensor([5999, 5999, 5999, 5999, 100, -1], dtype=torch.int32, device=DEV)
+    idx, cnt = pu.gpu_topk(s, q_pos, 2048)
+    pu.assert_topk_exact(to_numpy(idx), to_numpy(cnt), to_numpy(s).astype(np.float64),
+                         to_numpy(q_pos), 2048)
+    assert to_numpy(cnt).tolist()[-2:] == [101, 0]
+
+
+# ------------------------------------------------------------------ attention
+
+def _random_selection(wl, counts, sort=True, holes=False, seed=0):
+    rng = np.random.default_rng(seed)
+    q_pos = to_numpy(wl.q_pos)
+    k = 2048
+    idx = np.full((wl.T, k), -1, np.int32)
+    for t, c in enumerate(counts):
+        n = int(q_pos[t]) + 1
+        c = min(c, n)
+        sel = rng.choice(n, c, replace=False)
+        if sort:
+            sel = np.sort(sel)
+        idx[t, :c] = sel
+        if holes and c > 10:
+            idx[t, 3] = -1      # skipped entries inside the counted prefix
+    cnt = np.array([min(c, int(q_pos[t]) + 1) for t, c in enumerate(counts)], np.int32)
+    return idx, cnt
+
+
+@pytest.mark.parametrize("d_rope", [64, 0])
+@pytest.mark.parametrize("sort", [True, False])
+def test_attention_matches_oracle_split_path(d_rope, sort):
+    # 5 queries: the kernel splits each selection across several CTAs and merges.
+    case = small_case("attn_split", (4096, 3000, 2100, 600, 50), layers=(d_rope,), seed=17)
+    wl = make_workload(case, DEV)
+    idx, cnt = _random_selection(wl, [2048, 1500, 2048, 129, 37], sort=sort, holes=not sort, seed=3)
+    lay = wl.layers[0]
+    o, lse = pu.gpu_attend(wl, lay, torch.as_tensor(idx, device=DEV), torch.as_tensor(cnt, device=DEV))
+    ref_o, ref_l = pu.oracle_attend(wl, lay, list(range(wl.T)), idx, cnt)
+    pu.assert_attention_close(to_numpy(o), to_numpy(lse), ref_o, ref_l)
+
+
+@pytest.mark.parametrize("d_rope", [64, 0])
+def test_attention_matches_oracle_single_split_path(d_rope):
+    # Enough queries that each one is handled by one CTA (bf16 written directly).
+    lengths = tuple(int(x) for x in np.random.default_rng(4).integers(1, 3000, size=160))
+    case = small_case("attn_many", lengths, layers=(d_rope,), seed=18, mla_q_std=1.0)
+    wl = make_workload(case, DEV)
+    counts = [2048 if i % 3 else int(lengths[i]) for i in range(len(lengths))]
+    idx, cnt = _random_selection(wl, counts, seed=5)
+    lay = wl.layers[0]
+    o, lse = pu.gpu_attend(wl, lay, torch.as_tensor(idx, device=DEV), torch.as_tensor(cnt, device=DEV))
+    ts = list(range(0, wl.T, 7))
+    ref_o, ref_l = pu.oracle_attend(wl, lay, ts, idx, cnt)
+    pu.assert_attention_close(to_numpy(o)[ts], to_numpy(lse)[ts], ref_o, ref_l)
+
+
+def test_attention_empty_selection_gives_zero_and_minus_inf():
+    case = small_case("attn_empty", (300, 300), seed=19)
+    wl = make_workload(case, DEV)
+    idx = torch.full((2, 2048), -1, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros(2, dtype=torch.int32, device=DEV)
+    o, lse = pu.gpu_attend(wl, wl.layers[0], idx, cnt)
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_attention_softmax_rows_sum_to_one():
+    # sum_i exp(z_i - lse_gpu) = 1 with z recomputed by the oracle's definition.
+    case = small_case("attn_norm", (2500, 900), seed=20)
+    wl = make_workload(case, DEV)
+    idx, cnt = _random_selection(wl, [2048, 700], seed=6)
+    lay = wl.layers[0]
+    _, lse = pu.gpu_attend(wl, lay, torch.as_tensor(idx, device=DEV), torch.as_tensor(cnt, device=DEV))
+    lse = to_numpy(lse).astype(np.float64)
+    starts, q_seq, _ = pu.host_meta(wl)
+    cache = to_numpy(lay.cache).astype(np.float64)
+    for t in range(wl.T):
+        rows = cache[starts[q_seq[t]] + idx[t, :cnt[t]]]
+        z = (to_numpy(lay.q_nope[t]).astype(np.float64) @ rows[:, :512].T
+             + to_numpy(lay.q_pe[t]).astype(np.float64) @ rows[:, 512:576].T)
+        z *= SOFTMAX_SCALE * to_numpy(lay.qmul[t]).astype(np.float64)[:, None]
+        s = np.exp(z - lse[t][:, None]).sum(1)
+        np.testing.assert_allclose(s, 1.0, atol=2e-3)
+
+
+# ------------------------------------------------------------------ fused forward
+
+def test_forward_tiny_decode_config_end_to_end():
+    case = CONFIGS["tiny_decode"]
+    wl = make_workload(case, DEV)
+    T, ld = wl.T, case.ld
+    lay = wl.layers[0]
+    out = torch.empty((T, 64, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((T, 64), dtype=torch.float32, device=DEV)
+    idx = torch.empty((T, 2048), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((T,), dtype=torch.int32, device=DEV)
+    ops.sparse_mla_forward(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos,
+                           [dict(q_nope=lay.q_nope, q_pe=lay.q_pe, qmul=lay.qmul, cache=lay.cache,
+                                 d_rope=64, out=out, lse=lse)], ld, idx_out=idx, count_out=cnt)
+    torch.cuda.synchronize()
+    assert to_numpy(cnt).tolist() == [2048, 2048, 1500, 37]
+    ref_scores = pu.oracle_scores(wl, list(range(T)), ld)
+    idx_h, cnt_h = to_numpy(idx), to_numpy(cnt)
+    for t in range(T):
+        n = int(to_numpy(wl.q_pos)[t]) + 1
+        pu.assert_selection_overlap(idx_h[t, :cnt_h[t]], ref_scores[t, :n], 2048)
+    # attention parity on the GPU's own selection
+    ref_o, ref_l = pu.oracle_attend(wl, lay, list(range(T)), idx_h, cnt_h)
+    pu.assert_attention_close(to_numpy(out), to_numpy(lse), ref_o, ref_l)
+    # and the fused call equals the three separate calls bit for bit
+    s = pu.gpu_scores(wl)
+    idx2, cnt2 = pu.gpu_topk(s, wl.q_pos, 2048)
+    o2, l2 = pu.gpu_attend(wl, lay, idx2, cnt2)
+    assert torch.equal(idx2, idx) and torch.equal(o2, out) and torch.equal(l2, lse)
+
+
+def test_forward_one_selection_feeds_rope_and_nope_layers_with_chunking():
+    case = small_case("fwd_prefill", kind="prefill", cached=3000, new=40, layers=(64, 0), seed=21,
+                      mla_q_std=1.0)
+    wl = make_workload(case, DEV)
+    T, ld = wl.T, case.ld
+    outs = [torch.empty((T, 64, 512), dtype=torch.bfloat16, device=DEV) for _ in wl.layers]
+    lses = [torch.empty((T, 64), dtype=torch.float32, device=DEV) for _ in wl.layers]
+    layers = [dict(q_nope=L.q_nope, q_pe=L.q_pe, qmul=L.qmul, cache=L.cache, d_rope=L.d_rope, out=o,
+                   lse=l) for L, o, l in zip(wl.layers, outs, lses)]
+    idx = torch.empty((T, 2048), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((T,), dtype=torch.int32, device=DEV)
+    # a workspace for 16 queries forces three chunks (16 + 16 + 8)
+    ws = ops.workspace(ops.forward_workspace_bytes(16, ld, 2048, 8), DEV)
+    ops.sparse_mla_forward(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, layers, ld,
+                           q_group=8, idx_out=idx, count_out=cnt, ws=ws)
+    torch.cuda.synchronize()
+    idx_h, cnt_h = to_numpy(idx), to_numpy(cnt)
+    s_ref = pu.oracle_scores(wl, list(range(T)), ld)
+    for t in range(T):
+        n = int(to_numpy(wl.q_pos)[t]) + 1
+        pu.assert_selection_overlap(idx_h[t, :cnt_h[t]], s_ref[t, :n], 2048)
+    for L, o, l in zip(wl.layers, outs, lses):
+        ref_o, ref_l = pu.oracle_attend(wl, L, list(range(T)), idx_h, cnt_h)
+        pu.assert_attention_close(to_numpy(o), to_numpy(l), ref_o, ref_l)
+
+
+# ------------------------------------------------------------------ device-side checks
+
+def test_bad_indices_are_flagged_not_faulted():
+    case = small_case("bad_idx", (500, 500), seed=22)
+    wl = make_workload(case, DEV)
+    idx, cnt = _random_selection(wl, [300, 300], seed=7)
+    idx[0, 5] = 10_000_000          # far outside the cache
+    idx[1, 7] = -5                  # negative, not the -1 padding value
+    out = torch.empty((2, 64, 512), dtype=torch.bfloat16, device=DEV)
+    ops.sparse_mla_attend(wl.layers[0].q_nope, wl.layers[0].q_pe, wl.layers[0].qmul, wl.layers[0].cache,
+                          64, wl.seq_row_start, wl.q_seq, torch.as_tensor(idx, device=DEV),
+                          torch.as_tensor(cnt, device=DEV), out)
+    with pytest.raises(ops.DSAError) as e:
+        ops.check_errors()
+    assert "0x1" in str(e.value)
+    assert ops.check_errors() == 0   # cleared; the context is still usable
+    assert torch.isfinite(out.float()).all()
+
+
+def test_bad_sequence_ids_are_flagged():
+    case = small_case("bad_seq", (500, 500), seed=23)
+    wl = make_workload(case, DEV)
+    wl.q_seq[1] = 7                 # only 2 sequences exist
+    s = torch.empty((2, wl.case.ld), dtype=torch.float32, device=DEV)
+    ops.index_scores(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, s)
+    with pytest.raises(ops.DSAError):
+        ops.check_errors()
+    assert torch.isneginf(s[1]).all()
