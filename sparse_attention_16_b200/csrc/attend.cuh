@@ -269,6 +269,9 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
     const int quarter = warp;
     const int r = quarter * 32 + lane;         // tile row == TMEM lane
     const uint32_t lane_base = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    const int sb = p.q_seq[t];
+    const bool seq_ok = (sb >= 0 && sb < p.B);
+    const int64_t seq_base = seq_ok ? p.seq_row_start[sb] : 0;
     if (st < kHeads) {
       sc->fac[st] = p.qmul[(int64_t)t * kHeads + st] * p.scale_log2e;
       sc->m_used[st] = -INFINITY;
@@ -289,7 +292,13 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
       tmem_ld32(lane_base + C::S_COL, v0);
       tmem_ld32(lane_base + C::S_COL + 32, v1);
       tmem_wait_ld();
-      const bool valid = r < nvalid;
+      // A row takes part only if its index is a real position of the sequence
+      // (entries of -1 inside the counted prefix are skipped).
+      bool valid = false;
+      if (r < nvalid && seq_ok) {
+        const int32_t sidx = p.idx[(int64_t)t * p.k + r_begin + i * C::ROWS + r];
+        valid = sidx >= 0 && seq_base + sidx < p.n_rows;
+      }
       float z[kHeads];
 #pragma unroll
       for (int h = 0; h < 32; ++h) {
@@ -356,9 +365,11 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
           const int h0 = q8 * 8 + 2 * e;
           const float p0 = ex2_approx(z[h0] - sc->m_used[h0]);
           const float p1 = ex2_approx(z[h0 + 1] - sc->m_used[h0 + 1]);
-          l_part[h0] += p0;
-          l_part[h0 + 1] += p1;
           pk[e] = pack_bf16x2(p0, p1);
+          // Sum the bf16-rounded weights the tensor core multiplies, so the
+          // numerator and the denominator of the softmax use the same values.
+          l_part[h0] += __uint_as_float(pk[e] << 16);
+          l_part[h0 + 1] += __uint_as_float(pk[e] & 0xFFFF0000u);
         }
         st_shared_v4(pbase + ((q8 ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
       }

@@ -5,7 +5,7 @@ compare against the fp64 oracle with the tolerances the benchmark spec fixes:
   top-k     bit-exact when both select from the same (GPU) score array
   selection end to end: set overlap >= 99.9%, misses only where neighbouring
             scores differ by < 1e-3 relative
-  attention max |o_gpu - o_ref| <= 2e-2 (plus a relative bar: <= 2e-2 of rms(o_ref))
+  attention max |o_gpu - o_ref| <= 2e-2 (plus an internal bar: <= 1e-2 of max|o_ref| per query)
 """
 
 from __future__ import annotations
@@ -19,7 +19,7 @@ from sparse_attention_16_b200.workloads import SOFTMAX_SCALE, to_numpy
 
 SCORE_RTOL = 1e-3
 ATTN_ATOL = 2e-2
-ATTN_RRMS = 2e-2
+ATTN_REL = 1e-2     # internal bar: max error <= 1% of the query's largest |o|
 LSE_ATOL = 2e-3
 
 
@@ -134,9 +134,9 @@ def assert_attention_close(gpu_o, gpu_lse, ref_o, ref_lse):
     err = np.abs(g - ref_o)
     assert err.max() <= ATTN_ATOL, f"max abs err {err.max():.3e}"
     for t in range(ref_o.shape[0]):
-        rms = float(np.sqrt(np.mean(ref_o[t] ** 2)))
-        if rms > 0:
-            assert err[t].max() <= ATTN_RRMS * rms + 1e-6, f"query {t}: max err {err[t].max():.3e} vs rms {rms:.3e}"
+        mx = float(np.abs(ref_o[t]).max())
+        if mx > 0:
+            assert err[t].max() <= ATTN_REL * mx + 1e-6, f"query {t}: max err {err[t].max():.3e} vs max|o| {mx:.3e}"
     if gpu_lse is not None:
         both_inf = np.isneginf(gpu_lse) & np.isneginf(ref_lse)
         d = np.abs(np.where(both_inf, 0.0, gpu_lse.astype(np.float64) - ref_lse))
