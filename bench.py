@@ -39,6 +39,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from sparse_attention_16_b200 import accounting as acc  # noqa: E402
+from sparse_attention_16_b200 import replicas  # noqa: E402
 from sparse_attention_16_b200.workloads import CONFIGS, make_workload, small_case  # noqa: E402
 
 HEADLINE = "decode_b64_32k"
@@ -146,7 +147,7 @@ def run_ours(args, rank, world, local):
                                              device_id=dev)
     case = CONFIGS[args.config]
     # each rank owns an independent batch of the same shape (its own seed)
-    case = type(case)(**{**case.__dict__, "seed": case.seed + 1000 * rank})
+    case = type(case)(**{**case.__dict__, "seed": replicas.rank_seed(case.seed, rank)})
     wl = make_workload(case, dev)
     T, ld, k = wl.T, case.ld, case.topk
     q_group = 8 if case.kind == "prefill" else 1
@@ -202,11 +203,9 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     launches = ops.launch_count() - n0
     elapsed = t0.elapsed_time(t1) / 1e3
-    el = torch.tensor([elapsed], device=dev, dtype=torch.float64)
+    elapsed = replicas.max_over_ranks(elapsed, device=dev)
     if world > 1:
-        torch.distributed.all_reduce(el, op=torch.distributed.ReduceOp.MAX)
         torch.distributed.barrier()
-    elapsed = float(el.item())
     clocks = sampler.stop() if sampler else None
     ops.check_errors()
 
@@ -236,8 +235,7 @@ def run_ours(args, rank, world, local):
     # ---- end to end through the C ABI with host buffers
     e2e = run_e2e(args, wl, ld, k, q_group, dev) if not args.no_e2e else None
 
-    total_queries = T * world * args.steps
-    value = total_queries / elapsed
+    value = replicas.job_throughput(T, world, args.steps, elapsed)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "queries/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(elapsed / args.steps * 1e3, 4),
