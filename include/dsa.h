@@ -143,6 +143,42 @@ dsa_status_t sparse_mla_attend(const void* q_nope, const void* q_pe, const float
                                int32_t T, int32_t k, void* out, float* lse, void* workspace,
                                size_t ws_bytes, void* stream);
 
+/*
+ * sparse_mla_attend_noalloc - sparse_mla_attend for callers that cannot
+ * allocate device memory.
+ *
+ * The pages have no counterpart to this call: it is a convenience of this
+ * library.  Some callers are handed only their input and output buffers and
+ * may not allocate, for example code running inside another framework's
+ * memory pool or an inference-engine plugin, where a cudaMalloc would bypass
+ * the pool's accounting and can synchronize the whole device.  This call takes
+ * the arguments of sparse_mla_attend without the workspace and computes the
+ * same result with the same kernels; when a query's selection is split across
+ * several thread blocks, the partial results go to a fixed scratch array
+ * inside the library instead of a caller buffer.
+ *   - Scratch: a file-scope __device__ array of DSA_NOALLOC_MAX_PARTIALS x 64 x
+ *     514 floats (16.8 MB) that every GPU loading the library holds until the
+ *     process exits.  The call allocates nothing and calls no allocating routine.
+ *   - Limit: a call needs T x n_split partials, where n_split is the number of
+ *     blocks each query is split across (1 once T reaches the SM count, so no
+ *     scratch is used then).  Calls needing more than DSA_NOALLOC_MAX_PARTIALS
+ *     return DSA_ERR_WORKSPACE with a message that states the limit.
+ *   - Set-up: the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current.  Make that first call
+ *     before any stream capture.
+ *   - Sharing: all calls on a device use the same array, which keeps the last
+ *     call's contents.  Each call overwrites every entry it reads, so nothing
+ *     needs clearing, but calls that overlap on the GPU (other streams, other
+ *     host threads) race on the array: the caller must serialize them.
+ */
+#define DSA_NOALLOC_MAX_PARTIALS 128
+dsa_status_t sparse_mla_attend_noalloc(const void* q_nope, const void* q_pe, const float* qmul,
+                                       float softmax_scale, const void* cache, int64_t n_rows,
+                                       int32_t ld_c, int32_t d_rope, const int64_t* seq_row_start,
+                                       int32_t B, const int32_t* q_seq, const int32_t* idx,
+                                       const int32_t* count, int32_t T, int32_t k, void* out,
+                                       float* lse, void* stream);
+
 /* One attention layer fed by a shared selection (fields as in sparse_mla_attend). */
 typedef struct dsa_layer_args {
   const void* q_nope;   /* bf16 [T, 64, 512]                      */

@@ -334,6 +334,42 @@ dsa_status_t check_attend_args(const void* q_nope, const void* q_pe, const float
 
 }  // namespace
 
+// =================================================================== no-allocation variant
+// Scratch for sparse_mla_attend_noalloc: the split partials (numerators, then
+// max/sum pairs) of at most kNoAllocMaxPartials (query, split) work units, in
+// the layout launch_attend expects of a workspace.  Every GPU that loads this
+// library holds the array until the process exits.
+constexpr int kNoAllocMaxPartials = DSA_NOALLOC_MAX_PARTIALS;
+static __device__ __align__(256) float g_noalloc_scratch[(size_t)kNoAllocMaxPartials * 64 * (512 + 2)];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+constexpr int kNoAllocMaxDevices = 64;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once per
+// device (host code cannot use the array's name as a device pointer).
+dsa_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  DSA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return fail(DSA_ERR_UNSUPPORTED, "device %d: sparse_mla_attend_noalloc supports devices 0..%d", dev,
+                kNoAllocMaxDevices - 1);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(DSA_ERR_CUDA, "cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DSA_OK;
+}
+
+}  // namespace
+
 // =================================================================== C ABI
 extern "C" {
 
@@ -383,6 +419,36 @@ dsa_status_t sparse_mla_attend(const void* q_nope, const void* q_pe, const float
     return fail(DSA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need, ws_bytes);
   return attend_impl(q_nope, q_pe, qmul, softmax_scale, cache, n_rows, ld_c, d_rope, seq_row_start, B,
                      q_seq, idx, count, T, k, out, lse, workspace, static_cast<cudaStream_t>(stream));
+}
+
+// Same computation as sparse_mla_attend, for callers that may not allocate:
+// the split partials go to the library's fixed scratch array instead of a
+// caller workspace.  Launches exactly the kernels sparse_mla_attend launches.
+dsa_status_t sparse_mla_attend_noalloc(const void* q_nope, const void* q_pe, const float* qmul,
+                                       float softmax_scale, const void* cache, int64_t n_rows,
+                                       int32_t ld_c, int32_t d_rope, const int64_t* seq_row_start,
+                                       int32_t B, const int32_t* q_seq, const int32_t* idx,
+                                       const int32_t* count, int32_t T, int32_t k, void* out,
+                                       float* lse, void* stream) {
+  dsa_status_t st = check_attend_args(q_nope, q_pe, qmul, cache, n_rows, ld_c, d_rope, seq_row_start, B,
+                                      q_seq, idx, count, T, k, out);
+  if (st != DSA_OK) return st;
+  DSA_REQUIRE(lse == nullptr || aligned(lse, 4), "misaligned lse");
+  if (T == 0) return DSA_OK;
+  const SplitPlan sp = attend_plan(T, k);
+  void* scratch = nullptr;
+  if (sp.n_split > 1) {
+    const int64_t partials = (int64_t)T * sp.n_split;
+    if (partials > kNoAllocMaxPartials)
+      return fail(DSA_ERR_WORKSPACE,
+                  "sparse_mla_attend_noalloc: %d queries split %d ways need %lld partials; its fixed "
+                  "scratch holds %d (use sparse_mla_attend with a workspace, or fewer queries per call)",
+                  T, sp.n_split, (long long)partials, kNoAllocMaxPartials);
+    st = noalloc_scratch(&scratch);
+    if (st != DSA_OK) return st;
+  }
+  return attend_impl(q_nope, q_pe, qmul, softmax_scale, cache, n_rows, ld_c, d_rope, seq_row_start, B,
+                     q_seq, idx, count, T, k, out, lse, scratch, static_cast<cudaStream_t>(stream));
 }
 
 // Workspace of the fused call for a chunk of Tc queries:

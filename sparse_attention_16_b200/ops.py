@@ -46,6 +46,8 @@ SIGNATURES = {
     "sparse_mla_workspace_size": (_SZ, [_I32, _I32]),
     "sparse_mla_attend": (_I32, [_P, _P, _P, _F, _P, _I64, _I32, _I32, _P, _I32, _P, _P, _P, _I32,
                                  _I32, _P, _P, _P, _SZ, _P]),
+    "sparse_mla_attend_noalloc": (_I32, [_P, _P, _P, _F, _P, _I64, _I32, _I32, _P, _I32, _P, _P, _P,
+                                         _I32, _I32, _P, _P, _P]),
     "dsa_forward_workspace_size": (_SZ, [_I32, _I64, _I32, _I32]),
     "dsa_sparse_mla_forward": (_I32, [_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I64, _I32,
                                       ctypes.POINTER(LayerArgs), _F, _I32, _P, _P, _P, _SZ, _P]),
@@ -175,6 +177,33 @@ def sparse_mla_attend(q_nope, q_pe, qmul, cache, d_rope, seq_row_start, q_seq, i
                                  d_rope, _ptr(seq_row_start), seq_row_start.shape[0], _ptr(q_seq),
                                  _ptr(idx), _ptr(count), T, k, _ptr(out), _ptr(lse), _ptr(ws),
                                  0 if ws is None else ws.numel(), _stream(stream)))
+    return out, lse
+
+
+def sparse_mla_attend_noalloc(q_nope, q_pe, qmul, cache, d_rope, seq_row_start, q_seq, idx, count,
+                              out, lse=None, softmax_scale=SOFTMAX_SCALE, stream=None):
+    """Same as sparse_mla_attend without a workspace, for callers that may not
+    allocate device memory: the library's fixed scratch array holds the split
+    partials (see sparse_mla_attend_noalloc in include/dsa.h for the limit and
+    the rule that overlapping calls must be serialized)."""
+    T = q_nope.shape[0]
+    k = idx.shape[1]
+    _need(q_nope, torch.bfloat16, (T, 64, 512), "q_nope")
+    if d_rope:
+        _need(q_pe, torch.bfloat16, (T, 64, d_rope), "q_pe")
+    _need(qmul, torch.float32, (T, 64), "qmul")
+    _need(cache, torch.bfloat16, None, "cache")
+    _need(idx, torch.int32, (T, k), "idx")
+    _need(count, torch.int32, (T,), "count")
+    _need(out, torch.bfloat16, (T, 64, 512), "out")
+    if lse is not None:
+        _need(lse, torch.float32, (T, 64), "lse")
+    lib = load_library()
+    _check(lib.sparse_mla_attend_noalloc(_ptr(q_nope), _ptr(q_pe) if d_rope else None, _ptr(qmul),
+                                         float(softmax_scale), _ptr(cache), cache.shape[0], cache.shape[1],
+                                         d_rope, _ptr(seq_row_start), seq_row_start.shape[0], _ptr(q_seq),
+                                         _ptr(idx), _ptr(count), T, k, _ptr(out), _ptr(lse),
+                                         _stream(stream)))
     return out, lse
 
 

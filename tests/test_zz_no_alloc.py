@@ -1,0 +1,90 @@
+"""sparse_mla_attend_noalloc: the attention call for callers that cannot allocate
+device memory (code that is only handed its input and output buffers, such as a
+plugin inside another framework's memory pool, where cudaMalloc would bypass the
+pool and can synchronize the device).  Its split partials live in a fixed scratch
+array inside the library instead of a caller workspace.
+
+Checked through the C ABI against sparse_mla_attend (the entry point that takes a
+workspace) with the attention tolerances used everywhere else, on two calls in a
+row with different inputs, so stale scratch contents from the first call would
+show up in the second.  This file is collected last on purpose.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from sparse_attention_16_b200 import ops
+from sparse_attention_16_b200.workloads import make_workload, small_case, to_numpy
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    ops.load_library()
+    yield
+
+
+def _selection(wl, seed):
+    rng = np.random.default_rng(seed)
+    q_pos = to_numpy(wl.q_pos)
+    idx = np.full((wl.T, 2048), -1, np.int32)
+    cnt = np.zeros(wl.T, np.int32)
+    for t in range(wl.T):
+        n = int(q_pos[t]) + 1
+        c = min(2048, n)
+        idx[t, :c] = np.sort(rng.choice(n, c, replace=False))
+        cnt[t] = c
+    return torch.as_tensor(idx, device=DEV), torch.as_tensor(cnt, device=DEV)
+
+
+def _both(wl, lay, idx, cnt):
+    T = wl.T
+    ref_o = torch.empty((T, 64, 512), dtype=torch.bfloat16, device=DEV)
+    ref_l = torch.empty((T, 64), dtype=torch.float32, device=DEV)
+    ops.sparse_mla_attend(lay.q_nope, lay.q_pe, lay.qmul, lay.cache, lay.d_rope, wl.seq_row_start, wl.q_seq,
+                          idx, cnt, ref_o, ref_l)
+    o = torch.full((T, 64, 512), float("nan"), dtype=torch.bfloat16, device=DEV)
+    l = torch.full((T, 64), float("nan"), dtype=torch.float32, device=DEV)
+    ops.sparse_mla_attend_noalloc(lay.q_nope, lay.q_pe, lay.qmul, lay.cache, lay.d_rope, wl.seq_row_start,
+                                  wl.q_seq, idx, cnt, o, l)
+    torch.cuda.synchronize()
+    return o, l, ref_o, ref_l
+
+
+@pytest.mark.parametrize("d_rope", [64, 0])
+def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(d_rope):
+    # 6 queries: each selection is split across several blocks, so the scratch is used.
+    assert ops.attend_workspace_bytes(6, 2048) > 0
+    wl1 = make_workload(small_case("na1", (4096, 3000, 2500, 600, 2049, 90), layers=(d_rope,), seed=31), DEV)
+    wl2 = make_workload(small_case("na2", (5000, 2048, 100, 4000, 3333, 777), layers=(d_rope,), seed=32,
+                                   mla_q_std=1.0), DEV)
+    for wl, seed in ((wl1, 1), (wl2, 2)):
+        idx, cnt = _selection(wl, seed)
+        o, l, ref_o, ref_l = _both(wl, wl.layers[0], idx, cnt)
+        g, r = to_numpy(o).astype(np.float64), to_numpy(ref_o).astype(np.float64)
+        assert np.abs(g - r).max() <= pu.ATTN_ATOL
+        for t in range(wl.T):
+            assert np.abs(g[t] - r[t]).max() <= pu.ATTN_REL * np.abs(r[t]).max() + 1e-6
+        assert np.abs(to_numpy(l).astype(np.float64) - to_numpy(ref_l)).max() <= pu.LSE_ATOL
+    assert ops.check_errors() == 0
+
+
+def test_noalloc_rejects_more_partials_than_its_scratch_holds():
+    lib = ops.load_library()
+    per_partial = 64 * 512 * 4
+    # find a batch size whose split plan needs more partials than the fixed scratch holds
+    T = next(T for T in range(1, 4096)
+             if ops.attend_workspace_bytes(T, 2048) // per_partial > 128)
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the call returns before launching
+    st = lib.sparse_mla_attend_noalloc(fake, fake, fake, 0.07, fake, 1000, 576, 64, fake, 1, fake, fake, fake,
+                                       T, 2048, fake, None, None)
+    assert st == 6   # DSA_ERR_WORKSPACE
+    assert b"128" in lib.dsa_last_error()
