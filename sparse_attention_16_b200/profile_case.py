@@ -1,0 +1,75 @@
+"""Runs one kernel of the hot path a few times on a configuration's inputs, for
+profiler captures (ncu) of that kernel alone.
+
+    python -m sparse_attention_16_b200.profile_case --kernel indexer --config decode_b64_32k --launches 3
+
+Only the inputs the chosen kernel reads are drawn (the indexer and top-k never
+touch the latent caches), so a capture holds little device memory.  The
+selection fed to the attention kernel comes from one untimed indexer + top-k
+pass.  Prints the mean CUDA-event time per launch.
+"""
+
+from __future__ import annotations
+
+import argparse
+import dataclasses
+
+import torch
+
+from sparse_attention_16_b200 import ops
+from sparse_attention_16_b200.workloads import CONFIGS, make_workload
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--kernel", choices=["indexer", "topk", "attend"], required=True)
+    ap.add_argument("--config", default="decode_b64_32k", choices=sorted(CONFIGS))
+    ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--layer", type=int, default=0, help="attention: which layer of the configuration")
+    a = ap.parse_args()
+
+    case = CONFIGS[a.config]
+    if a.kernel != "attend":
+        case = dataclasses.replace(case, layers=())
+    dev = torch.device("cuda", 0)
+    wl = make_workload(case, dev)
+    T, ld, k = wl.T, case.ld, case.topk
+    q_group = 8 if case.kind == "prefill" else 1
+    scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((T,), dtype=torch.int32, device=dev)
+
+    def indexer():
+        ops.index_scores(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, scores, q_group=q_group)
+
+    def topk():
+        ops.topk(scores, wl.q_pos, k, idx, cnt)
+
+    if a.kernel in ("topk", "attend"):
+        indexer()
+        topk()
+    run = {"indexer": indexer, "topk": topk}.get(a.kernel)
+    if a.kernel == "attend":
+        lay = wl.layers[a.layer]
+        out = torch.empty((T, 64, 512), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((T, 64), dtype=torch.float32, device=dev)
+        ws = ops.workspace(ops.attend_workspace_bytes(T, k), dev)
+
+        def run():
+            ops.sparse_mla_attend(lay.q_nope, lay.q_pe, lay.qmul, lay.cache, lay.d_rope, wl.seq_row_start,
+                                  wl.q_seq, idx, cnt, out, lse, ws=ws)
+
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.launches):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ops.check_errors()
+    print(f"{a.kernel} on {a.config}: {e0.elapsed_time(e1) / a.launches:.4f} ms per launch "
+          f"({a.launches} launches)", flush=True)
+
+
+if __name__ == "__main__":
+    main()
