@@ -158,6 +158,10 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
 
   if (warp >= 5) {
     // ------------------------------------------------------------- producers
+    // Thread pt copies 16-byte piece (lane & 7) of rows prow, prow + 12, ... of
+    // every chunk.  The destination offsets (with the 128-byte swizzle) depend
+    // only on the row, so they are computed once; the source row addresses once
+    // per tile; each copy then costs two adds.
     const int pt = threadIdx.x - 160;  // 0..95
     if (pt == 0 && n_tiles > 0) {
       prefetch_tmap(&qn_map);
@@ -173,43 +177,47 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
     const bool seq_ok = (b >= 0 && b < p.B);
     if (!seq_ok && pt == 0 && n_tiles > 0) raise_error(kErrBadSeq);
     const int64_t base = seq_ok ? p.seq_row_start[b] : 0;
-    const int prow = 4 * (warp - 5) + (lane >> 3);  // first row; rows advance by 12
-    const int piece = lane & 7;                       // 16-byte piece within the 128-byte chunk row
+    const int prow = 4 * (warp - 5) + (lane >> 3);  // rows prow + 12 j
+    const int piece = lane & 7;                       // 16-byte piece of the 128-byte chunk row
+    constexpr int RPT = (C::ROWS + 11) / 12;          // rows per thread (10 or 11)
+    const uint32_t cs0 = smem_u32(cs);
+    uint32_t dst[RPT];
+#pragma unroll
+    for (int j = 0; j < RPT; ++j) {
+      const int r = prow + 12 * j;
+      dst[j] = cs0 + r * 128 + ((piece ^ (r & 7)) << 4);
+    }
+    const char* cache_bytes = reinterpret_cast<const char*>(p.cache);
     bool ok = true;
-    for (int i = 0; i < n_tiles; ++i) {
+    for (int i = 0; i < n_tiles && ok; ++i) {
       const int r0 = r_begin + i * C::ROWS;
       const int nvalid = min(C::ROWS, r_end - r0);
-      // The previous tile's row list is fully consumed; leave together if any
-      // producer thread gave up waiting.
-      if (named_bar_or(2, C::PRODUCERS, !ok)) {
-        ok = false;
-        break;
-      }
-      for (int rr = pt; rr < C::ROWS; rr += C::PRODUCERS) {
-        int32_t grow = -1;
-        if (rr < nvalid && seq_ok) {
-          const int32_t s = p.idx[(int64_t)t * p.k + r0 + rr];
-          if (s >= 0 && base + s < p.n_rows) {
-            grow = (int32_t)(base + s);
-          } else if (s != -1) {
+      const char* src[RPT];
+      uint32_t nbytes[RPT];
+#pragma unroll
+      for (int j = 0; j < RPT; ++j) {
+        const int r = prow + 12 * j;
+        src[j] = cache_bytes;
+        nbytes[j] = 0;
+        if (r < C::ROWS && r < nvalid && seq_ok) {
+          const int32_t sidx = p.idx[(int64_t)t * p.k + r0 + r];
+          if (sidx >= 0 && base + sidx < p.n_rows) {
+            src[j] = cache_bytes + ((base + sidx) * p.ld_c) * 2 + piece * 16;
+            nbytes[j] = 16;
+          } else if (sidx != -1 && piece == 0) {
             raise_error(kErrBadIndex);
           }
         }
-        sc->rowidx[rr] = grow;
       }
-      named_bar_sync(2, C::PRODUCERS);
       for (int c = 0; c < C::KCH; ++c) {
         if (i > 0 && !mbar_wait(&sc->c_free[c], (uint32_t)((i - 1) & 1), abort_flag)) {
           ok = false;
           break;
         }
-        const uint32_t cbase = smem_u32(cs + c * C::CHUNK_BYTES);
-#pragma unroll 4
-        for (int r = prow; r < C::ROWS; r += 12) {
-          const int32_t g = sc->rowidx[r];
-          const __nv_bfloat16* src = p.cache + (g >= 0 ? (int64_t)g * p.ld_c + c * 64 + piece * 8 : 0);
-          const uint32_t dst = cbase + r * 128 + ((piece ^ (r & 7)) << 4);
-          cp_async_16(dst, src, g >= 0 ? 16u : 0u);
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+          if (prow + 12 * j < C::ROWS)
+            cp_async_16(dst[j] + c * C::CHUNK_BYTES, src[j] + (nbytes[j] ? c * 128 : 0), nbytes[j]);
         }
         cp_async_arrive_noinc(&sc->c_full[c]);
       }
@@ -281,17 +289,12 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
 #pragma unroll
     for (int h = 0; h < kHeads; ++h) l_part[h] = 0.f;
     const uint32_t pbase = smem_u32(ps) + r * 128;
+    const float4* fac4 = reinterpret_cast<const float4*>(sc->fac);
+    const float4* mu4 = reinterpret_cast<const float4*>(sc->m_used);
     bool ok = true;
     for (int i = 0; i < n_tiles && ok; ++i) {
       const uint32_t ph = (uint32_t)(i & 1);
       const int nvalid = min(C::ROWS, r_end - (r_begin + i * C::ROWS));
-      const bool got_s = mbar_wait(&sc->s_full, ph, abort_flag);
-      if (named_bar_or(1, 128, !got_s)) { ok = false; break; }   // leave together
-      tc_fence_after();
-      uint32_t v0[32], v1[32];
-      tmem_ld32(lane_base + C::S_COL, v0);
-      tmem_ld32(lane_base + C::S_COL + 32, v1);
-      tmem_wait_ld();
       // A row takes part only if its index is a real position of the sequence
       // (entries of -1 inside the counted prefix are skipped).
       bool valid = false;
@@ -299,79 +302,123 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
         const int32_t sidx = p.idx[(int64_t)t * p.k + r_begin + i * C::ROWS + r];
         valid = sidx >= 0 && seq_base + sidx < p.n_rows;
       }
-      float z[kHeads];
+      const bool got_s = mbar_wait(&sc->s_full, ph, abort_flag);
+      if (named_bar_or(1, 128, !got_s)) { ok = false; break; }   // leave together
+      tc_fence_after();
+
+      // Common case: every logit of this tile is at most 2^8 above the head's
+      // reference m_used (the first tile always fails this test: m_used = -inf).
+      float dmax = -INFINITY;
 #pragma unroll
-      for (int h = 0; h < 32; ++h) {
-        z[h] = valid ? __uint_as_float(v0[h]) * sc->fac[h] : -INFINITY;
-        z[32 + h] = valid ? __uint_as_float(v1[h]) * sc->fac[32 + h] : -INFINITY;
-      }
-      int mine0 = 0, mine1 = 0;
+      for (int half = 0; half < 2; ++half) {
+        uint32_t v[32];
+        tmem_ld32(lane_base + C::S_COL + half * 32, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) {
-        const int m = warp_max_s32(f2ord(z[h]));
-        if (lane == (h & 31)) {
-          if (h < 32) mine0 = m; else mine1 = m;
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 f = fac4[half * 8 + q4];
+          const float4 m = mu4[half * 8 + q4];
+          dmax = fmaxf(dmax, fmaf(__uint_as_float(v[4 * q4 + 0]), f.x, -m.x));
+          dmax = fmaxf(dmax, fmaf(__uint_as_float(v[4 * q4 + 1]), f.y, -m.y));
+          dmax = fmaxf(dmax, fmaf(__uint_as_float(v[4 * q4 + 2]), f.z, -m.z));
+          dmax = fmaxf(dmax, fmaf(__uint_as_float(v[4 * q4 + 3]), f.w, -m.w));
         }
       }
-      sc->red[sw][lane] = mine0;
-      sc->red[sw][32 + lane] = mine1;
-      named_bar_sync(1, 128);
-      bool resc = false;
-      if (st < kHeads) {
-        float tmax = ord2f(sc->red[0][st]);
+      const bool grow = named_bar_or(1, 128, valid && !(dmax <= 8.f));
+      if (grow) {
+        // Exact per-head maxima of the tile: warp max-reductions, then across warps.
+        int mine0 = 0, mine1 = 0;
 #pragma unroll
-        for (int w2 = 1; w2 < 4; ++w2) tmax = fmaxf(tmax, ord2f(sc->red[w2][st]));
-        const float mo = sc->m_used[st];
-        float al = 1.f;
-        if (tmax > mo + 8.f) {
-          al = (mo == -INFINITY) ? 0.f : ex2_approx(mo - tmax);
-          resc = (mo != -INFINITY);
-          sc->m_used[st] = tmax;
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[32];
+          tmem_ld32(lane_base + C::S_COL + half * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int h = half * 32 + c;
+            const float z = valid ? __uint_as_float(v[c]) * sc->fac[h] : -INFINITY;
+            const int m = warp_max_s32(f2ord(z));
+            if (lane == c) {
+              if (half == 0) mine0 = m; else mine1 = m;
+            }
+          }
         }
-        sc->alpha[st] = al;
+        sc->red[sw][lane] = mine0;
+        sc->red[sw][32 + lane] = mine1;
+        named_bar_sync(1, 128);
+        bool resc = false;
+        if (st < kHeads) {
+          float tmax = ord2f(sc->red[0][st]);
+#pragma unroll
+          for (int w2 = 1; w2 < 4; ++w2) tmax = fmaxf(tmax, ord2f(sc->red[w2][st]));
+          const float mo = sc->m_used[st];
+          float al = 1.f;
+          if (tmax > mo) {
+            al = (mo == -INFINITY) ? 0.f : ex2_approx(mo - tmax);
+            resc = (mo != -INFINITY);
+            sc->m_used[st] = tmax;
+          }
+          sc->alpha[st] = al;
+        }
+        const bool any_resc = named_bar_or(1, 128, resc);
+        if (any_resc) {
+          // O(i-1) must be complete before O^T is rescaled in place.
+          const bool got_o = mbar_wait(&sc->o_done, (uint32_t)((i - 1) & 1), abort_flag);
+          if (named_bar_or(1, 128, !got_o)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int blk = 0; blk < 4; ++blk) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint32_t u[32];
+              const uint32_t a = lane_base + C::O_COL + blk * 64 + half * 32;
+              tmem_ld32(a, u);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                u[c] = __float_as_uint(__uint_as_float(u[c]) * sc->alpha[half * 32 + c]);
+              tmem_st32(a, u);
+            }
+          }
+          tmem_wait_st();
+#pragma unroll
+          for (int h = 0; h < kHeads; ++h) l_part[h] *= sc->alpha[h];
+        }
       }
-      const bool any_resc = named_bar_or(1, 128, resc);
       if (i > 0) {
-        // O(i-1) finished: needed before touching O^T or overwriting P^T.
+        // O(i-1) finished: P^T of the previous tile is no longer read.
         const bool got_o = mbar_wait(&sc->o_done, (uint32_t)((i - 1) & 1), abort_flag);
         if (named_bar_or(1, 128, !got_o)) { ok = false; break; }
         tc_fence_after();
       }
-      if (any_resc) {
-#pragma unroll 1
-        for (int blk = 0; blk < 4; ++blk) {
+      // p = 2^(z - m), this row of P^T (64 heads, bf16), and the row sums.
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t u[32];
-            const uint32_t a = lane_base + C::O_COL + blk * 64 + half * 32;
-            tmem_ld32(a, u);
-            tmem_wait_ld();
+      for (int half = 0; half < 2; ++half) {
+        uint32_t v[32];
+        tmem_ld32(lane_base + C::S_COL + half * 32, v);
+        tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              u[c] = __float_as_uint(__uint_as_float(u[c]) * sc->alpha[half * 32 + c]);
-            tmem_st32(a, u);
+        for (int q8 = 0; q8 < 4; ++q8) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = q8 * 8 + 2 * e;
+            const int h0 = half * 32 + c;
+            const float4 f = fac4[h0 >> 2];
+            const float4 m = mu4[h0 >> 2];
+            const float f0 = (h0 & 2) ? f.z : f.x, f1 = (h0 & 2) ? f.w : f.y;
+            const float m0 = (h0 & 2) ? m.z : m.x, m1 = (h0 & 2) ? m.w : m.y;
+            const float p0 = valid ? ex2_approx(fmaf(__uint_as_float(v[c]), f0, -m0)) : 0.f;
+            const float p1 = valid ? ex2_approx(fmaf(__uint_as_float(v[c + 1]), f1, -m1)) : 0.f;
+            pk[e] = pack_bf16x2(p0, p1);
+            // Sum the bf16-rounded weights the tensor core multiplies, so the
+            // numerator and the denominator of the softmax use the same values.
+            l_part[h0] += __uint_as_float(pk[e] << 16);
+            l_part[h0 + 1] += __uint_as_float(pk[e] & 0xFFFF0000u);
           }
+          const int q = half * 4 + q8;   // 16-byte group of 8 heads
+          st_shared_v4(pbase + ((q ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
         }
-        tmem_wait_st();
-#pragma unroll
-        for (int h = 0; h < kHeads; ++h) l_part[h] *= sc->alpha[h];
-      }
-      // p = 2^(z - m), accumulate row sums, write this row of P^T (64 heads, bf16).
-#pragma unroll
-      for (int q8 = 0; q8 < 8; ++q8) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int h0 = q8 * 8 + 2 * e;
-          const float p0 = ex2_approx(z[h0] - sc->m_used[h0]);
-          const float p1 = ex2_approx(z[h0 + 1] - sc->m_used[h0 + 1]);
-          pk[e] = pack_bf16x2(p0, p1);
-          // Sum the bf16-rounded weights the tensor core multiplies, so the
-          // numerator and the denominator of the softmax use the same values.
-          l_part[h0] += __uint_as_float(pk[e] << 16);
-          l_part[h0 + 1] += __uint_as_float(pk[e] & 0xFFFF0000u);
-        }
-        st_shared_v4(pbase + ((q8 ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -466,13 +513,13 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
 }
 
 // Merges the split partials of each (query, head): o = sum_j 2^(m_j - M) O_j / L,
-// L = sum_j 2^(m_j - M) l_j, lse = (M + log2 L) ln 2.  One block per query,
-// one thread per latent column.
+// L = sum_j 2^(m_j - M) l_j, lse = (M + log2 L) ln 2.  One block per
+// (query, group of 8 heads), one thread per latent column.
 __global__ void __launch_bounds__(512) attend_combine_kernel(const AttendParams p) {
   const int t = blockIdx.x;
   const int d = threadIdx.x;
   const int ns = p.n_split;
-  for (int h = 0; h < kHeads; ++h) {
+  for (int h = blockIdx.y * 8; h < blockIdx.y * 8 + 8; ++h) {
     float M = -INFINITY;
     for (int j = 0; j < ns; ++j) M = fmaxf(M, p.ws_ml[(((int64_t)t * ns + j) * kHeads + h) * 2]);
     float L = 0.f, acc = 0.f;

@@ -162,10 +162,13 @@ dsa_status_t launch_topk_cl(const dsa::TopkParams& p, cudaStream_t stream) {
   return DSA_OK;
 }
 
+// CTAs per query: as many as fit in one wave, then more only if a query's
+// candidates would not fit the shared-memory key stash.
 int topk_cluster_size(int32_t T, int64_t ld) {
   const int sms = sm_count();
   int cl = 1;
-  while (cl < 8 && ((int64_t)T * cl < sms || (ld + cl - 1) / cl > dsa::kTopkStashCap)) cl *= 2;
+  while (cl < 8 && (int64_t)T * cl * 2 <= sms) cl *= 2;
+  while (cl < 8 && (ld + cl - 1) / cl > dsa::kTopkStashCap) cl *= 2;
   return cl;
 }
 
@@ -260,7 +263,7 @@ dsa_status_t launch_attend(const void* q_nope, const void* q_pe, const float* qm
   DSA_CUDA(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (sp.n_split > 1) {
-    dsa::attend_combine_kernel<<<T, dsa::kLatent, 0, stream>>>(p);
+    dsa::attend_combine_kernel<<<dim3(T, dsa::kHeads / 8), dsa::kLatent, 0, stream>>>(p);
     DSA_CUDA(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
