@@ -196,13 +196,16 @@ struct SplitPlan {
   int rows_per_split;
 };
 
+// Splits each query's selection across CTAs so that T x n_split is about one
+// wave of the GPU; rows per split are a multiple of the 64-row tile.
 SplitPlan attend_plan(int32_t T, int32_t k) {
-  const int max_tiles = (k + 127) / 128;
+  const int tile = dsa::AttCfg<64>::ROWS;
+  const int max_tiles = (k + tile - 1) / tile;
   int want = std::max(1, sm_count() / std::max(1, T));
-  want = std::min(want, max_tiles);
+  want = std::min(want, std::min(max_tiles, dsa::kMaxSplits));
   int tiles_per = (max_tiles + want - 1) / want;
   SplitPlan sp;
-  sp.rows_per_split = tiles_per * 128;
+  sp.rows_per_split = tiles_per * tile;
   sp.n_split = (k + sp.rows_per_split - 1) / sp.rows_per_split;
   return sp;
 }
@@ -263,7 +266,7 @@ dsa_status_t launch_attend(const void* q_nope, const void* q_pe, const float* qm
   DSA_CUDA(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (sp.n_split > 1) {
-    dsa::attend_combine_kernel<<<dim3(T, dsa::kHeads / 8), dsa::kLatent, 0, stream>>>(p);
+    dsa::attend_combine_kernel<<<T * dsa::kHeads, 128, 0, stream>>>(p);
     DSA_CUDA(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
   }
