@@ -51,10 +51,13 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 constexpr int kMaxK = 16384;
 
 int sm_count() {
+  static std::atomic<int> cached[64] = {};
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && (n = cached[dev].load(std::memory_order_relaxed)) > 0) return n;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     return 148;
+  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -88,9 +91,17 @@ dsa_status_t make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_
   return DSA_OK;
 }
 
-template <typename K>
-dsa_status_t set_smem(K kernel, int bytes) {
-  DSA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+// Raises a kernel's dynamic shared-memory limit once per device (the
+// attribute persists, so later launches skip the driver call).
+template <auto Kernel>
+dsa_status_t set_smem(int bytes) {
+  static std::atomic<uint64_t> done{0};   // one flag set per kernel (not per signature)
+  int dev = 0;
+  DSA_CUDA(cudaGetDevice(&dev));
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load(std::memory_order_relaxed) & bit)) return DSA_OK;
+  DSA_CUDA(cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  if (bit) done.fetch_or(bit, std::memory_order_relaxed);
   return DSA_OK;
 }
 
@@ -121,7 +132,7 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   const int64_t n_groups = (T + QG - 1) / QG;
   p.n_units = n_groups * p.n_kt;
   const int grid = (int)std::min<int64_t>(p.n_units, sm_count());
-  st = set_smem(dsa::indexer_kernel<QG>, C::SMEM_BYTES);
+  st = set_smem<dsa::indexer_kernel<QG>>(C::SMEM_BYTES);
   if (st != DSA_OK) return st;
   dsa::indexer_kernel<QG><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(kmap, qmap, p);
   DSA_CUDA(cudaGetLastError());
@@ -143,8 +154,16 @@ dsa_status_t indexer_impl(const void* q_idx, const float* w, const void* k_idx, 
 // ----------------------------------------------------------------- top-k
 template <int CL>
 dsa_status_t launch_topk_cl(const dsa::TopkParams& p, cudaStream_t stream) {
-  dsa_status_t st = set_smem(dsa::topk_kernel<CL>, dsa::kTopkSmemBytes);
+  dsa_status_t st = set_smem<dsa::topk_kernel<CL>>(dsa::kTopkSmemBytes);
   if (st != DSA_OK) return st;
+  if (CL > 8) {
+    static std::once_flag once;
+    cudaError_t e = cudaSuccess;
+    std::call_once(once, [&] {
+      e = cudaFuncSetAttribute(dsa::topk_kernel<CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    });
+    if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "cluster attribute: %s", cudaGetErrorString(e));
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(p.T * CL));
   cfg.blockDim = dim3(dsa::kTopkThreads);
@@ -162,14 +181,44 @@ dsa_status_t launch_topk_cl(const dsa::TopkParams& p, cudaStream_t stream) {
   return DSA_OK;
 }
 
-// CTAs per query: as many as fit in one wave, then more only if a query's
-// candidates would not fit the shared-memory key stash.
+// CTAs per query: enough that each CTA owns at least ~16K candidates' worth of
+// work, within one wave of the GPU; more (up to 16) when a query's slice would
+// not fit the shared-memory key stash and the batch is small.
 int topk_cluster_size(int32_t T, int64_t ld) {
   const int sms = sm_count();
   int cl = 1;
-  while (cl < 8 && (int64_t)T * cl * 2 <= sms) cl *= 2;
-  while (cl < 8 && (ld + cl - 1) / cl > dsa::kTopkStashCap) cl *= 2;
+  while (cl < 8 && (ld + cl - 1) / cl > 16384 && (int64_t)T * cl * 2 <= sms) cl *= 2;
+  while (cl < 16 && (ld + cl - 1) / cl > dsa::kTopkStashCap && (int64_t)T * cl * 2 <= sms) cl *= 2;
   return cl;
+}
+
+// Largest cluster size that can be co-scheduled for the top-k kernel (16 needs
+// the non-portable attribute and a GPC with 16 free SMs).
+template <int CL>
+bool topk_cluster_fits() {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CL);
+  cfg.blockDim = dim3(dsa::kTopkThreads);
+  cfg.dynamicSmemBytes = dsa::kTopkSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaFuncSetAttribute(dsa::topk_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           dsa::kTopkSmemBytes) != cudaSuccess)
+    return false;
+  if (CL > 8 &&
+      cudaFuncSetAttribute(dsa::topk_kernel<CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+    return false;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, dsa::topk_kernel<CL>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return n > 0;
 }
 
 dsa_status_t topk_impl(const float* scores, int64_t ld, const int32_t* q_pos, int32_t T, int32_t k,
@@ -186,7 +235,12 @@ dsa_status_t topk_impl(const float* scores, int64_t ld, const int32_t* q_pos, in
     case 1: return launch_topk_cl<1>(p, stream);
     case 2: return launch_topk_cl<2>(p, stream);
     case 4: return launch_topk_cl<4>(p, stream);
-    default: return launch_topk_cl<8>(p, stream);
+    case 8: return launch_topk_cl<8>(p, stream);
+    default: {
+      static int fits16 = -1;   // probed once per process
+      if (fits16 < 0) fits16 = topk_cluster_fits<16>() ? 1 : 0;
+      return fits16 ? launch_topk_cl<16>(p, stream) : launch_topk_cl<8>(p, stream);
+    }
   }
 }
 
@@ -260,7 +314,7 @@ dsa_status_t launch_attend(const void* q_nope, const void* q_pe, const float* qm
     p.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
                                        round_up(units * dsa::kHeads * dsa::kLatent * 4, 256));
   }
-  st = set_smem(dsa::attend_kernel<DR>, C::SMEM_BYTES);
+  st = set_smem<dsa::attend_kernel<DR>>(C::SMEM_BYTES);
   if (st != DSA_OK) return st;
   dsa::attend_kernel<DR><<<T * sp.n_split, C::THREADS, C::SMEM_BYTES, stream>>>(qn_map, qp_map, p);
   DSA_CUDA(cudaGetLastError());

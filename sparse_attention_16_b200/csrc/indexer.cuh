@@ -288,18 +288,30 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
       if (kt * kKeyTile <= gi.maxpos) {
         if (!mbar_wait(&acc_full[as.idx], as.phase, abort_flag)) { *abort_flag = 1; break; }
         tc_fence_after();
+        // Per query: ReLU of the 32 head dot products, weighted head sum (two
+        // partial sums to halve the dependent FMA chain; weights as float4).
+        const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(as.idx * C::N);
 #pragma unroll
-        for (int qi = 0; qi < QPW; ++qi) {
-          uint32_t v[32];
-          const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) +
-                                 (uint32_t)(as.idx * C::N + (qbase + qi) * 32);
-          tmem_ld32(taddr, v);
+        for (int qp = 0; qp < QPW; qp += (QPW > 1 ? 2 : 1)) {
+          uint32_t v[2][32];
+#pragma unroll
+          for (int u = 0; u < (QPW > 1 ? 2 : 1); ++u)
+            tmem_ld32(lane_addr + (uint32_t)((qbase + qp + u) * 32), v[u]);
           tmem_wait_ld();
-          const float* wq = w_my + qi * kIdxHeads;
-          float s = 0.f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) s = fmaf(wq[j], fmaxf(__uint_as_float(v[j]), 0.f), s);
-          res[qi] = s;
+          for (int u = 0; u < (QPW > 1 ? 2 : 1); ++u) {
+            const float4* wq = reinterpret_cast<const float4*>(w_my + (qp + u) * kIdxHeads);
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+              const float4 wv = wq[j4];
+              s0 = fmaf(wv.x, fmaxf(__uint_as_float(v[u][4 * j4 + 0]), 0.f), s0);
+              s1 = fmaf(wv.y, fmaxf(__uint_as_float(v[u][4 * j4 + 1]), 0.f), s1);
+              s0 = fmaf(wv.z, fmaxf(__uint_as_float(v[u][4 * j4 + 2]), 0.f), s0);
+              s1 = fmaf(wv.w, fmaxf(__uint_as_float(v[u][4 * j4 + 3]), 0.f), s1);
+            }
+            res[qp + u] = s0 + s1;
+          }
         }
         tc_fence_before();
         __syncwarp();

@@ -28,8 +28,9 @@ namespace cg = cooperative_groups;
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkBins = 2048;                 // passes 1 and 2 (11 bits); pass 3 uses 1024
-constexpr int kTopkStashCap = 49152;            // keys staged in shared memory per CTA
-constexpr int kTopkSmemBytes = 2 * kTopkBins * 4 + 1024 + kTopkStashCap * 4;
+constexpr int kTopkStashCap = 32768;            // keys staged in shared memory per CTA
+constexpr int kTopkCandCap = 10240;             // (key, position) candidates per CTA
+constexpr int kTopkSmemBytes = 2 * kTopkBins * 4 + 1024 + kTopkStashCap * 4 + kTopkCandCap * 8;
 
 struct TopkParams {
   const float* scores;   // [T, ld]
@@ -111,22 +112,33 @@ __device__ __forceinline__ void cluster_barrier() {
   }
 }
 
-// Sums the NB-bin histograms of all CTAs in the cluster into `tot`.
+// Sums the NB-bin histograms of all CTAs in the cluster into `tot` of every
+// CTA.  CTA r reduces bins [r NB/CL, (r+1) NB/CL) over all ranks into rank 0's
+// `tot`; then every CTA copies rank 0's `tot`.  Each CTA thus reads 2 NB words
+// through distributed shared memory instead of CL x NB.
 template <int CL, int NB>
 __device__ __forceinline__ void cluster_sum_hist(uint32_t* hist, uint32_t* tot) {
-  cluster_barrier<CL>();
   if constexpr (CL > 1) {
     cg::cluster_group cl = cg::this_cluster();
-    for (int b = threadIdx.x; b < NB; b += kTopkThreads) {
+    const int rank = (int)cl.block_rank();
+    cluster_barrier<CL>();                 // every histogram is complete
+    uint32_t* tot0 = cl.map_shared_rank(tot, 0);
+    constexpr int SL = NB / CL;
+    for (int b = rank * SL + threadIdx.x; b < (rank + 1) * SL; b += kTopkThreads) {
       uint32_t s = 0;
 #pragma unroll
       for (int r = 0; r < CL; ++r) s += cl.map_shared_rank(hist, r)[b];
-      tot[b] = s;
+      tot0[b] = s;
     }
+    cluster_barrier<CL>();                 // rank 0 holds the sums; peers' hists no longer read
+    if (rank != 0)
+      for (int b = threadIdx.x; b < NB; b += kTopkThreads) tot[b] = tot0[b];
+    __syncthreads();
   } else {
+    __syncthreads();
     for (int b = threadIdx.x; b < NB; b += kTopkThreads) tot[b] = hist[b];
+    __syncthreads();
   }
-  cluster_barrier<CL>();  // peers are done reading `hist` before it is reused
 }
 
 template <int CL>
@@ -165,26 +177,36 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   const int64_t len = hi - lo;
   const bool staged = len <= kTopkStashCap;
 
-  // ---- pass 1: top 11 bits
+  // ---- pass 1: histogram of the top 11 bits (loads batched 4 x float4 per thread)
   for (int b = threadIdx.x; b < kTopkBins; b += kTopkThreads) hist[b] = 0;
   __syncthreads();
-  {
-    const int64_t n4 = len >> 2;
-    const float4* row4 = reinterpret_cast<const float4*>(row + lo);
-    for (int64_t i = threadIdx.x; i < n4; i += kTopkThreads) {
-      const float4 f = row4[i];
-      const uint32_t k0 = score_key(f.x), k1 = score_key(f.y), k2 = score_key(f.z), k3 = score_key(f.w);
-      atomicAdd(&hist[k0 >> 21], 1u);
-      atomicAdd(&hist[k1 >> 21], 1u);
-      atomicAdd(&hist[k2 >> 21], 1u);
-      atomicAdd(&hist[k3 >> 21], 1u);
-      if (staged) reinterpret_cast<uint4*>(stash)[i] = make_uint4(k0, k1, k2, k3);
+  const int64_t n4 = len >> 2;
+  const float4* row4 = reinterpret_cast<const float4*>(row + lo);
+  for (int64_t i0 = 0; i0 < n4; i0 += 4 * kTopkThreads) {
+    float4 f[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * kTopkThreads + threadIdx.x;
+      f[u] = (i < n4) ? row4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (int64_t i = (n4 << 2) + threadIdx.x; i < len; i += kTopkThreads) {
-      const uint32_t kk = score_key(row[lo + i]);
-      atomicAdd(&hist[kk >> 21], 1u);
-      if (staged) stash[i] = kk;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * kTopkThreads + threadIdx.x;
+      if (i < n4) {
+        const uint32_t k0 = score_key(f[u].x), k1 = score_key(f[u].y), k2 = score_key(f[u].z),
+                       k3 = score_key(f[u].w);
+        atomicAdd(&hist[k0 >> 21], 1u);
+        atomicAdd(&hist[k1 >> 21], 1u);
+        atomicAdd(&hist[k2 >> 21], 1u);
+        atomicAdd(&hist[k3 >> 21], 1u);
+        if (staged) reinterpret_cast<uint4*>(stash)[i] = make_uint4(k0, k1, k2, k3);
+      }
     }
+  }
+  for (int64_t i = (n4 << 2) + threadIdx.x; i < len; i += kTopkThreads) {
+    const uint32_t kk = score_key(row[lo + i]);
+    atomicAdd(&hist[kk >> 21], 1u);
+    if (staged) stash[i] = kk;
   }
   __syncthreads();
   cluster_sum_hist<CL, kTopkBins>(hist, tot);
@@ -193,13 +215,66 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   uint32_t above = res[1];
   uint32_t need = (uint32_t)p.k - above;
 
-  auto key_at = [&](int64_t i) -> uint32_t { return staged ? stash[i] : score_key(row[lo + i]); };
+  // ---- filter: keys in bins >= b1 (all of the selection) with their positions,
+  // compacted in position order into shared memory.  Rounds of 4 consecutive
+  // candidates per thread.
+  uint32_t* cand_key = stash + kTopkStashCap;
+  int32_t* cand_pos = reinterpret_cast<int32_t*>(cand_key + kTopkCandCap);
+  uint32_t nc = 0;
+  for (int64_t r0 = 0; r0 < len; r0 += 4 * kTopkThreads) {
+    const int64_t e0 = r0 + 4 * (int64_t)threadIdx.x;
+    uint32_t kk[4];
+    if (staged) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) kk[e] = (e0 + e < len) ? stash[e0 + e] : 0u;
+    } else if (e0 + 3 < len) {
+      const float4 f = *reinterpret_cast<const float4*>(row + lo + e0);
+      kk[0] = score_key(f.x); kk[1] = score_key(f.y); kk[2] = score_key(f.z); kk[3] = score_key(f.w);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) kk[e] = (e0 + e < len) ? score_key(row[lo + e0 + e]) : 0u;
+    }
+    uint32_t c = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c += (e0 + e < len) && ((kk[e] >> 21) >= b1);
+    uint32_t total;
+    uint32_t pos = nc + block_excl_scan(c, tmp, &total);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if ((e0 + e < len) && ((kk[e] >> 21) >= b1)) {
+        if (pos < (uint32_t)kTopkCandCap) {
+          cand_key[pos] = kk[e];
+          cand_pos[pos] = (int32_t)(lo + e0 + e);
+        }
+        ++pos;
+      }
+    }
+    nc += total;
+  }
+  // Every CTA of the cluster takes the candidate path, or none does.
+  if (threadIdx.x == 0) cnt[2] = (nc > (uint32_t)kTopkCandCap) ? 1u : 0u;
+  cluster_barrier<CL>();
+  bool overflow = false;
+  if constexpr (CL > 1) {
+    cg::cluster_group cl = cg::this_cluster();
+    for (int r = 0; r < CL; ++r) overflow |= cl.map_shared_rank(cnt, r)[2] != 0u;
+  } else {
+    overflow = cnt[2] != 0u;
+  }
+  cluster_barrier<CL>();   // flags read before cnt is reused
+
+  const uint32_t n_items = overflow ? (uint32_t)len : nc;
+  auto item_key = [&](uint32_t i) -> uint32_t {
+    if (!overflow) return cand_key[i];
+    return staged ? stash[i] : score_key(row[lo + i]);
+  };
+  auto item_pos = [&](uint32_t i) -> int32_t { return overflow ? (int32_t)(lo + i) : cand_pos[i]; };
 
   // ---- pass 2: next 11 bits of keys in bin b1
   for (int b = threadIdx.x; b < kTopkBins; b += kTopkThreads) hist[b] = 0;
   __syncthreads();
-  for (int64_t i = threadIdx.x; i < len; i += kTopkThreads) {
-    const uint32_t kk = key_at(i);
+  for (uint32_t i = threadIdx.x; i < n_items; i += kTopkThreads) {
+    const uint32_t kk = item_key(i);
     if ((kk >> 21) == b1) atomicAdd(&hist[(kk >> 10) & 0x7FFu], 1u);
   }
   __syncthreads();
@@ -212,8 +287,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   // ---- pass 3: last 10 bits of keys with prefix pre2
   for (int b = threadIdx.x; b < 1024; b += kTopkThreads) hist[b] = 0;
   __syncthreads();
-  for (int64_t i = threadIdx.x; i < len; i += kTopkThreads) {
-    const uint32_t kk = key_at(i);
+  for (uint32_t i = threadIdx.x; i < n_items; i += kTopkThreads) {
+    const uint32_t kk = item_key(i);
     if ((kk >> 10) == pre2) atomicAdd(&hist[kk & 0x3FFu], 1u);
   }
   __syncthreads();
@@ -225,15 +300,14 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
 
   // ---- counts of this slice, exchanged so each CTA knows what precedes it
   uint32_t my_gt = 0, my_eq = 0;
-  for (int64_t i = threadIdx.x; i < len; i += kTopkThreads) {
-    const uint32_t kk = key_at(i);
+  for (uint32_t i = threadIdx.x; i < n_items; i += kTopkThreads) {
+    const uint32_t kk = item_key(i);
     my_gt += (kk > tau);
     my_eq += (kk == tau);
   }
   {
     uint32_t tt;
-    const uint32_t g_total_dummy = block_excl_scan(my_gt, tmp, &tt);
-    (void)g_total_dummy;
+    block_excl_scan(my_gt, tmp, &tt);
     my_gt = tt;
     block_excl_scan(my_eq, tmp, &tt);
     my_eq = tt;
@@ -254,29 +328,29 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   }
   cluster_barrier<CL>();  // peers finished reading cnt (the CTA may exit after this)
 
-  // ---- ordered compaction: 4 consecutive candidates per thread per round
-  for (int64_t r0 = 0; r0 < len; r0 += 4 * kTopkThreads) {
-    const int64_t i0 = r0 + 4 * (int64_t)threadIdx.x;
+  // ---- ordered output: 4 consecutive items (in position order) per thread per round
+  for (uint32_t r0 = 0; r0 < n_items; r0 += 4 * kTopkThreads) {
+    const uint32_t i0 = r0 + 4 * threadIdx.x;
     uint32_t kk[4];
     uint32_t c_gt = 0, c_eq = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      kk[e] = (i0 + e < len) ? key_at(i0 + e) : 0u;
-      c_gt += (i0 + e < len) && (kk[e] > tau);
-      c_eq += (i0 + e < len) && (kk[e] == tau);
+      kk[e] = (i0 + e < n_items) ? item_key(i0 + e) : 0u;
+      c_gt += (i0 + e < n_items) && (kk[e] > tau);
+      c_eq += (i0 + e < n_items) && (kk[e] == tau);
     }
     uint32_t total;
     const uint32_t ex = block_excl_scan((c_gt << 16) | c_eq, tmp, &total);
     uint32_t g = base_gt + (ex >> 16), q = base_eq + (ex & 0xFFFFu);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      if (i0 + e < len) {
+      if (i0 + e < n_items) {
         if (kk[e] > tau) {
           const uint32_t slot = g + min(q, need_eq);
-          if (slot < (uint32_t)p.k) out[slot] = (int32_t)(lo + i0 + e);
+          if (slot < (uint32_t)p.k) out[slot] = item_pos(i0 + e);
           ++g;
         } else if (kk[e] == tau) {
-          if (q < need_eq && g + q < (uint32_t)p.k) out[g + q] = (int32_t)(lo + i0 + e);
+          if (q < need_eq && g + q < (uint32_t)p.k) out[g + q] = item_pos(i0 + e);
           ++q;
         }
       }
