@@ -215,60 +215,131 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   uint32_t above = res[1];
   uint32_t need = (uint32_t)p.k - above;
 
-  // ---- filter: keys in bins >= b1 (all of the selection) with their positions,
-  // compacted in position order into shared memory.  Rounds of 4 consecutive
-  // candidates per thread.
+  // ---- filter: keys in bins >= b1 (all of the selection) with their positions.
+  // Warp w owns a contiguous segment of this CTA's slice; pass (a) counts its
+  // candidates, pass (b) writes them in position order (ballot compaction).
   uint32_t* cand_key = stash + kTopkStashCap;
   int32_t* cand_pos = reinterpret_cast<int32_t*>(cand_key + kTopkCandCap);
-  uint32_t nc = 0;
-  for (int64_t r0 = 0; r0 < len; r0 += 4 * kTopkThreads) {
-    const int64_t e0 = r0 + 4 * (int64_t)threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kWarps = kTopkThreads / 32;
+  const int64_t seg = ((len + kWarps - 1) / kWarps + 127) & ~int64_t(127);
+  const int64_t s_lo = (warp * seg < len) ? warp * seg : len;
+  const int64_t s_hi = (s_lo + seg < len) ? s_lo + seg : len;
+  auto key_at = [&](int64_t i) -> uint32_t { return staged ? stash[i] : score_key(row[lo + i]); };
+  // (a) count, 4 keys per lane per step (vector loads when not staged)
+  uint32_t wcount = 0;
+  for (int64_t i0 = s_lo; i0 < s_hi; i0 += 128) {
+    const int64_t e0 = i0 + 4 * lane;
     uint32_t kk[4];
-    if (staged) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) kk[e] = (e0 + e < len) ? stash[e0 + e] : 0u;
-    } else if (e0 + 3 < len) {
+    if (!staged && e0 + 3 < s_hi) {
       const float4 f = *reinterpret_cast<const float4*>(row + lo + e0);
       kk[0] = score_key(f.x); kk[1] = score_key(f.y); kk[2] = score_key(f.z); kk[3] = score_key(f.w);
     } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) kk[e] = (e0 + e < len) ? score_key(row[lo + e0 + e]) : 0u;
+      for (int e = 0; e < 4; ++e) kk[e] = (e0 + e < s_hi) ? key_at(e0 + e) : 0u;
     }
-    uint32_t c = 0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) c += (e0 + e < len) && ((kk[e] >> 21) >= b1);
-    uint32_t total;
-    uint32_t pos = nc + block_excl_scan(c, tmp, &total);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if ((e0 + e < len) && ((kk[e] >> 21) >= b1)) {
-        if (pos < (uint32_t)kTopkCandCap) {
-          cand_key[pos] = kk[e];
-          cand_pos[pos] = (int32_t)(lo + e0 + e);
-        }
-        ++pos;
-      }
-    }
-    nc += total;
+    for (int e = 0; e < 4; ++e) wcount += (e0 + e < s_hi) && ((kk[e] >> 21) >= b1);
   }
-  // Every CTA of the cluster takes the candidate path, or none does.
-  if (threadIdx.x == 0) cnt[2] = (nc > (uint32_t)kTopkCandCap) ? 1u : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wcount += __shfl_xor_sync(0xffffffffu, wcount, o);
+  if (lane == 0) tmp[warp] = wcount;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t w = tmp[lane];
+    uint32_t x = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    tmp[lane] = x - w;                 // exclusive prefix of warp counts
+    if (lane == 31) res[4] = x;        // candidates of this CTA
+  }
+  __syncthreads();
+  const uint32_t nc = res[4];
+  // (b) write in position order into the local candidate arrays
+  if (nc <= (uint32_t)kTopkCandCap) {
+    uint32_t wpos = tmp[warp];
+    for (int64_t i0 = s_lo; i0 < s_hi; i0 += 128) {
+      const int64_t e0 = i0 + 4 * lane;
+      uint32_t kk[4];
+      if (!staged && e0 + 3 < s_hi) {
+        const float4 f = *reinterpret_cast<const float4*>(row + lo + e0);
+        kk[0] = score_key(f.x); kk[1] = score_key(f.y); kk[2] = score_key(f.z); kk[3] = score_key(f.w);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) kk[e] = (e0 + e < s_hi) ? key_at(e0 + e) : 0u;
+      }
+      uint32_t flags = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) flags |= ((e0 + e < s_hi) && ((kk[e] >> 21) >= b1)) ? (1u << e) : 0u;
+      const uint32_t mine = __popc(flags);
+      uint32_t before = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, before, o);
+        if (lane >= o) before += y;
+      }
+      const uint32_t total = __shfl_sync(0xffffffffu, before, 31);
+      uint32_t at = wpos + before - mine;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (flags & (1u << e)) {
+          cand_key[at] = kk[e];
+          cand_pos[at] = (int32_t)(lo + e0 + e);
+          ++at;
+        }
+      }
+      wpos += total;
+    }
+  }
+  // ---- gather the cluster's candidates, in rank (= position) order, in rank 0
+  if (threadIdx.x == 0) cnt[3] = nc;
   cluster_barrier<CL>();
-  bool overflow = false;
+  uint32_t off = 0, n_all = 0;
   if constexpr (CL > 1) {
     cg::cluster_group cl = cg::this_cluster();
-    for (int r = 0; r < CL; ++r) overflow |= cl.map_shared_rank(cnt, r)[2] != 0u;
+    for (int r = 0; r < CL; ++r) {
+      const uint32_t c = cl.map_shared_rank(cnt, r)[3];
+      if (r < rank) off += c;
+      n_all += c;
+    }
   } else {
-    overflow = cnt[2] != 0u;
+    n_all = nc;
   }
-  cluster_barrier<CL>();   // flags read before cnt is reused
+  const bool overflow = n_all > (uint32_t)kTopkCandCap;   // the same in every CTA
+  if (!overflow) {
+    if constexpr (CL > 1) {
+      if (rank != 0) {
+        cg::cluster_group cl = cg::this_cluster();
+        uint32_t* dk = cl.map_shared_rank(cand_key, 0);
+        int32_t* dp = cl.map_shared_rank(cand_pos, 0);
+        for (uint32_t i = threadIdx.x; i < nc; i += kTopkThreads) {
+          dk[off + i] = cand_key[i];
+          dp[off + i] = cand_pos[i];
+        }
+      }
+    }
+    cluster_barrier<CL>();   // rank 0 holds every candidate; the other CTAs are done
+    if (rank != 0) return;
+  }
 
-  const uint32_t n_items = overflow ? (uint32_t)len : nc;
-  auto item_key = [&](uint32_t i) -> uint32_t {
-    if (!overflow) return cand_key[i];
-    return staged ? stash[i] : score_key(row[lo + i]);
-  };
+  // From here: rank 0 alone on the gathered candidates, or (overflow) every CTA
+  // of the cluster on its whole slice with cluster-wide reductions.
+  const uint32_t n_items = overflow ? (uint32_t)len : n_all;
+  auto item_key = [&](uint32_t i) -> uint32_t { return overflow ? key_at(i) : cand_key[i]; };
   auto item_pos = [&](uint32_t i) -> int32_t { return overflow ? (int32_t)(lo + i) : cand_pos[i]; };
+  auto sum_hist = [&](int nb) {
+    if (overflow) {
+      if (nb == kTopkBins) cluster_sum_hist<CL, kTopkBins>(hist, tot);
+      else cluster_sum_hist<CL, 1024>(hist, tot);
+    } else {
+      __syncthreads();
+      for (int b = threadIdx.x; b < nb; b += kTopkThreads) tot[b] = hist[b];
+      __syncthreads();
+    }
+  };
 
   // ---- pass 2: next 11 bits of keys in bin b1
   for (int b = threadIdx.x; b < kTopkBins; b += kTopkThreads) hist[b] = 0;
@@ -278,7 +349,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     if ((kk >> 21) == b1) atomicAdd(&hist[(kk >> 10) & 0x7FFu], 1u);
   }
   __syncthreads();
-  cluster_sum_hist<CL, kTopkBins>(hist, tot);
+  sum_hist(kTopkBins);
   find_threshold_bin<kTopkBins>(tot, need, tmp, res);
   const uint32_t pre2 = (b1 << 11) | res[0];
   above += res[1];
@@ -292,41 +363,40 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     if ((kk >> 10) == pre2) atomicAdd(&hist[kk & 0x3FFu], 1u);
   }
   __syncthreads();
-  cluster_sum_hist<CL, 1024>(hist, tot);
+  sum_hist(1024);
   find_threshold_bin<1024>(tot, need, tmp, res);
   const uint32_t tau = (pre2 << 10) | res[0];
   need -= res[1];                 // keys == tau still to take (>= 1)
   const uint32_t need_eq = need;
 
-  // ---- counts of this slice, exchanged so each CTA knows what precedes it
-  uint32_t my_gt = 0, my_eq = 0;
-  for (uint32_t i = threadIdx.x; i < n_items; i += kTopkThreads) {
-    const uint32_t kk = item_key(i);
-    my_gt += (kk > tau);
-    my_eq += (kk == tau);
-  }
-  {
-    uint32_t tt;
-    block_excl_scan(my_gt, tmp, &tt);
-    my_gt = tt;
-    block_excl_scan(my_eq, tmp, &tt);
-    my_eq = tt;
-  }
-  if (threadIdx.x == 0) {
-    cnt[0] = my_gt;
-    cnt[1] = my_eq;
-  }
-  cluster_barrier<CL>();
+  // ---- what precedes this CTA's items in position order (only with overflow
+  // is the selection spread over several CTAs)
   uint32_t base_gt = 0, base_eq = 0;
-  if constexpr (CL > 1) {
-    cg::cluster_group cl = cg::this_cluster();
-    for (int r = 0; r < rank; ++r) {
-      const uint32_t* pc = cl.map_shared_rank(cnt, r);
-      base_gt += pc[0];
-      base_eq += pc[1];
+  if (overflow) {
+    uint32_t my_gt = 0, my_eq = 0;
+    for (uint32_t i = threadIdx.x; i < n_items; i += kTopkThreads) {
+      const uint32_t kk = item_key(i);
+      my_gt += (kk > tau);
+      my_eq += (kk == tau);
     }
+    uint32_t tg, te;
+    block_excl_scan(my_gt, tmp, &tg);
+    block_excl_scan(my_eq, tmp, &te);
+    if (threadIdx.x == 0) {
+      cnt[0] = tg;
+      cnt[1] = te;
+    }
+    cluster_barrier<CL>();
+    if constexpr (CL > 1) {
+      cg::cluster_group cl = cg::this_cluster();
+      for (int r = 0; r < rank; ++r) {
+        const uint32_t* pc = cl.map_shared_rank(cnt, r);
+        base_gt += pc[0];
+        base_eq += pc[1];
+      }
+    }
+    cluster_barrier<CL>();  // peers finished reading cnt (the CTA may exit after this)
   }
-  cluster_barrier<CL>();  // peers finished reading cnt (the CTA may exit after this)
 
   // ---- ordered output: 4 consecutive items (in position order) per thread per round
   for (uint32_t r0 = 0; r0 < n_items; r0 += 4 * kTopkThreads) {
