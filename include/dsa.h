@@ -157,7 +157,7 @@ dsa_status_t sparse_mla_attend(const void* q_nope, const void* q_pe, const float
  * several thread blocks, the partial results go to a fixed scratch array
  * inside the library instead of a caller buffer.
  *   - Scratch: a file-scope __device__ array of DSA_NOALLOC_MAX_PARTIALS x 64 x
- *     514 floats (16.8 MB) that every GPU loading the library holds until the
+ *     516 floats (16.9 MB) that every GPU loading the library holds until the
  *     process exits.  The call allocates nothing and calls no allocating routine.
  *   - Limit: a call needs T x n_split partials, where n_split is the number of
  *     blocks each query is split across (1 once T reaches the SM count, so no

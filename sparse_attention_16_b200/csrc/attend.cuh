@@ -7,30 +7,47 @@
 // Every gathered 1,152-byte row (1,024 on NoPE layers) is read once and used by
 // all 64 heads.
 //
-// Work unit = (query t, split j): rows [j*R, min(count, (j+1)*R)) of idx[t], in
-// tiles of 128 rows.  Per tile:
-//   producer warps 5-7   gather the 128 rows with 16-byte cp.async into a
-//                        chunk-major tile: chunk c (64 columns) holds 128 rows x
-//                        128 B in the 128-byte-swizzled layout the tensor core
-//                        reads (K-major for the logits, MN-major for the output)
-//   warp 4               TMEM owner; one thread issues
-//                          S^T[128 rows x 64 heads] = C[rows, 576] . Q^T   (K-major A, B)
-//                          O^T[512 x 64] += C^T[512, rows] . P^T[rows, 64] (MN-major A, B)
-//   warps 0-3            softmax: TMEM lane r = row r holds that row's 64 head
-//                        logits; per-head maxima come from warp max-reductions;
-//                        exp2 with scale*m*log2(e) folded in; P^T (bf16) is
-//                        written to shared memory for the second product.
+// Heads are the M dimension of both tensor-core products, so each head's
+// softmax state lives in one pair of threads.  Tensor memory (512 columns x
+// 128 lanes) holds, in lanes 0-15 of every 32-lane quarter, the query Q
+// [64 heads x 576] (bf16, two per column) and two logit buffers S [64 heads x
+// 64 rows] (f32), and in lanes 16-31 the output O [64 heads x 512] (f32).  That
+// leaves shared memory for three 64-row tile buffers (3 x 72 KB), so two tiles
+// are in flight while a third is computed on.  Q arrives by TMA in the third
+// tile buffer (free until tile 2) and is moved to TMEM by the softmax warps.
+//
+// Work unit = (query t, split j) = rows [j*R, min(count, (j+1)*R)) of idx[t].
+// Per 64-row tile i (buffer i % 3):
+//   producer warps 5-7  gather the rows with 16-byte cp.async into a
+//                       chunk-major tile: chunk c (64 columns) = 64 rows x 128 B
+//                       in the 128-byte-swizzled layout (K-major for the
+//                       logits, MN-major for the output product).  The copies
+//                       of a row are issued back to back (a warp covers four
+//                       whole rows in 9 instructions), so each row reaches the
+//                       memory system as one 1,152-byte request stream.
+//   warp 4              TMEM owner; one thread issues
+//                         S = Q . C^T   M = 64 heads, N = 64 rows, K = 576, Q read from TMEM
+//                         O += P . C    M = 64 heads, N = 2 x 256 columns, K = 64 rows
+//                       in order of readiness (S of the next tile usually runs
+//                       while the softmax of this one does)
+//   warps 0-3           softmax: lane L of warp w owns head 16 w + (L & 15) and
+//                       rows 32 (L >> 4) .. + 31 of the tile; writes P (bf16,
+//                       K-major) to shared memory for the output product.
 // The running max is updated lazily: O and the row sums are rescaled only when
 // a head's maximum grows by more than 2^8, so p <= 256 and the final
 // normalisation uses the same reference for numerator and denominator.
-// The rotary chunk of the tile is no longer needed once S^T is done, so P^T is
-// written over it on RoPE layers.  Splits write fp32 partials (o, max, sum)
-// that a small combine kernel merges; a single split writes bf16 output
-// directly.
+// A single split writes bf16 output directly.  When a query's selection is
+// split over 2-8 CTAs, those CTAs form a thread-block cluster: each stages its
+// unnormalised O and per-head (max, sum) in its own shared memory, and rank r
+// merges columns [r 512 / n, (r + 1) 512 / n) of all heads from every CTA
+// through distributed shared memory.  Larger splits write fp32 partials that a
+// small combine kernel merges.
 #pragma once
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+
+#include <cooperative_groups.h>
 
 #include <cstddef>
 
@@ -44,25 +61,29 @@ constexpr int kLatent = 512;
 template <int DR>
 struct AttCfg {
   static constexpr int KCH = (kLatent + DR) / 64;        // 64-column chunks: 9 or 8
-  static constexpr int ROWS = 64;                        // rows per tile (M of the logit MMA)
+  static constexpr int ROWS = 64;                        // rows per tile (N of the logit MMA)
+  static constexpr int NBUF = 3;                         // tile buffers
   static constexpr int CHUNK_BYTES = ROWS * 128;         // 8 KB: 64 rows x 64 columns
   static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;   // 72 KB (RoPE) / 64 KB (NoPE)
-  static constexpr int QCHUNK_BYTES = kHeads * 128;      // 8 KB
-  static constexpr int Q_BYTES = KCH * QCHUNK_BYTES;
-  static constexpr int P_BYTES = ROWS * 128;             // P^T: 64 rows x 64 heads bf16
-  static constexpr int DATA_BYTES = Q_BYTES + 2 * TILE_BYTES + P_BYTES;
-  static constexpr int SCRATCH_BYTES = 2048;
+  static constexpr int P_BYTES = kHeads * 128;           // P: 64 heads x 64 rows bf16
+  static constexpr int DATA_BYTES = NBUF * TILE_BYTES + P_BYTES;
+  static constexpr int SCRATCH_BYTES = 1024;
   static constexpr int SMEM_BYTES = DATA_BYTES + SCRATCH_BYTES;
   static constexpr int THREADS = 8 * 32;
   static constexpr int PRODUCERS = 96;                   // warps 5-7
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t S_COL = 0;                   // S^T of tile j in TMEM lane half (j & 1)
-  static constexpr uint32_t O_COL = 128;                 // O^T: 4 blocks x 64 columns
-  static constexpr uint32_t IDESC_S = idesc_bf16_f32(64, kHeads, 0, 0);
-  static constexpr uint32_t IDESC_O = idesc_bf16_f32(128, kHeads, 1, 1);
+  static constexpr uint32_t Q_COL = 0;                   // lanes 0-15: Q, KCH x 32 columns
+  static constexpr uint32_t S_COL = KCH * 32;            // lanes 0-15: S buffer b at S_COL + 64 b
+  static constexpr uint32_t O_LANE = 16;                 // lanes 16-31: O, 512 columns
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(kHeads, ROWS, 0, 0);
+  static constexpr uint32_t IDESC_O = idesc_bf16_f32(kHeads, 256, 0, 1);
+  static_assert(S_COL + 2 * ROWS <= TMEM_COLS, "Q and two logit buffers must fit in 512 columns");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 };
 
 struct AttendParams {
+  const __nv_bfloat16* q_nope;    // [T, 64, 512]
+  const __nv_bfloat16* q_pe;      // [T, 64, 64] (RoPE layers)
   const __nv_bfloat16* cache;     // [n_rows, ld_c]
   const float* qmul;              // [T, 64]
   const int64_t* seq_row_start;   // [B]
@@ -72,7 +93,8 @@ struct AttendParams {
   __nv_bfloat16* out;             // [T, 64, 512]
   float* lse;                     // [T, 64] or null
   float* ws_o;                    // [T, n_split, 64, 512] partial numerators (n_split > 1)
-  float* ws_ml;                   // [T, n_split, 64, 2] (max in log2 units, sum)
+  float* ws_ml;                   // [T, n_split, 64, 4] (max in log2 units, sum of the bf16 weights,
+                                  //  sum of the fp32 weights, unused)
   int64_t ld_c;
   int64_t n_rows;
   float scale_log2e;              // softmax_scale * log2(e)
@@ -81,26 +103,23 @@ struct AttendParams {
   int32_t k;
   int32_t n_split;
   int32_t rows_per_split;         // multiple of 64
+  int32_t merge;                  // 1: the n_split CTAs of a query are a cluster and merge in DSMEM
 };
 
 struct AttScratch {
-  uint64_t q_full;
-  uint64_t s_full[2];             // S^T of a tile is in TMEM (per lane half)
-  uint64_t p_full;                // P^T of a tile is in shared memory
+  uint64_t q_smem;                // Q has landed in tile buffer 2 (TMA)
+  uint64_t q_full;                // Q is in tensor memory (128 arrivals)
+  uint64_t s_full[2];             // logits of a tile are in S buffer b
+  uint64_t s_free[2];             // S buffer b has been read by the softmax (128 arrivals)
+  uint64_t p_full;                // P of a tile is in shared memory (128 arrivals)
   uint64_t o_done;                // the output product of a tile has completed
   uint64_t mma_done;
-  uint64_t full[2][9];            // chunk c of tile buffer b loaded
-  uint64_t free_[2];              // tile buffer no longer read (per buffer)
+  uint64_t full[3];               // tile buffer b loaded
+  uint64_t free_[3];              // tile buffer b no longer read
   uint32_t tmem_slot;
   int abort_flag;
-  alignas(16) float fac[64];      // scale * m[t,h] * log2(e)   (read as float4)
-  alignas(16) float m_used[64];   // running (lazy) max per head, log2 units (float4)
-  alignas(16) float alpha[64];    // rescale factor of the current tile
-  alignas(16) int32_t red[4][64]; // per-warp head maxima (order-mapped ints) / sums
 };
-static_assert(sizeof(AttScratch) <= 2048, "scratch overflow");
-static_assert(offsetof(AttScratch, fac) % 16 == 0 && offsetof(AttScratch, m_used) % 16 == 0,
-              "vector-read arrays must be 16-byte aligned");
+static_assert(sizeof(AttScratch) <= 1024, "scratch overflow");
 
 __device__ __forceinline__ void unit_rows(const AttendParams& p, int t, int j, int& r_begin,
                                           int& r_end, bool report) {
@@ -114,17 +133,122 @@ __device__ __forceinline__ void unit_rows(const AttendParams& p, int t, int j, i
   if (r_end < r_begin) r_end = r_begin;
 }
 
-// Work unit = (query t, split j) = rows [j*R, min(count, (j+1)*R)) of idx[t], in
-// tiles of 64 rows held in two buffers:
-//   producers (warps 5-7) gather tile j into buffer j & 1 with 16-byte cp.async,
-//     in the 128-byte-swizzled chunk-major layout (chunk = 64 rows x 64 columns)
-//   the MMA thread (warp 4) issues, per tile,
-//     S^T[64 rows x 64 heads] = C . Q^T     M = 64, into TMEM lane half (j & 1)
-//     O^T[512 x 64] += C^T . P^T            M = 128 latent columns x 4, K = 64 rows
-//     and issues S(j+1) before O(j), so the logits of the next tile are ready
-//     while the softmax of this one runs and the tile after that is loading
-//   softmax warps 0-3: lane L of warp w holds row 16 w + (L & 15) of the tile
-//     whose lane half is L >> 4.
+// tcgen05.st over the 16 lanes [taddr.lane, +16): threads 0-15 write columns
+// [col, col + N), threads 16-31 columns [col + N, col + 2N).
+__device__ __forceinline__ void tmem_st16x2_32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 32, "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+      "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]),
+      "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]),
+      "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16x2_16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 16, "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] . B[smem]: A read from tensor memory.  A and D must sit
+// in the same TMEM lanes (for M = 64: lanes 0-15 of every 32-lane quarter).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Merge of a query's split partials inside its cluster (n = p.n_split CTAs,
+// rank = split).  Each CTA has staged O_j[64][512] (unnormalised, fp32, pieces
+// swizzled by h & 7) and (m_j, l_j, lx_j) per head at the start of its shared
+// memory (l: sum of the bf16 weights the products used, lx: of the fp32
+// weights); rank r produces columns [r 512 / n, (r + 1) 512 / n) of every head:
+//   M = max_j m_j,  w_j = 2^(m_j - M),  L = sum_j w_j l_j,
+//   o[h, c] = sum_j (w_j / L) O_j[h, c],
+//   lse[h] = (M + log2 sum_j w_j lx_j) ln 2 (rank 0).
+__device__ __forceinline__ void cluster_merge(const AttendParams& p, uint8_t* cs, uint8_t* ps, int t,
+                                              int rank) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int n = p.n_split;
+  cl.sync();   // every CTA's partial is staged
+  float* wt = reinterpret_cast<float*>(ps);   // [64 heads][8]: w_j / L
+  const int tid = threadIdx.x;
+  if (tid < kHeads) {
+    const int h = tid;
+    float m[8], l[8], lx[8];
+    float M = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      m[j] = -INFINITY;
+      l[j] = 0.f;
+      lx[j] = 0.f;
+      if (j < n) {
+        const float* xml = cl.map_shared_rank(reinterpret_cast<float*>(cs + kHeads * kLatent * 4), j);
+        m[j] = xml[4 * h];
+        l[j] = xml[4 * h + 1];
+        lx[j] = xml[4 * h + 2];
+        M = fmaxf(M, m[j]);
+      }
+    }
+    float w[8], L = 0.f, Lx = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      w[j] = (m[j] == -INFINITY) ? 0.f : ex2_approx(m[j] - M);
+      L += w[j] * l[j];
+      Lx += w[j] * lx[j];
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wt[h * 8 + j] = (L > 0.f) ? w[j] / L : 0.f;
+    if (rank == 0 && p.lse != nullptr)
+      p.lse[(int64_t)t * kHeads + h] = (Lx > 0.f) ? (M + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
+  }
+  __syncthreads();
+  const int c0 = rank * (kLatent / 4) / n, c1 = (rank + 1) * (kLatent / 4) / n;   // float4 columns
+  const int nc = c1 - c0;
+  const float4* xo[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    xo[j] = cl.map_shared_rank(reinterpret_cast<const float4*>(cs), j < n ? j : 0);
+  for (int i = tid; i < kHeads * nc; i += blockDim.x) {
+    const int h = i / nc;
+    const int c = c0 + (i - h * nc);
+    const int piece = h * (kLatent / 4) + (c ^ (h & 7));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float wj = (j < n) ? wt[h * 8 + j] : 0.f;
+      if (wj != 0.f) {
+        const float4 v = xo[j][piece];
+        acc.x = fmaf(wj, v.x, acc.x);
+        acc.y = fmaf(wj, v.y, acc.y);
+        acc.z = fmaf(wj, v.z, acc.z);
+        acc.w = fmaf(wj, v.w, acc.w);
+      }
+    }
+    uint2 o;
+    o.x = pack_bf16x2(acc.x, acc.y);
+    o.y = pack_bf16x2(acc.z, acc.w);
+    *reinterpret_cast<uint2*>(p.out + ((int64_t)t * kHeads + h) * kLatent + 4 * c) = o;
+  }
+  cl.sync();   // no CTA leaves while its staged partial may still be read
+}
+
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c,
+                                             uint32_t& d) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr));
+}
+
 template <int DR>
 __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
     attend_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_constant__ CUtensorMap qp_map,
@@ -133,13 +257,10 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // The swizzled layouts need 1024-byte alignment; dynamic shared memory starts
   // there when the kernel has no static shared memory.
-  if ((smem_u32(smem_raw) & 1023u) != 0) {
-    if (threadIdx.x == 0) raise_error(kErrBadSeq);
-    return;
-  }
-  uint8_t* qs = smem_raw;
-  uint8_t* cs = smem_raw + C::Q_BYTES;                  // two tile buffers
-  uint8_t* ps = cs + 2 * C::TILE_BYTES;
+  const bool smem_ok = (smem_u32(smem_raw) & 1023u) == 0;
+  if (!smem_ok && threadIdx.x == 0) raise_error(kErrBadSeq);
+  uint8_t* cs = smem_raw;                               // three tile buffers
+  uint8_t* ps = cs + C::NBUF * C::TILE_BYTES;
   AttScratch* sc = reinterpret_cast<AttScratch*>(ps + C::P_BYTES);
   volatile int* abort_flag = &sc->abort_flag;
 
@@ -149,14 +270,17 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
   const int jsplit = blockIdx.x % p.n_split;
 
   if (threadIdx.x == 0) {
-    mbar_init(&sc->q_full, 1);
-    mbar_init(&sc->s_full[0], 1);
-    mbar_init(&sc->s_full[1], 1);
+    mbar_init(&sc->q_smem, 1);
+    mbar_init(&sc->q_full, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sc->s_full[b], 1);
+      mbar_init(&sc->s_free[b], 128);
+    }
     mbar_init(&sc->p_full, 128);
     mbar_init(&sc->o_done, 1);
     mbar_init(&sc->mma_done, 1);
-    for (int b = 0; b < 2; ++b) {
-      for (int c = 0; c < C::KCH; ++c) mbar_init(&sc->full[b][c], C::PRODUCERS);
+    for (int b = 0; b < C::NBUF; ++b) {
+      mbar_init(&sc->full[b], C::PRODUCERS);
       mbar_init(&sc->free_[b], 1);
     }
     sc->abort_flag = 0;
@@ -173,169 +297,159 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
 
   int r_begin, r_end;
   unit_rows(p, t, jsplit, r_begin, r_end, threadIdx.x == 0);
+  if (!smem_ok) r_end = r_begin;   // nothing is computed; cluster barriers are still met
   const int n_tiles = (r_end - r_begin + C::ROWS - 1) / C::ROWS;
 
   if (warp >= 5) {
     // ------------------------------------------------------------- producers
-    // Thread pt copies 16-byte piece (lane & 7) of rows prow, prow + 12, ... of
-    // every chunk.  Destination offsets (with the 128-byte swizzle) depend only
-    // on the row; source row addresses are computed once per tile.
-    const int pt = threadIdx.x - 160;  // 0..95
-    if (pt == 0 && n_tiles > 0) {
-      prefetch_tmap(&qn_map);
-      mbar_arrive_expect_tx(&sc->q_full, C::Q_BYTES);
-      for (int c = 0; c < 8; ++c)
-        tma_load_2d(qs + c * C::QCHUNK_BYTES, &qn_map, c * 64, t * kHeads, &sc->q_full);
-      if (DR == 64) {
-        prefetch_tmap(&qp_map);
-        tma_load_2d(qs + 8 * C::QCHUNK_BYTES, &qp_map, 0, t * kHeads, &sc->q_full);
-      }
-    }
+    // Warp pw = 0..2 gathers row quads pw, pw + 3, ... of each tile.  The
+    // 4 x KCH x 8 sixteen-byte pieces of a quad are KCH warp-wide copies;
+    // piece g = 32 j + lane of instruction j is piece g % (8 KCH) of quad row
+    // g / (8 KCH).  Lane l holds the index of the warp's row 4 (l >> 2) + (l & 3)
+    // (quad pw + 3 (l >> 2)); other lanes read it with a shuffle.
+    const int pw = warp - 5;
+    constexpr int PPR = 8 * C::KCH;          // 16-byte pieces per row
+    constexpr int NQ = C::ROWS / 4;          // row quads per tile
+    constexpr int QPW = (NQ + 2) / 3;        // quads per warp, at most
+    static_assert(4 * PPR == 32 * C::KCH, "a quad is KCH warp-wide copies");
+    static_assert(4 * QPW <= 32, "one index per lane");
     const int b = p.q_seq[t];
     const bool seq_ok = (b >= 0 && b < p.B);
-    if (!seq_ok && pt == 0 && n_tiles > 0) raise_error(kErrBadSeq);
+    if (!seq_ok && threadIdx.x == 160 && n_tiles > 0) raise_error(kErrBadSeq);
     const int64_t base = seq_ok ? p.seq_row_start[b] : 0;
-    const int prow = 4 * (warp - 5) + (lane >> 3);  // rows prow + 12 jj
-    const int piece = lane & 7;
-    constexpr int RPT = (C::ROWS + 11) / 12;          // 6 rows per thread at most
-    const uint32_t cs0 = smem_u32(cs);
-    uint32_t dst[RPT];
-#pragma unroll
-    for (int jj = 0; jj < RPT; ++jj) {
-      const int r = prow + 12 * jj;
-      dst[jj] = r * 128 + ((piece ^ (r & 7)) << 4);
+    if (threadIdx.x == 160 && n_tiles > 0) {
+      // Q [64 heads x (512 + DR)] into tile buffer 2, chunk-major, 128-byte swizzled.
+      uint8_t* qs = cs + 2 * C::TILE_BYTES;
+      prefetch_tmap(&qn_map);
+      mbar_arrive_expect_tx(&sc->q_smem, C::KCH * kHeads * 128);
+      for (int c = 0; c < 8; ++c) tma_load_2d(qs + c * kHeads * 128, &qn_map, c * 64, t * kHeads, &sc->q_smem);
+      if (DR == 64) {
+        prefetch_tmap(&qp_map);
+        tma_load_2d(qs + 8 * kHeads * 128, &qp_map, 0, t * kHeads, &sc->q_smem);
+      }
     }
+    const int my_quad = pw + 3 * (lane >> 2);
+    const int my_row = 4 * my_quad + (lane & 3);
+    const uint32_t cs0 = smem_u32(cs);
     const char* cache_bytes = reinterpret_cast<const char*>(p.cache);
     const int32_t* idx_t = p.idx + (int64_t)t * p.k;
-    // Index loads are software-pipelined one tile ahead so that a global
+    // The index of this lane's row, loaded one tile ahead so that a global
     // round trip never sits between a buffer becoming free and its copies.
-    // Rows of the tile three ahead are bulk-prefetched into L2, so their
-    // cp.async copies later hit L2.
-    constexpr int kPrefetchTiles = 3;
-    auto load_rows = [&](int i, int32_t (&out)[RPT]) {
-      const int r0 = r_begin + i * C::ROWS;
-#pragma unroll
-      for (int jj = 0; jj < RPT; ++jj) {
-        const int r = prow + 12 * jj;
-        out[jj] = (i < n_tiles && r < C::ROWS && r0 + r < r_end && seq_ok) ? idx_t[r0 + r] : -1;
-      }
+    auto load_idx = [&](int i) -> int32_t {
+      const int rr = r_begin + i * C::ROWS + my_row;
+      return (i < n_tiles && my_quad < NQ && rr < r_end && seq_ok) ? idx_t[rr] : -1;
     };
-    auto load_pf = [&](int i) -> int32_t {
-      const int rr = r_begin + i * C::ROWS + pt;
-      return (i < n_tiles && pt < C::ROWS && rr < r_end && seq_ok) ? idx_t[rr] : -1;
-    };
-    auto prefetch_row = [&](int32_t sidx) {
-      if (sidx >= 0 && base + sidx < p.n_rows)
-        prefetch_l2_bulk(cache_bytes + (base + sidx) * p.ld_c * 2, (kLatent + DR) * 2);
-    };
-    for (int i = 0; i < kPrefetchTiles && i < n_tiles; ++i) prefetch_row(load_pf(i));
-    int32_t cur[RPT];
-    load_rows(0, cur);
-    int32_t pf_next = load_pf(kPrefetchTiles);
+    int32_t cur = load_idx(0);
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
-      const int buf = i & 1;
-      prefetch_row(pf_next);
-      pf_next = load_pf(i + kPrefetchTiles + 1);
-      if (i >= 2 && !mbar_wait(&sc->free_[buf], (uint32_t)(((i >> 1) - 1) & 1), abort_flag)) {
+      const int buf = i % C::NBUF;
+      if (i >= C::NBUF &&
+          !mbar_wait(&sc->free_[buf], (uint32_t)((i / C::NBUF - 1) & 1), abort_flag)) {
         ok = false;
         break;
       }
-      const char* src[RPT];
-      uint32_t nbytes[RPT];
-#pragma unroll
-      for (int jj = 0; jj < RPT; ++jj) {
-        const int32_t sidx = cur[jj];
-        src[jj] = cache_bytes;
-        nbytes[jj] = 0;
-        if (sidx >= 0 && base + sidx < p.n_rows) {
-          src[jj] = cache_bytes + ((base + sidx) * p.ld_c) * 2 + piece * 16;
-          nbytes[jj] = 16;
-        } else if (sidx != -1 && piece == 0) {
-          raise_error(kErrBadIndex);
-        }
+      // Buffer 2 holds Q until the softmax warps have moved it to TMEM.
+      if (i == 2 && !mbar_wait(&sc->q_full, 0, abort_flag)) {
+        ok = false;
+        break;
       }
-      load_rows(i + 1, cur);   // next tile's indices, in flight while this tile is copied
+      int32_t row = -1;   // row of the cache, or -1: the copy zero-fills
+      if (cur >= 0 && base + cur < p.n_rows) row = (int32_t)(base + cur);
+      else if (cur != -1) raise_error(kErrBadIndex);
+      cur = load_idx(i + 1);
       const uint32_t tb = cs0 + buf * C::TILE_BYTES;
 #pragma unroll 1
-      for (int c = 0; c < C::KCH; ++c) {
+      for (int k = 0; k < QPW; ++k) {
+        const int quad = pw + 3 * k;
+        if (quad >= NQ) break;
 #pragma unroll
-        for (int jj = 0; jj < RPT; ++jj) {
-          if (prow + 12 * jj < C::ROWS)
-            cp_async_16(tb + c * C::CHUNK_BYTES + dst[jj], src[jj] + (nbytes[jj] ? c * 128 : 0), nbytes[jj]);
+        for (int j = 0; j < C::KCH; ++j) {
+          const int g = 32 * j + lane;
+          const int riq = g / PPR;
+          const int pr = g - riq * PPR;
+          const int32_t src_row = __shfl_sync(0xffffffffu, row, 4 * k + riq);
+          const int r = 4 * quad + riq;
+          const uint32_t dst = tb + (pr >> 3) * C::CHUNK_BYTES + r * 128 + (((pr & 7) ^ (r & 7)) << 4);
+          const char* src = src_row >= 0 ? cache_bytes + (int64_t)src_row * p.ld_c * 2 + pr * 16 : cache_bytes;
+          cp_async_16(dst, src, src_row >= 0 ? 16u : 0u);
         }
-        cp_async_arrive_noinc(&sc->full[buf][c]);   // lands once this thread's copies so far have
       }
+      cp_async_arrive_noinc(&sc->full[buf]);   // lands once this thread's copies so far have
     }
     if (!ok) *abort_flag = 1;
     cp_async_wait_all();   // nothing may still be landing in shared memory at exit
-    if (pt == 0 && n_tiles > 0) mbar_wait(&sc->q_full, 0, nullptr);
+    if (threadIdx.x == 160 && n_tiles > 0) mbar_wait(&sc->q_smem, 0, nullptr);   // no TMA in flight at exit
   } else if (warp == 4) {
     // ------------------------------------------------------------- MMA issuer
-    // Issues, in order of readiness, the logit MMAs of the next tile chunk by
-    // chunk as its rows land, and the output MMAs of a tile as soon as its
-    // softmax weights are in shared memory.  Descriptors are built once; an
+    // Issues, in order of readiness, the logit MMAs of the next tile once its
+    // rows have landed and the output MMAs of a tile as soon as its softmax
+    // weights are in shared memory.  Descriptors are built once; an
     // operand at byte offset d from its base is the base descriptor + (d >> 4)
     // (shared addresses stay below 256 KB, so the start field cannot carry).
     if (lane == 0 && n_tiles > 0) {
       bool ok = mbar_wait(&sc->q_full, 0, abort_flag);
-      const uint64_t q_desc = sdesc_sw128(smem_u32(qs), 16, 1024);
-      const uint64_t s_desc0 = sdesc_sw128(smem_u32(cs), 16, 1024);                        // K-major C
-      const uint64_t o_desc0 = sdesc_sw128(smem_u32(cs), C::CHUNK_BYTES, 1024);            // MN-major C^T
-      const uint64_t p_desc = sdesc_sw128(smem_u32(ps), C::CHUNK_BYTES, 1024);             // MN-major P^T
-      int s_tile = 0, s_chunk = 0;   // next logit chunk to issue
+      tc_fence_after();
+      const uint64_t s_desc0 = sdesc_sw128(smem_u32(cs), 16, 1024);                 // K-major C
+      const uint64_t o_desc0 = sdesc_sw128(smem_u32(cs), C::CHUNK_BYTES, 1024);     // MN-major C
+      const uint64_t p_desc = sdesc_sw128(smem_u32(ps), 16, 1024);                  // K-major P
+      const uint32_t o_tmem = tmem_base + (C::O_LANE << 16);
+      int s_tile = 0;                // next logit product to issue
+      bool s_buf_free = true;        // S buffer of s_tile has been read by its previous softmax
       int o_tile = 0;                // next output product to issue
-      uint64_t t_idle = global_timer_ns();
+      uint64_t t_idle = 0;
       uint32_t spins = 0;
       while (ok && o_tile < n_tiles) {
         bool progressed = false;
-        // Output product of tile o_tile once its P^T is written.
+        // Output product of tile o_tile once its P is written.
         if (o_tile < s_tile && mbar_test(&sc->p_full, (uint32_t)(o_tile & 1))) {
           tc_fence_after();
-          fence_proxy_async_smem();     // P^T was written with st.shared
-          const uint64_t ob = o_desc0 + (uint64_t)(((o_tile & 1) * C::TILE_BYTES) >> 4);
+          const int buf = o_tile % C::NBUF;
 #pragma unroll
-          for (int blk = 0; blk < 4; ++blk) {
+          for (int kk = 0; kk < C::ROWS / 16; ++kk) {
 #pragma unroll
-            for (int kk = 0; kk < C::ROWS / 16; ++kk)
-              mma_bf16_ss(tmem_base + C::O_COL + blk * 64,
-                          ob + (uint64_t)((2 * blk * C::CHUNK_BYTES + kk * 2048) >> 4),
-                          p_desc + (uint64_t)((kk * 2048) >> 4), C::IDESC_O, (o_tile > 0 || kk > 0) ? 1u : 0u);
+            for (int nh = 0; nh < 2; ++nh)
+              mma_bf16_ss(o_tmem + nh * 256, p_desc + (uint64_t)((kk * 32) >> 4),
+                          o_desc0 + (uint64_t)((buf * C::TILE_BYTES + 4 * nh * C::CHUNK_BYTES + kk * 2048) >> 4),
+                          C::IDESC_O, (o_tile > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&sc->free_[o_tile & 1]);
+          mma_commit(&sc->free_[buf]);
           mma_commit(&sc->o_done);
           ++o_tile;
           progressed = true;
         }
-        // Logits of tile s_tile, one chunk at a time.  Its TMEM lane half was
-        // last read by the softmax of tile s_tile - 2, whose weights the
-        // output product o_tile > s_tile - 2 has already consumed.
-        if (s_tile < n_tiles && o_tile >= s_tile - 1) {
-          const int buf = s_tile & 1;
-          if (mbar_test(&sc->full[buf][s_chunk], (uint32_t)((s_tile >> 1) & 1))) {
-            fence_proxy_async_smem();   // cp.async wrote through the generic proxy
+        // Logits of tile s_tile once its rows have landed and its S buffer has
+        // been read by the softmax of tile s_tile - 2: all KCH x 4 MMAs at once.
+        if (s_tile < n_tiles) {
+          const int sb = s_tile & 1;
+          if (!s_buf_free)
+            s_buf_free = mbar_test(&sc->s_free[sb], (uint32_t)(((s_tile - 2) >> 1) & 1));
+          const int buf = s_tile % C::NBUF;
+          if (s_buf_free && mbar_test(&sc->full[buf], (uint32_t)((s_tile / C::NBUF) & 1))) {
+            fence_proxy_async_smem();   // cp.async wrote the tile through the generic proxy
             tc_fence_after();
-            const uint64_t sb = s_desc0 + (uint64_t)((buf * C::TILE_BYTES + s_chunk * C::CHUNK_BYTES) >> 4);
-            const uint64_t qb = q_desc + (uint64_t)((s_chunk * C::QCHUNK_BYTES) >> 4);
-            const uint32_t d = tmem_base + ((uint32_t)(16 * buf) << 16) + C::S_COL;
+            const uint64_t sbd = s_desc0 + (uint64_t)((buf * C::TILE_BYTES) >> 4);
+            const uint32_t d = tmem_base + C::S_COL + 64 * sb;
+#pragma unroll 1
+            for (int c = 0; c < C::KCH; ++c) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(d, sb + (uint64_t)((kk * 32) >> 4), qb + (uint64_t)((kk * 32) >> 4), C::IDESC_S,
-                          (s_chunk | kk) ? 1u : 0u);
-            if (++s_chunk == C::KCH) {
-              mma_commit(&sc->s_full[buf]);
-              s_chunk = 0;
-              ++s_tile;
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ts(d, tmem_base + C::Q_COL + 32 * c + 8 * kk,
+                            sbd + (uint64_t)((c * C::CHUNK_BYTES + kk * 32) >> 4), C::IDESC_S, (c | kk) ? 1u : 0u);
             }
+            mma_commit(&sc->s_full[sb]);
+            ++s_tile;
+            s_buf_free = s_tile < 2;
             progressed = true;
           }
         }
         if (progressed) {
           spins = 0;
-          t_idle = global_timer_ns();
         } else if ((++spins & 255u) == 0) {
+          // The idle clock starts at the first check after progress stopped.
+          const uint64_t now = global_timer_ns();
           if (*abort_flag) ok = false;
-          else if (global_timer_ns() - t_idle > kWaitLimitNs) {
+          else if (spins == 256u) t_idle = now;
+          else if (now - t_idle > kWaitLimitNs) {
             raise_error(kErrTimeout);
             ok = false;
           }
@@ -347,228 +461,220 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------- softmax + epilogue
-    // Lane L of warp w owns row 16 w + (L & 15) of the current tile and heads
-    // 32 (L >> 4) .. 32 (L >> 4) + 31 (the 16x32bx2 TMEM load pattern).
-    const int st = threadIdx.x;                // 0..127
-    const int sw = warp;                       // softmax warp 0..3 == TMEM lane quarter
-    const int hh = lane >> 4;                  // head half
-    const int row = 16 * warp + (lane & 15);   // tile row
-    const int r = 32 * warp + lane;            // epilogue: latent column within a 128-block
-    const uint32_t lane_base = tmem_base + ((uint32_t)(warp * 32) << 16);
-    const int sb = p.q_seq[t];
-    const bool seq_ok = (sb >= 0 && sb < p.B);
-    const int64_t seq_base = seq_ok ? p.seq_row_start[sb] : 0;
-    if (st < kHeads) {
-      sc->fac[st] = p.qmul[(int64_t)t * kHeads + st] * p.scale_log2e;
-      sc->m_used[st] = -INFINITY;
-    }
-    named_bar_sync(1, 128);
-    float fac[32], mref[32], l_part[32];
+    // Lane L of warp w owns head h = 16 w + (L & 15) and rows 32 hf .. 32 hf + 31
+    // of each tile, hf = L >> 4 (the 16x32bx2 TMEM access pattern).
+    const int hf = lane >> 4;
+    const int h = 16 * warp + (lane & 15);
+    const uint32_t lo_base = tmem_base + ((uint32_t)(warp * 32) << 16);          // Q, S lanes
+    const uint32_t hi_base = tmem_base + ((uint32_t)(warp * 32 + C::O_LANE) << 16);  // O lanes
+    const int sb_seq = p.q_seq[t];
+    const bool seq_ok = (sb_seq >= 0 && sb_seq < p.B);
+    const int64_t seq_base = seq_ok ? p.seq_row_start[sb_seq] : 0;
+    const float fac = p.qmul[(int64_t)t * kHeads + h] * p.scale_log2e;
+    if (n_tiles > 0) {
+      // Q[t, h] into TMEM from its staging copy in tile buffer 2: this thread
+      // moves elements [128 s + 64 hf, + 64) of the NoPE part (chunk 2 s + hf)
+      // and [32 hf, + 32) of the rotary part (chunk 8, pieces 4 hf ..).
+      const bool got_q = mbar_wait(&sc->q_smem, 0, abort_flag);
+      const uint32_t qrow = smem_u32(cs + 2 * C::TILE_BYTES) + h * 128;
+#pragma unroll 1
+      for (int s = 0; s < 4; ++s) {
+        uint32_t v[32];
+        const uint32_t ca = qrow + (2 * s + hf) * (kHeads * 128);
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      fac[c] = sc->fac[hh * 32 + c];
-      mref[c] = -INFINITY;
-      l_part[c] = 0.f;
+        for (int u = 0; u < 8; ++u) ld_shared_v4(ca + ((u ^ (h & 7)) << 4), v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        tmem_st16x2_32(lo_base + C::Q_COL + 64 * s, v);
+      }
+      if (DR == 64) {
+        uint32_t v[16];
+        const uint32_t ca = qrow + 8 * (kHeads * 128);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          ld_shared_v4(ca + (((4 * hf + u) ^ (h & 7)) << 4), v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+        tmem_st16x2_16(lo_base + C::Q_COL + 256, v);
+      }
+      if (!got_q) *abort_flag = 1;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sc->q_full);
     }
-    const uint32_t pbase = smem_u32(ps) + row * 128;
-    // A row takes part only if its index is a real position of the sequence
-    // (entries of -1 inside the counted prefix are skipped).  The index of the
-    // next tile's row is loaded one tile ahead.
-    auto row_index = [&](int i) -> int32_t {
-      const int rr = r_begin + i * C::ROWS + row;
-      return (i < n_tiles && rr < r_end && seq_ok) ? p.idx[(int64_t)t * p.k + rr] : -1;
+    // Rows that take part: a real position of the sequence inside the unit
+    // (entries of -1 inside the counted prefix are skipped).  Lane L tests
+    // rows L and 32 + L; a ballot gives every lane the masks of both halves.
+    auto valid_mask = [&](int i) -> uint32_t {
+      uint32_t m[2];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int rr = r_begin + i * C::ROWS + 32 * half + lane;
+        const int32_t sidx = (i < n_tiles && rr < r_end && seq_ok) ? p.idx[(int64_t)t * p.k + rr] : -1;
+        m[half] = __ballot_sync(0xffffffffu, sidx >= 0 && seq_base + sidx < p.n_rows);
+      }
+      return hf ? m[1] : m[0];
     };
-    int32_t sidx_next = row_index(0);
+    const uint32_t pbase = smem_u32(ps) + h * 128;
+    float m_used = -INFINITY;   // reference max of this head, log2 units
+    float l_sum = 0.f;          // this thread's share of the row sum of the bf16 weights (normalises o)
+    float l_ex = 0.f;           // ... and of the fp32 weights (gives lse)
+    uint32_t vm_next = valid_mask(0);
     bool ok = true;
     for (int i = 0; i < n_tiles && ok; ++i) {
-      const int buf = i & 1;
-      const int32_t sidx = sidx_next;
-      sidx_next = row_index(i + 1);
-      const bool valid = sidx >= 0 && seq_base + sidx < p.n_rows;
-      const bool got_s = mbar_wait(&sc->s_full[buf], (uint32_t)((i >> 1) & 1), abort_flag);
+      const int sbuf = i & 1;
+      const uint32_t vm = vm_next;
+      vm_next = valid_mask(i + 1);
+      const bool got_s = mbar_wait(&sc->s_full[sbuf], (uint32_t)((i >> 1) & 1), abort_flag);
       if (named_bar_or(1, 128, !got_s)) { ok = false; break; }   // leave together
       tc_fence_after();
       uint32_t v[32];
-      tmem_ld16x2_32(lane_base + ((uint32_t)(16 * buf) << 16) + C::S_COL, v);
+      tmem_ld16x2_32(lo_base + C::S_COL + 64 * sbuf, v);
       tmem_wait_ld();
-      // Speculative weights against the current references; valid unless a
-      // logit exceeds its head's reference by more than 2^8.
-      float dmax = -INFINITY;
+      tc_fence_before();
+      mbar_arrive(&sc->s_free[sbuf]);
+      float z[32];
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        z[c] = ((vm >> c) & 1u) ? __uint_as_float(v[c]) * fac : -INFINITY;
+        mt = fmaxf(mt, z[c]);
+      }
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+      // Lazy reference: move it only when the tile max exceeds it by more than 2^8.
+      float alpha = 1.f;
+      bool resc = false;
+      if (mt > m_used + 8.f) {
+        alpha = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - mt);
+        resc = (m_used != -INFINITY);
+        m_used = mt;
+        l_sum *= alpha;
+        l_ex *= alpha;
+      }
       uint32_t pk[16];
 #pragma unroll
       for (int c = 0; c < 32; c += 2) {
-        const float d0 = fmaf(__uint_as_float(v[c]), fac[c], -mref[c]);
-        const float d1 = fmaf(__uint_as_float(v[c + 1]), fac[c + 1], -mref[c + 1]);
-        dmax = fmaxf(dmax, fmaxf(d0, d1));
-        pk[c >> 1] = pack_bf16x2(ex2_approx(d0), ex2_approx(d1));
-      }
-      const bool grow = named_bar_or(1, 128, valid && !(dmax <= 8.f));
-      if (grow) {
-        // Exact per-head maxima of the tile (always on the first tile).
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float z = valid ? __uint_as_float(v[c]) * fac[c] : -INFINITY;
-          const int zl = (hh == 0) ? f2ord(z) : f2ord(-INFINITY);
-          const int zh = (hh == 1) ? f2ord(z) : f2ord(-INFINITY);
-          const int m_lo = warp_max_s32(zl);   // head c      over this warp's 16 rows
-          const int m_hi = warp_max_s32(zh);   // head 32 + c over this warp's 16 rows
-          if (lane == c) {
-            sc->red[sw][c] = m_lo;
-            sc->red[sw][32 + c] = m_hi;
-          }
-        }
-        named_bar_sync(1, 128);
-        bool resc = false;
-        if (st < kHeads) {
-          float tmax = ord2f(sc->red[0][st]);
-#pragma unroll
-          for (int w2 = 1; w2 < 4; ++w2) tmax = fmaxf(tmax, ord2f(sc->red[w2][st]));
-          const float mo = sc->m_used[st];
-          float al = 1.f;
-          if (tmax > mo) {
-            al = (mo == -INFINITY) ? 0.f : ex2_approx(mo - tmax);
-            resc = (mo != -INFINITY);
-            sc->m_used[st] = tmax;
-          }
-          sc->alpha[st] = al;
-        }
-        const bool any_resc = named_bar_or(1, 128, resc);
-        if (any_resc) {
-          // O(i-1) must be complete before O^T is rescaled in place.
-          const bool got_o = mbar_wait(&sc->o_done, (uint32_t)((i - 1) & 1), abort_flag);
-          if (named_bar_or(1, 128, !got_o)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll 1
-          for (int blk = 0; blk < 4; ++blk) {
-#pragma unroll 1
-            for (int h2 = 0; h2 < 2; ++h2) {
-              uint32_t u[32];
-              const uint32_t a = lane_base + C::O_COL + blk * 64 + h2 * 32;
-              tmem_ld32(a, u);
-              tmem_wait_ld();
-#pragma unroll
-              for (int c = 0; c < 32; ++c)
-                u[c] = __float_as_uint(__uint_as_float(u[c]) * sc->alpha[h2 * 32 + c]);
-              tmem_st32(a, u);
-            }
-          }
-          tmem_wait_st();
-        }
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          l_part[c] *= sc->alpha[hh * 32 + c];
-          mref[c] = sc->m_used[hh * 32 + c];
-        }
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float d0 = fmaf(__uint_as_float(v[c]), fac[c], -mref[c]);
-          const float d1 = fmaf(__uint_as_float(v[c + 1]), fac[c + 1], -mref[c + 1]);
-          pk[c >> 1] = pack_bf16x2(ex2_approx(d0), ex2_approx(d1));
-        }
-      }
-      if (!valid) {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) pk[c] = 0u;
+        const float p0 = ((vm >> c) & 1u) ? ex2_approx(z[c] - m_used) : 0.f;
+        const float p1 = ((vm >> (c + 1)) & 1u) ? ex2_approx(z[c + 1] - m_used) : 0.f;
+        l_ex += p0 + p1;
+        pk[c >> 1] = pack_bf16x2(p0, p1);
       }
       if (i > 0) {
-        // O(i-1) finished: P^T of the previous tile is no longer read.
+        // O(i-1) finished: P of the previous tile is no longer read, and O may
+        // be rescaled in place.
         const bool got_o = mbar_wait(&sc->o_done, (uint32_t)((i - 1) & 1), abort_flag);
         if (named_bar_or(1, 128, !got_o)) { ok = false; break; }
         tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+          for (int cb = 0; cb < kLatent; cb += 64) {
+            uint32_t u[32];
+            tmem_ld16x2_32(hi_base + cb, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
+            tmem_st16x2_32(hi_base + cb, u);
+          }
+          tmem_wait_st();
+        }
       }
-      // This thread's 32 heads of the row's P^T (bf16) and the row sums of the
-      // rounded weights the tensor core multiplies.
+      // P row h, rows 32 hf .. + 31 of the tile = 16-byte pieces 4 hf .. 4 hf + 3,
+      // and the row sum of the rounded weights the tensor core multiplies.
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        const int q = hh * 4 + q4;   // 16-byte group of 8 heads
-        st_shared_v4(pbase + ((q ^ (row & 7)) << 4), pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        const int q = 4 * hf + q4;
+        st_shared_v4(pbase + ((q ^ (h & 7)) << 4), pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
       }
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        l_part[2 * c] += __uint_as_float(pk[c] << 16);
-        l_part[2 * c + 1] += __uint_as_float(pk[c] & 0xFFFF0000u);
-      }
+      for (int c = 0; c < 16; ++c)
+        l_sum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&sc->p_full);
     }
     if (!ok) *abort_flag = 1;
 
-    // ---- epilogue: per-head row sums, then normalised output or partials
+    // ---- epilogue: normalised output or partials
     bool have_o = ok && n_tiles > 0;
     if (have_o) {
       const bool got_o = mbar_wait(&sc->o_done, (uint32_t)((n_tiles - 1) & 1), abort_flag);
       have_o = !named_bar_or(1, 128, !got_o);
       tc_fence_after();
     }
-    float* lsum = reinterpret_cast<float*>(&sc->red[0][0]);
-    named_bar_sync(1, 128);
-    // Sum each head over the 16 rows of this warp (lanes sharing a head half).
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      float s = l_part[c];
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      l_part[c] = s;
-    }
-    if ((lane & 15) == 0) {
-#pragma unroll
-      for (int c = 0; c < 32; ++c) lsum[sw * kHeads + hh * 32 + c] = l_part[c];
-    }
-    named_bar_sync(1, 128);
-    if (st < kHeads) {
-      const float L = lsum[st] + lsum[kHeads + st] + lsum[2 * kHeads + st] + lsum[3 * kHeads + st];
-      sc->alpha[st] = L;   // reuse: final row sum per head
-    }
-    named_bar_sync(1, 128);
+    const float L = l_sum + __shfl_xor_sync(0xffffffffu, l_sum, 16);
+    const float Lx = l_ex + __shfl_xor_sync(0xffffffffu, l_ex, 16);
     const int64_t unit = (int64_t)t * p.n_split + jsplit;
     if (p.n_split == 1) {
-      __nv_bfloat16* o_t = p.out + (int64_t)t * kHeads * kLatent;
+      const float inv = (have_o && L > 0.f) ? 1.f / L : 0.f;
+      uint4* o_t = reinterpret_cast<uint4*>(p.out + ((int64_t)t * kHeads + h) * kLatent + 32 * hf);
 #pragma unroll 1
-      for (int blk = 0; blk < 4; ++blk) {
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t u[32];
-          if (have_o) {
-            tmem_ld32(lane_base + C::O_COL + blk * 64 + hh * 32, u);
-            tmem_wait_ld();
-          }
+      for (int cb = 0; cb < kLatent; cb += 64) {
+        uint32_t u[32];
+        if (have_o) {
+          tmem_ld16x2_32(hi_base + cb, u);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int h = hh * 32 + c;
-            const float L = sc->alpha[h];
-            const float o = (have_o && L > 0.f) ? __uint_as_float(u[c]) / L : 0.f;
-            o_t[(int64_t)h * kLatent + blk * 128 + r] = __float2bfloat16_rn(o);
-          }
+          for (int c = 0; c < 32; ++c) u[c] = 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(u[8 * q]) * inv, __uint_as_float(u[8 * q + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(u[8 * q + 2]) * inv, __uint_as_float(u[8 * q + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(u[8 * q + 4]) * inv, __uint_as_float(u[8 * q + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(u[8 * q + 6]) * inv, __uint_as_float(u[8 * q + 7]) * inv);
+          o_t[cb / 8 + q] = w;
         }
       }
-      if (p.lse != nullptr && st < kHeads) {
-        const float L = sc->alpha[st];
-        p.lse[(int64_t)t * kHeads + st] =
-            (have_o && L > 0.f) ? (sc->m_used[st] + lg2_approx(L)) * 0.69314718055994531f : -INFINITY;
+      if (p.lse != nullptr && hf == 0)
+        p.lse[(int64_t)t * kHeads + h] =
+            (have_o && Lx > 0.f) ? (m_used + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
+    } else if (p.merge) {
+      // Stage unnormalised O[h, :] (fp32, 16-byte pieces XOR-swizzled by h & 7
+      // within 128-byte groups) and (max, sum) in this CTA's tile buffers,
+      // which no copy or product touches any more.
+      const uint32_t xrow = smem_u32(cs) + h * (kLatent * 4);
+#pragma unroll 1
+      for (int cb = 0; cb < kLatent; cb += 64) {
+        uint32_t u[32];
+        if (have_o) {
+          tmem_ld16x2_32(hi_base + cb, u);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) u[c] = 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int piece = (cb / 4 + 8 * hf + q) ^ (h & 7);
+          st_shared_v4(xrow + piece * 16, u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
+        }
+      }
+      if (hf == 0) {
+        float* xml = reinterpret_cast<float*>(cs + kHeads * kLatent * 4);
+        xml[4 * h] = have_o ? m_used : -INFINITY;
+        xml[4 * h + 1] = have_o ? L : 0.f;
+        xml[4 * h + 2] = have_o ? Lx : 0.f;
       }
     } else {
-      float* wo = p.ws_o + unit * kHeads * kLatent;
+      float4* wo = reinterpret_cast<float4*>(p.ws_o + (unit * kHeads + h) * kLatent + 32 * hf);
 #pragma unroll 1
-      for (int blk = 0; blk < 4; ++blk) {
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t u[32];
-          if (have_o) {
-            tmem_ld32(lane_base + C::O_COL + blk * 64 + hh * 32, u);
-            tmem_wait_ld();
-          }
+      for (int cb = 0; cb < kLatent; cb += 64) {
+        uint32_t u[32];
+        if (have_o) {
+          tmem_ld16x2_32(hi_base + cb, u);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int h = hh * 32 + c;
-            wo[(int64_t)h * kLatent + blk * 128 + r] = have_o ? __uint_as_float(u[c]) : 0.f;
-          }
+          for (int c = 0; c < 32; ++c) u[c] = 0u;
         }
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          wo[cb / 4 + q] = make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
+                                       __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
       }
-      if (st < kHeads) {
-        float* ml = p.ws_ml + (unit * kHeads + st) * 2;
-        ml[0] = have_o ? sc->m_used[st] : -INFINITY;
-        ml[1] = have_o ? sc->alpha[st] : 0.f;
+      if (hf == 0) {
+        float* ml = p.ws_ml + (unit * kHeads + h) * 4;
+        ml[0] = have_o ? m_used : -INFINITY;
+        ml[1] = have_o ? L : 0.f;
+        ml[2] = have_o ? Lx : 0.f;
       }
     }
   }
@@ -579,10 +685,11 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
+  if (p.merge) cluster_merge(p, cs, ps, t, jsplit);
 }
 
 // Merges the split partials of each (query, head): o = sum_j 2^(m_j - M) O_j / L,
-// L = sum_j 2^(m_j - M) l_j, lse = (M + log2 L) ln 2.  One block per
+// L = sum_j 2^(m_j - M) l_j, lse = (M + log2 sum_j 2^(m_j - M) lx_j) ln 2.  One block per
 // (query, head); each of the 128 threads owns 4 latent columns.
 constexpr int kMaxSplits = 32;
 __global__ void __launch_bounds__(128) attend_combine_kernel(const AttendParams p) {
@@ -590,23 +697,27 @@ __global__ void __launch_bounds__(128) attend_combine_kernel(const AttendParams 
   const int h = blockIdx.x % kHeads;
   const int ns = p.n_split;
   __shared__ float wsc[kMaxSplits];
-  __shared__ float stats[2];
+  __shared__ float stats[2];   // M, sum_j 2^(m_j - M) lx_j
   if (threadIdx.x < 32) {
     const int j = threadIdx.x;
     const int64_t u = (int64_t)t * ns + j;
-    const float m = (j < ns) ? p.ws_ml[(u * kHeads + h) * 2] : -INFINITY;
-    const float l = (j < ns) ? p.ws_ml[(u * kHeads + h) * 2 + 1] : 0.f;
+    const float m = (j < ns) ? p.ws_ml[(u * kHeads + h) * 4] : -INFINITY;
+    const float l = (j < ns) ? p.ws_ml[(u * kHeads + h) * 4 + 1] : 0.f;
+    const float lx = (j < ns) ? p.ws_ml[(u * kHeads + h) * 4 + 2] : 0.f;
     float M = m;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     const float sc = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
-    float L = sc * l;
+    float L = sc * l, Lx = sc * lx;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    for (int o = 16; o > 0; o >>= 1) {
+      L += __shfl_xor_sync(0xffffffffu, L, o);
+      Lx += __shfl_xor_sync(0xffffffffu, Lx, o);
+    }
     wsc[j] = (L > 0.f) ? sc / L : 0.f;
     if (j == 0) {
       stats[0] = M;
-      stats[1] = L;
+      stats[1] = Lx;
     }
   }
   __syncthreads();

@@ -248,7 +248,38 @@ dsa_status_t topk_impl(const float* scores, int64_t ld, const int32_t* q_pos, in
 struct SplitPlan {
   int n_split;
   int rows_per_split;
+  bool merge;   // the n_split CTAs of a query form a cluster and merge in distributed shared memory
 };
+
+// How many clusters of CL attention CTAs (one per SM, 225 KB of shared memory
+// each) can be resident at once (0: none, or CL outside 2..8).  A cluster must
+// sit inside one GPC, so this can be well below SMs / CL.
+int attend_max_clusters(int CL) {
+  static std::atomic<int> count[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+  if (CL < 2 || CL > 8) return 0;
+  const int known = count[CL].load(std::memory_order_relaxed);
+  if (known >= 0) return known;
+  using C = dsa::AttCfg<64>;
+  int n = 0;
+  if (cudaFuncSetAttribute(dsa::attend_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM_BYTES) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(CL);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, dsa::attend_kernel<64>, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  count[CL].store(n, std::memory_order_relaxed);
+  return n;
+}
 
 // Splits each query's selection across CTAs so that T x n_split is about one
 // wave of the GPU; rows per split are a multiple of the 64-row tile.
@@ -261,14 +292,17 @@ SplitPlan attend_plan(int32_t T, int32_t k) {
   SplitPlan sp;
   sp.rows_per_split = tiles_per * tile;
   sp.n_split = (k + sp.rows_per_split - 1) / sp.rows_per_split;
+  // Merge in clusters only when every query's cluster is resident at once;
+  // otherwise the partials go through the workspace and the combine kernel.
+  sp.merge = sp.n_split >= 2 && sp.n_split <= 8 && T <= attend_max_clusters(sp.n_split);
   return sp;
 }
 
 size_t attend_ws_bytes(int32_t T, int32_t k) {
   const SplitPlan sp = attend_plan(T, k);
-  if (sp.n_split <= 1) return 0;
+  if (sp.n_split <= 1 || sp.merge) return 0;
   const size_t units = (size_t)T * sp.n_split;
-  return round_up(units * dsa::kHeads * dsa::kLatent * 4, 256) + round_up(units * dsa::kHeads * 2 * 4, 256);
+  return round_up(units * dsa::kHeads * dsa::kLatent * 4, 256) + round_up(units * dsa::kHeads * 4 * 4, 256);
 }
 
 template <int DR>
@@ -290,6 +324,8 @@ dsa_status_t launch_attend(const void* q_nope, const void* q_pe, const float* qm
   }
   const SplitPlan sp = attend_plan(T, k);
   dsa::AttendParams p;
+  p.q_nope = static_cast<const __nv_bfloat16*>(q_nope);
+  p.q_pe = static_cast<const __nv_bfloat16*>(q_pe);
   p.cache = static_cast<const __nv_bfloat16*>(cache);
   p.qmul = qmul;
   p.seq_row_start = seq_row_start;
@@ -306,9 +342,10 @@ dsa_status_t launch_attend(const void* q_nope, const void* q_pe, const float* qm
   p.k = k;
   p.n_split = sp.n_split;
   p.rows_per_split = sp.rows_per_split;
+  p.merge = sp.merge ? 1 : 0;
   p.ws_o = nullptr;
   p.ws_ml = nullptr;
-  if (sp.n_split > 1) {
+  if (sp.n_split > 1 && !sp.merge) {
     const size_t units = (size_t)T * sp.n_split;
     p.ws_o = static_cast<float*>(ws);
     p.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
@@ -316,10 +353,26 @@ dsa_status_t launch_attend(const void* q_nope, const void* q_pe, const float* qm
   }
   st = set_smem<dsa::attend_kernel<DR>>(C::SMEM_BYTES);
   if (st != DSA_OK) return st;
-  dsa::attend_kernel<DR><<<T * sp.n_split, C::THREADS, C::SMEM_BYTES, stream>>>(qn_map, qp_map, p);
+  if (sp.merge) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(T * sp.n_split));
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)sp.n_split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    DSA_CUDA(cudaLaunchKernelEx(&cfg, dsa::attend_kernel<DR>, qn_map, qp_map, p));
+  } else {
+    dsa::attend_kernel<DR><<<T * sp.n_split, C::THREADS, C::SMEM_BYTES, stream>>>(qn_map, qp_map, p);
+  }
   DSA_CUDA(cudaGetLastError());
   g_launches.fetch_add(1, std::memory_order_relaxed);
-  if (sp.n_split > 1) {
+  if (sp.n_split > 1 && !sp.merge) {
     dsa::attend_combine_kernel<<<T * dsa::kHeads, 128, 0, stream>>>(p);
     DSA_CUDA(cudaGetLastError());
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -396,11 +449,11 @@ dsa_status_t check_attend_args(const void* q_nope, const void* q_pe, const float
 
 // =================================================================== no-allocation variant
 // Scratch for sparse_mla_attend_noalloc: the split partials (numerators, then
-// max/sum pairs) of at most kNoAllocMaxPartials (query, split) work units, in
+// four statistics per head) of at most kNoAllocMaxPartials (query, split) work units, in
 // the layout launch_attend expects of a workspace.  Every GPU that loads this
 // library holds the array until the process exits.
 constexpr int kNoAllocMaxPartials = DSA_NOALLOC_MAX_PARTIALS;
-static __device__ __align__(256) float g_noalloc_scratch[(size_t)kNoAllocMaxPartials * 64 * (512 + 2)];
+static __device__ __align__(256) float g_noalloc_scratch[(size_t)kNoAllocMaxPartials * 64 * (512 + 4)];
 
 namespace {
 
@@ -497,7 +550,7 @@ dsa_status_t sparse_mla_attend_noalloc(const void* q_nope, const void* q_pe, con
   if (T == 0) return DSA_OK;
   const SplitPlan sp = attend_plan(T, k);
   void* scratch = nullptr;
-  if (sp.n_split > 1) {
+  if (sp.n_split > 1 && !sp.merge) {
     const int64_t partials = (int64_t)T * sp.n_split;
     if (partials > kNoAllocMaxPartials)
       return fail(DSA_ERR_WORKSPACE,

@@ -108,6 +108,8 @@ def test_forward_rejects_missing_workspace(lib):
 def test_workspace_sizes_are_host_only(lib):
     assert lib.dsa_topk_workspace_size(64, 32768, 2048) == 0
     assert lib.sparse_mla_workspace_size(0, 2048) == 0
-    # 64 queries are split across SMs: partial numerators are needed
-    assert lib.sparse_mla_workspace_size(64, 2048) > 64 * 64 * 512 * 4
+    # 4 queries are split 16+ ways (more than one cluster merges): partial
+    # numerators go through the workspace.  2-8 way splits merge inside a
+    # cluster when the GPU allows it, so their size depends on the device.
+    assert lib.sparse_mla_workspace_size(4, 2048) >= 4 * 16 * 64 * 512 * 4
     assert lib.dsa_forward_workspace_size(64, 32768, 2048, 1) >= 64 * 32768 * 4

@@ -163,6 +163,26 @@ def test_attention_matches_oracle_single_split_path(d_rope):
     pu.assert_attention_close(to_numpy(o)[ts], to_numpy(lse)[ts], ref_o, ref_l)
 
 
+@pytest.mark.parametrize("T", [64, 40, 36, 27, 24, 21, 14, 10])
+def test_attention_matches_oracle_cluster_merge_path(T):
+    # With 2-8 CTAs per query (2 to 8 for these batch sizes on 148 SMs)
+    # the CTAs of a query merge their partials in distributed shared memory and
+    # no workspace is needed.  Short selections leave trailing CTAs empty.
+    if ops.attend_workspace_bytes(T, 2048) != 0:
+        pytest.skip("this GPU's split plan for this batch size uses the combine kernel")
+    rng = np.random.default_rng(T)
+    lengths = tuple(int(x) for x in rng.integers(2100, 6000, size=T))
+    case = small_case(f"attn_merge{T}", lengths, layers=(64,), seed=40 + T, mla_q_std=1.0)
+    wl = make_workload(case, DEV)
+    counts = [2048 if i % 4 else int(rng.integers(1, 700)) for i in range(T)]
+    idx, cnt = _random_selection(wl, counts, sort=(T % 2 == 0), holes=True, seed=T)
+    lay = wl.layers[0]
+    o, lse = pu.gpu_attend(wl, lay, torch.as_tensor(idx, device=DEV), torch.as_tensor(cnt, device=DEV))
+    ts = sorted(set(range(0, T, 3)) | {T - 1})
+    ref_o, ref_l = pu.oracle_attend(wl, lay, ts, idx, cnt)
+    pu.assert_attention_close(to_numpy(o)[ts], to_numpy(lse)[ts], ref_o, ref_l)
+
+
 def test_attention_empty_selection_gives_zero_and_minus_inf():
     case = small_case("attn_empty", (300, 300), seed=19)
     wl = make_workload(case, DEV)

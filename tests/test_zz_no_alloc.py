@@ -10,8 +10,6 @@ row with different inputs, so stale scratch contents from the first call would
 show up in the second.  This file is collected last on purpose.
 """
 
-import ctypes
-
 import numpy as np
 import pytest
 import torch
@@ -78,13 +76,22 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(d_rope):
 
 
 def test_noalloc_rejects_more_partials_than_its_scratch_holds():
-    lib = ops.load_library()
-    per_partial = 64 * 512 * 4
-    # find a batch size whose split plan needs more partials than the fixed scratch holds
+    # A workspace partial is 64 heads x (512 numerators + 4 statistics) floats.
+    per_partial = 64 * (512 + 4) * 4
+    # a batch size whose split plan needs more partials than the fixed scratch holds
     T = next(T for T in range(1, 4096)
              if ops.attend_workspace_bytes(T, 2048) // per_partial > 128)
-    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the call returns before launching
-    st = lib.sparse_mla_attend_noalloc(fake, fake, fake, 0.07, fake, 1000, 576, 64, fake, 1, fake, fake, fake,
-                                       T, 2048, fake, None, None)
-    assert st == 6   # DSA_ERR_WORKSPACE
-    assert b"128" in lib.dsa_last_error()
+    # Real buffers of the right sizes: the call must refuse before launching,
+    # and nothing could read out of bounds even if it did not.
+    wl = make_workload(small_case("na_rej", (2100,) * T, layers=(64,), seed=33), DEV)
+    lay = wl.layers[0]
+    idx = torch.zeros((T, 2048), dtype=torch.int32, device=DEV)
+    cnt = torch.ones((T,), dtype=torch.int32, device=DEV)
+    out = torch.empty((T, 64, 512), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ops.DSAError) as err:
+        ops.sparse_mla_attend_noalloc(lay.q_nope, lay.q_pe, lay.qmul, lay.cache, lay.d_rope, wl.seq_row_start,
+                                      wl.q_seq, idx, cnt, out)
+    assert err.value.status == 6   # DSA_ERR_WORKSPACE
+    assert "128" in str(err.value)
+    torch.cuda.synchronize()
+    assert ops.check_errors() == 0
