@@ -181,44 +181,60 @@ dsa_status_t launch_topk_cl(const dsa::TopkParams& p, cudaStream_t stream) {
   return DSA_OK;
 }
 
-// CTAs per query: enough that each CTA owns at least ~16K candidates' worth of
-// work, within one wave of the GPU; more (up to 16) when a query's slice would
-// not fit the shared-memory key stash and the batch is small.
-int topk_cluster_size(int32_t T, int64_t ld) {
-  const int sms = sm_count();
-  int cl = 1;
-  while (cl < 8 && (ld + cl - 1) / cl > 16384 && (int64_t)T * cl * 2 <= sms) cl *= 2;
-  while (cl < 16 && (ld + cl - 1) / cl > dsa::kTopkStashCap && (int64_t)T * cl * 2 <= sms) cl *= 2;
-  return cl;
+// How many top-k clusters of CL CTAs can be resident at once (16 needs the
+// non-portable attribute and a GPC with 16 free SMs); 0 if none.
+template <int CL>
+int topk_max_clusters_t() {
+  static std::atomic<int> count{-1};
+  const int known = count.load(std::memory_order_relaxed);
+  if (known >= 0) return known;
+  int n = 0;
+  bool ok = cudaFuncSetAttribute(dsa::topk_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::kTopkSmemBytes) == cudaSuccess;
+  if (ok && CL > 8)
+    ok = cudaFuncSetAttribute(dsa::topk_kernel<CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+         cudaSuccess;
+  if (ok) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(CL);
+    cfg.blockDim = dim3(dsa::kTopkThreads);
+    cfg.dynamicSmemBytes = dsa::kTopkSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, dsa::topk_kernel<CL>, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  count.store(n, std::memory_order_relaxed);
+  return n;
 }
 
-// Largest cluster size that can be co-scheduled for the top-k kernel (16 needs
-// the non-portable attribute and a GPC with 16 free SMs).
-template <int CL>
-bool topk_cluster_fits() {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(CL);
-  cfg.blockDim = dim3(dsa::kTopkThreads);
-  cfg.dynamicSmemBytes = dsa::kTopkSmemBytes;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaFuncSetAttribute(dsa::topk_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           dsa::kTopkSmemBytes) != cudaSuccess)
-    return false;
-  if (CL > 8 &&
-      cudaFuncSetAttribute(dsa::topk_kernel<CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-    return false;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, dsa::topk_kernel<CL>, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    return false;
+int topk_max_clusters(int CL) {
+  switch (CL) {
+    case 1: return sm_count();
+    case 2: return topk_max_clusters_t<2>();
+    case 4: return topk_max_clusters_t<4>();
+    case 8: return topk_max_clusters_t<8>();
+    case 16: return topk_max_clusters_t<16>();
+    default: return 0;
   }
-  return n > 0;
+}
+
+// CTAs per query: enough that each CTA owns at least ~16K candidates' worth of
+// work while the batch takes at most half the SMs (the rest stay free for the
+// next kernel) and every cluster is resident at once; more (up to 16) when a
+// query's slice would not fit the shared-memory key stash and the batch is small.
+int topk_cluster_size(int32_t T, int64_t ld) {
+  const int sms = sm_count();
+  auto fits = [&](int c) { return (int64_t)T * c * 2 <= sms && T <= topk_max_clusters(c); };
+  int cl = 1;
+  while (cl < 8 && (ld + cl - 1) / cl > 16384 && fits(cl * 2)) cl *= 2;
+  while (cl < 16 && (ld + cl - 1) / cl > dsa::kTopkStashCap && fits(cl * 2)) cl *= 2;
+  return cl;
 }
 
 dsa_status_t topk_impl(const float* scores, int64_t ld, const int32_t* q_pos, int32_t T, int32_t k,
@@ -236,11 +252,7 @@ dsa_status_t topk_impl(const float* scores, int64_t ld, const int32_t* q_pos, in
     case 2: return launch_topk_cl<2>(p, stream);
     case 4: return launch_topk_cl<4>(p, stream);
     case 8: return launch_topk_cl<8>(p, stream);
-    default: {
-      static int fits16 = -1;   // probed once per process
-      if (fits16 < 0) fits16 = topk_cluster_fits<16>() ? 1 : 0;
-      return fits16 ? launch_topk_cl<16>(p, stream) : launch_topk_cl<8>(p, stream);
-    }
+    default: return launch_topk_cl<16>(p, stream);   // chosen only when its clusters fit
   }
 }
 

@@ -11,9 +11,11 @@
 // (output slot of a kept element = #(> tau before it) + min(#(== tau before it),
 // need_eq)), so the result is unique and deterministic.
 //
-// One query is processed by a cluster of CL CTAs (CL in {1, 2, 4, 8}); each CTA
-// owns a contiguous slice of the candidates, stages its keys in shared memory
-// when they fit, and the per-CTA histograms and counts are combined through
+// One query is processed by a cluster of CL CTAs (CL in {1, 2, 4, 8, 16}); each
+// CTA owns a contiguous slice of the candidates and stages its keys in shared
+// memory: whole keys up to 32K per CTA, the top 16 bits of each key up to 64K
+// (enough for the first pass's 11-bit bins; the few candidates then read their
+// full key from the scores).  The per-CTA histograms and counts are combined through
 // distributed shared memory with cluster barriers (hardware barriers: every
 // CTA of a cluster is co-resident, so no software spin is involved).
 #pragma once
@@ -175,7 +177,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   const int64_t lo = ((int64_t)rank * n / CL) & ~int64_t(3);
   const int64_t hi = (rank == CL - 1) ? n : (((int64_t)(rank + 1) * n / CL) & ~int64_t(3));
   const int64_t len = hi - lo;
-  const bool staged = len <= kTopkStashCap;
+  const bool staged = len <= kTopkStashCap;                          // 32-bit keys
+  const bool staged16 = !staged && len <= 2 * kTopkStashCap;       // top 16 bits of each key
+  uint16_t* stash16 = reinterpret_cast<uint16_t*>(stash);
 
   // ---- pass 1: histogram of the top 11 bits (loads batched 4 x float4 per thread)
   for (int b = threadIdx.x; b < kTopkBins; b += kTopkThreads) hist[b] = 0;
@@ -200,6 +204,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
         atomicAdd(&hist[k2 >> 21], 1u);
         atomicAdd(&hist[k3 >> 21], 1u);
         if (staged) reinterpret_cast<uint4*>(stash)[i] = make_uint4(k0, k1, k2, k3);
+        else if (staged16) reinterpret_cast<uint2*>(stash16)[i] = make_uint2((k0 >> 16) | (k1 & 0xFFFF0000u),
+                                                                             (k2 >> 16) | (k3 & 0xFFFF0000u));
       }
     }
   }
@@ -207,6 +213,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     const uint32_t kk = score_key(row[lo + i]);
     atomicAdd(&hist[kk >> 21], 1u);
     if (staged) stash[i] = kk;
+    else if (staged16) stash16[i] = (uint16_t)(kk >> 16);
   }
   __syncthreads();
   cluster_sum_hist<CL, kTopkBins>(hist, tot);
@@ -226,18 +233,33 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   const int64_t s_lo = (warp * seg < len) ? warp * seg : len;
   const int64_t s_hi = (s_lo + seg < len) ? s_lo + seg : len;
   auto key_at = [&](int64_t i) -> uint32_t { return staged ? stash[i] : score_key(row[lo + i]); };
-  // (a) count, 4 keys per lane per step (vector loads when not staged)
-  uint32_t wcount = 0;
-  for (int64_t i0 = s_lo; i0 < s_hi; i0 += 128) {
-    const int64_t e0 = i0 + 4 * lane;
-    uint32_t kk[4];
-    if (!staged && e0 + 3 < s_hi) {
-      const float4 f = *reinterpret_cast<const float4*>(row + lo + e0);
-      kk[0] = score_key(f.x); kk[1] = score_key(f.y); kk[2] = score_key(f.z); kk[3] = score_key(f.w);
+  // Four consecutive keys per lane per step: one 16-byte load from the stash
+  // (conflict-free) or from the scores, scalar loads only in a segment's tail.
+  // With the 16-bit stash the loaded keys hold only their top 16 bits (the
+  // filter tests bits 31..21); full keys come from the scores when written.
+  auto load4 = [&](int64_t e0, uint32_t (&kk)[4]) {
+    if (e0 + 3 < s_hi) {
+      if (staged) {
+        const uint4 v = reinterpret_cast<const uint4*>(stash)[e0 >> 2];
+        kk[0] = v.x; kk[1] = v.y; kk[2] = v.z; kk[3] = v.w;
+      } else if (staged16) {
+        const uint2 v = reinterpret_cast<const uint2*>(stash16)[e0 >> 2];
+        kk[0] = v.x << 16; kk[1] = v.x & 0xFFFF0000u; kk[2] = v.y << 16; kk[3] = v.y & 0xFFFF0000u;
+      } else {
+        const float4 f = *reinterpret_cast<const float4*>(row + lo + e0);
+        kk[0] = score_key(f.x); kk[1] = score_key(f.y); kk[2] = score_key(f.z); kk[3] = score_key(f.w);
+      }
     } else {
 #pragma unroll
       for (int e = 0; e < 4; ++e) kk[e] = (e0 + e < s_hi) ? key_at(e0 + e) : 0u;
     }
+  };
+  // (a) count
+  uint32_t wcount = 0;
+  for (int64_t i0 = s_lo; i0 < s_hi; i0 += 128) {
+    const int64_t e0 = i0 + 4 * lane;
+    uint32_t kk[4];
+    load4(e0, kk);
 #pragma unroll
     for (int e = 0; e < 4; ++e) wcount += (e0 + e < s_hi) && ((kk[e] >> 21) >= b1);
   }
@@ -261,32 +283,28 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   // (b) write in position order into the local candidate arrays
   if (nc <= (uint32_t)kTopkCandCap) {
     uint32_t wpos = tmp[warp];
+    const uint32_t lanes_below = (1u << lane) - 1u;
     for (int64_t i0 = s_lo; i0 < s_hi; i0 += 128) {
       const int64_t e0 = i0 + 4 * lane;
       uint32_t kk[4];
-      if (!staged && e0 + 3 < s_hi) {
-        const float4 f = *reinterpret_cast<const float4*>(row + lo + e0);
-        kk[0] = score_key(f.x); kk[1] = score_key(f.y); kk[2] = score_key(f.z); kk[3] = score_key(f.w);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) kk[e] = (e0 + e < s_hi) ? key_at(e0 + e) : 0u;
-      }
+      load4(e0, kk);
       uint32_t flags = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) flags |= ((e0 + e < s_hi) && ((kk[e] >> 21) >= b1)) ? (1u << e) : 0u;
-      const uint32_t mine = __popc(flags);
-      uint32_t before = mine;
+      // Candidates of lower lanes come first (position order): one ballot per
+      // element slot gives both this lane's offset and the warp's total.
+      uint32_t before = 0, total = 0;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, before, o);
-        if (lane >= o) before += y;
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t bal = __ballot_sync(0xffffffffu, (flags >> e) & 1u);
+        before += __popc(bal & lanes_below);
+        total += __popc(bal);
       }
-      const uint32_t total = __shfl_sync(0xffffffffu, before, 31);
-      uint32_t at = wpos + before - mine;
+      uint32_t at = wpos + before;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         if (flags & (1u << e)) {
-          cand_key[at] = kk[e];
+          cand_key[at] = staged16 ? score_key(row[lo + e0 + e]) : kk[e];
           cand_pos[at] = (int32_t)(lo + e0 + e);
           ++at;
         }

@@ -87,12 +87,26 @@ def test_topk_bit_exact_on_gpu_scores(k):
                          to_numpy(wl.q_pos), k)
 
 
-@pytest.mark.parametrize("T,ld", [(1, 100_000), (1, 500_000), (200, 40_000), (100, 5_000), (3, 131_072)])
+@pytest.mark.parametrize("T,ld", [(1, 100_000), (1, 500_000), (200, 40_000), (100, 5_000), (3, 131_072),
+                                  (2, 1_000_000)])
 def test_topk_cluster_sizes_and_ties(T, ld):
     # Integer-valued scores: heavy ties everywhere, including at the threshold.
     g = torch.Generator(device=DEV).manual_seed(T * 7 + ld)
     scores = torch.randint(-40, 41, (T, ld), generator=g, device=DEV).float()
     scores[:, ::5] = -0.0
+    q_pos = torch.randint(ld // 2, ld, (T,), generator=g, device=DEV, dtype=torch.int32)
+    q_pos[0] = ld - 1
+    idx, cnt = pu.gpu_topk(scores, q_pos, 2048)
+    pu.assert_topk_exact(to_numpy(idx), to_numpy(cnt), to_numpy(scores).astype(np.float64),
+                         to_numpy(q_pos), 2048)
+
+
+@pytest.mark.parametrize("T,ld", [(200, 40_000), (2, 1_000_000), (64, 32_768)])
+def test_topk_continuous_scores_all_stash_modes(T, ld):
+    # Slices of up to 32K keys per CTA stage whole keys, 32K-64K stage their top
+    # 16 bits; continuous scores keep the candidate set small (no overflow path).
+    g = torch.Generator(device=DEV).manual_seed(T + ld)
+    scores = torch.randn((T, ld), generator=g, device=DEV)
     q_pos = torch.randint(ld // 2, ld, (T,), generator=g, device=DEV, dtype=torch.int32)
     q_pos[0] = ld - 1
     idx, cnt = pu.gpu_topk(scores, q_pos, 2048)
