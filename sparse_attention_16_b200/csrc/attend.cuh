@@ -286,6 +286,7 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
     sc->abort_flag = 0;
     fence_mbar_init();
   }
+  griddep_wait();
   if (warp == 4) {
     tmem_alloc(&sc->tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
@@ -693,6 +694,7 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
 // (query, head); each of the 128 threads owns 4 latent columns.
 constexpr int kMaxSplits = 32;
 __global__ void __launch_bounds__(128) attend_combine_kernel(const AttendParams p) {
+  griddep_wait();
   const int t = blockIdx.x / kHeads;
   const int h = blockIdx.x % kHeads;
   const int ns = p.n_split;

@@ -10,9 +10,11 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "dsa.h"
 #include "attend.cuh"
@@ -105,6 +107,49 @@ dsa_status_t set_smem(int bytes) {
   return DSA_OK;
 }
 
+// Launches a kernel, as clusters of cl CTAs for cl > 1.  With DSA_PDL=1 in the
+// environment the launch also allows programmatic stream serialization: every
+// kernel waits in griddepcontrol.wait before touching global memory, so it may
+// be scheduled while the previous kernel of the stream drains.  Off by
+// default: on the decode and prefill steps measured it gained nothing (the
+// kernels' set-up is short and each fills the GPU).
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("DSA_PDL");
+    return v != nullptr && v[0] == '1';
+  }();
+  return on;
+}
+
+template <typename... KArgs, typename... Args>
+dsa_status_t launch(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                    unsigned cl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cl > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cl;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  DSA_CUDA(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return DSA_OK;
+}
+
 // ----------------------------------------------------------------- indexer
 template <int QG>
 dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx, int64_t n_rows,
@@ -134,10 +179,7 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   const int grid = (int)std::min<int64_t>(p.n_units, sm_count());
   st = set_smem<dsa::indexer_kernel<QG>>(C::SMEM_BYTES);
   if (st != DSA_OK) return st;
-  dsa::indexer_kernel<QG><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(kmap, qmap, p);
-  DSA_CUDA(cudaGetLastError());
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return DSA_OK;
+  return launch(dsa::indexer_kernel<QG>, (unsigned)grid, C::THREADS, C::SMEM_BYTES, stream, 1, kmap, qmap, p);
 }
 
 dsa_status_t indexer_impl(const void* q_idx, const float* w, const void* k_idx, int64_t n_rows,
@@ -164,21 +206,8 @@ dsa_status_t launch_topk_cl(const dsa::TopkParams& p, cudaStream_t stream) {
     });
     if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "cluster attribute: %s", cudaGetErrorString(e));
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(p.T * CL));
-  cfg.blockDim = dim3(dsa::kTopkThreads);
-  cfg.dynamicSmemBytes = dsa::kTopkSmemBytes;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  DSA_CUDA(cudaLaunchKernelEx(&cfg, dsa::topk_kernel<CL>, p));
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return DSA_OK;
+  return launch(dsa::topk_kernel<CL>, (unsigned)(p.T * CL), dsa::kTopkThreads, dsa::kTopkSmemBytes, stream,
+                (unsigned)CL, p);
 }
 
 // How many top-k clusters of CL CTAs can be resident at once (16 needs the
@@ -365,31 +394,10 @@ dsa_status_t launch_attend(const void* q_nope, const void* q_pe, const float* qm
   }
   st = set_smem<dsa::attend_kernel<DR>>(C::SMEM_BYTES);
   if (st != DSA_OK) return st;
-  if (sp.merge) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(T * sp.n_split));
-    cfg.blockDim = dim3(C::THREADS);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)sp.n_split;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    DSA_CUDA(cudaLaunchKernelEx(&cfg, dsa::attend_kernel<DR>, qn_map, qp_map, p));
-  } else {
-    dsa::attend_kernel<DR><<<T * sp.n_split, C::THREADS, C::SMEM_BYTES, stream>>>(qn_map, qp_map, p);
-  }
-  DSA_CUDA(cudaGetLastError());
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  if (sp.n_split > 1 && !sp.merge) {
-    dsa::attend_combine_kernel<<<T * dsa::kHeads, 128, 0, stream>>>(p);
-    DSA_CUDA(cudaGetLastError());
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-  }
-  return DSA_OK;
+  st = launch(dsa::attend_kernel<DR>, (unsigned)(T * sp.n_split), C::THREADS, C::SMEM_BYTES, stream,
+              sp.merge ? (unsigned)sp.n_split : 1u, qn_map, qp_map, p);
+  if (st != DSA_OK || sp.n_split == 1 || sp.merge) return st;
+  return launch(dsa::attend_combine_kernel, (unsigned)(T * dsa::kHeads), 128, 0, stream, 1, p);
 }
 
 dsa_status_t attend_impl(const void* q_nope, const void* q_pe, const float* qmul, float scale,

@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  griddep_wait();
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();

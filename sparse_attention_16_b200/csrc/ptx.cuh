@@ -121,6 +121,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return true;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// With DSA_PDL=1 the library launches its kernels with programmatic stream
+// serialization, so a kernel may be scheduled while the previous kernel of its
+// stream drains.  Before griddep_wait() a kernel touches only its own shared
+// memory (barrier set-up); the wait returns once the previous kernel has
+// completed and its writes are visible, whatever that kernel was.  Without
+// the launch attribute the wait returns at once.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ proxies / fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   uint32_t* cnt = res + 8;                   // this CTA's (#gt, #eq), read by peers
   uint32_t* stash = reinterpret_cast<uint32_t*>(smem_raw + 2 * kTopkBins * 4 + 1024);
 
+  griddep_wait();
   const int t = blockIdx.x / CL;
   int rank = 0;
   if constexpr (CL > 1) rank = (int)cg::this_cluster().block_rank();
