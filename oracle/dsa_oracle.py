@@ -20,7 +20,7 @@ Sources (the web pages about Mistral Large 4 this library follows):
         avisoori1x.github.io/mistral_large_4, DSA paragraph: the indexer picks
         the top 2,048 keys per query, chosen per query.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   * the query's own position is a candidate: candidates are 0..q_pos[t];
   * ties go to the lower position; -0.0 equals +0.0; NaN scores rank as -inf;
   * the selection is returned sorted by ascending position, padded with -1;
