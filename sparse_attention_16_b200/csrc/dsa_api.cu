@@ -254,12 +254,12 @@ int topk_max_clusters(int CL) {
 }
 
 // CTAs per query: enough that each CTA owns at least ~16K candidates' worth of
-// work while the batch takes at most half the SMs (the rest stay free for the
-// next kernel) and every cluster is resident at once; more (up to 16) when a
-// query's slice would not fit the shared-memory key stash and the batch is small.
+// work while the batch stays within one wave (T x CL <= SMs, every cluster
+// resident at once); more (up to 16) when a query's slice would not fit the
+// shared-memory key stash.
 int topk_cluster_size(int32_t T, int64_t ld) {
   const int sms = sm_count();
-  auto fits = [&](int c) { return (int64_t)T * c * 2 <= sms && T <= topk_max_clusters(c); };
+  auto fits = [&](int c) { return (int64_t)T * c <= sms && T <= topk_max_clusters(c); };
   int cl = 1;
   while (cl < 8 && (ld + cl - 1) / cl > 16384 && fits(cl * 2)) cl *= 2;
   while (cl < 16 && (ld + cl - 1) / cl > dsa::kTopkStashCap && fits(cl * 2)) cl *= 2;
