@@ -23,10 +23,17 @@ Parity status per function (what pins it, see tests/test_oracle_pins.py):
   dense_causal_mla  pinned through the same equalities (independent code path).
   explicit_mla      pinned through the same equality (independent code path).
   forward           composition of the above; no separate pin needed.
+  e4m3_decode       pinned: every one of the 256 codes against torch's float8_e4m3fn
+                    conversion, and the format's landmark values (1, 448, 2^-6, 2^-9).
+  index_scores_fp8  pinned: hand-worked example with integer codes, positive
+                    homogeneity in each key scale and in each query's scales, zero
+                    scale gives zero scores, causal/offset checks.
 """
 
 from .dsa_oracle import (  # noqa: F401
     index_scores,
+    e4m3_decode,
+    index_scores_fp8,
     topk_select,
     sparse_mla,
     dense_causal_mla,

@@ -75,6 +75,48 @@ def index_scores(q_idx, w, k_idx, seq_row_start, q_seq, q_pos, ld):
     return out
 
 
+def e4m3_decode(codes):
+    """Value of FP8 E4M3 codes (the OCP 8-bit floating-point format, E4M3 variant),
+    written out from the format's definition:
+      bit 7 sign; bits 6..3 exponent e (bias 7); bits 2..0 mantissa m;
+      e == 0: subnormal, value (m / 8) * 2^-6;  e > 0: (1 + m / 8) * 2^(e - 7);
+      S.1111.111 is NaN; there are no infinities (largest finite: 448).
+    Returns float64 of the same shape."""
+    c = np.asarray(codes).astype(np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64)))
+    return np.where((c & 0x7F) == 0x7F, np.nan, sign * mag)
+
+
+def index_scores_fp8(q8, q_scale, w, k8, k_scale, seq_row_start, q_seq, q_pos, ld):
+    """Lightning-indexer scores on FP8 (E4M3) keys and queries with per-row scales.
+
+    The concept page stores the indexer keys in FP8 in production ("1M-token
+    serving scenario": 128 B per position per indexer layer) and does not give
+    a scale convention.  The reading taken: key row s is
+        k[s, :] = k_scale[s] * e4m3(k8[row(s), :])
+    and query head j of query t is
+        q[t, j, :] = q_scale[t, j] * e4m3(q8[t, j, :]),
+    with positive fp32 scales; the scores are then the indexer's definition
+        I[t, s] = sum_j w[t, j] * max(0, q[t, j, :] . k[s, :])
+    on those values (columns q_pos[t] < s < ld hold -inf).  Returns float64 [T, ld].
+    """
+    wt = _f64(w)
+    T = wt.shape[0]
+    out = np.full((T, int(ld)), -np.inf, dtype=np.float64)
+    for t in range(T):
+        n = int(q_pos[t]) + 1
+        if n <= 0:
+            continue
+        base = int(seq_row_start[int(q_seq[t])])
+        q = e4m3_decode(q8[t]) * _f64(q_scale[t])[:, None]                              # [H_I, d_I]
+        k_rows = e4m3_decode(k8[base:base + n]) * _f64(k_scale[base:base + n])[:, None]  # [n, d_I]
+        out[t, :n] = np.maximum(k_rows @ q.T, 0.0) @ wt[t]
+    return out
+
+
 def topk_select(scores, q_pos, k):
     """Per-query top-k selection, [CP] "Sparse attention" and [TR] DSA paragraph.
 

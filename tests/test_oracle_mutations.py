@@ -34,6 +34,16 @@ MUTATIONS = {
                                  "z = z + qp @ rows[:, :qp.shape[1]].T"),
     "attn_lse_without_max": ("lse = zmax[:, 0] + np.log(", "lse = np.log("),
     "attn_values_shifted_window": ("return p @ rows[:, :d_c], lse", "return p @ rows[:, -d_c:], lse"),
+    "e4m3_exponent_bias_8": ("np.exp2((e - 7).astype(np.float64))", "np.exp2((e - 8).astype(np.float64))"),
+    "e4m3_no_subnormals": ("np.where(e == 0, (m / 8.0) * 2.0 ** -6,", "np.where(e == 0, 0.0 * m,"),
+    "fp8_indexer_ignores_key_scale": (
+        "k_rows = e4m3_decode(k8[base:base + n]) * _f64(k_scale[base:base + n])[:, None]",
+        "k_rows = e4m3_decode(k8[base:base + n])"),
+    "fp8_indexer_key_scale_of_wrong_row": (
+        "k_rows = e4m3_decode(k8[base:base + n]) * _f64(k_scale[base:base + n])[:, None]",
+        "k_rows = e4m3_decode(k8[base:base + n]) * _f64(k_scale[:n])[:, None]"),
+    "fp8_indexer_relu_after_weighting": ("out[t, :n] = np.maximum(k_rows @ q.T, 0.0) @ wt[t]",
+                                         "out[t, :n] = np.maximum(k_rows @ q.T @ wt[t], 0.0)"),
 }
 
 
@@ -47,7 +57,7 @@ def _mutant(name):
 
 def _run_pins(mod, golden_dir, monkeypatch):
     for fn in ("index_scores", "topk_select", "sparse_mla", "dense_causal_mla", "explicit_mla",
-               "forward"):
+               "forward", "e4m3_decode", "index_scores_fp8"):
         monkeypatch.setattr(pins, fn, getattr(mod, fn))
     failures = 0
     for tname, test in inspect.getmembers(pins, inspect.isfunction):

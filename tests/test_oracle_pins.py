@@ -14,8 +14,8 @@ import os
 import numpy as np
 import pytest
 
-from oracle import (dense_causal_mla, explicit_mla, forward, index_scores,
-                    sparse_mla, topk_select)
+from oracle import (dense_causal_mla, e4m3_decode, explicit_mla, forward, index_scores,
+                    index_scores_fp8, sparse_mla, topk_select)
 
 RNG = np.random.default_rng(1234)
 
@@ -119,6 +119,68 @@ def test_indexer_causal_range_and_sequence_offsets():
     s3 = index_scores(q, w, k, starts, q_seq, q_pos3, ld)
     np.testing.assert_allclose(s3[1, :31], s[1, :31], rtol=1e-12, atol=1e-12)
     assert np.isneginf(s3[1, 31:]).all()
+
+
+# --------------------------------------------------------------------------- FP8 (E4M3) index keys
+
+def test_e4m3_decode_matches_library_conversion_for_every_code():
+    # torch's float8_e4m3fn is the same OCP E4M3 format; all 256 codes agree (NaN where it has NaN).
+    torch = pytest.importorskip("torch")
+    c = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(c.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = e4m3_decode(c)
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    assert np.array_equal(mine[~np.isnan(mine)], ref[~np.isnan(ref)])
+
+
+def test_e4m3_decode_landmark_values():
+    # The format's definition: 1.0 = 0.0111.000, largest finite 448 = 0.1111.110, smallest normal
+    # 2^-6 = 0.0001.000, smallest subnormal 2^-9 = 0.0000.001, sign bit, NaN = S.1111.111.
+    v = e4m3_decode(np.array([0x38, 0x7E, 0x08, 0x01, 0xB8, 0x00, 0x40, 0x44, 0x7F, 0xFF], np.uint8))
+    assert v[:8].tolist() == [1.0, 448.0, 2.0 ** -6, 2.0 ** -9, -1.0, 0.0, 2.0, 3.0]
+    assert np.isnan(v[8]) and np.isnan(v[9])
+
+
+def test_indexer_fp8_hand_worked_example():
+    # Two heads x 2 dims, integer codes: q0 = (1, 2), q1 = (-1, 1); keys (1, 1) and (2, 0); w = (1, 0.5).
+    #   s=0: head0 1+2 = 3, head1 -1+1 = 0  -> I = 1*3 + 0.5*0 = 3, times k_scale 2 -> 6
+    #   s=1: head0 2+0 = 2, head1 -2+0 = -2 -> I = 1*2 + 0.5*ReLU(-2) = 2 (not ReLU(2 - 1) = 1)
+    one, two, mone, zero = 0x38, 0x40, 0xB8, 0x00
+    q8 = np.array([[[one, two], [mone, one]]], np.uint8)
+    k8 = np.array([[one, one], [two, zero]], np.uint8)
+    I = index_scores_fp8(q8, np.ones((1, 2)), np.array([[1.0, 0.5]]), k8, np.array([2.0, 1.0]),
+                         np.array([0]), np.array([0]), np.array([1]), 4)
+    assert I[0, :2].tolist() == [6.0, 2.0]
+    assert np.all(np.isneginf(I[0, 2:]))
+
+
+def test_indexer_fp8_scale_homogeneity_and_offsets():
+    # Each key scale multiplies its own column; each query's scales multiply its row (ReLU of a
+    # positively scaled argument); a zero scale zeroes the scores; sequences read their own rows.
+    rng = np.random.default_rng(8)
+    T, H, d, rows = 3, 4, 16, 90
+    q8 = rng.integers(0, 256, (T, H, d)).astype(np.uint8)
+    k8 = rng.integers(0, 256, (rows, d)).astype(np.uint8)
+    q8[(q8 & 0x7F) == 0x7F] = 0x38     # no NaN codes
+    k8[(k8 & 0x7F) == 0x7F] = 0x38
+    qs = rng.uniform(0.01, 0.1, (T, H))
+    ks = rng.uniform(0.01, 0.1, rows)
+    w = rng.normal(size=(T, H))
+    starts, q_seq, q_pos = np.array([0, 40]), np.array([0, 1, 1]), np.array([39, 49, 20])
+    base = index_scores_fp8(q8, qs, w, k8, ks, starts, q_seq, q_pos, 64)
+    ks2 = ks.copy()
+    ks2[40 + 7] *= 4.0                   # row 7 of sequence 1
+    b2 = index_scores_fp8(q8, qs, w, k8, ks2, starts, q_seq, q_pos, 64)
+    np.testing.assert_allclose(b2[1:, 7], 4.0 * base[1:, 7], rtol=1e-12)
+    np.testing.assert_array_equal(np.delete(b2[1:], 7, axis=1), np.delete(base[1:], 7, axis=1))
+    np.testing.assert_array_equal(b2[0], base[0])   # sequence 0 never reads row 47's scale at s = 7
+    qs3 = qs.copy()
+    qs3[2] *= 3.0
+    b3 = index_scores_fp8(q8, qs3, w, k8, ks, starts, q_seq, q_pos, 64)
+    np.testing.assert_allclose(b3[2, :21], 3.0 * base[2, :21], rtol=1e-12)
+    b0 = index_scores_fp8(q8, np.zeros_like(qs), w, k8, ks, starts, q_seq, q_pos, 64)
+    assert np.all(b0[0, :40] == 0.0) and np.all(np.isneginf(b0[0, 40:]))
+    assert np.all(np.isneginf(base[2, 21:]))
 
 
 # --------------------------------------------------------------------------- top-k
@@ -281,7 +343,9 @@ def test_single_row_and_uniform_closed_forms():
     sel = np.array([3, 9, 10, 44, 59])
     idx[0, :5] = sel
     o, lse = sparse_mla(qn, qp, np.zeros_like(m), scale, cache, 64, starts, q_seq, idx, np.array([5]))
-    np.testing.assert_allclose(o[0], np.broadcast_to(cache[sel, :512].astype(np.float64).mean(0), (64, 512)), rtol=1e-12)
+    # (atol: a column whose mean is ~0 differs by float64 rounding of the two summation orders, ~1e-17)
+    np.testing.assert_allclose(o[0], np.broadcast_to(cache[sel, :512].astype(np.float64).mean(0), (64, 512)),
+                               rtol=1e-12, atol=1e-15)
     np.testing.assert_allclose(lse[0], math.log(5), rtol=1e-12)
 
 
