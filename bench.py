@@ -40,7 +40,7 @@ sys.path.insert(0, ROOT)
 
 from sparse_attention_16_b200 import accounting as acc  # noqa: E402
 from sparse_attention_16_b200 import replicas  # noqa: E402
-from sparse_attention_16_b200.workloads import CONFIGS, make_workload, small_case  # noqa: E402
+from sparse_attention_16_b200.workloads import CONFIGS, make_workload, quantize_e4m3_rows, small_case  # noqa: E402
 
 HEADLINE = "decode_b64_32k"
 METRIC = "sparse-MLA+DSA decode queries/s per layer; achieved HBM TB/s vs peak"
@@ -63,8 +63,8 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-KERNEL_SOURCES = {"indexer": ["indexer.cuh", "ptx.cuh"], "topk": ["topk.cuh", "ptx.cuh"],
-                  "attend": ["attend.cuh", "ptx.cuh"]}
+KERNEL_SOURCES = {"indexer": ["indexer.cuh", "ptx.cuh"], "indexer_fp8": ["indexer.cuh", "ptx.cuh"],
+                  "topk": ["topk.cuh", "ptx.cuh"], "attend": ["attend.cuh", "ptx.cuh"]}
 
 
 def kernel_source_hash(kernel):
@@ -165,6 +165,12 @@ def run_ours(args, rank, world, local):
     lses = [torch.empty((T, 64), dtype=torch.float32, device=dev) for _ in wl.layers]
     att_ws = ops.workspace(ops.attend_workspace_bytes(T, k), dev)
     stream = torch.cuda.current_stream()
+    if args.fp8_keys:
+        # E4M3 codes + per-row scales of the same seeded keys/queries (input preparation, untimed)
+        q8, q8_scale = quantize_e4m3_rows(wl.q_idx)
+        k8, k8_scale = quantize_e4m3_rows(wl.k_idx)
+        wl.k_idx = None          # the bf16 keys are not read in this mode
+        torch.cuda.empty_cache()
 
     # events around the indexer launch of every timed step (same stream)
     ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(args.steps)]
@@ -173,8 +179,12 @@ def run_ours(args, rank, world, local):
         e = ev[i] if i is not None else None
         if e:
             e[0].record(stream)
-        ops.index_scores(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, scores,
-                         q_group=q_group)
+        if args.fp8_keys:
+            ops.index_scores_fp8(q8, q8_scale, wl.w, k8, k8_scale, wl.seq_row_start, wl.q_seq, wl.q_pos, scores,
+                                 q_group=q_group)
+        else:
+            ops.index_scores(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, scores,
+                             q_group=q_group)
         if e:
             e[1].record(stream)
         ops.topk(scores, wl.q_pos, k, idx, cnt)
@@ -257,25 +267,31 @@ def run_ours(args, rank, world, local):
     peaks, peak_src = load_peaks()
     q_pos = wl.q_pos.to("cpu").numpy().astype(np.int64)
     n_scored = int((q_pos + 1).sum())
-    idx_bytes = acc.indexer_bytes(n_scored, T, T * ld)
+    idx_bytes = acc.indexer_bytes(n_scored, T, T * ld, fp8=args.fp8_keys)
+    idx_kernel = "indexer_fp8" if args.fp8_keys else "indexer"
+    idx_name = "indexer_kernel<{},{}>".format(q_group, "fp8" if args.fp8_keys else "bf16")
     idx_dur = statistics.mean(idx_ms) / 1e3
     if q_group == 1:
         achieved_gbs = idx_bytes / idx_dur / 1e9
-        roofline = {"kernel": "indexer_kernel<1>", "bound": "hbm",
+        roofline = {"kernel": idx_name, "bound": "hbm",
                     "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": round(achieved_gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} hbm_gbs",
-                    "traffic": profiled_traffic("indexer", args.config),
+                    "traffic": profiled_traffic(idx_kernel, args.config),
                     "algorithmic_bytes_per_launch": idx_bytes, "avg_launch_ms": round(idx_dur * 1e3, 4)}
     else:
         flops = acc.indexer_flops(n_scored)
         achieved_tf = flops / idx_dur / 1e12
-        peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        roofline = {"kernel": "indexer_kernel<8>", "bound": "tensor",
+        # an FP8 contraction is measured against the bf16 peak x 2 (the nominal fp8 : bf16 ratio, 4.5 : 2.25)
+        ratio = 2.0 if args.fp8_keys else 1.0
+        peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * ratio
+        roofline = {"kernel": idx_name, "bound": "tensor",
                     "achieved": round(achieved_tf, 1), "peak": peak_tf, "unit": "TFLOP/s",
                     "frac": round(achieved_tf / peak_tf, 4),
-                    "frac_of_burst_peak": round(achieved_tf / peaks["bf16_tflops"], 4),
-                    "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a multi-ms step)",
-                    "traffic": profiled_traffic("indexer", args.config),
+                    "frac_of_burst_peak": round(achieved_tf / (peaks["bf16_tflops"] * ratio), 4),
+                    "peak_source": (f"{peak_src} bf16_tflops_sustained" + (" x 2 (nominal fp8:bf16)" if args.fp8_keys
+                                                                          else "")
+                                    + " (kernel timed inside a multi-ms step)"),
+                    "traffic": profiled_traffic(idx_kernel, args.config),
                     "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": idx_bytes,
                     "avg_launch_ms": round(idx_dur * 1e3, 4)}
 
@@ -286,7 +302,8 @@ def run_ours(args, rank, world, local):
         step_bytes += acc.attend_bytes(n_rows_att, T, L.d_rope)
 
     # ---- end to end through the C ABI with host buffers
-    e2e = run_e2e(args, wl, ld, k, q_group, dev) if not args.no_e2e else None
+    # the fused C-ABI call takes bf16 index keys; no end-to-end line in FP8-key mode
+    e2e = run_e2e(args, wl, ld, k, q_group, dev) if not (args.no_e2e or args.fp8_keys) else None
 
     value = replicas.job_throughput(T, world, args.steps, elapsed)
     line = {
@@ -294,7 +311,8 @@ def run_ours(args, rank, world, local):
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(elapsed / args.steps * 1e3, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded, shapes/distributions of the configuration)",
-        "config": {"workload": args.config, "queries_per_gpu": T, "context": list(case.seq_lengths)[:1],
+        "config": {"workload": args.config + ("+fp8_index_keys" if args.fp8_keys else ""),
+                   "queries_per_gpu": T, "context": list(case.seq_lengths)[:1],
                    "layers": [("rope" if L.d_rope else "nope") for L in wl.layers], "topk": k,
                    "parallelism": f"replicas{world}" if world > 1 else "1gpu",
                    "l2": f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB per step)"},
@@ -448,6 +466,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--eager", action="store_true", help="launch every step from the host instead of a CUDA graph")
+    ap.add_argument("--fp8-keys", action="store_true",
+                    help="score with FP8 (E4M3) index keys and queries, per-row scales (dsa_index_scores_fp8); "
+                         "the selection and attention are unchanged")
     args = ap.parse_args()
     rank, world, local = dist_env()
     if args.impl == "reference":

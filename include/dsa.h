@@ -96,6 +96,32 @@ dsa_status_t dsa_index_scores(const void* q_idx, const float* w, const void* k_i
                               int32_t q_group, float* scores, int64_t ld, void* stream);
 
 /*
+ * dsa_index_scores_fp8 - lightning-indexer scores on FP8 (E4M3) keys and queries.
+ * Concept page, "Where to look" and "Sparse attention" (the scorer), and the
+ * 1M-token serving scenario (indexer keys kept in FP8, 128 B per position per
+ * indexer layer).  The page gives no scale convention; this call takes one fp32
+ * scale per key row and per query head:
+ *     k[s]   = k_scale[s]   * e4m3(k8[s, :])
+ *     q[t,j] = q_scale[t,j] * e4m3(q8[t, j, :])
+ * and writes I[t,s] = sum_j w[t,j] * max(0, q[t,j] . k[s]) exactly as
+ * dsa_index_scores does for bf16 inputs.
+ *
+ *   q8      uint8 [T, 32, 128]  E4M3 codes (OCP FP8 E4M3: bias 7, max 448, NaN = S.1111.111)
+ *   q_scale f32   [T, 32]       > 0
+ *   w       f32   [T, 32]
+ *   k8      uint8 [n_rows, 128] E4M3 codes, rows located by seq_row_start
+ *   k_scale f32   [n_rows]      > 0
+ *   the remaining arguments, layouts, q_group and errors as dsa_index_scores;
+ *   additionally DSA_ERR_INVALID_ARG for a null or misaligned q_scale / k_scale.
+ * Scales must be positive (the ReLU is applied to the unscaled dot product
+ * times the scales); codes must not be NaN.
+ */
+dsa_status_t dsa_index_scores_fp8(const void* q8, const float* q_scale, const float* w, const void* k8,
+                                  const float* k_scale, int64_t n_rows, const int64_t* seq_row_start,
+                                  int32_t B, const int32_t* q_seq, const int32_t* q_pos, int32_t T,
+                                  int32_t q_group, float* scores, int64_t ld, void* stream);
+
+/*
  * dsa_topk - per-query top-k of a score array.
  * Concept page, "Sparse attention" (keeps the top 2,048) and the report's DSA
  * paragraph (chosen per query).  Candidates of query t are columns

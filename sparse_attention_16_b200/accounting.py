@@ -123,12 +123,17 @@ class ModelSchedule:
 
 # ---- per-call algorithmic traffic (compulsory bytes, read once / written once) ----
 
-def indexer_bytes(n_scored_total: int, n_queries: int, n_cols_written: int) -> int:
+def indexer_bytes(n_scored_total: int, n_queries: int, n_cols_written: int, fp8: bool = False) -> int:
     """Index keys read once, q and w per query, and the fp32 score row written.
 
     n_scored_total: key rows read (sum over queries of q_pos + 1 for decode).
     n_cols_written: score entries written (T x ld).
+    fp8: E4M3 keys and queries (1 B per value) plus one fp32 scale per key row
+         and per query head.
     """
+    if fp8:
+        q_w = n_queries * (N_IDX_HEADS * D_IDX * 1 + 2 * N_IDX_HEADS * F32)
+        return n_scored_total * (D_IDX * 1 + F32) + q_w + n_cols_written * F32
     q_w = n_queries * (N_IDX_HEADS * D_IDX * BF16 + N_IDX_HEADS * F32)
     return n_scored_total * D_IDX * BF16 + q_w + n_cols_written * F32
 

@@ -79,14 +79,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 2-D bf16 tensor map with the 128-byte swizzle: `inner` contiguous elements
 // per row, `outer` rows `row_bytes` apart, box of box_inner x box_outer.
 dsa_status_t make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                       CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto enc = encode_fn();
   if (enc == nullptr) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+  CUresult r = enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -151,20 +152,28 @@ dsa_status_t launch(void (*kernel)(KArgs...), unsigned grid, unsigned block, siz
 }
 
 // ----------------------------------------------------------------- indexer
-template <int QG>
-dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx, int64_t n_rows,
-                            const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
-                            const int32_t* q_pos, int32_t T, float* scores, int64_t ld,
+// F8: q_idx / k_idx hold E4M3 codes (one byte per value) and q_scale / k_scale
+// their per-head / per-row scales; otherwise bf16 values and null scales.
+template <int QG, bool F8>
+dsa_status_t launch_indexer(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
+                            const float* k_scale, int64_t n_rows, const int64_t* seq_row_start, int32_t B,
+                            const int32_t* q_seq, const int32_t* q_pos, int32_t T, float* scores, int64_t ld,
                             cudaStream_t stream) {
-  using C = dsa::IdxCfg<QG>;
+  using C = dsa::IdxCfg<QG, F8>;
+  // One 128-byte swizzled block per box row: 64 bf16 or 128 fp8 values.  TMA
+  // moves bytes, so an fp8 row (128 B) is described as 64 two-byte elements:
+  // the same bytes and the same swizzle as a bf16 half row.
+  const uint64_t row_elems = F8 ? dsa::kIdxDim / 2 : dsa::kIdxDim;
+  const uint64_t row_bytes = F8 ? dsa::kIdxDim : dsa::kIdxDim * 2;
   CUtensorMap kmap, qmap;
-  dsa_status_t st = make_tmap(&kmap, k_idx, dsa::kIdxDim, (uint64_t)n_rows, dsa::kIdxDim * 2, 64,
-                              dsa::kKeyTile);
+  dsa_status_t st = make_tmap(&kmap, k_idx, row_elems, (uint64_t)n_rows, row_bytes, 64, dsa::kKeyTile);
   if (st != DSA_OK) return st;
-  st = make_tmap(&qmap, q_idx, dsa::kIdxDim, (uint64_t)T * dsa::kIdxHeads, dsa::kIdxDim * 2, 64, C::N);
+  st = make_tmap(&qmap, q_idx, row_elems, (uint64_t)T * dsa::kIdxHeads, row_bytes, 64, C::N);
   if (st != DSA_OK) return st;
   dsa::IndexerParams p;
   p.w = w;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
   p.seq_row_start = seq_row_start;
   p.q_seq = q_seq;
   p.q_pos = q_pos;
@@ -177,9 +186,10 @@ dsa_status_t launch_indexer(const void* q_idx, const float* w, const void* k_idx
   const int64_t n_groups = (T + QG - 1) / QG;
   p.n_units = n_groups * p.n_kt;
   const int grid = (int)std::min<int64_t>(p.n_units, sm_count());
-  st = set_smem<dsa::indexer_kernel<QG>>(C::SMEM_BYTES);
+  st = set_smem<dsa::indexer_kernel<QG, F8>>(C::SMEM_BYTES);
   if (st != DSA_OK) return st;
-  return launch(dsa::indexer_kernel<QG>, (unsigned)grid, C::THREADS, C::SMEM_BYTES, stream, 1, kmap, qmap, p);
+  return launch(dsa::indexer_kernel<QG, F8>, (unsigned)grid, C::THREADS, C::SMEM_BYTES, stream, 1, kmap, qmap,
+                p);
 }
 
 dsa_status_t indexer_impl(const void* q_idx, const float* w, const void* k_idx, int64_t n_rows,
@@ -187,10 +197,10 @@ dsa_status_t indexer_impl(const void* q_idx, const float* w, const void* k_idx, 
                           const int32_t* q_pos, int32_t T, int32_t q_group, float* scores,
                           int64_t ld, cudaStream_t stream) {
   if (q_group == 8)
-    return launch_indexer<8>(q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T, scores, ld,
-                             stream);
-  return launch_indexer<1>(q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T, scores, ld,
-                           stream);
+    return launch_indexer<8, false>(q_idx, nullptr, w, k_idx, nullptr, n_rows, seq_row_start, B, q_seq, q_pos,
+                                    T, scores, ld, stream);
+  return launch_indexer<1, false>(q_idx, nullptr, w, k_idx, nullptr, n_rows, seq_row_start, B, q_seq, q_pos, T,
+                                  scores, ld, stream);
 }
 
 // ----------------------------------------------------------------- top-k
@@ -517,6 +527,24 @@ dsa_status_t dsa_index_scores(const void* q_idx, const float* w, const void* k_i
   if (T == 0) return DSA_OK;
   return indexer_impl(q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, scores, ld,
                       static_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_index_scores_fp8(const void* q8, const float* q_scale, const float* w, const void* k8,
+                                  const float* k_scale, int64_t n_rows, const int64_t* seq_row_start,
+                                  int32_t B, const int32_t* q_seq, const int32_t* q_pos, int32_t T,
+                                  int32_t q_group, float* scores, int64_t ld, void* stream) {
+  dsa_status_t st = check_index_args(q8, w, k8, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, ld);
+  if (st != DSA_OK) return st;
+  DSA_REQUIRE(q_scale && k_scale && aligned(q_scale, 4) && aligned(k_scale, 4),
+              "q_scale and k_scale must be non-null and 4-byte aligned");
+  DSA_REQUIRE(scores && aligned(scores, 16), "scores must be non-null and 16-byte aligned");
+  if (T == 0) return DSA_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (q_group == 8)
+    return launch_indexer<8, true>(q8, q_scale, w, k8, k_scale, n_rows, seq_row_start, B, q_seq, q_pos, T,
+                                   scores, ld, s);
+  return launch_indexer<1, true>(q8, q_scale, w, k8, k_scale, n_rows, seq_row_start, B, q_seq, q_pos, T, scores,
+                                 ld, s);
 }
 
 size_t dsa_topk_workspace_size(int32_t, int64_t, int32_t) { return 0; }

@@ -12,6 +12,15 @@
 // the group.  The epilogue applies ReLU, the head weights and the head sum in
 // registers, so each key row costs one TMEM row read and a 32-term FMA chain.
 //
+// FP8 keys (F8 = true): key rows and query heads are E4M3 codes with one fp32
+// scale per key row and per query head (k = k_scale[s] e4m3(k8[s]),
+// q_j = q_scale[t,j] e4m3(q8[t,j]); the concept page keeps indexer keys in FP8,
+// "1M-token serving scenario", without a scale convention).  Both scales are
+// positive, so ReLU commutes with them: the MMA runs on the raw codes
+// (kind::f8f6f4, K = 32), q_scale is folded into the head weights and k_scale
+// multiplies each key's head sum.  A key row is 128 B, one swizzle row, so a
+// key tile is 16 KB and twice as many tiles are in flight.
+//
 // Warp roles (persistent CTA, one per SM, contiguous range of tiles):
 //   warp 0        TMA producer (key tiles ring, query block buffers)
 //   warp 1        TMEM owner + single-thread MMA issuer
@@ -28,25 +37,38 @@ constexpr int kIdxHeads = 32;
 constexpr int kIdxDim = 128;
 constexpr int kKeyTile = 128;
 
-template <int QG>
+// Instruction descriptor of tcgen05.mma kind::f8f6f4 with E4M3 A and B (format
+// code 0), f32 accumulate, both K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                          // D format: f32
+         | ((uint32_t)(N >> 3) << 17)       // N / 8
+         | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+template <int QG, bool F8 = false>
 struct IdxCfg {
   static constexpr int N = 32 * QG;                     // MMA N: heads x queries
-  static constexpr int STAGES = (QG == 1) ? 6 : 4;      // key tiles in flight
+  static constexpr int KBLK = F8 ? 1 : 2;               // 128-byte column blocks per row
+  static constexpr int STAGES = F8 ? ((QG == 1) ? 12 : 8) : ((QG == 1) ? 6 : 4);   // key tiles in flight
   static constexpr int QBUFS = (QG == 1) ? 2 : 1;       // query blocks in flight
-  static constexpr int KHALF = kKeyTile * 128;          // bytes of one 64-column half
-  static constexpr int KT_BYTES = 2 * KHALF;            // 32 KB per key tile
+  static constexpr int KHALF = kKeyTile * 128;          // bytes of one 128-byte column block
+  static constexpr int KT_BYTES = KBLK * KHALF;         // 32 KB (bf16) / 16 KB (fp8) per key tile
   static constexpr int QHALF = N * 128;
-  static constexpr int Q_BYTES = 2 * QHALF;
+  static constexpr int Q_BYTES = KBLK * QHALF;
+  static constexpr int KSTEPS = F8 ? kIdxDim / 32 : kIdxDim / 16;   // MMAs per tile (K = 32 / 16)
   static constexpr int EPI_WARPS = (QG == 1) ? 4 : 8;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr int TMEM_COLS = (2 * N < 32) ? 32 : 2 * N;
+  static constexpr int NACC = (F8 && QG == 1) ? 4 : 2;   // TMEM accumulators in flight (measured best)
+  static constexpr int TMEM_COLS = (NACC * N < 32) ? 32 : NACC * N;
   static constexpr int SMEM_TILES = STAGES * KT_BYTES + QBUFS * Q_BYTES;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024 + EPI_WARPS * ((QG == 1) ? 1 : 4) * kIdxHeads * 4;
-  static constexpr uint32_t IDESC = idesc_bf16_f32(128, N, 0, 0);
+  static constexpr uint32_t IDESC = F8 ? idesc_e4m3_f32(128, N) : idesc_bf16_f32(128, N, 0, 0);
 };
 
 struct IndexerParams {
   const float* w;                 // [T, 32]
+  const float* q_scale;           // [T, 32] (FP8 keys only)
+  const float* k_scale;           // [n_rows] (FP8 keys only)
   const int64_t* seq_row_start;   // [B]
   const int32_t* q_seq;           // [T]
   const int32_t* q_pos;           // [T]
@@ -95,6 +117,15 @@ __device__ __forceinline__ GroupInfo load_group(const IndexerParams& p, int g, b
   return gi;
 }
 
+// Group and key tile of work unit u (u = g * n_kt + kt).  The FP8 kernel
+// advances (g, kt) incrementally instead; on the bf16 kernel the division per
+// unit measured faster (its slower issue loop paces the key loads better on
+// the decode batches), so it keeps it.
+__device__ __forceinline__ void unit_of(int64_t u, int32_t n_kt, int& g, int& kt) {
+  g = (int)(u / n_kt);
+  kt = (int)(u % n_kt);
+}
+
 struct Ring {
   int idx;
   uint32_t phase;
@@ -106,11 +137,22 @@ struct Ring {
   }
 };
 
-template <int QG>
-__global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
+// D[tmem] (+)= A . B with E4M3 operands from shared memory, fp32 accumulate.
+__device__ __forceinline__ void mma_e4m3_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <int QG, bool F8>
+__global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                    const IndexerParams p) {
-  using C = IdxCfg<QG>;
+  using C = IdxCfg<QG, F8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -122,8 +164,8 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
   uint64_t* q_full = k_empty + C::STAGES;
   uint64_t* q_empty = q_full + C::QBUFS;
   uint64_t* acc_full = q_empty + C::QBUFS;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* mma_done = acc_empty + 2;
+  uint64_t* acc_empty = acc_full + C::NACC;
+  uint64_t* mma_done = acc_empty + C::NACC;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* w_s = reinterpret_cast<float*>(smem + C::SMEM_TILES + 1024);
@@ -140,7 +182,7 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::NACC; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], C::EPI_WARPS);
     }
@@ -174,9 +216,9 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
       bool qused[C::QBUFS] = {};
       uint32_t qlast[C::QBUFS] = {};
       bool ok = true;
-      for (int64_t u = u_begin; u < u_end && ok; ++u) {
-        const int g = (int)(u / p.n_kt);
-        const int kt = (int)(u % p.n_kt);
+      int g = (int)(u_begin / p.n_kt), kt = (int)(u_begin % p.n_kt);   // unit u = g * n_kt + kt
+      for (int64_t u = u_begin; u < u_end && ok; ++u, kt = (kt + 1 == p.n_kt) ? 0 : kt + 1, g += (kt == 0)) {
+        if constexpr (!F8) unit_of(u, p.n_kt, g, kt);
         if (g != cur_g) {
           gi = load_group<QG>(p, g, true);
           cur_g = g;
@@ -184,8 +226,8 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
           if (!mbar_wait(&q_empty[qs.idx], qs.phase ^ 1u, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&q_full[qs.idx], C::Q_BYTES);
           uint8_t* qb = qbufs + qs.idx * C::Q_BYTES;
-          tma_load_2d(qb, &qmap, 0, g * C::N, &q_full[qs.idx]);
-          tma_load_2d(qb + C::QHALF, &qmap, 64, g * C::N, &q_full[qs.idx]);
+          for (int blk = 0; blk < C::KBLK; ++blk)   // 128-byte column blocks (64 bf16 / 128 fp8)
+            tma_load_2d(qb + blk * C::QHALF, &qmap, blk * 64, g * C::N, &q_full[qs.idx]);
           qused[qs.idx] = true;
           qlast[qs.idx] = qs.phase;
         }
@@ -194,8 +236,8 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
         mbar_arrive_expect_tx(&k_full[ks.idx], C::KT_BYTES);
         uint8_t* kb = ktiles + ks.idx * C::KT_BYTES;
         const int32_t row0 = (int32_t)(gi.row_base + (int64_t)kt * kKeyTile);
-        tma_load_2d(kb, &kmap, 0, row0, &k_full[ks.idx]);
-        tma_load_2d(kb + C::KHALF, &kmap, 64, row0, &k_full[ks.idx]);
+        for (int blk = 0; blk < C::KBLK; ++blk)
+          tma_load_2d(kb + blk * C::KHALF, &kmap, blk * 64, row0, &k_full[ks.idx]);
         kused[ks.idx] = true;
         klast[ks.idx] = ks.phase;
         ks.next(C::STAGES);
@@ -214,10 +256,10 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
       int cur_g = -1;
       GroupInfo gi{0, -1};
       bool ok = true;
-      for (int64_t u = u_begin; u < u_end && ok; ++u) {
+      int g = (int)(u_begin / p.n_kt), kt = (int)(u_begin % p.n_kt);   // unit u = g * n_kt + kt
+      for (int64_t u = u_begin; u < u_end && ok; ++u, kt = (kt + 1 == p.n_kt) ? 0 : kt + 1, g += (kt == 0)) {
+        if constexpr (!F8) unit_of(u, p.n_kt, g, kt);
         if (*abort_flag) { ok = false; break; }
-        const int g = (int)(u / p.n_kt);
-        const int kt = (int)(u % p.n_kt);
         if (g != cur_g) {
           gi = load_group<QG>(p, g, false);
           if (cur_g >= 0) mma_commit(&q_empty[qs.idx]);   // old query block free once drained
@@ -232,17 +274,19 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
         const uint32_t kaddr = smem_u32(ktiles + ks.idx * C::KT_BYTES);
         const uint32_t qaddr = smem_u32(qbufs + qs.idx * C::Q_BYTES);
         const uint32_t d_tmem = tmem_base + (uint32_t)(as.idx * C::N);
+        // K steps of 32 bytes (16 bf16 or 32 fp8 values) inside each 128-byte block
 #pragma unroll
-        for (int kk = 0; kk < kIdxDim / 16; ++kk) {
+        for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const uint32_t off = (uint32_t)((kk & 3) * 32);
           const uint64_t ad = sdesc_sw128(kaddr + (kk >> 2) * C::KHALF + off, 16, 1024);
           const uint64_t bd = sdesc_sw128(qaddr + (kk >> 2) * C::QHALF + off, 16, 1024);
-          mma_bf16_ss(d_tmem, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+          if constexpr (F8) mma_e4m3_ss(d_tmem, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+          else mma_bf16_ss(d_tmem, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
         }
         mma_commit(&k_empty[ks.idx]);
         mma_commit(&acc_full[as.idx]);
         ks.next(C::STAGES);
-        as.next(2);
+        as.next(C::NACC);
       }
       if (!ok) *abort_flag = 1;
       // Drain: every MMA issued by this thread has finished before TMEM is freed.
@@ -261,10 +305,10 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
     int cur_g = -1;
     GroupInfo gi{0, -1};
     int qpos_q[QPW];
-    for (int64_t u = u_begin; u < u_end; ++u) {
+    int g = (int)(u_begin / p.n_kt), kt = (int)(u_begin % p.n_kt);   // unit u = g * n_kt + kt
+    for (int64_t u = u_begin; u < u_end; ++u, kt = (kt + 1 == p.n_kt) ? 0 : kt + 1, g += (kt == 0)) {
+      if constexpr (!F8) unit_of(u, p.n_kt, g, kt);
       if (*abort_flag) break;
-      const int g = (int)(u / p.n_kt);
-      const int kt = (int)(u % p.n_kt);
       if (g != cur_g) {
         gi = load_group<QG>(p, g, false);
         cur_g = g;
@@ -273,7 +317,9 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
 #pragma unroll
         for (int qi = 0; qi < QPW; ++qi) {
           const int t = g * QG + qbase + qi;
-          w_my[qi * kIdxHeads + lane] = (t < p.T) ? p.w[(int64_t)t * kIdxHeads + lane] : 0.f;
+          float wv = (t < p.T) ? p.w[(int64_t)t * kIdxHeads + lane] : 0.f;
+          if (F8 && t < p.T) wv *= p.q_scale[(int64_t)t * kIdxHeads + lane];   // ReLU(a x) = a ReLU(x), a > 0
+          w_my[qi * kIdxHeads + lane] = wv;
         }
         __syncwarp();
 #pragma unroll
@@ -286,6 +332,9 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
       }
       const int64_t pos = (int64_t)kt * kKeyTile + row;
       float res[QPW];
+      float kscale = 1.f;
+      if (F8 && pos <= gi.maxpos && gi.row_base + pos < p.n_rows)
+        kscale = p.k_scale[gi.row_base + pos];   // issued before the wait
       if (kt * kKeyTile <= gi.maxpos) {
         if (!mbar_wait(&acc_full[as.idx], as.phase, abort_flag)) { *abort_flag = 1; break; }
         tc_fence_after();
@@ -311,13 +360,13 @@ __global__ void __launch_bounds__(IdxCfg<QG>::THREADS, 1)
               s0 = fmaf(wv.z, fmaxf(__uint_as_float(v[u][4 * j4 + 2]), 0.f), s0);
               s1 = fmaf(wv.w, fmaxf(__uint_as_float(v[u][4 * j4 + 3]), 0.f), s1);
             }
-            res[qp + u] = s0 + s1;
+            res[qp + u] = (s0 + s1) * kscale;
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[as.idx]);
-        as.next(2);
+        as.next(C::NACC);
       } else {
 #pragma unroll
         for (int qi = 0; qi < QPW; ++qi) res[qi] = -INFINITY;

@@ -41,6 +41,7 @@ class LayerArgs(ctypes.Structure):
 
 SIGNATURES = {
     "dsa_index_scores": (_I32, [_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _P, _I64, _P]),
+    "dsa_index_scores_fp8": (_I32, [_P, _P, _P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _P, _I64, _P]),
     "dsa_topk_workspace_size": (_SZ, [_I32, _I64, _I32]),
     "dsa_topk": (_I32, [_P, _I64, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "sparse_mla_workspace_size": (_SZ, [_I32, _I32]),
@@ -124,6 +125,35 @@ def index_scores(q_idx, w, k_idx, seq_row_start, q_seq, q_pos, scores, q_group=1
     _check(lib.dsa_index_scores(_ptr(q_idx), _ptr(w), _ptr(k_idx), k_idx.shape[0], _ptr(seq_row_start),
                                 seq_row_start.shape[0], _ptr(q_seq), _ptr(q_pos), T, q_group,
                                 _ptr(scores), scores.shape[1], _stream(stream)))
+    return scores
+
+
+def _codes(t, shape, name):
+    """E4M3 codes as torch.float8_e4m3fn or their uint8 bytes."""
+    if t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    _need(t, torch.uint8, shape, name)
+    return t
+
+
+def index_scores_fp8(q8, q_scale, w, k8, k_scale, seq_row_start, q_seq, q_pos, scores, q_group=1,
+                     stream=None):
+    """I[t, s] on FP8 (E4M3) keys and queries with per-row scales into ``scores``
+    [T, ld] (see dsa_index_scores_fp8)."""
+    T = q8.shape[0]
+    q8 = _codes(q8, (T, 32, 128), "q8")
+    k8 = _codes(k8, None, "k8")
+    _need(q_scale, torch.float32, (T, 32), "q_scale")
+    _need(w, torch.float32, (T, 32), "w")
+    _need(k_scale, torch.float32, (k8.shape[0],), "k_scale")
+    _need(seq_row_start, torch.int64, None, "seq_row_start")
+    _need(q_seq, torch.int32, (T,), "q_seq")
+    _need(q_pos, torch.int32, (T,), "q_pos")
+    _need(scores, torch.float32, None, "scores")
+    lib = load_library()
+    _check(lib.dsa_index_scores_fp8(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), k8.shape[0],
+                                    _ptr(seq_row_start), seq_row_start.shape[0], _ptr(q_seq), _ptr(q_pos), T,
+                                    q_group, _ptr(scores), scores.shape[1], _stream(stream)))
     return scores
 
 

@@ -17,7 +17,7 @@ import dataclasses
 import torch
 
 from sparse_attention_16_b200 import ops
-from sparse_attention_16_b200.workloads import CONFIGS, make_workload
+from sparse_attention_16_b200.workloads import CONFIGS, make_workload, quantize_e4m3_rows
 
 
 def main():
@@ -26,6 +26,7 @@ def main():
     ap.add_argument("--config", default="decode_b64_32k", choices=sorted(CONFIGS))
     ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--layer", type=int, default=0, help="attention: which layer of the configuration")
+    ap.add_argument("--fp8", action="store_true", help="indexer: FP8 (E4M3) keys and queries, per-row scales")
     a = ap.parse_args()
 
     case = CONFIGS[a.config]
@@ -39,8 +40,17 @@ def main():
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     cnt = torch.empty((T,), dtype=torch.int32, device=dev)
 
+    if a.fp8:
+        q8, q8_scale = quantize_e4m3_rows(wl.q_idx)
+        k8, k8_scale = quantize_e4m3_rows(wl.k_idx)
+
     def indexer():
-        ops.index_scores(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, scores, q_group=q_group)
+        if a.fp8:
+            ops.index_scores_fp8(q8, q8_scale, wl.w, k8, k8_scale, wl.seq_row_start, wl.q_seq, wl.q_pos, scores,
+                                 q_group=q_group)
+        else:
+            ops.index_scores(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, scores,
+                             q_group=q_group)
 
     def topk():
         ops.topk(scores, wl.q_pos, k, idx, cnt)

@@ -194,6 +194,19 @@ def make_workload(case: Case, device="cpu") -> Workload:
                     q_idx=q_idx, w=w, k_idx=k_idx, layers=layers, planted_pos=planted)
 
 
+def quantize_e4m3_rows(x: torch.Tensor):
+    """Per-row FP8 (E4M3) encoding of an input tensor, for the FP8-key indexer:
+    scale = max |x| over the last dimension / 448 (the largest E4M3 value; 1
+    for an all-zero row) and codes = e4m3(x / scale) with torch's
+    float8_e4m3fn conversion.  Returns (codes uint8 [..., d], scales f32 [...]).
+    Input preparation only: both the library and the oracle receive these bytes."""
+    xf = x.float()
+    amax = xf.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    codes = (xf / scale.unsqueeze(-1)).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), scale.contiguous()
+
+
 def small_case(name, lengths=None, *, kind="decode", cached=0, new=0, layers=(64,),
                qmul="uniform", mla_q_std=1.0 / math.sqrt(192.0), seed=7, topk=2048,
                planted=0) -> Case:

@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from sparse_attention_16_b200 import ops
-from sparse_attention_16_b200.workloads import SOFTMAX_SCALE, to_numpy
+from sparse_attention_16_b200.workloads import SOFTMAX_SCALE, quantize_e4m3_rows, to_numpy
 
 SCORE_RTOL = 1e-3
 ATTN_ATOL = 2e-2
@@ -62,6 +62,35 @@ def oracle_scores(wl, ts, ld):
         k = to_numpy(wl.k_idx[int(starts[b]):int(starts[b]) + n])
         rows.append(oracle.index_scores(to_numpy(wl.q_idx[t:t + 1]), to_numpy(wl.w[t:t + 1]), k,
                                         np.array([0]), np.array([0]), np.array([q_pos[t]]), ld)[0])
+    return np.stack(rows)
+
+
+def fp8_inputs(wl):
+    """E4M3 codes and per-row scales of the workload's indexer queries and keys."""
+    q8, qs = quantize_e4m3_rows(wl.q_idx)
+    k8, ks = quantize_e4m3_rows(wl.k_idx)
+    return q8, qs, k8, ks
+
+
+def gpu_scores_fp8(wl, q8, qs, k8, ks, ld=None, q_group=1):
+    ld = ld or wl.case.ld
+    scores = torch.empty((wl.T, ld), dtype=torch.float32, device=wl.q_idx.device)
+    ops.index_scores_fp8(q8, qs, wl.w, k8, ks, wl.seq_row_start, wl.q_seq, wl.q_pos, scores,
+                         q_group=q_group)
+    return scores
+
+
+def oracle_scores_fp8(wl, q8, qs, k8, ks, ts, ld):
+    """Oracle FP8-key score rows for the queries in ``ts`` (fetches only their key rows)."""
+    starts, q_seq, q_pos = host_meta(wl)
+    rows = []
+    for t in ts:
+        b = int(q_seq[t])
+        n = int(q_pos[t]) + 1
+        lo = int(starts[b])
+        rows.append(oracle.index_scores_fp8(to_numpy(q8[t:t + 1]), to_numpy(qs[t:t + 1]), to_numpy(wl.w[t:t + 1]),
+                                            to_numpy(k8[lo:lo + n]), to_numpy(ks[lo:lo + n]), np.array([0]),
+                                            np.array([0]), np.array([q_pos[t]]), ld)[0])
     return np.stack(rows)
 
 
