@@ -158,7 +158,12 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, int
  *   out    bf16 [T, 64, 512]   o[t,h] = sum_i p_i c_{s_i}   (round to nearest even)
  *   lse    f32  [T, 64] or NULL: natural-log log-sum-exp of the logits
  *   count == 0 gives out = 0 and lse = -inf.
- *   workspace: sparse_mla_workspace_size(T, k) bytes, 256-byte aligned.
+ *   workspace: sparse_mla_workspace_size(T, k) bytes, 256-byte aligned (may be
+ *              NULL when that size is 0).  The size is 0 when each query is
+ *              handled by one thread block, or split over 2-8 blocks that run as
+ *              a thread-block cluster and merge their partials in distributed
+ *              shared memory (used when every cluster of the call can be
+ *              resident at once); otherwise it holds the fp32 split partials.
  */
 size_t sparse_mla_workspace_size(int32_t T, int32_t k);
 dsa_status_t sparse_mla_attend(const void* q_nope, const void* q_pe, const float* qmul,
@@ -186,9 +191,11 @@ dsa_status_t sparse_mla_attend(const void* q_nope, const void* q_pe, const float
  *     516 floats (16.9 MB) that every GPU loading the library holds until the
  *     process exits.  The call allocates nothing and calls no allocating routine.
  *   - Limit: a call needs T x n_split partials, where n_split is the number of
- *     blocks each query is split across (1 once T reaches the SM count, so no
- *     scratch is used then).  Calls needing more than DSA_NOALLOC_MAX_PARTIALS
- *     return DSA_ERR_WORKSPACE with a message that states the limit.
+ *     blocks each query is split across, unless those blocks merge on chip
+ *     (n_split of 2-8 with every cluster resident: no scratch; n_split = 1 once
+ *     T reaches the SM count: no scratch).  Calls needing more than
+ *     DSA_NOALLOC_MAX_PARTIALS return DSA_ERR_WORKSPACE with a message that
+ *     states the limit.
  *   - Set-up: the first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current.  Make that first call
  *     before any stream capture.

@@ -75,6 +75,16 @@ def test_decode_bytes_of_the_batch64_config():
     assert (idx_b + att_b) / 1e6 == pytest.approx(698, abs=1)
 
 
+def test_fp8_indexer_bytes_per_key_and_query():
+    # E4M3 keys: 128 B of codes + a 4 B fp32 scale per scored key; per query 32 x 128 B of codes,
+    # 32 fp32 scales and 32 fp32 weights; the score row as before.
+    T, L = 64, 32768
+    b = acc.indexer_bytes(T * L, T, T * L, fp8=True)
+    assert b == T * L * (128 + 4) + T * (4096 + 128 + 128) + T * L * 4
+    # about half of the bf16 stream for the same work
+    assert b / acc.indexer_bytes(T * L, T, T * L) == pytest.approx(136 / 260, rel=1e-3)
+
+
 def test_flop_counts():
     assert acc.attend_flops(1, 64) == 2 * 64 * 1088
     assert acc.attend_flops(1, 0) == 2 * 64 * 1024
