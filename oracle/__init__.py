@@ -25,6 +25,10 @@ Parity status per function (what pins it, see tests/test_oracle_pins.py):
   forward           composition of the above; no separate pin needed.
   e4m3_decode       pinned: every one of the 256 codes against torch's float8_e4m3fn
                     conversion, and the format's landmark values (1, 448, 2^-6, 2^-9).
+  topk_merge        pinned: the merge of per-shard top-k lists equals topk_select on the
+                    whole row (tied and random rows, several shard counts).
+  lse_combine       pinned: combining sparse_mla over disjoint parts of a selection equals
+                    sparse_mla over the whole selection; empty parts contribute nothing.
   index_scores_fp8  pinned: hand-worked example with integer codes, positive
                     homogeneity in each key scale and in each query's scales, zero
                     scale gives zero scores, causal/offset checks.
@@ -35,6 +39,8 @@ from .dsa_oracle import (  # noqa: F401
     e4m3_decode,
     index_scores_fp8,
     topk_select,
+    topk_merge,
+    lse_combine,
     sparse_mla,
     dense_causal_mla,
     explicit_mla,

@@ -146,6 +146,46 @@ def topk_select(scores, q_pos, k):
     return idx, count
 
 
+def topk_merge(cand_scores, cand_pos, k):
+    """Global top-k of one query from the union of per-shard candidate lists.
+
+    Context-parallel decode ([TR] serving section, Figure 16: each rank selects
+    among its own positions, the candidates are exchanged, then merged):
+    cand_scores [n] and cand_pos [n] hold every shard's candidates with their
+    global positions (-1 marks an empty slot).  The rule is topk_select's:
+    score descending, then position ascending; -0.0 == +0.0; NaN ranks as -inf.
+    Returns the k_eff = min(k, valid candidates) best positions, ascending.
+    """
+    sc = np.asarray(cand_scores, dtype=np.float64) + 0.0
+    ps = np.asarray(cand_pos, dtype=np.int64)
+    keep = ps >= 0
+    sc, ps = sc[keep], ps[keep]
+    sc = np.where(np.isnan(sc), -np.inf, sc)
+    order = np.lexsort((ps, -sc))
+    return np.sort(ps[order[:min(int(k), ps.size)]])
+
+
+def lse_combine(o_parts, lse_parts):
+    """Attention over a selection split into disjoint parts, merged exactly.
+
+    For one query, parts r = 0..R-1 each give o_r = sum_{i in r} exp(z_i - lse_r) c_i
+    and lse_r = log sum_{i in r} exp(z_i) (-inf and o_r = 0 for an empty part).
+    Over the whole selection, lse = log sum_r exp(lse_r) and
+    o = sum_r exp(lse_r - lse) o_r: the context-parallel "output combine"
+    ([TR] serving section, Figure 16).  o_parts [R, H, d], lse_parts [R, H].
+    Returns (o [H, d], lse [H]); a head with every part empty gives 0 and -inf.
+    """
+    o_p = np.asarray(o_parts, dtype=np.float64)
+    l_p = np.asarray(lse_parts, dtype=np.float64)
+    top = np.max(l_p, axis=0)                                  # [H]
+    safe = np.where(np.isneginf(top), 0.0, top)
+    w = np.where(np.isneginf(l_p), 0.0, np.exp(l_p - safe))   # [R, H]
+    tot = w.sum(axis=0)
+    lse = np.where(tot > 0, safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    o = np.einsum("rh,rhd->hd", w, o_p) / np.where(tot > 0, tot, 1.0)[:, None]
+    return o, lse
+
+
 def _attend_rows(qn, qp, mult, scale, rows, d_c):
     """Softmax attention of one query (all heads) over the given cache rows.
 

@@ -1,7 +1,10 @@
 """Multi-rank bookkeeping on CPU with the gloo backend (world size 2): sequence
 sharding, the max-over-ranks time, the job-wide throughput, and that running the
 path rank by rank on disjoint sequences reproduces the single-process result
-(checked with the CPU oracle, so no GPU is needed)."""
+(checked with the CPU oracle, so no GPU is needed).  Also the context-parallel
+exchange for one long sequence (per-rank selection, candidate all-gather and
+merge, per-rank attention, output combine), computed with the oracle: the
+decomposition a context-parallel decode must reproduce."""
 
 import os
 import socket
@@ -73,6 +76,72 @@ def test_replicas_world_size_2():
                                 SOFTMAX_SCALE, k=256)
     for q in range(5):
         np.testing.assert_allclose(r0["all"][q], outs[0][0][q], rtol=1e-12, atol=1e-14)
+
+
+def _cp_worker(rank, world, port, out):
+    # Context-parallel decode of one long sequence (the exchange the technical report's
+    # serving section describes): each rank scores and selects among its own positions,
+    # the candidates are all-gathered and merged, each rank attends over the selected rows
+    # it owns, and the partial outputs are all-gathered and combined.
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        from sparse_attention_16_b200.workloads import SOFTMAX_SCALE, make_workload, small_case, to_numpy
+
+        k = 256
+        wl = make_workload(small_case("cp", (5000,), layers=(64,), seed=4), "cpu")
+        lay = wl.layers[0]
+        L = 5000
+        lo, hi = rank * L // world, (rank + 1) * L // world
+        keys = to_numpy(wl.k_idx[lo:hi])
+        s = oracle.index_scores(to_numpy(wl.q_idx), to_numpy(wl.w), keys, np.array([0]), np.array([0]),
+                                np.array([hi - lo - 1]), hi - lo)
+        sel, cnt = oracle.topk_select(s, np.array([hi - lo - 1]), k)
+        pos = np.full(k, -1, np.int64)
+        sc = np.full(k, -np.inf)
+        pos[:cnt[0]] = sel[0, :cnt[0]] + lo
+        sc[:cnt[0]] = s[0, sel[0, :cnt[0]]]
+        all_pos = [torch.empty(k, dtype=torch.int64) for _ in range(world)]
+        all_sc = [torch.empty(k, dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(all_pos, torch.from_numpy(pos))
+        dist.all_gather(all_sc, torch.from_numpy(sc))
+        chosen = oracle.topk_merge(torch.cat(all_sc).numpy(), torch.cat(all_pos).numpy(), k)
+        mine = chosen[(chosen >= lo) & (chosen < hi)] - lo
+        idx = np.full((1, 2048), -1, np.int32)
+        idx[0, :mine.size] = mine
+        o, lse = oracle.sparse_mla(to_numpy(lay.q_nope), to_numpy(lay.q_pe), to_numpy(lay.qmul), SOFTMAX_SCALE,
+                                   to_numpy(lay.cache[lo:hi]), 64, np.array([0]), np.array([0]), idx,
+                                   np.array([mine.size]))
+        all_o = [torch.empty(o[0].shape, dtype=torch.float64) for _ in range(world)]
+        all_l = [torch.empty(lse[0].shape, dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(all_o, torch.from_numpy(o[0]))
+        dist.all_gather(all_l, torch.from_numpy(lse[0]))
+        oc, lc = oracle.lse_combine(torch.stack(all_o).numpy(), torch.stack(all_l).numpy())
+        out[rank] = {"chosen": chosen.tolist(), "o": oc, "lse": lc}
+    finally:
+        dist.destroy_process_group()
+
+
+def test_context_parallel_exchange_world_size_2():
+    import oracle
+    from sparse_attention_16_b200.workloads import SOFTMAX_SCALE, make_workload, small_case, to_numpy
+
+    world = 2
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.start_processes(_cp_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
+    wl = make_workload(small_case("cp", (5000,), layers=(64,), seed=4), "cpu")
+    lay = wl.layers[0]
+    s = oracle.index_scores(to_numpy(wl.q_idx), to_numpy(wl.w), to_numpy(wl.k_idx), np.array([0]), np.array([0]),
+                            np.array([4999]), 5000)
+    idx, cnt = oracle.topk_select(s, np.array([4999]), 256)
+    o, lse = oracle.sparse_mla(to_numpy(lay.q_nope), to_numpy(lay.q_pe), to_numpy(lay.qmul), SOFTMAX_SCALE,
+                               to_numpy(lay.cache), 64, np.array([0]), np.array([0]), idx, cnt)
+    for r in range(world):
+        assert out[r]["chosen"] == idx[0, :cnt[0]].tolist()
+        np.testing.assert_allclose(out[r]["o"], o[0], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(out[r]["lse"], lse[0], rtol=1e-12)
 
 
 def test_shards_cover_and_balance():

@@ -42,6 +42,11 @@ MUTATIONS = {
     "fp8_indexer_key_scale_of_wrong_row": (
         "k_rows = e4m3_decode(k8[base:base + n]) * _f64(k_scale[base:base + n])[:, None]",
         "k_rows = e4m3_decode(k8[base:base + n]) * _f64(k_scale[:n])[:, None]"),
+    "merge_ties_to_higher_position": ("order = np.lexsort((ps, -sc))", "order = np.lexsort((-ps, -sc))"),
+    "merge_keeps_empty_slots": ("    keep = ps >= 0\n", "    keep = ps >= -1\n"),
+    "combine_plain_average": ('o = np.einsum("rh,rhd->hd", w, o_p) / np.where(tot > 0, tot, 1.0)[:, None]',
+                              'o = o_p.mean(axis=0)'),
+    "combine_lse_without_shift": ("lse = np.where(tot > 0, safe + np.log(", "lse = np.where(tot > 0, 0.0 + np.log("),
     "fp8_indexer_relu_after_weighting": ("out[t, :n] = np.maximum(k_rows @ q.T, 0.0) @ wt[t]",
                                          "out[t, :n] = np.maximum(k_rows @ q.T @ wt[t], 0.0)"),
 }
@@ -57,7 +62,7 @@ def _mutant(name):
 
 def _run_pins(mod, golden_dir, monkeypatch):
     for fn in ("index_scores", "topk_select", "sparse_mla", "dense_causal_mla", "explicit_mla",
-               "forward", "e4m3_decode", "index_scores_fp8"):
+               "forward", "e4m3_decode", "index_scores_fp8", "topk_merge", "lse_combine"):
         monkeypatch.setattr(pins, fn, getattr(mod, fn))
     failures = 0
     for tname, test in inspect.getmembers(pins, inspect.isfunction):

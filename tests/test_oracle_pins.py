@@ -15,7 +15,7 @@ import numpy as np
 import pytest
 
 from oracle import (dense_causal_mla, e4m3_decode, explicit_mla, forward, index_scores,
-                    index_scores_fp8, sparse_mla, topk_select)
+                    index_scores_fp8, lse_combine, sparse_mla, topk_merge, topk_select)
 
 RNG = np.random.default_rng(1234)
 
@@ -270,6 +270,58 @@ def test_topk_invariants_random():
 
 
 # --------------------------------------------------------------------------- attention
+
+# --------------------------------------------------------------------------- context-parallel pieces
+
+@pytest.mark.parametrize("trial", range(12))
+def test_topk_merge_of_shard_selections_equals_whole_row(trial):
+    # Every element of the global top-k is in its own shard's top-k (the tie rule is the
+    # same global-position order inside a shard), so merging the shards' lists is exact.
+    rng = np.random.default_rng(100 + trial)
+    n = int(rng.integers(5, 400))
+    k = int(rng.integers(1, 60))
+    row = rng.integers(-4, 5, n).astype(float) if trial % 2 else rng.normal(size=n)
+    row[rng.random(n) < 0.1] = -0.0
+    whole, cnt = topk_select(row[None, :], np.array([n - 1]), k)
+    G = int(rng.integers(2, 6))
+    edges = np.linspace(0, n, G + 1).astype(int)
+    cs, cp = [], []
+    for a, b in zip(edges[:-1], edges[1:]):
+        if b <= a:
+            continue
+        sel, c = topk_select(row[None, a:b], np.array([b - a - 1]), k)
+        pos = sel[0, :c[0]].astype(np.int64) + a
+        cs.append(row[pos])
+        cp.append(pos)
+    cs.append(np.array([np.inf, 3.0]))     # empty slots (position -1) never take part, whatever their score
+    cp.append(np.array([-1, -1]))
+    merged = topk_merge(np.concatenate(cs), np.concatenate(cp), k)
+    assert merged.tolist() == whole[0, :cnt[0]].tolist()
+
+
+def test_lse_combine_of_parts_equals_whole_selection():
+    qn, qp, m, cache, starts, q_seq, q_pos = _rand_attn_case(T=1, lens=(300,))
+    scale = 0.2
+    for n_parts in (2, 3, 5):
+        sel = np.sort(np.random.default_rng(n_parts).choice(300, 97, replace=False))
+        idx = np.full((1, 2048), -1, np.int32)
+        idx[0, :97] = sel
+        o_all, l_all = sparse_mla(qn, qp, m, scale, cache, 64, starts, q_seq, idx, np.array([97]))
+        parts = np.array_split(np.random.default_rng(7).permutation(sel), n_parts)
+        parts.append(np.array([], dtype=np.int64))          # an empty part contributes nothing
+        o_p, l_p = [], []
+        for part in parts:
+            ip = np.full((1, 2048), -1, np.int32)
+            ip[0, :part.size] = part
+            o, l = sparse_mla(qn, qp, m, scale, cache, 64, starts, q_seq, ip, np.array([part.size]))
+            o_p.append(o[0])
+            l_p.append(l[0])
+        o, l = lse_combine(np.stack(o_p), np.stack(l_p))
+        np.testing.assert_allclose(o, o_all[0], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(l, l_all[0], rtol=1e-12)
+    o0, l0 = lse_combine(np.zeros((2, 64, 512)), np.full((2, 64), -np.inf))
+    assert np.all(o0 == 0) and np.all(np.isneginf(l0))
+
 
 def test_attention_hand_worked_example(golden_dir):
     g = _toy(golden_dir)["attention"]
