@@ -79,15 +79,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 2-D bf16 tensor map with the 128-byte swizzle: `inner` contiguous elements
 // per row, `outer` rows `row_bytes` apart, box of box_inner x box_outer.
 dsa_status_t make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-                       CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
   auto enc = encode_fn();
   if (enc == nullptr) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box,
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
