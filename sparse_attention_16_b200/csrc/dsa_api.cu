@@ -16,6 +16,8 @@
 #include <string>
 #include <utility>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "dsa.h"
 #include "attend.cuh"
 #include "indexer.cuh"
@@ -92,6 +94,15 @@ dsa_status_t make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_
   if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return DSA_OK;
 }
+
+// NVTX range around each C-ABI call (header-only NVTX 3: free unless a
+// profiler is attached), so traces show the library's calls by name.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Raises a kernel's dynamic shared-memory limit once per device (the
 // attribute persists, so later launches skip the driver call).
@@ -519,6 +530,7 @@ dsa_status_t dsa_index_scores(const void* q_idx, const float* w, const void* k_i
                               const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
                               const int32_t* q_pos, int32_t T, int32_t q_group, float* scores,
                               int64_t ld, void* stream) {
+  NvtxRange nvtx_range("dsa_index_scores");
   dsa_status_t st = check_index_args(q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T,
                                      q_group, ld);
   if (st != DSA_OK) return st;
@@ -532,6 +544,7 @@ dsa_status_t dsa_index_scores_fp8(const void* q8, const float* q_scale, const fl
                                   const float* k_scale, int64_t n_rows, const int64_t* seq_row_start,
                                   int32_t B, const int32_t* q_seq, const int32_t* q_pos, int32_t T,
                                   int32_t q_group, float* scores, int64_t ld, void* stream) {
+  NvtxRange nvtx_range("dsa_index_scores_fp8");
   dsa_status_t st = check_index_args(q8, w, k8, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, ld);
   if (st != DSA_OK) return st;
   DSA_REQUIRE(q_scale && k_scale && aligned(q_scale, 4) && aligned(k_scale, 4),
@@ -550,6 +563,7 @@ size_t dsa_topk_workspace_size(int32_t, int64_t, int32_t) { return 0; }
 
 dsa_status_t dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, int32_t T, int32_t k,
                       int32_t* idx, int32_t* count, void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("dsa_topk");
   (void)workspace;
   (void)ws_bytes;
   dsa_status_t st = check_topk_args(scores, ld, q_pos, T, k, idx, count);
@@ -569,6 +583,7 @@ dsa_status_t sparse_mla_attend(const void* q_nope, const void* q_pe, const float
                                const int32_t* q_seq, const int32_t* idx, const int32_t* count,
                                int32_t T, int32_t k, void* out, float* lse, void* workspace,
                                size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("sparse_mla_attend");
   dsa_status_t st = check_attend_args(q_nope, q_pe, qmul, cache, n_rows, ld_c, d_rope, seq_row_start, B,
                                       q_seq, idx, count, T, k, out);
   if (st != DSA_OK) return st;
@@ -590,6 +605,7 @@ dsa_status_t sparse_mla_attend_noalloc(const void* q_nope, const void* q_pe, con
                                        int32_t B, const int32_t* q_seq, const int32_t* idx,
                                        const int32_t* count, int32_t T, int32_t k, void* out,
                                        float* lse, void* stream) {
+  NvtxRange nvtx_range("sparse_mla_attend_noalloc");
   dsa_status_t st = check_attend_args(q_nope, q_pe, qmul, cache, n_rows, ld_c, d_rope, seq_row_start, B,
                                       q_seq, idx, count, T, k, out);
   if (st != DSA_OK) return st;
@@ -635,6 +651,7 @@ dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const voi
                                     float softmax_scale, int32_t k, int32_t* idx_out,
                                     int32_t* count_out, void* workspace, size_t ws_bytes,
                                     void* stream) {
+  NvtxRange nvtx_range("dsa_sparse_mla_forward");
   dsa_status_t st = check_index_args(q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T,
                                      q_group, ld);
   if (st != DSA_OK) return st;
