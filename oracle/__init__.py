@@ -22,7 +22,11 @@ Parity status per function (what pins it, see tests/test_oracle_pins.py):
                     row and zero-multiplier closed forms; permutation invariance.
   dense_causal_mla  pinned through the same equalities (independent code path).
   explicit_mla      pinned through the same equality (independent code path).
-  forward           composition of the above; no separate pin needed.
+  forward           pinned: hand-worked two-layer example (RoPE + NoPE layer sharing one
+                    selection, k = 1, 2 and more than the candidates); its selection equals a
+                    brute-force top-k (repeated argmax) of each query's own scores over its
+                    causal range; five planted mistakes (k ignored, ld one short, selection past
+                    q_pos, every layer reading the first cache, last layer dropped) are caught.
   e4m3_decode       pinned: every one of the 256 codes against torch's float8_e4m3fn
                     conversion, and the format's landmark values (1, 448, 2^-6, 2^-9).
   topk_merge        pinned: the merge of per-shard top-k lists equals topk_select on the

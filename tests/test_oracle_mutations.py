@@ -47,6 +47,14 @@ MUTATIONS = {
     "combine_plain_average": ('o = np.einsum("rh,rhd->hd", w, o_p) / np.where(tot > 0, tot, 1.0)[:, None]',
                               'o = o_p.mean(axis=0)'),
     "combine_lse_without_shift": ("lse = np.where(tot > 0, safe + np.log(", "lse = np.where(tot > 0, 0.0 + np.log("),
+    "forward_ignores_k": ("idx, count = topk_select(scores, q_pos, k)",
+                          "idx, count = topk_select(scores, q_pos, 2048)"),
+    "forward_ld_one_short": ("ld = int(np.max(q_pos)) + 1", "ld = int(np.max(q_pos))"),
+    "forward_selects_past_q_pos": ("idx, count = topk_select(scores, q_pos, k)",
+                                   "idx, count = topk_select(scores, np.full(len(q_pos), ld - 1), k)"),
+    "forward_every_layer_reads_first_cache": ('lay["cache"], lay["d_rope"], seq_row_start',
+                                              'layers[0]["cache"], lay["d_rope"], seq_row_start'),
+    "forward_drops_last_layer": ("    for lay in layers:\n", "    for lay in layers[:-1]:\n"),
     "fp8_indexer_relu_after_weighting": ("out[t, :n] = np.maximum(k_rows @ q.T, 0.0) @ wt[t]",
                                          "out[t, :n] = np.maximum(k_rows @ q.T @ wt[t], 0.0)"),
 }

@@ -458,6 +458,64 @@ def test_empty_selection():
 
 # --------------------------------------------------------------------------- composition
 
+def _forward_toy(golden_dir):
+    g = _toy(golden_dir)
+    ix, fw = g["indexer"], g["forward"]
+    layers = []
+    for lay in fw["layers"]:
+        layers.append(dict(q_nope=np.array(lay["q_nope"], float)[:, None, :],
+                           q_pe=None if lay["q_pe"] is None else np.array(lay["q_pe"], float)[:, None, :],
+                           qmul=np.ones((2, 1)), cache=np.array(lay["cache"], float), d_rope=lay["d_rope"]))
+    args = (np.array(ix["q_idx"], float), np.array(ix["w"]), np.array(ix["k_idx"], float),
+            np.array(ix["seq_row_start"]), np.array(ix["q_seq"]), np.array(fw["q_pos"]))
+    return fw, args, layers
+
+
+def test_forward_hand_worked_example(golden_dir):
+    # Hand-worked selection and per-layer outputs (one RoPE and one NoPE layer
+    # sharing one selection) for k = 1, 2 and 4 (more than the candidates).
+    fw, args, layers = _forward_toy(golden_dir)
+    want_scores = np.array([[float(v) for v in row] for row in fw["scores"]])
+    np.testing.assert_array_equal(index_scores(*args, 3), want_scores)
+    for key, kk in (("k1", 1), ("k2", 2), ("k4", 4)):
+        c = fw["cases"][key]
+        idx, cnt, outs = forward(*args, layers, 1.0, k=kk)
+        assert idx.tolist() == c["idx"], key
+        assert cnt.tolist() == c["count"], key
+        assert len(outs) == len(layers)
+        for (o, lse), o_want, l_want in zip(outs, c["o"], c["lse"]):
+            np.testing.assert_allclose(o, np.array(o_want), rtol=1e-12, atol=1e-15)
+            np.testing.assert_allclose(lse, np.array(l_want), rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("trial", range(6))
+def test_forward_selection_is_the_top_k_of_the_indexer_scores(trial):
+    # The shared selection is the top-k of the indexer's own scores, over the
+    # causal range of each query, with the given k (random sizes, some queries
+    # with fewer than k candidates, several queries per sequence).
+    rng = np.random.default_rng(500 + trial)
+    lens = tuple(int(x) for x in rng.integers(5, 90, size=3))
+    q, w, k, starts, q_seq, q_pos, ld = _rand_index_case(T=3, lens=lens)
+    q_pos = np.array([int(rng.integers(0, lens[b])) for b in q_seq])
+    qn, qp, m, cache, _, _, _ = _rand_attn_case(T=3, lens=lens)
+    layers = [dict(q_nope=qn, q_pe=qp, qmul=m, cache=cache, d_rope=64)]
+    kk = int(rng.integers(1, 70))
+    idx, cnt, outs = forward(q, w, k, starts, q_seq, q_pos, layers, 0.1, k=kk)
+    for t in range(3):
+        n = q_pos[t] + 1
+        b = q_seq[t]
+        # brute force on this query alone: scores of its candidates, best kk by repeated argmax
+        row = index_scores(q[t:t + 1], w[t:t + 1], k[starts[b]:starts[b] + n], np.array([0]), np.array([0]),
+                           np.array([n - 1]), n)[0]
+        want = _select_by_repeated_argmax(list(row), kk)
+        assert cnt[t] == len(want) == min(kk, n)
+        assert idx[t, :cnt[t]].tolist() == want
+        assert (idx[t, cnt[t]:] == -1).all()
+    o_ref, l_ref = sparse_mla(qn, qp, m, 0.1, cache, 64, starts, q_seq, idx, cnt)
+    np.testing.assert_array_equal(outs[0][0], o_ref)
+    np.testing.assert_array_equal(outs[0][1], l_ref)
+
+
 def test_forward_shares_one_selection_across_layers():
     q, w, k, starts, q_seq, q_pos, ld = _rand_index_case(T=2, lens=(300, 120))
     qn, qp, m, cache, _, _, _ = _rand_attn_case(T=2, lens=(300, 120))
