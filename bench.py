@@ -4,24 +4,38 @@
 
 A step is one pass of the whole hot path over one batch: the indexer scores
 every earlier position of every query, the top-k kernel selects 2,048 per
-query, and every layer of the configuration attends over that selection.  The
-default configuration is the decode batch the headline metric is quoted on: 64
-sequences x 32,768 positions, one RoPE layer.  Inputs are resident in HBM when
-the timed region starts (698 MB per step, larger than the 126 MB L2, so every
-step streams from HBM).
+query, and every layer of the configuration attends over that selection (one
+attention launch for all layers).  The default configuration is the largest
+that fits one GPU: 4 sequences x 2^20 positions, one selection reused by 3 RoPE
+layers and 1 NoPE layer (1.11 GB of compulsory HBM traffic per step).  The
+metric is per layer, so `value` counts query-layers per second.  Inputs are
+resident in HBM when the timed region starts; every step streams more than
+the 126 MB L2 holds, so no flush is needed between steps.
 
-Multi-GPU (torchrun, one process per GPU): decode sequences are independent,
-so each rank runs its own batch with no collective on the data path; the only
-collectives are the barrier and the max-over-ranks reduction of the device
-time ("scaling": "weak").
+Timing: the K steps are captured into one CUDA graph; the timed region replays
+that graph R times (R chosen so the region lasts at least --min-seconds,
+default 1 s, long enough for a clock record), bracketed by a barrier and
+synchronisation, timed with CUDA events on the launching stream, max over
+ranks.  `ms_per_step` = region / (K x R).
+
+The same run also measures the 64 x 32,768 decode batch and the chunked
+prefill (8,192 queries over 40,960 positions; the indexer's tensor-core rate)
+as extra keys.
+
+Multi-GPU: `--gpus N` without torchrun spawns N processes itself (one per GPU,
+NCCL); under torchrun each rank is one process.  Decode sequences are
+independent, so each rank runs its own batch with no collective on the data
+path; the only collectives are the barrier and the max-over-ranks reduction of
+the device time ("scaling": "weak").
 
 The reference arm (--impl reference) times the fp64 CPU oracle on a bounded
-sample of the same workload (a few queries per step) on the host cores.
+sample of the same workload (one query per step) on the host cores.
 """
 
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -42,7 +56,8 @@ from sparse_attention_16_b200 import accounting as acc  # noqa: E402
 from sparse_attention_16_b200 import replicas  # noqa: E402
 from sparse_attention_16_b200.workloads import CONFIGS, make_workload, quantize_e4m3_rows, small_case  # noqa: E402
 
-HEADLINE = "decode_b64_32k"
+HEADLINE = "decode_b4_1m_4layers"
+EXTRAS = ("decode_b64_32k", "prefill_32k_plus_8k")
 METRIC = "sparse-MLA+DSA decode queries/s per layer; achieved HBM TB/s vs peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -140,46 +155,43 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- our arm
 
-def run_ours(args, rank, world, local):
+def measure(name, dev, steps, warmup, rank, world, local, min_seconds=0.0, sample_clocks=False, fp8=False,
+            eager=False, e2e=False, e2e_steps=20):
+    """Times `steps` steps of configuration `name` (see the module docstring).
+    Returns a dict with the timing, the per-kernel breakdown and the rooflines."""
     from sparse_attention_16_b200 import ops
 
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    if world > 1:
-        import datetime
-
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=dev)
-    case = CONFIGS[args.config]
+    case = CONFIGS[name]
     # each rank owns an independent batch of the same shape (its own seed)
-    case = type(case)(**{**case.__dict__, "seed": replicas.rank_seed(case.seed, rank)})
+    case = dataclasses.replace(case, seed=replicas.rank_seed(case.seed, rank))
     wl = make_workload(case, dev)
     T, ld, k = wl.T, case.ld, case.topk
+    n_layers = len(wl.layers)
     q_group = 8 if case.kind == "prefill" else 1
-    ops.load_library()
 
     scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     cnt = torch.empty((T,), dtype=torch.int32, device=dev)
     outs = [torch.empty((T, 64, 512), dtype=torch.bfloat16, device=dev) for _ in wl.layers]
     lses = [torch.empty((T, 64), dtype=torch.float32, device=dev) for _ in wl.layers]
-    att_ws = ops.workspace(ops.attend_workspace_bytes(T, k), dev)
+    layers = [dict(q_nope=L.q_nope, q_pe=L.q_pe, qmul=L.qmul, cache=L.cache, d_rope=L.d_rope, out=o, lse=l)
+              for L, o, l in zip(wl.layers, outs, lses)]
+    n_rows = wl.layers[0].cache.shape[0]
+    att_ws = ops.workspace(ops.layers_workspace_bytes(T, n_layers, k), dev)
     stream = torch.cuda.current_stream()
-    if args.fp8_keys:
+    if fp8:
         # E4M3 codes + per-row scales of the same seeded keys/queries (input preparation, untimed)
         q8, q8_scale = quantize_e4m3_rows(wl.q_idx)
         k8, k8_scale = quantize_e4m3_rows(wl.k_idx)
-        wl.k_idx = None          # the bf16 keys are not read in this mode
-        torch.cuda.empty_cache()
 
-    # events around the indexer launch of every timed step (same stream)
-    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(args.steps)]
+    # events around each kernel of every step of the breakdown graph (same stream)
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(steps)]
 
     def step(i=None):
         e = ev[i] if i is not None else None
         if e:
             e[0].record(stream)
-        if args.fp8_keys:
+        if fp8:
             ops.index_scores_fp8(q8, q8_scale, wl.w, k8, k8_scale, wl.seq_row_start, wl.q_seq, wl.q_pos, scores,
                                  q_group=q_group)
         else:
@@ -190,41 +202,48 @@ def run_ours(args, rank, world, local):
         ops.topk(scores, wl.q_pos, k, idx, cnt)
         if e:
             e[2].record(stream)
-        for L, o, l in zip(wl.layers, outs, lses):
-            ops.sparse_mla_attend(L.q_nope, L.q_pe, L.qmul, L.cache, L.d_rope, wl.seq_row_start,
-                                  wl.q_seq, idx, cnt, o, l, ws=att_ws)
+        ops.sparse_mla_attend_layers(layers, n_rows, wl.seq_row_start, wl.q_seq, idx, cnt, q_pos=wl.q_pos,
+                                     ws=att_ws)
         if e:
             e[3].record(stream)
 
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         step()
     torch.cuda.synchronize()
     ops.check_errors()
 
-    # The K timed steps are captured once into a CUDA graph and replayed, so
-    # host-side launch overhead does not leak into the device timings.  Every
-    # kernel of every step still runs.  The timed graph has no event nodes
-    # between kernels (they would stop each kernel from being scheduled while
-    # the previous one drains); a second graph of the same steps with events
-    # around each kernel gives the per-kernel breakdown, after the timed region.
+    # The K timed steps are captured once into a CUDA graph, so host launch
+    # overhead does not leak into the device timings; every kernel of every step
+    # still runs.  The timed graph has no event nodes between kernels; a second
+    # graph of the same steps with events around each kernel gives the
+    # per-kernel breakdown, replayed after the timed region.
     graph = graph_ev = None
     n0 = ops.launch_count()
-    if not args.eager:
+    if not eager:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            for i in range(args.steps):
+            for _ in range(steps):
                 step()
-        launches = ops.launch_count() - n0
+        launches_per_graph = ops.launch_count() - n0
         graph_ev = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph_ev):
             stream = torch.cuda.current_stream()
-            for i in range(args.steps):
+            for i in range(steps):
                 step(i)
         stream = torch.cuda.current_stream()
-        graph.replay()            # one untimed replay
+        # one untimed replay, timed to size the region
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
         torch.cuda.synchronize()
+        one = a.elapsed_time(b) / 1e3
+        replays = max(1, math.ceil(1.1 * min_seconds / max(one, 1e-6)))
+        replays = int(replicas.max_over_ranks(float(replays), device=dev)) if world > 1 else replays
+    else:
+        replays = 1
 
-    sampler = ClockSampler(local) if rank == 0 else None
+    sampler = ClockSampler(local) if (sample_clocks and rank == 0) else None
     if sampler:
         sampler.start()
         time.sleep(0.3)
@@ -235,15 +254,15 @@ def run_ours(args, rank, world, local):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     if graph is not None:
-        graph.replay()
+        for _ in range(replays):
+            graph.replay()
     else:
         n0 = ops.launch_count()
-        for i in range(args.steps):
+        for _ in range(steps):
             step()
     t1.record(stream)
     torch.cuda.synchronize()
-    if graph is None:
-        launches = ops.launch_count() - n0
+    launches = (launches_per_graph * replays) if graph is not None else ops.launch_count() - n0
     elapsed = t0.elapsed_time(t1) / 1e3
     elapsed = replicas.max_over_ranks(elapsed, device=dev)
     if world > 1:
@@ -254,92 +273,74 @@ def run_ours(args, rank, world, local):
     if graph_ev is not None:
         graph_ev.replay()
     else:
-        for i in range(args.steps):
+        for i in range(steps):
             step(i)
     torch.cuda.synchronize()
+    idx_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    topk_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    att_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
 
-    idx_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    topk_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    att_ms = [e[2].elapsed_time(e[3]) for e in ev]
-
-    # ---- roofline of the dominant kernel: the indexer (HBM-bound in decode,
-    # tensor-bound in chunked prefill, where 8 queries share each key tile)
+    # ---- algorithmic bytes / flops and rooflines
     peaks, peak_src = load_peaks()
     q_pos = wl.q_pos.to("cpu").numpy().astype(np.int64)
     n_scored = int((q_pos + 1).sum())
-    idx_bytes = acc.indexer_bytes(n_scored, T, T * ld, fp8=args.fp8_keys)
-    idx_kernel = "indexer_fp8" if args.fp8_keys else "indexer"
-    idx_name = "indexer_kernel<{},{}>".format(q_group, "fp8" if args.fp8_keys else "bf16")
-    idx_dur = statistics.mean(idx_ms) / 1e3
+    idx_bytes = acc.indexer_bytes(n_scored, T, T * ld, fp8=fp8)
+    n_rows_att = int(np.minimum(q_pos + 1, k).sum())
+    att_bytes = sum(acc.attend_bytes(n_rows_att, T, L.d_rope) for L in wl.layers)
+    step_bytes = idx_bytes + acc.topk_bytes(n_scored, T, k) + att_bytes
+    timed_steps = steps * replays
+    step_s = elapsed / timed_steps
+    idx_name = "indexer_kernel<{},{}>".format(q_group, "fp8" if fp8 else "bf16")
+    idx_kernel = "indexer_fp8" if fp8 else "indexer"
+    res = {
+        "config": case.name, "T": T, "n_layers": n_layers, "ld": ld, "steps": steps, "graph_replays": replays,
+        "timed_steps": timed_steps, "timed_region_s": round(elapsed, 4), "ms_per_step": round(step_s * 1e3, 4),
+        "queries_per_s": T * world / step_s, "query_layers_per_s": T * n_layers * world / step_s,
+        "launches": launches, "clocks": clocks,
+        "kernel_ms": {"indexer": round(idx_ms, 4), "topk": round(topk_ms, 4),
+                      "attention_all_layers": round(att_ms, 4)},
+        "step_hbm": {"algorithmic_bytes": step_bytes, "achieved_tbs": round(step_bytes / step_s / 1e12, 3),
+                     "frac_of_measured_copy": round(step_bytes / step_s / 1e9 / peaks["hbm_gbs"], 4),
+                     "frac_of_8tbs": round(step_bytes / step_s / 8e12, 4)},
+        "attention_hbm": {"algorithmic_bytes": att_bytes,
+                          "achieved_tbs": round(att_bytes / (att_ms / 1e3) / 1e12, 3),
+                          "frac_of_measured_copy": round(att_bytes / (att_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)},
+    }
+    idx_dur = idx_ms / 1e3
     if q_group == 1:
-        achieved_gbs = idx_bytes / idx_dur / 1e9
-        roofline = {"kernel": idx_name, "bound": "hbm",
-                    "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(achieved_gbs / peaks["hbm_gbs"], 4), "peak_source": f"{peak_src} hbm_gbs",
-                    "traffic": profiled_traffic(idx_kernel, args.config),
-                    "algorithmic_bytes_per_launch": idx_bytes, "avg_launch_ms": round(idx_dur * 1e3, 4)}
+        achieved = idx_bytes / idx_dur / 1e9
+        res["roofline"] = {"kernel": idx_name, "bound": "hbm", "achieved": round(achieved, 1),
+                           "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                           "peak_source": f"{peak_src} hbm_gbs", "traffic": profiled_traffic(idx_kernel, case.name),
+                           "algorithmic_bytes_per_launch": idx_bytes, "avg_launch_ms": round(idx_ms, 4)}
     else:
         flops = acc.indexer_flops(n_scored)
-        achieved_tf = flops / idx_dur / 1e12
+        achieved = flops / idx_dur / 1e12
         # an FP8 contraction is measured against the bf16 peak x 2 (the nominal fp8 : bf16 ratio, 4.5 : 2.25)
-        ratio = 2.0 if args.fp8_keys else 1.0
+        ratio = 2.0 if fp8 else 1.0
         peak_tf = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * ratio
-        roofline = {"kernel": idx_name, "bound": "tensor",
-                    "achieved": round(achieved_tf, 1), "peak": peak_tf, "unit": "TFLOP/s",
-                    "frac": round(achieved_tf / peak_tf, 4),
-                    "frac_of_burst_peak": round(achieved_tf / (peaks["bf16_tflops"] * ratio), 4),
-                    "peak_source": (f"{peak_src} bf16_tflops_sustained" + (" x 2 (nominal fp8:bf16)" if args.fp8_keys
-                                                                          else "")
-                                    + " (kernel timed inside a multi-ms step)"),
-                    "traffic": profiled_traffic(idx_kernel, args.config),
-                    "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": idx_bytes,
-                    "avg_launch_ms": round(idx_dur * 1e3, 4)}
-
-    # whole-step algorithmic bytes (all kernels) and the fraction of HBM peak they imply
-    n_rows_att = int(np.minimum(q_pos + 1, k).sum())
-    step_bytes = idx_bytes + acc.topk_bytes(n_scored, T, k)
-    for L in wl.layers:
-        step_bytes += acc.attend_bytes(n_rows_att, T, L.d_rope)
-
-    # ---- end to end through the C ABI with host buffers
-    # the fused C-ABI call takes bf16 index keys; no end-to-end line in FP8-key mode
-    e2e = run_e2e(args, wl, ld, k, q_group, dev) if not (args.no_e2e or args.fp8_keys) else None
-
-    value = replicas.job_throughput(T, world, args.steps, elapsed)
-    line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "queries/s", "n_gpus": world,
-        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(elapsed / args.steps * 1e3, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded, shapes/distributions of the configuration)",
-        "config": {"workload": args.config + ("+fp8_index_keys" if args.fp8_keys else ""),
-                   "queries_per_gpu": T, "context": list(case.seq_lengths)[:1],
-                   "layers": [("rope" if L.d_rope else "nope") for L in wl.layers], "topk": k,
-                   "parallelism": f"replicas{world}" if world > 1 else "1gpu",
-                   "l2": f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB per step)"},
-        "step_hbm": {"algorithmic_bytes": step_bytes,
-                     "achieved_tbs": round(step_bytes / (elapsed / args.steps) / 1e12, 3),
-                     "frac_of_measured_copy": round(step_bytes / (elapsed / args.steps) / 1e9 / peaks["hbm_gbs"], 4),
-                     "frac_of_8tbs": round(step_bytes / (elapsed / args.steps) / 8e12, 4)},
-        "kernel_ms": {"indexer": round(statistics.mean(idx_ms), 4), "topk": round(statistics.mean(topk_ms), 4),
-                      "attention_all_layers": round(statistics.mean(att_ms), 4)},
-        "roofline": roofline, "gpu_launches": launches, "clocks": clocks, "e2e": e2e,
-        "timing": ("CUDA graph of the timed steps, one replay; kernel_ms from a second graph of the same "
-                   "steps with events around each kernel" if graph is not None else "eager launches"),
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.config, budget_s=args.cpu_seconds)
-    if world > 1:
-        torch.distributed.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+        res["roofline"] = {"kernel": idx_name, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak_tf,
+                           "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
+                           "frac_of_burst_peak": round(achieved / (peaks["bf16_tflops"] * ratio), 4),
+                           "peak_source": (f"{peak_src} bf16_tflops_sustained"
+                                           + (" x 2 (nominal fp8:bf16)" if fp8 else "")
+                                           + " (kernel timed inside a multi-ms step)"),
+                           "traffic": profiled_traffic(idx_kernel, case.name),
+                           "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": idx_bytes,
+                           "avg_launch_ms": round(idx_ms, 4)}
+    if e2e and not fp8:
+        res["e2e"] = run_e2e(wl, ld, k, q_group, dev, e2e_steps)
+    del graph, graph_ev
+    return res
 
 
-def run_e2e(args, wl, ld, k, q_group, dev):
+def run_e2e(wl, ld, k, q_group, dev, steps):
     """Same metric through dsa_sparse_mla_forward with pinned host inputs/outputs:
     each step copies the step's queries host->device and the outputs back."""
     from sparse_attention_16_b200 import ops
 
     T = wl.T
+    n_layers = len(wl.layers)
     host_in = {"q_idx": wl.q_idx, "w": wl.w, "q_seq": wl.q_seq, "q_pos": wl.q_pos}
     for i, L in enumerate(wl.layers):
         host_in[f"q_nope{i}"] = L.q_nope
@@ -350,7 +351,7 @@ def run_e2e(args, wl, ld, k, q_group, dev):
     dev_in = {n: torch.empty_like(t) for n, t in host_in.items()}
     outs = [torch.empty((T, 64, 512), dtype=torch.bfloat16, device=dev) for _ in wl.layers]
     host_out = [torch.empty((T, 64, 512), dtype=torch.bfloat16).pin_memory() for _ in wl.layers]
-    ws = ops.workspace(ops.forward_workspace_bytes(T, ld, k, q_group), dev)
+    ws = ops.workspace(ops.forward_workspace_bytes(T, ld, k, q_group, n_layers), dev)
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out)
 
@@ -371,21 +372,83 @@ def run_e2e(args, wl, ld, k, q_group, dev):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(s)
-    for _ in range(args.steps):
+    for _ in range(steps):
         step()
     t1.record(s)
     torch.cuda.synchronize()
     el = t0.elapsed_time(t1) / 1e3
-    return {"value": round(T * args.steps / el, 1), "unit": "queries/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": round(el / args.steps * 1e3, 4),
-            "api": "dsa_sparse_mla_forward"}
+    return {"value": round(T * n_layers * steps / el, 1), "unit": "query-layers/s", "queries_per_s": round(T * steps / el, 1),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(el / steps * 1e3, 4),
+            "steps": steps, "api": "dsa_sparse_mla_forward"}
+
+
+def run_ours(args, rank, world, local):
+    from sparse_attention_16_b200 import ops
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    ops.load_library()
+    head = measure(args.config, dev, args.steps, args.warmup, rank, world, local, min_seconds=args.min_seconds,
+                   sample_clocks=True, fp8=args.fp8_keys, eager=args.eager, e2e=not args.no_e2e)
+    torch.cuda.empty_cache()
+    case = CONFIGS[args.config]
+    wl_T = head["T"]
+    line = {
+        "metric": METRIC, "value": round(head["query_layers_per_s"], 1), "unit": "query-layers/s",
+        "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded, shapes/distributions of the configuration)",
+        "config": {"workload": args.config + ("+fp8_index_keys" if args.fp8_keys else ""),
+                   "queries_per_gpu": wl_T, "context": list(case.seq_lengths)[:1],
+                   "layers": [("rope" if d else "nope") for d in case.layers], "topk": case.topk,
+                   "parallelism": f"replicas{world}" if world > 1 else "1gpu",
+                   "l2": f"inputs larger than L2 ({head['step_hbm']['algorithmic_bytes'] / 1e6:.0f} MB per step)"},
+        "queries_per_s": round(head["queries_per_s"], 1),
+        "timing": {"graph_steps": args.steps, "graph_replays": head["graph_replays"],
+                   "timed_steps": head["timed_steps"], "timed_region_s": head["timed_region_s"],
+                   "how": ("CUDA graph of the K steps replayed R times inside one event-timed region; "
+                           "kernel_ms from a second graph of the same steps with events around each kernel")},
+        "step_hbm": head["step_hbm"], "attention_hbm": head["attention_hbm"], "kernel_ms": head["kernel_ms"],
+        "roofline": head["roofline"], "gpu_launches": head["launches"], "clocks": head["clocks"],
+        "e2e": head.get("e2e"),
+    }
+    if world == 1 and not args.no_extras:
+        extras = {}
+        for name in EXTRAS:
+            if name == args.config:
+                continue
+            r = measure(name, dev, 3 if CONFIGS[name].kind == "prefill" else args.steps, 3, rank, world, local,
+                        min_seconds=0.0 if CONFIGS[name].kind == "prefill" else 0.3, fp8=args.fp8_keys)
+            torch.cuda.empty_cache()
+            keep = ("ms_per_step", "queries_per_s", "query_layers_per_s", "kernel_ms", "step_hbm", "attention_hbm",
+                    "roofline", "timed_steps")
+            extras[name] = {k_: (round(v, 4) if isinstance(v, float) else v) for k_, v in r.items() if k_ in keep}
+        line["extra_configs"] = extras
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.config, budget_s=args.cpu_seconds)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 # --------------------------------------------------------------------------- oracle (CPU) arm
 
-def _oracle_sample_workload(config, n_queries):
+SAMPLE_CACHE_LIMIT = 1 << 30   # host bytes of latent cache beyond which the sample draws only the selected rows
+
+
+def _oracle_sample(config, n_queries):
     """A bounded slice of the configuration: ``n_queries`` sequences (or prefill
-    queries) of the same shape and distributions, drawn on the CPU."""
+    queries) of the same shape and distributions, drawn on the CPU.  Returns
+    (indexer workload, attention workload or None).  When the sequences' latent
+    caches would exceed SAMPLE_CACHE_LIMIT (the 2^20-position configuration:
+    4.7 GB per sequence), the attention side is drawn as `topk` rows per query
+    and layer (iid rows of the same distribution) that stand for the selected
+    positions: the oracle does the same arithmetic on them."""
     case = CONFIGS[config]
     if case.kind == "decode":
         sub = small_case(config + "_sample", case.lengths[:n_queries], layers=case.layers, qmul=case.qmul,
@@ -394,17 +457,37 @@ def _oracle_sample_workload(config, n_queries):
         sub = small_case(config + "_sample", kind="prefill", cached=case.cached + case.new - n_queries,
                          new=n_queries, layers=case.layers, qmul=case.qmul, mla_q_std=case.mla_q_std,
                          seed=case.seed)
-    return make_workload(sub, "cpu")
+    cache_bytes = sum(sub.seq_lengths) * sum(512 + d for d in case.layers) * 2
+    if cache_bytes <= SAMPLE_CACHE_LIMIT:
+        return make_workload(sub, "cpu"), None
+    idx_part = make_workload(dataclasses.replace(sub, layers=()), "cpu")
+    att_part = make_workload(small_case(config + "_rows", (case.topk,) * idx_part.T, layers=case.layers,
+                                        qmul=case.qmul, mla_q_std=case.mla_q_std, seed=case.seed + 1), "cpu")
+    return idx_part, att_part
 
 
-def _oracle_step(wl):
+def _oracle_step(sample):
     import oracle
     from sparse_attention_16_b200.workloads import SOFTMAX_SCALE, to_numpy
 
-    layers = [dict(q_nope=to_numpy(L.q_nope), q_pe=None if L.q_pe is None else to_numpy(L.q_pe),
-                   qmul=to_numpy(L.qmul), cache=to_numpy(L.cache), d_rope=L.d_rope) for L in wl.layers]
-    return oracle.forward(to_numpy(wl.q_idx), to_numpy(wl.w), to_numpy(wl.k_idx), to_numpy(wl.seq_row_start),
-                          to_numpy(wl.q_seq), to_numpy(wl.q_pos), layers, SOFTMAX_SCALE, k=wl.case.topk)
+    wl, att = sample
+    if att is None:
+        layers = [dict(q_nope=to_numpy(L.q_nope), q_pe=None if L.q_pe is None else to_numpy(L.q_pe),
+                       qmul=to_numpy(L.qmul), cache=to_numpy(L.cache), d_rope=L.d_rope) for L in wl.layers]
+        return oracle.forward(to_numpy(wl.q_idx), to_numpy(wl.w), to_numpy(wl.k_idx), to_numpy(wl.seq_row_start),
+                              to_numpy(wl.q_seq), to_numpy(wl.q_pos), layers, SOFTMAX_SCALE, k=wl.case.topk)
+    q_pos = to_numpy(wl.q_pos)
+    scores = oracle.index_scores(to_numpy(wl.q_idx), to_numpy(wl.w), to_numpy(wl.k_idx), to_numpy(wl.seq_row_start),
+                                 to_numpy(wl.q_seq), q_pos, int(q_pos.max()) + 1)
+    idx, count = oracle.topk_select(scores, q_pos, wl.case.topk)
+    # the i-th selected position of query t is row i of its drawn rows
+    local = np.where(idx >= 0, np.arange(idx.shape[1])[None, :], -1).astype(np.int32)
+    outs = []
+    for L in att.layers:
+        outs.append(oracle.sparse_mla(to_numpy(L.q_nope), None if L.q_pe is None else to_numpy(L.q_pe),
+                                      to_numpy(L.qmul), SOFTMAX_SCALE, to_numpy(L.cache), L.d_rope,
+                                      to_numpy(att.seq_row_start), to_numpy(att.q_seq), local, count))
+    return idx, count, outs
 
 
 def _threads_used():
@@ -417,42 +500,71 @@ def _threads_used():
 
 
 def cpu_baseline(config, budget_s=20.0, n_queries=1):
-    wl = _oracle_sample_workload(config, n_queries)
+    sample = _oracle_sample(config, n_queries)
+    n_layers = len(CONFIGS[config].layers)
     t = time.perf_counter()
     reps = 0
     while True:
-        _oracle_step(wl)
+        _oracle_step(sample)
         reps += 1
         if time.perf_counter() - t > budget_s or reps >= 50:
             break
     el = time.perf_counter() - t
-    return {"value": round(reps * wl.T / el, 4), "unit": "queries/s", "cores": _threads_used(), "kind": "oracle",
-            "sample": f"{reps} x {wl.T} queries of {config} (same shape, CPU-drawn), fp64 numpy oracle"}
+    T = sample[0].T
+    how = "attention rows drawn at the selected positions only" if sample[1] is not None else "full caches"
+    return {"value": round(reps * T * n_layers / el, 4), "unit": "query-layers/s",
+            "queries_per_s": round(reps * T / el, 4), "cores": _threads_used(), "kind": "oracle",
+            "sample": f"{reps} x {T} queries of {config} (same shape, CPU-drawn, {how}), fp64 numpy oracle"}
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    wl = _oracle_sample_workload(args.config, 1)
+    sample = _oracle_sample(args.config, 1)
+    n_layers = len(CONFIGS[args.config].layers)
     for _ in range(args.warmup):
-        _oracle_step(wl)
+        _oracle_step(sample)
     t = time.perf_counter()
     for _ in range(args.steps):
-        _oracle_step(wl)
+        _oracle_step(sample)
     el = time.perf_counter() - t
-    value = args.steps * wl.T / el
+    T = sample[0].T
+    value = args.steps * T * n_layers / el
     cores = _threads_used()
-    sample = f"each step = {wl.T} query of {args.config} (same shape), fp64 numpy oracle on host cores"
-    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "queries/s",
+    how = "attention rows drawn at the selected positions only" if sample[1] is not None else "full caches"
+    desc = f"each step = {T} query of {args.config} (same shape, {how}), fp64 numpy oracle on host cores"
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "query-layers/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.config},
-            "cpu_baseline": {"value": round(value, 4), "unit": "queries/s", "cores": cores, "kind": "oracle",
-                             "sample": sample},
-            "e2e": {"value": round(value, 4), "unit": "queries/s", "h2d_bytes_per_step": 0,
+            "cpu_baseline": {"value": round(value, 4), "unit": "query-layers/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(value, 4), "unit": "query-layers/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- launcher
+
+def _spawned_rank(local, world, port, argv):
+    os.environ.update(RANK=str(local), LOCAL_RANK=str(local), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
+                      MASTER_PORT=str(port), LOCAL_WORLD_SIZE=str(world))
+    sys.argv = [sys.argv[0]] + argv
+    main()
+
+
+def spawn_ranks(n, argv):
+    """`--gpus N` without torchrun: one process per GPU (spawn), ranks 0..N-1 on
+    this node, rendezvous on 127.0.0.1.  Rank 0 prints the JSON line."""
+    import socket
+
+    import torch.multiprocessing as mp
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    mp.start_processes(_spawned_rank, args=(n, port, argv), nprocs=n, start_method="spawn")
 
 
 def main():
@@ -462,7 +574,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default=HEADLINE, choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--min-seconds", type=float, default=1.0, help="shortest timed region (graph replays)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--eager", action="store_true", help="launch every step from the host instead of a CUDA graph")
@@ -471,6 +585,9 @@ def main():
                          "the selection and attention are unchanged")
     args = ap.parse_args()
     rank, world, local = dist_env()
+    if args.gpus > 1 and "RANK" not in os.environ:
+        spawn_ranks(args.gpus, sys.argv[1:])
+        return
     if args.impl == "reference":
         run_reference(args, rank, world)
         return

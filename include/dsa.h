@@ -61,7 +61,8 @@ typedef enum dsa_status {
 } dsa_status_t;
 
 /* Device error word bits (returned through dsa_check_errors' out argument). */
-#define DSA_DEVERR_BAD_INDEX    0x1u  /* a selected position outside its sequence's rows */
+#define DSA_DEVERR_BAD_INDEX    0x1u  /* a selected position < 0 (other than -1 padding), past q_pos
+                                         when q_pos is given, or outside the cache; or count < 0 or > k */
 #define DSA_DEVERR_BAD_SEQ      0x2u  /* q_seq out of range or q_pos >= ld               */
 #define DSA_DEVERR_MIXED_GROUP  0x4u  /* q_group > 1 but a group spans several sequences */
 #define DSA_DEVERR_TIMEOUT      0x8u  /* a pipeline barrier wait hit its iteration limit */
@@ -153,6 +154,11 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, int
  *   cache  bf16 [n_rows, ld_c] rows [c_s (512) | kR_s (d_rope)]; ld_c >= 512 + d_rope,
  *                              ld_c % 8 == 0;  d_rope in {0, 64}
  *   seq_row_start int64 [B], q_seq int32 [T]; B >= 1
+ *   q_pos  int32 [T] or NULL   when given, a selected position s of query t is
+ *                              used only if s <= q_pos[t] (the causal bound:
+ *                              decode q_pos = L - 1); a position past it is
+ *                              skipped and flagged DSA_DEVERR_BAD_INDEX.  With
+ *                              NULL only the cache bound is checked.
  *   idx    int32 [T, k] positions (ascending or not; -1 entries are skipped),
  *   count  int32 [T]    number of leading idx entries to use (<= k)
  *   out    bf16 [T, 64, 512]   o[t,h] = sum_i p_i c_{s_i}   (round to nearest even)
@@ -164,13 +170,14 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, int
  *              a thread-block cluster and merge their partials in distributed
  *              shared memory (used when every cluster of the call can be
  *              resident at once); otherwise it holds the fp32 split partials.
+ *              dsa_plan_attend tells which case a batch size falls in.
  */
 size_t sparse_mla_workspace_size(int32_t T, int32_t k);
 dsa_status_t sparse_mla_attend(const void* q_nope, const void* q_pe, const float* qmul,
                                float softmax_scale, const void* cache, int64_t n_rows,
                                int32_t ld_c, int32_t d_rope, const int64_t* seq_row_start,
-                               int32_t B, const int32_t* q_seq, const int32_t* idx,
-                               const int32_t* count,
+                               int32_t B, const int32_t* q_seq, const int32_t* q_pos,
+                               const int32_t* idx, const int32_t* count,
                                int32_t T, int32_t k, void* out, float* lse, void* workspace,
                                size_t ws_bytes, void* stream);
 
@@ -195,10 +202,13 @@ dsa_status_t sparse_mla_attend(const void* q_nope, const void* q_pe, const float
  *     (n_split of 2-8 with every cluster resident: no scratch; n_split = 1 once
  *     T reaches the SM count: no scratch).  Calls needing more than
  *     DSA_NOALLOC_MAX_PARTIALS return DSA_ERR_WORKSPACE with a message that
- *     states the limit.
- *   - Set-up: the first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current.  Make that first call
- *     before any stream capture.
+ *     states the limit.  The need is not monotone in T: a smaller batch splits
+ *     each query wider, so retrying with fewer queries can be refused again;
+ *     dsa_plan_attend(T, 1, k, NULL, &plan) predicts it (plan.workspace_bytes
+ *     > 0 means T x plan.n_split partials are needed).
+ *   - Set-up: the first call on each device (and again after a device reset)
+ *     looks up the array's device address (cudaGetSymbolAddress) with that
+ *     device current.  Make that first call before any stream capture.
  *   - Sharing: all calls on a device use the same array, which keeps the last
  *     call's contents.  Each call overwrites every entry it reads, so nothing
  *     needs clearing, but calls that overlap on the GPU (other streams, other
@@ -208,9 +218,9 @@ dsa_status_t sparse_mla_attend(const void* q_nope, const void* q_pe, const float
 dsa_status_t sparse_mla_attend_noalloc(const void* q_nope, const void* q_pe, const float* qmul,
                                        float softmax_scale, const void* cache, int64_t n_rows,
                                        int32_t ld_c, int32_t d_rope, const int64_t* seq_row_start,
-                                       int32_t B, const int32_t* q_seq, const int32_t* idx,
-                                       const int32_t* count, int32_t T, int32_t k, void* out,
-                                       float* lse, void* stream);
+                                       int32_t B, const int32_t* q_seq, const int32_t* q_pos,
+                                       const int32_t* idx, const int32_t* count, int32_t T, int32_t k,
+                                       void* out, float* lse, void* stream);
 
 /* One attention layer fed by a shared selection (fields as in sparse_mla_attend). */
 typedef struct dsa_layer_args {
@@ -225,19 +235,41 @@ typedef struct dsa_layer_args {
 } dsa_layer_args;
 
 /*
+ * sparse_mla_attend_layers - sparse_mla_attend for several layers that share
+ * one selection.  Concept page bullet "28 layers reuse the selection made by
+ * the most recent layer that ran its indexer": every layer in `layers` (host
+ * array of n_layers entries, device pointers inside; RoPE and NoPE layers may
+ * be mixed) attends over idx / count.  Up to 8 layers run in one launch whose
+ * work units are layers x queries x splits, so a small decode batch still
+ * fills the GPU.  The remaining arguments are those of sparse_mla_attend;
+ * workspace: sparse_mla_layers_workspace_size(T, n_layers, k) bytes, 256-byte
+ * aligned (may be NULL when that size is 0).
+ */
+size_t sparse_mla_layers_workspace_size(int32_t T, int32_t n_layers, int32_t k);
+dsa_status_t sparse_mla_attend_layers(int32_t n_layers, const dsa_layer_args* layers, float softmax_scale,
+                                      int64_t n_rows, const int64_t* seq_row_start, int32_t B,
+                                      const int32_t* q_seq, const int32_t* q_pos, const int32_t* idx,
+                                      const int32_t* count, int32_t T, int32_t k, void* workspace,
+                                      size_t ws_bytes, void* stream);
+
+/*
  * dsa_sparse_mla_forward - one selection reused by several layers.
  * Concept page bullet "28 layers reuse the selection made by the most recent
  * layer that ran its indexer": the indexer and top-k run once, then every
  * layer in `layers` (host array of n_layers entries, device pointers inside)
- * attends over that selection.  Queries are processed in chunks so that the
- * fp32 score rows fit the workspace (chunked prefill).
+ * attends over that selection.  Up to 8 layers run in one attention launch
+ * (work units = layers x queries x splits), so a small decode batch still
+ * fills the GPU; RoPE and NoPE layers may be mixed.  Queries are processed in
+ * chunks so that the fp32 score rows fit the workspace (chunked prefill);
+ * every chunk, the last one included, stays inside the workspace.
  *
  *   idx_out / count_out: optional [T, k] / [T] copies of the selection (NULL = not needed).
- *   workspace: at least dsa_forward_workspace_size(T, ld, k, q_group) bytes for
- *   one pass over all queries; a smaller workspace (>= the size for q_group
- *   queries) makes the call process queries in chunks.
+ *   workspace: at least dsa_forward_workspace_size(T, ld, k, q_group, n_layers)
+ *   bytes for one pass over all queries; a smaller workspace (>= the size for
+ *   q_group queries) makes the call process queries in chunks
+ *   (dsa_plan_forward shows the chunking and the workspace layout).
  */
-size_t dsa_forward_workspace_size(int32_t T, int64_t ld, int32_t k, int32_t q_group);
+size_t dsa_forward_workspace_size(int32_t T, int64_t ld, int32_t k, int32_t q_group, int32_t n_layers);
 dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const void* k_idx,
                                     int64_t n_rows, const int64_t* seq_row_start, int32_t B,
                                     const int32_t* q_seq, const int32_t* q_pos, int32_t T,
@@ -245,6 +277,73 @@ dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const voi
                                     const dsa_layer_args* layers, float softmax_scale,
                                     int32_t k, int32_t* idx_out, int32_t* count_out,
                                     void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Launch planning queries (host only: no device work, no allocation).  They
+ * return what the calls above will do, from the current device's properties or
+ * from `props` when it is non-NULL (then they work without a GPU).
+ *
+ * dsa_get_device_props: SM count of the current device and, for c = 2..8, how
+ * many clusters of c attention blocks it can keep resident at once.
+ *
+ * dsa_plan_attend: how sparse_mla_attend (n_layers = 1) or one attention
+ * launch of dsa_sparse_mla_forward (n_layers <= 8 layers) splits T queries:
+ * n_split blocks per (layer, query) of rows_per_split selected rows each;
+ * merge = 1 when those blocks form a cluster and merge on chip; and
+ * workspace_bytes, the split partials that otherwise go through the workspace.
+ *
+ * dsa_plan_forward: how dsa_sparse_mla_forward cuts T queries into chunks for
+ * a workspace of ws_bytes, and where each region sits in it (byte offsets;
+ * SIZE_MAX for idx / count regions replaced by the caller's idx_out /
+ * count_out, i.e. has_idx_out / has_count_out != 0).  Returns
+ * DSA_ERR_WORKSPACE (chunk = 0) when even q_group queries do not fit.
+ */
+typedef struct dsa_device_props {
+  int32_t sms;                 /* streaming multiprocessors                              */
+  int32_t max_clusters[9];     /* [c], c = 2..8: resident clusters of c attention blocks */
+} dsa_device_props;
+
+typedef struct dsa_attend_plan {
+  int32_t n_split;             /* blocks per (layer, query)                        */
+  int32_t rows_per_split;      /* selected rows per block (a multiple of 64)       */
+  int32_t merge;               /* 1: the blocks of a (layer, query) merge on chip  */
+  int32_t reserved;
+  size_t workspace_bytes;      /* split partials in the workspace (0: none)        */
+} dsa_attend_plan;
+
+typedef struct dsa_forward_plan {
+  int32_t chunk;               /* queries per chunk (a multiple of q_group, or T) */
+  int32_t n_chunks;
+  int32_t last_chunk;          /* queries in the final chunk                      */
+  int32_t reserved;
+  size_t idx_offset;           /* [chunk, k] int32 selection (SIZE_MAX: idx_out)  */
+  size_t count_offset;         /* [chunk] int32 counts (SIZE_MAX: count_out)      */
+  size_t attend_offset;        /* attention split partials                        */
+  size_t attend_bytes;         /* the largest need of any chunk's launches        */
+  size_t scores_offset;        /* [chunk, ld] f32 scores                          */
+  size_t end;                  /* bytes used (<= ws_bytes)                        */
+} dsa_forward_plan;
+
+dsa_status_t dsa_get_device_props(dsa_device_props* out);
+dsa_status_t dsa_plan_attend(int32_t T, int32_t n_layers, int32_t k, const dsa_device_props* props,
+                             dsa_attend_plan* out);
+dsa_status_t dsa_plan_forward(int32_t T, int64_t ld, int32_t k, int32_t q_group, int32_t n_layers,
+                              int32_t has_idx_out, int32_t has_count_out, size_t ws_bytes,
+                              const dsa_device_props* props, dsa_forward_plan* out);
+
+/*
+ * dsa_set_fault_test - testing hook for the failure-detection path of the
+ * attention kernel (process-wide; affects later launches only).  The pages have
+ * no counterpart to it.
+ *   wait_limit_ns  limit of the kernel's pipeline waits (0: the default, 4 s)
+ *   stall_tile     >= 0: every block skips gathering that 64-row tile, so the
+ *                  wait for it runs out after wait_limit_ns; the kernel then
+ *                  unwinds (copies drained, MMAs completed, tensor memory
+ *                  freed), sets DSA_DEVERR_TIMEOUT and returns, leaving the
+ *                  outputs of the affected queries undefined.  -1: off.
+ * A call after dsa_set_fault_test(0, -1) behaves normally again.
+ */
+dsa_status_t dsa_set_fault_test(uint64_t wait_limit_ns, int32_t stall_tile);
 
 /*
  * dsa_check_errors - synchronizes `stream`, returns DSA_ERR_DEVICE_CHECK (or
@@ -264,7 +363,7 @@ uint64_t dsa_launch_count(void);
 /* Text of the last failure reported on the calling thread ("" if none). */
 const char* dsa_last_error(void);
 
-/* ABI version of this library (major * 100 + minor). */
+/* ABI version of this library (major * 100 + minor): 200. */
 int32_t dsa_version(void);
 
 #ifdef __cplusplus

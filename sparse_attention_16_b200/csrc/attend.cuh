@@ -1,11 +1,15 @@
-// attend.cuh - absorbed MLA over the selected rows of a latent cache (sm_100a).
+// attend.cuh - absorbed MLA over the selected rows of latent caches (sm_100a).
 //
-// For query t and head h (concept page "What to keep", "Sparse attention",
-// "Query scaling"):
+// For query t, head h and layer l (concept page "What to keep", "Sparse
+// attention", "Query scaling"):
 //   z[h,i] = (q_nope[t,h] . c_{s_i} + q_pe[t,h] . kR_{s_i}) * scale * m[t,h]
 //   o[t,h] = sum_i softmax_i(z[h]) c_{s_i}
 // Every gathered 1,152-byte row (1,024 on NoPE layers) is read once and used by
-// all 64 heads.
+// all 64 heads.  One launch covers up to kMaxAttLayers layers that share one
+// selection (the concept page's bullet on layers reusing the selection of the
+// most recent layer that ran its indexer), so a small decode batch still fills
+// the GPU: the work units are (layer, query, split).  RoPE (576-wide rows) and
+// NoPE (512-wide) layers may be mixed in one launch.
 //
 // Heads are the M dimension of both tensor-core products, so each head's
 // softmax state lives in one pair of threads.  Tensor memory (512 columns x
@@ -13,20 +17,20 @@
 // [64 heads x 576] (bf16, two per column) and two logit buffers S [64 heads x
 // 64 rows] (f32), and in lanes 16-31 the output O [64 heads x 512] (f32).  That
 // leaves shared memory for three 64-row tile buffers (3 x 72 KB), so two tiles
-// are in flight while a third is computed on.  Q arrives by TMA in the third
-// tile buffer (free until tile 2) and is moved to TMEM by the softmax warps.
+// are in flight while a third is computed on.  Q is gathered into the third
+// tile buffer (free until tile 2) and moved to TMEM by the softmax warps.
 //
-// Work unit = (query t, split j) = rows [j*R, min(count, (j+1)*R)) of idx[t].
-// Per 64-row tile i (buffer i % 3):
+// Work unit = (pair = layer * T + t, split j) = rows [j*R, min(count, (j+1)*R))
+// of idx[t].  Per 64-row tile i (buffer i % 3):
 //   producer warps 5-7  gather the rows with 16-byte cp.async into a
 //                       chunk-major tile: chunk c (64 columns) = 64 rows x 128 B
 //                       in the 128-byte-swizzled layout (K-major for the
 //                       logits, MN-major for the output product).  The copies
 //                       of a row are issued back to back (a warp covers four
-//                       whole rows in 9 instructions), so each row reaches the
-//                       memory system as one 1,152-byte request stream.
+//                       whole rows in KCH instructions), so each row reaches
+//                       the memory system as one request stream.
 //   warp 4              TMEM owner; one thread issues
-//                         S = Q . C^T   M = 64 heads, N = 64 rows, K = 576, Q read from TMEM
+//                         S = Q . C^T   M = 64 heads, N = 64 rows, K = 576 | 512, Q read from TMEM
 //                         O += P . C    M = 64 heads, N = 2 x 256 columns, K = 64 rows
 //                       in order of readiness (S of the next tile usually runs
 //                       while the softmax of this one does)
@@ -40,8 +44,12 @@
 // split over 2-8 CTAs, those CTAs form a thread-block cluster: each stages its
 // unnormalised O and per-head (max, sum) in its own shared memory, and rank r
 // merges columns [r 512 / n, (r + 1) 512 / n) of all heads from every CTA
-// through distributed shared memory.  Larger splits write fp32 partials that a
-// small combine kernel merges.
+// through distributed shared memory.  Otherwise the splits write fp32 partials
+// that a small combine kernel merges.
+//
+// A selected position is used only if it lies in [0, q_pos[t]] (when q_pos is
+// given) and inside the cache; anything else except the -1 padding is skipped
+// and flagged (kErrBadIndex).
 #pragma once
 
 #include <cuda.h>
@@ -49,6 +57,7 @@
 
 #include <cooperative_groups.h>
 
+#include <climits>
 #include <cstddef>
 
 #include "ptx.cuh"
@@ -57,14 +66,15 @@ namespace dsa {
 
 constexpr int kHeads = 64;
 constexpr int kLatent = 512;
+constexpr int kMaxAttLayers = 8;   // layers per attention launch
+constexpr int kMaxSplits = 32;     // CTAs per (layer, query)
 
-template <int DR>
 struct AttCfg {
-  static constexpr int KCH = (kLatent + DR) / 64;        // 64-column chunks: 9 or 8
+  static constexpr int KCH_MAX = 9;                      // 64-column chunks of a RoPE row (NoPE: 8)
   static constexpr int ROWS = 64;                        // rows per tile (N of the logit MMA)
   static constexpr int NBUF = 3;                         // tile buffers
   static constexpr int CHUNK_BYTES = ROWS * 128;         // 8 KB: 64 rows x 64 columns
-  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;   // 72 KB (RoPE) / 64 KB (NoPE)
+  static constexpr int TILE_BYTES = KCH_MAX * CHUNK_BYTES;   // 72 KB per buffer
   static constexpr int P_BYTES = kHeads * 128;           // P: 64 heads x 64 rows bf16
   static constexpr int DATA_BYTES = NBUF * TILE_BYTES + P_BYTES;
   static constexpr int SCRATCH_BYTES = 1024;
@@ -73,41 +83,53 @@ struct AttCfg {
   static constexpr int PRODUCERS = 96;                   // warps 5-7
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t Q_COL = 0;                   // lanes 0-15: Q, KCH x 32 columns
-  static constexpr uint32_t S_COL = KCH * 32;            // lanes 0-15: S buffer b at S_COL + 64 b
+  static constexpr uint32_t S_COL = KCH_MAX * 32;        // lanes 0-15: S buffer b at S_COL + 64 b
   static constexpr uint32_t O_LANE = 16;                 // lanes 16-31: O, 512 columns
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(kHeads, ROWS, 0, 0);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(kHeads, 256, 0, 1);
   static_assert(S_COL + 2 * ROWS <= TMEM_COLS, "Q and two logit buffers must fit in 512 columns");
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+  static_assert(kHeads == ROWS, "Q is staged as one tile of 64 'rows' (heads)");
+};
+
+// One attention layer of a launch.
+struct AttLayer {
+  const __nv_bfloat16* q_nope;    // [T, 64, 512]
+  const __nv_bfloat16* q_pe;      // [T, 64, 64] (RoPE layers) or null
+  const float* qmul;              // [T, 64]
+  const __nv_bfloat16* cache;     // [n_rows, ld_c]
+  __nv_bfloat16* out;             // [T, 64, 512]
+  float* lse;                     // [T, 64] or null
+  int64_t ld_c;                   // row stride of the cache, elements
+  int32_t d_rope;                 // 64 (RoPE) or 0 (NoPE)
+  int32_t pad_;
 };
 
 struct AttendParams {
-  const __nv_bfloat16* q_nope;    // [T, 64, 512]
-  const __nv_bfloat16* q_pe;      // [T, 64, 64] (RoPE layers)
-  const __nv_bfloat16* cache;     // [n_rows, ld_c]
-  const float* qmul;              // [T, 64]
+  AttLayer layer[kMaxAttLayers];
   const int64_t* seq_row_start;   // [B]
   const int32_t* q_seq;           // [T]
+  const int32_t* q_pos;           // [T] or null: positions beyond q_pos[t] are rejected
   const int32_t* idx;             // [T, k]
   const int32_t* count;           // [T]
-  __nv_bfloat16* out;             // [T, 64, 512]
-  float* lse;                     // [T, 64] or null
-  float* ws_o;                    // [T, n_split, 64, 512] partial numerators (n_split > 1)
-  float* ws_ml;                   // [T, n_split, 64, 4] (max in log2 units, sum of the bf16 weights,
+  float* ws_o;                    // [units, n_split, 64, 512] partial numerators (combine path)
+  float* ws_ml;                   // [units, n_split, 64, 4] (max in log2 units, sum of the bf16 weights,
                                   //  sum of the fp32 weights, unused)
-  int64_t ld_c;
   int64_t n_rows;
+  uint64_t wait_limit_ns;         // limit of the pipeline waits (kWaitLimitNs unless a test lowers it)
   float scale_log2e;              // softmax_scale * log2(e)
+  int32_t n_layers;
   int32_t B;
   int32_t T;
   int32_t k;
   int32_t n_split;
   int32_t rows_per_split;         // multiple of 64
-  int32_t merge;                  // 1: the n_split CTAs of a query are a cluster and merge in DSMEM
+  int32_t merge;                  // 1: the n_split CTAs of a (layer, query) are a cluster and merge in DSMEM
+  int32_t stall_tile;             // testing hook: >= 0 -> that tile is never gathered, so its wait runs out
 };
 
 struct AttScratch {
-  uint64_t q_smem;                // Q has landed in tile buffer 2 (TMA)
+  uint64_t q_smem;                // Q has landed in tile buffer 2 (96 producer arrivals)
   uint64_t q_full;                // Q is in tensor memory (128 arrivals)
   uint64_t s_full[2];             // logits of a tile are in S buffer b
   uint64_t s_free[2];             // S buffer b has been read by the softmax (128 arrivals)
@@ -168,6 +190,11 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c,
+                                             uint32_t& d) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr));
+}
+
 // Merge of a query's split partials inside its cluster (n = p.n_split CTAs,
 // rank = split).  Each CTA has staged O_j[64][512] (unnormalised, fp32, pieces
 // swizzled by h & 7) and (m_j, l_j, lx_j) per head at the start of its shared
@@ -176,8 +203,8 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 //   M = max_j m_j,  w_j = 2^(m_j - M),  L = sum_j w_j l_j,
 //   o[h, c] = sum_j (w_j / L) O_j[h, c],
 //   lse[h] = (M + log2 sum_j w_j lx_j) ln 2 (rank 0).
-__device__ __forceinline__ void cluster_merge(const AttendParams& p, uint8_t* cs, uint8_t* ps, int t,
-                                              int rank) {
+__device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLayer& L, uint8_t* cs,
+                                              uint8_t* ps, int t, int rank) {
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int n = p.n_split;
@@ -201,17 +228,17 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, uint8_t* cs
         M = fmaxf(M, m[j]);
       }
     }
-    float w[8], L = 0.f, Lx = 0.f;
+    float w[8], Ls = 0.f, Lx = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       w[j] = (m[j] == -INFINITY) ? 0.f : ex2_approx(m[j] - M);
-      L += w[j] * l[j];
+      Ls += w[j] * l[j];
       Lx += w[j] * lx[j];
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) wt[h * 8 + j] = (L > 0.f) ? w[j] / L : 0.f;
-    if (rank == 0 && p.lse != nullptr)
-      p.lse[(int64_t)t * kHeads + h] = (Lx > 0.f) ? (M + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
+    for (int j = 0; j < 8; ++j) wt[h * 8 + j] = (Ls > 0.f) ? w[j] / Ls : 0.f;
+    if (rank == 0 && L.lse != nullptr)
+      L.lse[(int64_t)t * kHeads + h] = (Lx > 0.f) ? (M + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
   }
   __syncthreads();
   const int c0 = rank * (kLatent / 4) / n, c1 = (rank + 1) * (kLatent / 4) / n;   // float4 columns
@@ -239,67 +266,34 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, uint8_t* cs
     uint2 o;
     o.x = pack_bf16x2(acc.x, acc.y);
     o.y = pack_bf16x2(acc.z, acc.w);
-    *reinterpret_cast<uint2*>(p.out + ((int64_t)t * kHeads + h) * kLatent + 4 * c) = o;
+    *reinterpret_cast<uint2*>(L.out + ((int64_t)t * kHeads + h) * kLatent + 4 * c) = o;
   }
   cl.sync();   // no CTA leaves while its staged partial may still be read
 }
 
-__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c,
-                                             uint32_t& d) {
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr));
-}
-
-template <int DR>
-__global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
-    attend_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_constant__ CUtensorMap qp_map,
-                  const AttendParams p) {
-  using C = AttCfg<DR>;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // The swizzled layouts need 1024-byte alignment; dynamic shared memory starts
-  // there when the kernel has no static shared memory.
-  const bool smem_ok = (smem_u32(smem_raw) & 1023u) == 0;
-  if (!smem_ok && threadIdx.x == 0) raise_error(kErrBadSeq);
-  uint8_t* cs = smem_raw;                               // three tile buffers
-  uint8_t* ps = cs + C::NBUF * C::TILE_BYTES;
-  AttScratch* sc = reinterpret_cast<AttScratch*>(ps + C::P_BYTES);
+// The work of one CTA on one unit; KCH = 64-column chunks per row (9 RoPE, 8 NoPE).
+template <int KCH>
+__device__ __forceinline__ void attend_unit(const AttendParams& p, const AttLayer& L, uint8_t* cs, uint8_t* ps,
+                                            AttScratch* sc, uint32_t tmem_base, int t, int jsplit,
+                                            bool smem_ok) {
+  using C = AttCfg;
   volatile int* abort_flag = &sc->abort_flag;
-
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x / p.n_split;
-  const int jsplit = blockIdx.x % p.n_split;
-
-  if (threadIdx.x == 0) {
-    mbar_init(&sc->q_smem, 1);
-    mbar_init(&sc->q_full, 128);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sc->s_full[b], 1);
-      mbar_init(&sc->s_free[b], 128);
-    }
-    mbar_init(&sc->p_full, 128);
-    mbar_init(&sc->o_done, 1);
-    mbar_init(&sc->mma_done, 1);
-    for (int b = 0; b < C::NBUF; ++b) {
-      mbar_init(&sc->full[b], C::PRODUCERS);
-      mbar_init(&sc->free_[b], 1);
-    }
-    sc->abort_flag = 0;
-    fence_mbar_init();
-  }
-  griddep_wait();
-  if (warp == 4) {
-    tmem_alloc(&sc->tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = sc->tmem_slot;
+  const uint64_t limit = p.wait_limit_ns;
 
   int r_begin, r_end;
   unit_rows(p, t, jsplit, r_begin, r_end, threadIdx.x == 0);
   if (!smem_ok) r_end = r_begin;   // nothing is computed; cluster barriers are still met
   const int n_tiles = (r_end - r_begin + C::ROWS - 1) / C::ROWS;
+  const int b = p.q_seq[t];
+  const bool seq_ok = (b >= 0 && b < p.B);
+  const int64_t base = seq_ok ? p.seq_row_start[b] : 0;
+  const int32_t qpos = (p.q_pos != nullptr) ? p.q_pos[t] : INT_MAX;
+
+  bool have_o = false;        // softmax threads: O of this unit is complete
+  float m_used = -INFINITY;   // reference max of this thread's head, log2 units
+  float Lsum = 0.f, Lx = 0.f;
 
   if (warp >= 5) {
     // ------------------------------------------------------------- producers
@@ -309,30 +303,38 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
     // g / (8 KCH).  Lane l holds the index of the warp's row 4 (l >> 2) + (l & 3)
     // (quad pw + 3 (l >> 2)); other lanes read it with a shuffle.
     const int pw = warp - 5;
-    constexpr int PPR = 8 * C::KCH;          // 16-byte pieces per row
+    constexpr int PPR = 8 * KCH;             // 16-byte pieces per row
     constexpr int NQ = C::ROWS / 4;          // row quads per tile
     constexpr int QPW = (NQ + 2) / 3;        // quads per warp, at most
-    static_assert(4 * PPR == 32 * C::KCH, "a quad is KCH warp-wide copies");
+    static_assert(4 * PPR == 32 * KCH, "a quad is KCH warp-wide copies");
     static_assert(4 * QPW <= 32, "one index per lane");
-    const int b = p.q_seq[t];
-    const bool seq_ok = (b >= 0 && b < p.B);
     if (!seq_ok && threadIdx.x == 160 && n_tiles > 0) raise_error(kErrBadSeq);
-    const int64_t base = seq_ok ? p.seq_row_start[b] : 0;
-    if (threadIdx.x == 160 && n_tiles > 0) {
-      // Q [64 heads x (512 + DR)] into tile buffer 2, chunk-major, 128-byte swizzled.
-      uint8_t* qs = cs + 2 * C::TILE_BYTES;
-      prefetch_tmap(&qn_map);
-      mbar_arrive_expect_tx(&sc->q_smem, C::KCH * kHeads * 128);
-      for (int c = 0; c < 8; ++c) tma_load_2d(qs + c * kHeads * 128, &qn_map, c * 64, t * kHeads, &sc->q_smem);
-      if (DR == 64) {
-        prefetch_tmap(&qp_map);
-        tma_load_2d(qs + 8 * kHeads * 128, &qp_map, 0, t * kHeads, &sc->q_smem);
+    const uint32_t cs0 = smem_u32(cs);
+    if (n_tiles > 0) {
+      // Q [64 heads x (512 + 64)] into tile buffer 2 in the tile layout (heads as rows).
+      const char* qn = reinterpret_cast<const char*>(L.q_nope + (int64_t)t * kHeads * kLatent);
+      const char* qp = (KCH == 9) ? reinterpret_cast<const char*>(L.q_pe + (int64_t)t * kHeads * 64) : qn;
+      const uint32_t qb = cs0 + 2 * C::TILE_BYTES;
+#pragma unroll 1
+      for (int kq = 0; kq < QPW; ++kq) {
+        const int quad = pw + 3 * kq;
+        if (quad >= NQ) break;
+#pragma unroll
+        for (int j = 0; j < KCH; ++j) {
+          const int g = 32 * j + lane;
+          const int riq = g / PPR;
+          const int pr = g - riq * PPR;
+          const int h = 4 * quad + riq;
+          const uint32_t dst = qb + (pr >> 3) * C::CHUNK_BYTES + h * 128 + (((pr & 7) ^ (h & 7)) << 4);
+          const char* src = (pr < 64) ? qn + h * (kLatent * 2) + pr * 16 : qp + h * 128 + (pr - 64) * 16;
+          cp_async_16(dst, src, 16u);
+        }
       }
+      cp_async_arrive_noinc(&sc->q_smem);   // completes once this thread's Q copies have landed
     }
     const int my_quad = pw + 3 * (lane >> 2);
     const int my_row = 4 * my_quad + (lane & 3);
-    const uint32_t cs0 = smem_u32(cs);
-    const char* cache_bytes = reinterpret_cast<const char*>(p.cache);
+    const char* cache_bytes = reinterpret_cast<const char*>(L.cache);
     const int32_t* idx_t = p.idx + (int64_t)t * p.k;
     // The index of this lane's row, loaded one tile ahead so that a global
     // round trip never sits between a buffer becoming free and its copies.
@@ -345,41 +347,41 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
     for (int i = 0; i < n_tiles; ++i) {
       const int buf = i % C::NBUF;
       if (i >= C::NBUF &&
-          !mbar_wait(&sc->free_[buf], (uint32_t)((i / C::NBUF - 1) & 1), abort_flag)) {
+          !mbar_wait(&sc->free_[buf], (uint32_t)((i / C::NBUF - 1) & 1), abort_flag, limit)) {
         ok = false;
         break;
       }
       // Buffer 2 holds Q until the softmax warps have moved it to TMEM.
-      if (i == 2 && !mbar_wait(&sc->q_full, 0, abort_flag)) {
+      if (i == 2 && !mbar_wait(&sc->q_full, 0, abort_flag, limit)) {
         ok = false;
         break;
       }
       int32_t row = -1;   // row of the cache, or -1: the copy zero-fills
-      if (cur >= 0 && base + cur < p.n_rows) row = (int32_t)(base + cur);
+      if (cur >= 0 && cur <= qpos && base + cur < p.n_rows) row = (int32_t)(base + cur);
       else if (cur != -1) raise_error(kErrBadIndex);
       cur = load_idx(i + 1);
+      if (i == p.stall_tile) continue;   // testing hook: this tile never arrives
       const uint32_t tb = cs0 + buf * C::TILE_BYTES;
 #pragma unroll 1
-      for (int k = 0; k < QPW; ++k) {
-        const int quad = pw + 3 * k;
+      for (int kq = 0; kq < QPW; ++kq) {
+        const int quad = pw + 3 * kq;
         if (quad >= NQ) break;
 #pragma unroll
-        for (int j = 0; j < C::KCH; ++j) {
+        for (int j = 0; j < KCH; ++j) {
           const int g = 32 * j + lane;
           const int riq = g / PPR;
           const int pr = g - riq * PPR;
-          const int32_t src_row = __shfl_sync(0xffffffffu, row, 4 * k + riq);
+          const int32_t src_row = __shfl_sync(0xffffffffu, row, 4 * kq + riq);
           const int r = 4 * quad + riq;
           const uint32_t dst = tb + (pr >> 3) * C::CHUNK_BYTES + r * 128 + (((pr & 7) ^ (r & 7)) << 4);
-          const char* src = src_row >= 0 ? cache_bytes + (int64_t)src_row * p.ld_c * 2 + pr * 16 : cache_bytes;
+          const char* src = src_row >= 0 ? cache_bytes + (int64_t)src_row * L.ld_c * 2 + pr * 16 : cache_bytes;
           cp_async_16(dst, src, src_row >= 0 ? 16u : 0u);
         }
       }
       cp_async_arrive_noinc(&sc->full[buf]);   // lands once this thread's copies so far have
     }
     if (!ok) *abort_flag = 1;
-    cp_async_wait_all();   // nothing may still be landing in shared memory at exit
-    if (threadIdx.x == 160 && n_tiles > 0) mbar_wait(&sc->q_smem, 0, nullptr);   // no TMA in flight at exit
+    cp_async_wait_all();   // nothing may still be landing in shared memory at the barrier below
   } else if (warp == 4) {
     // ------------------------------------------------------------- MMA issuer
     // Issues, in order of readiness, the logit MMAs of the next tile once its
@@ -388,7 +390,7 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
     // operand at byte offset d from its base is the base descriptor + (d >> 4)
     // (shared addresses stay below 256 KB, so the start field cannot carry).
     if (lane == 0 && n_tiles > 0) {
-      bool ok = mbar_wait(&sc->q_full, 0, abort_flag);
+      bool ok = mbar_wait(&sc->q_full, 0, abort_flag, limit);
       tc_fence_after();
       const uint64_t s_desc0 = sdesc_sw128(smem_u32(cs), 16, 1024);                 // K-major C
       const uint64_t o_desc0 = sdesc_sw128(smem_u32(cs), C::CHUNK_BYTES, 1024);     // MN-major C
@@ -431,7 +433,7 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
             const uint64_t sbd = s_desc0 + (uint64_t)((buf * C::TILE_BYTES) >> 4);
             const uint32_t d = tmem_base + C::S_COL + 64 * sb;
 #pragma unroll 1
-            for (int c = 0; c < C::KCH; ++c) {
+            for (int c = 0; c < KCH; ++c) {
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
                 mma_bf16_ts(d, tmem_base + C::Q_COL + 32 * c + 8 * kk,
@@ -450,7 +452,7 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
           const uint64_t now = global_timer_ns();
           if (*abort_flag) ok = false;
           else if (spins == 256u) t_idle = now;
-          else if (now - t_idle > kWaitLimitNs) {
+          else if (now - t_idle > limit) {
             raise_error(kErrTimeout);
             ok = false;
           }
@@ -458,37 +460,34 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
       }
       if (!ok) *abort_flag = 1;
       mma_commit(&sc->mma_done);
-      mbar_wait(&sc->mma_done, 0, nullptr);
+      mbar_wait(&sc->mma_done, 0, nullptr);   // every issued MMA has finished (default limit)
     }
   } else {
-    // ------------------------------------------------------------- softmax + epilogue
+    // ------------------------------------------------------------- softmax
     // Lane L of warp w owns head h = 16 w + (L & 15) and rows 32 hf .. 32 hf + 31
     // of each tile, hf = L >> 4 (the 16x32bx2 TMEM access pattern).
     const int hf = lane >> 4;
     const int h = 16 * warp + (lane & 15);
     const uint32_t lo_base = tmem_base + ((uint32_t)(warp * 32) << 16);          // Q, S lanes
     const uint32_t hi_base = tmem_base + ((uint32_t)(warp * 32 + C::O_LANE) << 16);  // O lanes
-    const int sb_seq = p.q_seq[t];
-    const bool seq_ok = (sb_seq >= 0 && sb_seq < p.B);
-    const int64_t seq_base = seq_ok ? p.seq_row_start[sb_seq] : 0;
-    const float fac = p.qmul[(int64_t)t * kHeads + h] * p.scale_log2e;
+    const float fac = L.qmul[(int64_t)t * kHeads + h] * p.scale_log2e;
     if (n_tiles > 0) {
       // Q[t, h] into TMEM from its staging copy in tile buffer 2: this thread
       // moves elements [128 s + 64 hf, + 64) of the NoPE part (chunk 2 s + hf)
       // and [32 hf, + 32) of the rotary part (chunk 8, pieces 4 hf ..).
-      const bool got_q = mbar_wait(&sc->q_smem, 0, abort_flag);
+      const bool got_q = mbar_wait(&sc->q_smem, 0, abort_flag, limit);
       const uint32_t qrow = smem_u32(cs + 2 * C::TILE_BYTES) + h * 128;
 #pragma unroll 1
       for (int s = 0; s < 4; ++s) {
         uint32_t v[32];
-        const uint32_t ca = qrow + (2 * s + hf) * (kHeads * 128);
+        const uint32_t ca = qrow + (2 * s + hf) * C::CHUNK_BYTES;
 #pragma unroll
         for (int u = 0; u < 8; ++u) ld_shared_v4(ca + ((u ^ (h & 7)) << 4), v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
         tmem_st16x2_32(lo_base + C::Q_COL + 64 * s, v);
       }
-      if (DR == 64) {
+      if (KCH == 9) {
         uint32_t v[16];
-        const uint32_t ca = qrow + 8 * (kHeads * 128);
+        const uint32_t ca = qrow + 8 * C::CHUNK_BYTES;
 #pragma unroll
         for (int u = 0; u < 4; ++u)
           ld_shared_v4(ca + (((4 * hf + u) ^ (h & 7)) << 4), v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
@@ -508,12 +507,11 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
       for (int half = 0; half < 2; ++half) {
         const int rr = r_begin + i * C::ROWS + 32 * half + lane;
         const int32_t sidx = (i < n_tiles && rr < r_end && seq_ok) ? p.idx[(int64_t)t * p.k + rr] : -1;
-        m[half] = __ballot_sync(0xffffffffu, sidx >= 0 && seq_base + sidx < p.n_rows);
+        m[half] = __ballot_sync(0xffffffffu, sidx >= 0 && sidx <= qpos && base + sidx < p.n_rows);
       }
       return hf ? m[1] : m[0];
     };
     const uint32_t pbase = smem_u32(ps) + h * 128;
-    float m_used = -INFINITY;   // reference max of this head, log2 units
     float l_sum = 0.f;          // this thread's share of the row sum of the bf16 weights (normalises o)
     float l_ex = 0.f;           // ... and of the fp32 weights (gives lse)
     uint32_t vm_next = valid_mask(0);
@@ -522,7 +520,7 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
       const int sbuf = i & 1;
       const uint32_t vm = vm_next;
       vm_next = valid_mask(i + 1);
-      const bool got_s = mbar_wait(&sc->s_full[sbuf], (uint32_t)((i >> 1) & 1), abort_flag);
+      const bool got_s = mbar_wait(&sc->s_full[sbuf], (uint32_t)((i >> 1) & 1), abort_flag, limit);
       if (named_bar_or(1, 128, !got_s)) { ok = false; break; }   // leave together
       tc_fence_after();
       uint32_t v[32];
@@ -559,7 +557,7 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
       if (i > 0) {
         // O(i-1) finished: P of the previous tile is no longer read, and O may
         // be rescaled in place.
-        const bool got_o = mbar_wait(&sc->o_done, (uint32_t)((i - 1) & 1), abort_flag);
+        const bool got_o = mbar_wait(&sc->o_done, (uint32_t)((i - 1) & 1), abort_flag, limit);
         if (named_bar_or(1, 128, !got_o)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, resc)) {
@@ -590,95 +588,145 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
       mbar_arrive(&sc->p_full);
     }
     if (!ok) *abort_flag = 1;
-
-    // ---- epilogue: normalised output or partials
-    bool have_o = ok && n_tiles > 0;
+    have_o = ok && n_tiles > 0;
     if (have_o) {
-      const bool got_o = mbar_wait(&sc->o_done, (uint32_t)((n_tiles - 1) & 1), abort_flag);
+      const bool got_o = mbar_wait(&sc->o_done, (uint32_t)((n_tiles - 1) & 1), abort_flag, limit);
       have_o = !named_bar_or(1, 128, !got_o);
-      tc_fence_after();
     }
-    const float L = l_sum + __shfl_xor_sync(0xffffffffu, l_sum, 16);
-    const float Lx = l_ex + __shfl_xor_sync(0xffffffffu, l_ex, 16);
-    const int64_t unit = (int64_t)t * p.n_split + jsplit;
-    if (p.n_split == 1) {
-      const float inv = (have_o && L > 0.f) ? 1.f / L : 0.f;
-      uint4* o_t = reinterpret_cast<uint4*>(p.out + ((int64_t)t * kHeads + h) * kLatent + 32 * hf);
-#pragma unroll 1
-      for (int cb = 0; cb < kLatent; cb += 64) {
-        uint32_t u[32];
-        if (have_o) {
-          tmem_ld16x2_32(hi_base + cb, u);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) u[c] = 0u;
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(u[8 * q]) * inv, __uint_as_float(u[8 * q + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(u[8 * q + 2]) * inv, __uint_as_float(u[8 * q + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(u[8 * q + 4]) * inv, __uint_as_float(u[8 * q + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(u[8 * q + 6]) * inv, __uint_as_float(u[8 * q + 7]) * inv);
-          o_t[cb / 8 + q] = w;
-        }
-      }
-      if (p.lse != nullptr && hf == 0)
-        p.lse[(int64_t)t * kHeads + h] =
-            (have_o && Lx > 0.f) ? (m_used + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
-    } else if (p.merge) {
-      // Stage unnormalised O[h, :] (fp32, 16-byte pieces XOR-swizzled by h & 7
-      // within 128-byte groups) and (max, sum) in this CTA's tile buffers,
-      // which no copy or product touches any more.
-      const uint32_t xrow = smem_u32(cs) + h * (kLatent * 4);
-#pragma unroll 1
-      for (int cb = 0; cb < kLatent; cb += 64) {
-        uint32_t u[32];
-        if (have_o) {
-          tmem_ld16x2_32(hi_base + cb, u);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) u[c] = 0u;
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int piece = (cb / 4 + 8 * hf + q) ^ (h & 7);
-          st_shared_v4(xrow + piece * 16, u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
-        }
-      }
-      if (hf == 0) {
-        float* xml = reinterpret_cast<float*>(cs + kHeads * kLatent * 4);
-        xml[4 * h] = have_o ? m_used : -INFINITY;
-        xml[4 * h + 1] = have_o ? L : 0.f;
-        xml[4 * h + 2] = have_o ? Lx : 0.f;
-      }
+    Lsum = l_sum + __shfl_xor_sync(0xffffffffu, l_sum, 16);
+    Lx = l_ex + __shfl_xor_sync(0xffffffffu, l_ex, 16);
+  }
+
+  // Every role is done: the producers' copies have landed (cp.async.wait_all),
+  // every MMA has completed (mma_done), so the tile buffers may be reused for
+  // staging and O may be read from TMEM.
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp >= 4) return;
+
+  // ---- epilogue (softmax warps): normalised output, staged partial or workspace partial
+  const int hf = lane >> 4;
+  const int h = 16 * warp + (lane & 15);
+  const uint32_t hi_base = tmem_base + ((uint32_t)(warp * 32 + C::O_LANE) << 16);
+  const int64_t unit = blockIdx.x;   // (pair, split)
+  auto read_o = [&](int cb, uint32_t (&u)[32]) {
+    if (have_o) {
+      tmem_ld16x2_32(hi_base + cb, u);
+      tmem_wait_ld();
     } else {
-      float4* wo = reinterpret_cast<float4*>(p.ws_o + (unit * kHeads + h) * kLatent + 32 * hf);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) u[c] = 0u;
+    }
+  };
+  if (p.n_split == 1) {
+    const float inv = (have_o && Lsum > 0.f) ? 1.f / Lsum : 0.f;
+    uint4* o_t = reinterpret_cast<uint4*>(L.out + ((int64_t)t * kHeads + h) * kLatent + 32 * hf);
 #pragma unroll 1
-      for (int cb = 0; cb < kLatent; cb += 64) {
-        uint32_t u[32];
-        if (have_o) {
-          tmem_ld16x2_32(hi_base + cb, u);
-          tmem_wait_ld();
-        } else {
+    for (int cb = 0; cb < kLatent; cb += 64) {
+      uint32_t u[32];
+      read_o(cb, u);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) u[c] = 0u;
-        }
+      for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(u[8 * q]) * inv, __uint_as_float(u[8 * q + 1]) * inv);
+        w.y = pack_bf16x2(__uint_as_float(u[8 * q + 2]) * inv, __uint_as_float(u[8 * q + 3]) * inv);
+        w.z = pack_bf16x2(__uint_as_float(u[8 * q + 4]) * inv, __uint_as_float(u[8 * q + 5]) * inv);
+        w.w = pack_bf16x2(__uint_as_float(u[8 * q + 6]) * inv, __uint_as_float(u[8 * q + 7]) * inv);
+        o_t[cb / 8 + q] = w;
+      }
+    }
+    if (L.lse != nullptr && hf == 0)
+      L.lse[(int64_t)t * kHeads + h] =
+          (have_o && Lx > 0.f) ? (m_used + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
+  } else if (p.merge) {
+    // Stage unnormalised O[h, :] (fp32, 16-byte pieces XOR-swizzled by h & 7
+    // within 128-byte groups) and (max, sum) in this CTA's tile buffers.
+    const uint32_t xrow = smem_u32(cs) + h * (kLatent * 4);
+#pragma unroll 1
+    for (int cb = 0; cb < kLatent; cb += 64) {
+      uint32_t u[32];
+      read_o(cb, u);
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          wo[cb / 4 + q] = make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
-                                       __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
+      for (int q = 0; q < 8; ++q) {
+        const int piece = (cb / 4 + 8 * hf + q) ^ (h & 7);
+        st_shared_v4(xrow + piece * 16, u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
       }
-      if (hf == 0) {
-        float* ml = p.ws_ml + (unit * kHeads + h) * 4;
-        ml[0] = have_o ? m_used : -INFINITY;
-        ml[1] = have_o ? L : 0.f;
-        ml[2] = have_o ? Lx : 0.f;
-      }
+    }
+    if (hf == 0) {
+      float* xml = reinterpret_cast<float*>(cs + kHeads * kLatent * 4);
+      xml[4 * h] = have_o ? m_used : -INFINITY;
+      xml[4 * h + 1] = have_o ? Lsum : 0.f;
+      xml[4 * h + 2] = have_o ? Lx : 0.f;
+    }
+  } else {
+    float4* wo = reinterpret_cast<float4*>(p.ws_o + (unit * kHeads + h) * kLatent + 32 * hf);
+#pragma unroll 1
+    for (int cb = 0; cb < kLatent; cb += 64) {
+      uint32_t u[32];
+      read_o(cb, u);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        wo[cb / 4 + q] = make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
+                                     __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
+    }
+    if (hf == 0) {
+      float* ml = p.ws_ml + (unit * kHeads + h) * 4;
+      ml[0] = have_o ? m_used : -INFINITY;
+      ml[1] = have_o ? Lsum : 0.f;
+      ml[2] = have_o ? Lx : 0.f;
     }
   }
+}
+
+__global__ void __launch_bounds__(AttCfg::THREADS, 1)
+    attend_kernel(const __grid_constant__ AttendParams p) {
+  using C = AttCfg;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The swizzled layouts need 1024-byte alignment; dynamic shared memory starts
+  // there when the kernel has no static shared memory.
+  const bool smem_ok = (smem_u32(smem_raw) & 1023u) == 0;
+  if (!smem_ok && threadIdx.x == 0) raise_error(kErrBadSeq);
+  uint8_t* cs = smem_raw;                               // three tile buffers
+  uint8_t* ps = cs + C::NBUF * C::TILE_BYTES;
+  AttScratch* sc = reinterpret_cast<AttScratch*>(ps + C::P_BYTES);
+
+  const int warp = threadIdx.x >> 5;
+  const int pair = blockIdx.x / p.n_split;
+  const int jsplit = blockIdx.x % p.n_split;
+  const int lyr = pair / p.T;
+  const int t = pair - lyr * p.T;
+  const AttLayer& L = p.layer[lyr];
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sc->q_smem, C::PRODUCERS);
+    mbar_init(&sc->q_full, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sc->s_full[b], 1);
+      mbar_init(&sc->s_free[b], 128);
+    }
+    mbar_init(&sc->p_full, 128);
+    mbar_init(&sc->o_done, 1);
+    mbar_init(&sc->mma_done, 1);
+    for (int b = 0; b < C::NBUF; ++b) {
+      mbar_init(&sc->full[b], C::PRODUCERS);
+      mbar_init(&sc->free_[b], 1);
+    }
+    sc->abort_flag = 0;
+    fence_mbar_init();
+  }
+  griddep_wait();
+  if (warp == 4) {
+    tmem_alloc(&sc->tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = sc->tmem_slot;
+
+  if (L.d_rope == 64) attend_unit<9>(p, L, cs, ps, sc, tmem_base, t, jsplit, smem_ok);
+  else attend_unit<8>(p, L, cs, ps, sc, tmem_base, t, jsplit, smem_ok);
 
   tc_fence_before();
   __syncthreads();
@@ -686,23 +734,25 @@ __global__ void __launch_bounds__(AttCfg<DR>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
-  if (p.merge) cluster_merge(p, cs, ps, t, jsplit);
+  if (p.merge) cluster_merge(p, L, cs, ps, t, jsplit);
 }
 
-// Merges the split partials of each (query, head): o = sum_j 2^(m_j - M) O_j / L,
+// Merges the split partials of each (layer, query, head): o = sum_j 2^(m_j - M) O_j / L,
 // L = sum_j 2^(m_j - M) l_j, lse = (M + log2 sum_j 2^(m_j - M) lx_j) ln 2.  One block per
-// (query, head); each of the 128 threads owns 4 latent columns.
-constexpr int kMaxSplits = 32;
-__global__ void __launch_bounds__(128) attend_combine_kernel(const AttendParams p) {
+// (pair, head); each of the 128 threads owns 4 latent columns.
+__global__ void __launch_bounds__(128) attend_combine_kernel(const __grid_constant__ AttendParams p) {
   griddep_wait();
-  const int t = blockIdx.x / kHeads;
+  const int pair = blockIdx.x / kHeads;
   const int h = blockIdx.x % kHeads;
+  const int lyr = pair / p.T;
+  const int t = pair - lyr * p.T;
+  const AttLayer& L = p.layer[lyr];
   const int ns = p.n_split;
   __shared__ float wsc[kMaxSplits];
   __shared__ float stats[2];   // M, sum_j 2^(m_j - M) lx_j
   if (threadIdx.x < 32) {
     const int j = threadIdx.x;
-    const int64_t u = (int64_t)t * ns + j;
+    const int64_t u = (int64_t)pair * ns + j;
     const float m = (j < ns) ? p.ws_ml[(u * kHeads + h) * 4] : -INFINITY;
     const float l = (j < ns) ? p.ws_ml[(u * kHeads + h) * 4 + 1] : 0.f;
     const float lx = (j < ns) ? p.ws_ml[(u * kHeads + h) * 4 + 2] : 0.f;
@@ -710,13 +760,13 @@ __global__ void __launch_bounds__(128) attend_combine_kernel(const AttendParams 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     const float sc = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
-    float L = sc * l, Lx = sc * lx;
+    float Ls = sc * l, Lx = sc * lx;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      L += __shfl_xor_sync(0xffffffffu, L, o);
+      Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
       Lx += __shfl_xor_sync(0xffffffffu, Lx, o);
     }
-    wsc[j] = (L > 0.f) ? sc / L : 0.f;
+    wsc[j] = (Ls > 0.f) ? sc / Ls : 0.f;
     if (j == 0) {
       stats[0] = M;
       stats[1] = Lx;
@@ -727,18 +777,19 @@ __global__ void __launch_bounds__(128) attend_combine_kernel(const AttendParams 
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int j = 0; j < ns; ++j) {
     const float wj = wsc[j];
-    const float4 o4 = *reinterpret_cast<const float4*>(p.ws_o + (((int64_t)t * ns + j) * kHeads + h) * kLatent + d);
+    const float4 o4 =
+        *reinterpret_cast<const float4*>(p.ws_o + (((int64_t)pair * ns + j) * kHeads + h) * kLatent + d);
     acc.x = fmaf(wj, o4.x, acc.x);
     acc.y = fmaf(wj, o4.y, acc.y);
     acc.z = fmaf(wj, o4.z, acc.z);
     acc.w = fmaf(wj, o4.w, acc.w);
   }
-  __nv_bfloat16* o = p.out + ((int64_t)t * kHeads + h) * kLatent + d;
+  __nv_bfloat16* o = L.out + ((int64_t)t * kHeads + h) * kLatent + d;
   *reinterpret_cast<__nv_bfloat162*>(o) = __floats2bfloat162_rn(acc.x, acc.y);
   *reinterpret_cast<__nv_bfloat162*>(o + 2) = __floats2bfloat162_rn(acc.z, acc.w);
-  if (threadIdx.x == 0 && p.lse != nullptr) {
-    const float L = stats[1];
-    p.lse[(int64_t)t * kHeads + h] = (L > 0.f) ? (stats[0] + lg2_approx(L)) * 0.69314718055994531f : -INFINITY;
+  if (threadIdx.x == 0 && L.lse != nullptr) {
+    const float Lx = stats[1];
+    L.lse[(int64_t)t * kHeads + h] = (Lx > 0.f) ? (stats[0] + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
   }
 }
 

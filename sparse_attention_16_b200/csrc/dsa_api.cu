@@ -1,7 +1,8 @@
 // dsa_api.cu - host side of the C ABI declared in include/dsa.h: argument
-// validation, TMA descriptor encoding, launch configuration and the fused
-// indexer -> top-k -> per-layer attention sequence.  Every step of the hot
-// path runs in the kernels included below; nothing here computes on the host.
+// validation, TMA descriptor encoding, launch planning and configuration, and
+// the fused indexer -> top-k -> per-layer attention sequence.  Every step of
+// the hot path runs in the kernels included below; nothing here computes on
+// the host.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -21,12 +22,19 @@
 #include "dsa.h"
 #include "attend.cuh"
 #include "indexer.cuh"
+#include "plan.h"
 #include "topk.cuh"
+
+static_assert(dsa::kPlanMaxLayers == dsa::kMaxAttLayers, "planner and kernel agree on layers per launch");
+static_assert(dsa::kPlanMaxSplits == dsa::kMaxSplits, "planner and kernel agree on the split limit");
+static_assert(dsa::kPlanTileRows == dsa::AttCfg::ROWS, "planner and kernel agree on the tile height");
 
 namespace {
 
 thread_local std::string g_last_error;
 std::atomic<uint64_t> g_launches{0};
+std::atomic<uint64_t> g_wait_limit_ns{0};   // 0: kWaitLimitNs (testing hook)
+std::atomic<int32_t> g_stall_tile{-1};      // testing hook, off
 
 dsa_status_t fail(dsa_status_t st, const char* fmt, ...) {
   char buf[512];
@@ -49,37 +57,160 @@ dsa_status_t fail(dsa_status_t st, const char* fmt, ...) {
     if (e_ != cudaSuccess) return fail(DSA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
   } while (0)
 
+#define DSA_TRY(expr)                      \
+  do {                                     \
+    dsa_status_t st_ = (expr);             \
+    if (st_ != DSA_OK) return st_;         \
+  } while (0)
+
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kMaxK = 16384;
 
-int sm_count() {
-  static std::atomic<int> cached[64] = {};
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev >= 0 && dev < 64 && (n = cached[dev].load(std::memory_order_relaxed)) > 0) return n;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-    return 148;
-  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
-  return n;
+// ----------------------------------------------------------------- driver entry points
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess && q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<Fn>(p);
+  return nullptr;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
+  static const auto fn = driver_fn<PFN_cuTensorMapEncodeTiled_v12000>("cuTensorMapEncodeTiled");
   return fn;
 }
 
-// 2-D bf16 tensor map with the 128-byte swizzle: `inner` contiguous elements
-// per row, `outer` rows `row_bytes` apart, box of box_inner x box_outer.
+// Unique id of the calling thread's current context (0: none is current yet).
+// Per-device state is keyed by it, so a device reset (a new primary context)
+// starts from a clean slate instead of reusing addresses and attributes of the
+// old context.
+uint64_t current_context_id() {
+  static const auto get_cur = driver_fn<PFN_cuCtxGetCurrent_v4000>("cuCtxGetCurrent");
+  static const auto get_id = driver_fn<PFN_cuCtxGetId_v12000>("cuCtxGetId");
+  if (get_cur == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return (uint64_t)id + 1;   // never 0 for a real context
+}
+
+// ----------------------------------------------------------------- per-device state
+enum KernelId : uint32_t {
+  kKIdx1 = 0, kKIdx8, kKIdx1F8, kKIdx8F8, kKTopk1, kKTopk2, kKTopk4, kKTopk8, kKTopk16, kKAttend, kKCount
+};
+
+constexpr int kMaxDevices = 64;
+
+struct DevState {
+  std::mutex mu;
+  uint64_t ctx_id = ~0ull;        // context the cached values belong to
+  bool props_ok = false;
+  dsa::DevProps props;            // SMs and attention cluster residency
+  int topk_clusters[17] = {};     // [CL]: top-k clusters of CL blocks resident at once
+  uint32_t smem_done = 0;         // bit per KernelId: dynamic shared-memory limit raised
+  void* noalloc_ptr = nullptr;    // device address of the no-allocation scratch array
+};
+DevState g_dev[kMaxDevices];
+
+// The calling thread's device state, locked, reset when its context changed.
+struct DevLock {
+  DevState* s = nullptr;
+  int dev = 0;
+  std::unique_lock<std::mutex> lk;
+};
+
+dsa_status_t lock_device(DevLock& L) {
+  DSA_CUDA(cudaGetDevice(&L.dev));
+  if (L.dev < 0 || L.dev >= kMaxDevices)
+    return fail(DSA_ERR_UNSUPPORTED, "device %d: this library supports devices 0..%d", L.dev, kMaxDevices - 1);
+  L.s = &g_dev[L.dev];
+  L.lk = std::unique_lock<std::mutex>(L.s->mu);
+  const uint64_t id = current_context_id();
+  if (L.s->ctx_id != id) {
+    L.s->ctx_id = id;
+    L.s->props_ok = false;
+    L.s->smem_done = 0;
+    L.s->noalloc_ptr = nullptr;
+  }
+  return DSA_OK;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device and context.
+template <typename K>
+dsa_status_t set_smem(DevState& s, KernelId id, K kernel, int bytes) {
+  if (s.smem_done & (1u << id)) return DSA_OK;
+  DSA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  s.smem_done |= 1u << id;
+  return DSA_OK;
+}
+
+template <typename K>
+int max_active_clusters(K kernel, int threads, int smem, int cl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cl);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) n = 0;
+  cudaGetLastError();
+  return n;
+}
+
+// SM count and how many clusters of each size the attention and top-k kernels
+// can keep resident (a cluster must sit inside one GPC, so this can be well
+// below SMs / size).  Queried once per device and context.
+dsa_status_t device_props(DevLock& L, dsa::DevProps* out) {
+  DevState& s = *L.s;
+  if (!s.props_ok) {
+    dsa::DevProps d;
+    int n = 0;
+    DSA_CUDA(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, L.dev));
+    d.sms = n > 0 ? n : 1;
+    DSA_TRY(set_smem(s, kKAttend, dsa::attend_kernel, dsa::AttCfg::SMEM_BYTES));
+    for (int c = 2; c <= dsa::kPlanMaxMerge; ++c)
+      d.max_clusters[c] = max_active_clusters(dsa::attend_kernel, dsa::AttCfg::THREADS, dsa::AttCfg::SMEM_BYTES, c);
+    DSA_TRY(set_smem(s, kKTopk2, dsa::topk_kernel<2>, dsa::kTopkSmemBytes));
+    DSA_TRY(set_smem(s, kKTopk4, dsa::topk_kernel<4>, dsa::kTopkSmemBytes));
+    DSA_TRY(set_smem(s, kKTopk8, dsa::topk_kernel<8>, dsa::kTopkSmemBytes));
+    DSA_TRY(set_smem(s, kKTopk16, dsa::topk_kernel<16>, dsa::kTopkSmemBytes));
+    DSA_CUDA(cudaFuncSetAttribute(dsa::topk_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    s.topk_clusters[1] = d.sms;
+    s.topk_clusters[2] = max_active_clusters(dsa::topk_kernel<2>, dsa::kTopkThreads, dsa::kTopkSmemBytes, 2);
+    s.topk_clusters[4] = max_active_clusters(dsa::topk_kernel<4>, dsa::kTopkThreads, dsa::kTopkSmemBytes, 4);
+    s.topk_clusters[8] = max_active_clusters(dsa::topk_kernel<8>, dsa::kTopkThreads, dsa::kTopkSmemBytes, 8);
+    s.topk_clusters[16] = max_active_clusters(dsa::topk_kernel<16>, dsa::kTopkThreads, dsa::kTopkSmemBytes, 16);
+    s.props = d;
+    s.props_ok = true;
+  }
+  *out = s.props;
+  return DSA_OK;
+}
+
+// Props for a planning query: the caller's (on any machine) or the current device's.
+dsa_status_t props_for_query(const dsa_device_props* given, dsa::DevProps* out) {
+  if (given != nullptr) {
+    DSA_REQUIRE(given->sms >= 1, "props.sms must be >= 1");
+    dsa::DevProps d;
+    d.sms = given->sms;
+    for (int c = 0; c < 9; ++c) d.max_clusters[c] = std::max(0, given->max_clusters[c]);
+    *out = d;
+    return DSA_OK;
+  }
+  DevLock L;
+  DSA_TRY(lock_device(L));
+  return device_props(L, out);
+}
+
 dsa_status_t make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
   auto enc = encode_fn();
@@ -103,20 +234,6 @@ struct NvtxRange {
   NvtxRange(const NvtxRange&) = delete;
   NvtxRange& operator=(const NvtxRange&) = delete;
 };
-
-// Raises a kernel's dynamic shared-memory limit once per device (the
-// attribute persists, so later launches skip the driver call).
-template <auto Kernel>
-dsa_status_t set_smem(int bytes) {
-  static std::atomic<uint64_t> done{0};   // one flag set per kernel (not per signature)
-  int dev = 0;
-  DSA_CUDA(cudaGetDevice(&dev));
-  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
-  if (bit && (done.load(std::memory_order_relaxed) & bit)) return DSA_OK;
-  DSA_CUDA(cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
-  if (bit) done.fetch_or(bit, std::memory_order_relaxed);
-  return DSA_OK;
-}
 
 // Launches a kernel, as clusters of cl CTAs for cl > 1.  With DSA_PDL=1 in the
 // environment the launch also allows programmatic stream serialization: every
@@ -165,7 +282,7 @@ dsa_status_t launch(void (*kernel)(KArgs...), unsigned grid, unsigned block, siz
 // F8: q_idx / k_idx hold E4M3 codes (one byte per value) and q_scale / k_scale
 // their per-head / per-row scales; otherwise bf16 values and null scales.
 template <int QG, bool F8>
-dsa_status_t launch_indexer(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
+dsa_status_t launch_indexer(DevLock& L, const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                             const float* k_scale, int64_t n_rows, const int64_t* seq_row_start, int32_t B,
                             const int32_t* q_seq, const int32_t* q_pos, int32_t T, float* scores, int64_t ld,
                             cudaStream_t stream) {
@@ -176,10 +293,8 @@ dsa_status_t launch_indexer(const void* q_idx, const float* q_scale, const float
   const uint64_t row_elems = F8 ? dsa::kIdxDim / 2 : dsa::kIdxDim;
   const uint64_t row_bytes = F8 ? dsa::kIdxDim : dsa::kIdxDim * 2;
   CUtensorMap kmap, qmap;
-  dsa_status_t st = make_tmap(&kmap, k_idx, row_elems, (uint64_t)n_rows, row_bytes, 64, dsa::kKeyTile);
-  if (st != DSA_OK) return st;
-  st = make_tmap(&qmap, q_idx, row_elems, (uint64_t)T * dsa::kIdxHeads, row_bytes, 64, C::N);
-  if (st != DSA_OK) return st;
+  DSA_TRY(make_tmap(&kmap, k_idx, row_elems, (uint64_t)n_rows, row_bytes, 64, dsa::kKeyTile));
+  DSA_TRY(make_tmap(&qmap, q_idx, row_elems, (uint64_t)T * dsa::kIdxHeads, row_bytes, 64, C::N));
   dsa::IndexerParams p;
   p.w = w;
   p.q_scale = q_scale;
@@ -195,99 +310,50 @@ dsa_status_t launch_indexer(const void* q_idx, const float* q_scale, const float
   p.n_kt = (int32_t)((ld + dsa::kKeyTile - 1) / dsa::kKeyTile);
   const int64_t n_groups = (T + QG - 1) / QG;
   p.n_units = n_groups * p.n_kt;
-  const int grid = (int)std::min<int64_t>(p.n_units, sm_count());
-  st = set_smem<dsa::indexer_kernel<QG, F8>>(C::SMEM_BYTES);
-  if (st != DSA_OK) return st;
+  dsa::DevProps props;
+  DSA_TRY(device_props(L, &props));
+  const int grid = (int)std::min<int64_t>(p.n_units, props.sms);
+  const KernelId id = F8 ? (QG == 8 ? kKIdx8F8 : kKIdx1F8) : (QG == 8 ? kKIdx8 : kKIdx1);
+  DSA_TRY(set_smem(*L.s, id, dsa::indexer_kernel<QG, F8>, C::SMEM_BYTES));
   return launch(dsa::indexer_kernel<QG, F8>, (unsigned)grid, C::THREADS, C::SMEM_BYTES, stream, 1, kmap, qmap,
                 p);
 }
 
-dsa_status_t indexer_impl(const void* q_idx, const float* w, const void* k_idx, int64_t n_rows,
+dsa_status_t indexer_impl(DevLock& L, const void* q_idx, const float* w, const void* k_idx, int64_t n_rows,
                           const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
                           const int32_t* q_pos, int32_t T, int32_t q_group, float* scores,
                           int64_t ld, cudaStream_t stream) {
   if (q_group == 8)
-    return launch_indexer<8, false>(q_idx, nullptr, w, k_idx, nullptr, n_rows, seq_row_start, B, q_seq, q_pos,
+    return launch_indexer<8, false>(L, q_idx, nullptr, w, k_idx, nullptr, n_rows, seq_row_start, B, q_seq, q_pos,
                                     T, scores, ld, stream);
-  return launch_indexer<1, false>(q_idx, nullptr, w, k_idx, nullptr, n_rows, seq_row_start, B, q_seq, q_pos, T,
+  return launch_indexer<1, false>(L, q_idx, nullptr, w, k_idx, nullptr, n_rows, seq_row_start, B, q_seq, q_pos, T,
                                   scores, ld, stream);
 }
 
 // ----------------------------------------------------------------- top-k
 template <int CL>
-dsa_status_t launch_topk_cl(const dsa::TopkParams& p, cudaStream_t stream) {
-  dsa_status_t st = set_smem<dsa::topk_kernel<CL>>(dsa::kTopkSmemBytes);
-  if (st != DSA_OK) return st;
-  if (CL > 8) {
-    static std::once_flag once;
-    cudaError_t e = cudaSuccess;
-    std::call_once(once, [&] {
-      e = cudaFuncSetAttribute(dsa::topk_kernel<CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    });
-    if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "cluster attribute: %s", cudaGetErrorString(e));
-  }
+dsa_status_t launch_topk_cl(DevLock& L, KernelId id, const dsa::TopkParams& p, cudaStream_t stream) {
+  DSA_TRY(set_smem(*L.s, id, dsa::topk_kernel<CL>, dsa::kTopkSmemBytes));
   return launch(dsa::topk_kernel<CL>, (unsigned)(p.T * CL), dsa::kTopkThreads, dsa::kTopkSmemBytes, stream,
                 (unsigned)CL, p);
-}
-
-// How many top-k clusters of CL CTAs can be resident at once (16 needs the
-// non-portable attribute and a GPC with 16 free SMs); 0 if none.
-template <int CL>
-int topk_max_clusters_t() {
-  static std::atomic<int> count{-1};
-  const int known = count.load(std::memory_order_relaxed);
-  if (known >= 0) return known;
-  int n = 0;
-  bool ok = cudaFuncSetAttribute(dsa::topk_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dsa::kTopkSmemBytes) == cudaSuccess;
-  if (ok && CL > 8)
-    ok = cudaFuncSetAttribute(dsa::topk_kernel<CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-         cudaSuccess;
-  if (ok) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(CL);
-    cfg.blockDim = dim3(dsa::kTopkThreads);
-    cfg.dynamicSmemBytes = dsa::kTopkSmemBytes;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CL;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, dsa::topk_kernel<CL>, &cfg) != cudaSuccess) n = 0;
-  }
-  cudaGetLastError();
-  count.store(n, std::memory_order_relaxed);
-  return n;
-}
-
-int topk_max_clusters(int CL) {
-  switch (CL) {
-    case 1: return sm_count();
-    case 2: return topk_max_clusters_t<2>();
-    case 4: return topk_max_clusters_t<4>();
-    case 8: return topk_max_clusters_t<8>();
-    case 16: return topk_max_clusters_t<16>();
-    default: return 0;
-  }
 }
 
 // CTAs per query: enough that each CTA owns at least ~16K candidates' worth of
 // work while the batch stays within one wave (T x CL <= SMs, every cluster
 // resident at once); more (up to 16) when a query's slice would not fit the
 // shared-memory key stash.
-int topk_cluster_size(int32_t T, int64_t ld) {
-  const int sms = sm_count();
-  auto fits = [&](int c) { return (int64_t)T * c <= sms && T <= topk_max_clusters(c); };
+int topk_cluster_size(const DevState& s, int sms, int32_t T, int64_t ld) {
+  auto fits = [&](int c) { return (int64_t)T * c <= sms && T <= s.topk_clusters[c]; };
   int cl = 1;
   while (cl < 8 && (ld + cl - 1) / cl > 16384 && fits(cl * 2)) cl *= 2;
   while (cl < 16 && (ld + cl - 1) / cl > dsa::kTopkStashCap && fits(cl * 2)) cl *= 2;
   return cl;
 }
 
-dsa_status_t topk_impl(const float* scores, int64_t ld, const int32_t* q_pos, int32_t T, int32_t k,
+dsa_status_t topk_impl(DevLock& L, const float* scores, int64_t ld, const int32_t* q_pos, int32_t T, int32_t k,
                        int32_t* idx, int32_t* count, cudaStream_t stream) {
+  dsa::DevProps props;
+  DSA_TRY(device_props(L, &props));
   dsa::TopkParams p;
   p.scores = scores;
   p.q_pos = q_pos;
@@ -296,140 +362,97 @@ dsa_status_t topk_impl(const float* scores, int64_t ld, const int32_t* q_pos, in
   p.ld = ld;
   p.T = T;
   p.k = k;
-  switch (topk_cluster_size(T, ld)) {
-    case 1: return launch_topk_cl<1>(p, stream);
-    case 2: return launch_topk_cl<2>(p, stream);
-    case 4: return launch_topk_cl<4>(p, stream);
-    case 8: return launch_topk_cl<8>(p, stream);
-    default: return launch_topk_cl<16>(p, stream);   // chosen only when its clusters fit
+  switch (topk_cluster_size(*L.s, props.sms, T, ld)) {
+    case 1: return launch_topk_cl<1>(L, kKTopk1, p, stream);
+    case 2: return launch_topk_cl<2>(L, kKTopk2, p, stream);
+    case 4: return launch_topk_cl<4>(L, kKTopk4, p, stream);
+    case 8: return launch_topk_cl<8>(L, kKTopk8, p, stream);
+    default: return launch_topk_cl<16>(L, kKTopk16, p, stream);   // chosen only when its clusters fit
   }
 }
 
 // ----------------------------------------------------------------- attention
-struct SplitPlan {
-  int n_split;
-  int rows_per_split;
-  bool merge;   // the n_split CTAs of a query form a cluster and merge in distributed shared memory
-};
-
-// How many clusters of CL attention CTAs (one per SM, 225 KB of shared memory
-// each) can be resident at once (0: none, or CL outside 2..8).  A cluster must
-// sit inside one GPC, so this can be well below SMs / CL.
-int attend_max_clusters(int CL) {
-  static std::atomic<int> count[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
-  if (CL < 2 || CL > 8) return 0;
-  const int known = count[CL].load(std::memory_order_relaxed);
-  if (known >= 0) return known;
-  using C = dsa::AttCfg<64>;
-  int n = 0;
-  if (cudaFuncSetAttribute(dsa::attend_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           C::SMEM_BYTES) == cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(CL);
-    cfg.blockDim = dim3(C::THREADS);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CL;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, dsa::attend_kernel<64>, &cfg) != cudaSuccess) n = 0;
-  }
-  cudaGetLastError();
-  count[CL].store(n, std::memory_order_relaxed);
-  return n;
-}
-
-// Splits each query's selection across CTAs so that T x n_split is about one
-// wave of the GPU; rows per split are a multiple of the 64-row tile.
-SplitPlan attend_plan(int32_t T, int32_t k) {
-  const int tile = dsa::AttCfg<64>::ROWS;
-  const int max_tiles = (k + tile - 1) / tile;
-  int want = std::max(1, sm_count() / std::max(1, T));
-  want = std::min(want, std::min(max_tiles, dsa::kMaxSplits));
-  int tiles_per = (max_tiles + want - 1) / want;
-  SplitPlan sp;
-  sp.rows_per_split = tiles_per * tile;
-  sp.n_split = (k + sp.rows_per_split - 1) / sp.rows_per_split;
-  // Merge in clusters only when every query's cluster is resident at once;
-  // otherwise the partials go through the workspace and the combine kernel.
-  sp.merge = sp.n_split >= 2 && sp.n_split <= 8 && T <= attend_max_clusters(sp.n_split);
-  return sp;
-}
-
-size_t attend_ws_bytes(int32_t T, int32_t k) {
-  const SplitPlan sp = attend_plan(T, k);
-  if (sp.n_split <= 1 || sp.merge) return 0;
-  const size_t units = (size_t)T * sp.n_split;
-  return round_up(units * dsa::kHeads * dsa::kLatent * 4, 256) + round_up(units * dsa::kHeads * 4 * 4, 256);
-}
-
-template <int DR>
-dsa_status_t launch_attend(const void* q_nope, const void* q_pe, const float* qmul, float scale,
-                           const void* cache, int64_t n_rows, int32_t ld_c,
-                           const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
-                           const int32_t* idx, const int32_t* count, int32_t T, int32_t k, void* out,
-                           float* lse, void* ws, cudaStream_t stream) {
-  using C = dsa::AttCfg<DR>;
-  CUtensorMap qn_map, qp_map;
-  dsa_status_t st = make_tmap(&qn_map, q_nope, dsa::kLatent, (uint64_t)T * dsa::kHeads,
-                              dsa::kLatent * 2, 64, dsa::kHeads);
-  if (st != DSA_OK) return st;
-  if (DR == 64) {
-    st = make_tmap(&qp_map, q_pe, 64, (uint64_t)T * dsa::kHeads, 128, 64, dsa::kHeads);
-    if (st != DSA_OK) return st;
-  } else {
-    qp_map = qn_map;  // unused on NoPE layers
-  }
-  const SplitPlan sp = attend_plan(T, k);
+// One launch over up to kMaxAttLayers layers sharing one selection (grid =
+// layers x queries x splits), plus the combine kernel when the plan writes
+// partials.  `ws` must hold the plan's partials (checked).
+dsa_status_t launch_attend(DevLock& L, const dsa_layer_args* layers, int32_t n_layers, float scale,
+                           int64_t n_rows, const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
+                           const int32_t* q_pos, const int32_t* idx, const int32_t* count, int32_t T, int32_t k,
+                           void* ws, size_t ws_bytes, cudaStream_t stream) {
+  using C = dsa::AttCfg;
+  dsa::DevProps props;
+  DSA_TRY(device_props(L, &props));
+  const int64_t units = (int64_t)T * n_layers;
+  const dsa::SplitPlan sp = dsa::attend_plan(props, units, k);
   dsa::AttendParams p;
-  p.q_nope = static_cast<const __nv_bfloat16*>(q_nope);
-  p.q_pe = static_cast<const __nv_bfloat16*>(q_pe);
-  p.cache = static_cast<const __nv_bfloat16*>(cache);
-  p.qmul = qmul;
+  std::memset(&p, 0, sizeof(p));
+  for (int l = 0; l < n_layers; ++l) {
+    const dsa_layer_args& a = layers[l];
+    p.layer[l].q_nope = static_cast<const __nv_bfloat16*>(a.q_nope);
+    p.layer[l].q_pe = static_cast<const __nv_bfloat16*>(a.q_pe);
+    p.layer[l].qmul = a.qmul;
+    p.layer[l].cache = static_cast<const __nv_bfloat16*>(a.cache);
+    p.layer[l].out = static_cast<__nv_bfloat16*>(a.out);
+    p.layer[l].lse = a.lse;
+    p.layer[l].ld_c = a.ld_c;
+    p.layer[l].d_rope = a.d_rope;
+  }
   p.seq_row_start = seq_row_start;
   p.q_seq = q_seq;
+  p.q_pos = q_pos;
   p.idx = idx;
   p.count = count;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
-  p.ld_c = ld_c;
   p.n_rows = n_rows;
+  const uint64_t lim = g_wait_limit_ns.load(std::memory_order_relaxed);
+  p.wait_limit_ns = lim ? lim : dsa::kWaitLimitNs;
+  p.stall_tile = g_stall_tile.load(std::memory_order_relaxed);
   p.scale_log2e = scale * 1.4426950408889634f;
+  p.n_layers = n_layers;
   p.B = B;
   p.T = T;
   p.k = k;
   p.n_split = sp.n_split;
   p.rows_per_split = sp.rows_per_split;
   p.merge = sp.merge ? 1 : 0;
-  p.ws_o = nullptr;
-  p.ws_ml = nullptr;
-  if (sp.n_split > 1 && !sp.merge) {
-    const size_t units = (size_t)T * sp.n_split;
+  const bool partials = sp.n_split > 1 && !sp.merge;
+  if (partials) {
+    const size_t need = dsa::partial_bytes(units, sp.n_split);
+    if (ws == nullptr || ws_bytes < need || !aligned(ws, 256))
+      return fail(DSA_ERR_WORKSPACE, "attention partials need %zu bytes of 256-byte aligned workspace (got %zu)",
+                  need, ws_bytes);
     p.ws_o = static_cast<float*>(ws);
-    p.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
-                                       round_up(units * dsa::kHeads * dsa::kLatent * 4, 256));
+    p.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + dsa::partial_stats_offset(units, sp.n_split));
   }
-  st = set_smem<dsa::attend_kernel<DR>>(C::SMEM_BYTES);
-  if (st != DSA_OK) return st;
-  st = launch(dsa::attend_kernel<DR>, (unsigned)(T * sp.n_split), C::THREADS, C::SMEM_BYTES, stream,
-              sp.merge ? (unsigned)sp.n_split : 1u, qn_map, qp_map, p);
-  if (st != DSA_OK || sp.n_split == 1 || sp.merge) return st;
-  return launch(dsa::attend_combine_kernel, (unsigned)(T * dsa::kHeads), 128, 0, stream, 1, p);
+  DSA_TRY(set_smem(*L.s, kKAttend, dsa::attend_kernel, C::SMEM_BYTES));
+  DSA_TRY(launch(dsa::attend_kernel, (unsigned)(units * sp.n_split), C::THREADS, C::SMEM_BYTES, stream,
+                 sp.merge ? (unsigned)sp.n_split : 1u, p));
+  if (!partials) return DSA_OK;
+  return launch(dsa::attend_combine_kernel, (unsigned)(units * dsa::kHeads), 128, 0, stream, 1, p);
 }
 
-dsa_status_t attend_impl(const void* q_nope, const void* q_pe, const float* qmul, float scale,
-                         const void* cache, int64_t n_rows, int32_t ld_c, int32_t d_rope,
-                         const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
-                         const int32_t* idx, const int32_t* count, int32_t T, int32_t k, void* out,
-                         float* lse, void* ws, cudaStream_t stream) {
-  if (d_rope == 64)
-    return launch_attend<64>(q_nope, q_pe, qmul, scale, cache, n_rows, ld_c, seq_row_start, B, q_seq,
-                             idx, count, T, k, out, lse, ws, stream);
-  return launch_attend<0>(q_nope, q_pe, qmul, scale, cache, n_rows, ld_c, seq_row_start, B, q_seq,
-                          idx, count, T, k, out, lse, ws, stream);
+// Several layers over one selection: launches of up to kMaxAttLayers layers
+// each, in order on the stream (they reuse the same partials region).
+dsa_status_t attend_layers_impl(DevLock& L, const dsa_layer_args* layers, int32_t n_layers, float scale,
+                                int64_t n_rows, const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
+                                const int32_t* q_pos, const int32_t* idx, const int32_t* count, int32_t T,
+                                int32_t k, int64_t q_offset, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  for (int l0 = 0; l0 < n_layers; l0 += dsa::kMaxAttLayers) {
+    const int g = std::min(dsa::kMaxAttLayers, n_layers - l0);
+    dsa_layer_args sub[dsa::kMaxAttLayers];
+    const int64_t qo = q_offset * dsa::kHeads;
+    for (int i = 0; i < g; ++i) {
+      const dsa_layer_args& a = layers[l0 + i];
+      sub[i] = a;
+      sub[i].q_nope = static_cast<const __nv_bfloat16*>(a.q_nope) + qo * dsa::kLatent;
+      sub[i].q_pe = a.q_pe ? static_cast<const __nv_bfloat16*>(a.q_pe) + qo * 64 : nullptr;
+      sub[i].qmul = a.qmul + qo;
+      sub[i].out = static_cast<__nv_bfloat16*>(a.out) + qo * dsa::kLatent;
+      sub[i].lse = a.lse ? a.lse + qo : nullptr;
+    }
+    DSA_TRY(launch_attend(L, sub, g, scale, n_rows, seq_row_start, B, q_seq, q_pos, idx, count, T, k, ws,
+                          ws_bytes, stream));
+  }
+  return DSA_OK;
 }
 
 // ----------------------------------------------------------------- validation helpers
@@ -460,64 +483,85 @@ dsa_status_t check_topk_args(const float* scores, int64_t ld, const int32_t* q_p
   return DSA_OK;
 }
 
-dsa_status_t check_attend_args(const void* q_nope, const void* q_pe, const float* qmul,
-                               const void* cache, int64_t n_rows, int32_t ld_c, int32_t d_rope,
-                               const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
-                               const int32_t* idx, const int32_t* count, int32_t T, int32_t k,
-                               void* out) {
-  DSA_REQUIRE(T >= 0, "T must be >= 0");
-  DSA_REQUIRE(d_rope == 0 || d_rope == 64, "d_rope must be 0 or 64 (got %d)", d_rope);
-  DSA_REQUIRE(q_nope && qmul && cache && seq_row_start && q_seq && idx && count && out,
-              "null pointer argument");
-  DSA_REQUIRE((q_pe != nullptr) == (d_rope == 64), "q_pe must be given iff d_rope == 64");
-  DSA_REQUIRE(aligned(q_nope, 16) && aligned(cache, 16) && aligned(out, 16) &&
-                  (q_pe == nullptr || aligned(q_pe, 16)),
+// One layer's arguments (q_nope, q_pe, qmul, cache, ld_c, d_rope, out, lse).
+dsa_status_t check_layer_args(const dsa_layer_args& a, int64_t n_rows) {
+  DSA_REQUIRE(a.d_rope == 0 || a.d_rope == 64, "d_rope must be 0 or 64 (got %d)", a.d_rope);
+  DSA_REQUIRE(a.q_nope && a.qmul && a.cache && a.out, "null pointer argument");
+  DSA_REQUIRE((a.q_pe != nullptr) == (a.d_rope == 64), "q_pe must be given iff d_rope == 64");
+  DSA_REQUIRE(aligned(a.q_nope, 16) && aligned(a.cache, 16) && aligned(a.out, 16) &&
+                  (a.q_pe == nullptr || aligned(a.q_pe, 16)),
               "q_nope, q_pe, cache and out must be 16-byte aligned");
-  DSA_REQUIRE(aligned(qmul, 4) && aligned(idx, 4) && aligned(count, 4) && aligned(q_seq, 4) &&
-                  aligned(seq_row_start, 8),
-              "misaligned qmul/idx/count/q_seq/seq_row_start");
-  DSA_REQUIRE(ld_c >= dsa::kLatent + d_rope && ld_c % 8 == 0, "ld_c must be >= 512 + d_rope and a multiple of 8");
-  DSA_REQUIRE(n_rows >= 1 && n_rows * (int64_t)ld_c < (int64_t(1) << 62), "n_rows out of range");
-  DSA_REQUIRE(n_rows < (int64_t(1) << 31), "n_rows must be < 2^31");
+  DSA_REQUIRE(aligned(a.qmul, 4) && (a.lse == nullptr || aligned(a.lse, 4)), "misaligned qmul / lse");
+  DSA_REQUIRE(a.ld_c >= dsa::kLatent + a.d_rope && a.ld_c % 8 == 0,
+              "ld_c must be >= 512 + d_rope and a multiple of 8");
+  DSA_REQUIRE(n_rows * (int64_t)a.ld_c < (int64_t(1) << 62), "cache too large");
+  return DSA_OK;
+}
+
+dsa_status_t check_attend_common(int64_t n_rows, const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
+                                 const int32_t* q_pos, const int32_t* idx, const int32_t* count, int32_t T,
+                                 int32_t k) {
+  DSA_REQUIRE(T >= 0, "T must be >= 0");
+  DSA_REQUIRE(seq_row_start && q_seq && idx && count, "null pointer argument");
+  DSA_REQUIRE(aligned(idx, 4) && aligned(count, 4) && aligned(q_seq, 4) && aligned(seq_row_start, 8) &&
+                  (q_pos == nullptr || aligned(q_pos, 4)),
+              "misaligned idx/count/q_seq/q_pos/seq_row_start");
+  DSA_REQUIRE(n_rows >= 1 && n_rows < (int64_t(1) << 31), "n_rows must be in [1, 2^31)");
   DSA_REQUIRE(B >= 1, "B must be >= 1");
   DSA_REQUIRE(k >= 1 && k <= kMaxK, "k must be in [1, %d]", kMaxK);
   DSA_REQUIRE((int64_t)T * dsa::kHeads < (int64_t(1) << 31), "T too large");
   return DSA_OK;
 }
 
+dsa_layer_args one_layer(const void* q_nope, const void* q_pe, const float* qmul, const void* cache, int32_t ld_c,
+                         int32_t d_rope, void* out, float* lse) {
+  dsa_layer_args a;
+  a.q_nope = q_nope;
+  a.q_pe = q_pe;
+  a.qmul = qmul;
+  a.cache = cache;
+  a.ld_c = ld_c;
+  a.d_rope = d_rope;
+  a.out = out;
+  a.lse = lse;
+  return a;
+}
+
+void fill_attend_plan(const dsa::DevProps& d, int64_t units, int32_t k, dsa_attend_plan* out) {
+  const dsa::SplitPlan sp = dsa::attend_plan(d, units, k);
+  out->n_split = sp.n_split;
+  out->rows_per_split = sp.rows_per_split;
+  out->merge = sp.merge ? 1 : 0;
+  out->reserved = 0;
+  out->workspace_bytes = (sp.n_split > 1 && !sp.merge) ? dsa::partial_bytes(units, sp.n_split) : 0;
+}
+
 }  // namespace
 
 // =================================================================== no-allocation variant
 // Scratch for sparse_mla_attend_noalloc: the split partials (numerators, then
-// four statistics per head) of at most kNoAllocMaxPartials (query, split) work units, in
-// the layout launch_attend expects of a workspace.  Every GPU that loads this
-// library holds the array until the process exits.
+// four statistics per head) of at most kNoAllocMaxPartials (query, split) work
+// units, in the layout launch_attend expects of a workspace.  Every GPU that
+// loads this library holds the array until the process exits.
 constexpr int kNoAllocMaxPartials = DSA_NOALLOC_MAX_PARTIALS;
+constexpr size_t kNoAllocBytes = (size_t)kNoAllocMaxPartials * 64 * (512 + 4) * 4;
 static __device__ __align__(256) float g_noalloc_scratch[(size_t)kNoAllocMaxPartials * 64 * (512 + 4)];
+static_assert(dsa::kPlanHeads == 64 && dsa::kPlanLatent == 512, "scratch layout");
 
 namespace {
 
-std::mutex g_noalloc_mu;
-constexpr int kNoAllocMaxDevices = 64;
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
-
-// Device address of the scratch array on the current device, looked up once per
-// device (host code cannot use the array's name as a device pointer).
-dsa_status_t noalloc_scratch(void** out) {
-  int dev = 0;
-  DSA_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kNoAllocMaxDevices)
-    return fail(DSA_ERR_UNSUPPORTED, "device %d: sparse_mla_attend_noalloc supports devices 0..%d", dev,
-                kNoAllocMaxDevices - 1);
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+// Device address of the scratch array in the current context, looked up once
+// per device and context (host code cannot use the array's name as a device
+// pointer: there it is a host-side stand-in).
+dsa_status_t noalloc_scratch(DevLock& L, void** out) {
+  if (L.s->noalloc_ptr == nullptr) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr)
       return fail(DSA_ERR_CUDA, "cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
-    g_noalloc_ptr[dev] = p;
+    L.s->noalloc_ptr = p;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = L.s->noalloc_ptr;
   return DSA_OK;
 }
 
@@ -531,12 +575,12 @@ dsa_status_t dsa_index_scores(const void* q_idx, const float* w, const void* k_i
                               const int32_t* q_pos, int32_t T, int32_t q_group, float* scores,
                               int64_t ld, void* stream) {
   NvtxRange nvtx_range("dsa_index_scores");
-  dsa_status_t st = check_index_args(q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T,
-                                     q_group, ld);
-  if (st != DSA_OK) return st;
+  DSA_TRY(check_index_args(q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, ld));
   DSA_REQUIRE(scores && aligned(scores, 16), "scores must be non-null and 16-byte aligned");
   if (T == 0) return DSA_OK;
-  return indexer_impl(q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, scores, ld,
+  DevLock L;
+  DSA_TRY(lock_device(L));
+  return indexer_impl(L, q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, scores, ld,
                       static_cast<cudaStream_t>(stream));
 }
 
@@ -545,17 +589,18 @@ dsa_status_t dsa_index_scores_fp8(const void* q8, const float* q_scale, const fl
                                   int32_t B, const int32_t* q_seq, const int32_t* q_pos, int32_t T,
                                   int32_t q_group, float* scores, int64_t ld, void* stream) {
   NvtxRange nvtx_range("dsa_index_scores_fp8");
-  dsa_status_t st = check_index_args(q8, w, k8, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, ld);
-  if (st != DSA_OK) return st;
+  DSA_TRY(check_index_args(q8, w, k8, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, ld));
   DSA_REQUIRE(q_scale && k_scale && aligned(q_scale, 4) && aligned(k_scale, 4),
               "q_scale and k_scale must be non-null and 4-byte aligned");
   DSA_REQUIRE(scores && aligned(scores, 16), "scores must be non-null and 16-byte aligned");
   if (T == 0) return DSA_OK;
+  DevLock L;
+  DSA_TRY(lock_device(L));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (q_group == 8)
-    return launch_indexer<8, true>(q8, q_scale, w, k8, k_scale, n_rows, seq_row_start, B, q_seq, q_pos, T,
+    return launch_indexer<8, true>(L, q8, q_scale, w, k8, k_scale, n_rows, seq_row_start, B, q_seq, q_pos, T,
                                    scores, ld, s);
-  return launch_indexer<1, true>(q8, q_scale, w, k8, k_scale, n_rows, seq_row_start, B, q_seq, q_pos, T, scores,
+  return launch_indexer<1, true>(L, q8, q_scale, w, k8, k_scale, n_rows, seq_row_start, B, q_seq, q_pos, T, scores,
                                  ld, s);
 }
 
@@ -566,34 +611,35 @@ dsa_status_t dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, int
   NvtxRange nvtx_range("dsa_topk");
   (void)workspace;
   (void)ws_bytes;
-  dsa_status_t st = check_topk_args(scores, ld, q_pos, T, k, idx, count);
-  if (st != DSA_OK) return st;
+  DSA_TRY(check_topk_args(scores, ld, q_pos, T, k, idx, count));
   if (T == 0) return DSA_OK;
-  return topk_impl(scores, ld, q_pos, T, k, idx, count, static_cast<cudaStream_t>(stream));
+  DevLock L;
+  DSA_TRY(lock_device(L));
+  return topk_impl(L, scores, ld, q_pos, T, k, idx, count, static_cast<cudaStream_t>(stream));
 }
 
 size_t sparse_mla_workspace_size(int32_t T, int32_t k) {
   if (T <= 0 || k <= 0) return 0;
-  return attend_ws_bytes(T, k);
+  dsa::DevProps d;
+  if (props_for_query(nullptr, &d) != DSA_OK) return 0;
+  return dsa::attend_ws_bytes(d, T, k);
 }
 
 dsa_status_t sparse_mla_attend(const void* q_nope, const void* q_pe, const float* qmul,
                                float softmax_scale, const void* cache, int64_t n_rows, int32_t ld_c,
                                int32_t d_rope, const int64_t* seq_row_start, int32_t B,
-                               const int32_t* q_seq, const int32_t* idx, const int32_t* count,
-                               int32_t T, int32_t k, void* out, float* lse, void* workspace,
-                               size_t ws_bytes, void* stream) {
+                               const int32_t* q_seq, const int32_t* q_pos, const int32_t* idx,
+                               const int32_t* count, int32_t T, int32_t k, void* out, float* lse,
+                               void* workspace, size_t ws_bytes, void* stream) {
   NvtxRange nvtx_range("sparse_mla_attend");
-  dsa_status_t st = check_attend_args(q_nope, q_pe, qmul, cache, n_rows, ld_c, d_rope, seq_row_start, B,
-                                      q_seq, idx, count, T, k, out);
-  if (st != DSA_OK) return st;
-  DSA_REQUIRE(lse == nullptr || aligned(lse, 4), "misaligned lse");
+  const dsa_layer_args a = one_layer(q_nope, q_pe, qmul, cache, ld_c, d_rope, out, lse);
+  DSA_TRY(check_attend_common(n_rows, seq_row_start, B, q_seq, q_pos, idx, count, T, k));
+  DSA_TRY(check_layer_args(a, n_rows));
   if (T == 0) return DSA_OK;
-  const size_t need = attend_ws_bytes(T, k);
-  if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)))
-    return fail(DSA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need, ws_bytes);
-  return attend_impl(q_nope, q_pe, qmul, softmax_scale, cache, n_rows, ld_c, d_rope, seq_row_start, B,
-                     q_seq, idx, count, T, k, out, lse, workspace, static_cast<cudaStream_t>(stream));
+  DevLock L;
+  DSA_TRY(lock_device(L));
+  return launch_attend(L, &a, 1, softmax_scale, n_rows, seq_row_start, B, q_seq, q_pos, idx, count, T, k,
+                       workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 // Same computation as sparse_mla_attend, for callers that may not allocate:
@@ -602,46 +648,68 @@ dsa_status_t sparse_mla_attend(const void* q_nope, const void* q_pe, const float
 dsa_status_t sparse_mla_attend_noalloc(const void* q_nope, const void* q_pe, const float* qmul,
                                        float softmax_scale, const void* cache, int64_t n_rows,
                                        int32_t ld_c, int32_t d_rope, const int64_t* seq_row_start,
-                                       int32_t B, const int32_t* q_seq, const int32_t* idx,
-                                       const int32_t* count, int32_t T, int32_t k, void* out,
-                                       float* lse, void* stream) {
+                                       int32_t B, const int32_t* q_seq, const int32_t* q_pos,
+                                       const int32_t* idx, const int32_t* count, int32_t T, int32_t k,
+                                       void* out, float* lse, void* stream) {
   NvtxRange nvtx_range("sparse_mla_attend_noalloc");
-  dsa_status_t st = check_attend_args(q_nope, q_pe, qmul, cache, n_rows, ld_c, d_rope, seq_row_start, B,
-                                      q_seq, idx, count, T, k, out);
-  if (st != DSA_OK) return st;
-  DSA_REQUIRE(lse == nullptr || aligned(lse, 4), "misaligned lse");
+  const dsa_layer_args a = one_layer(q_nope, q_pe, qmul, cache, ld_c, d_rope, out, lse);
+  DSA_TRY(check_attend_common(n_rows, seq_row_start, B, q_seq, q_pos, idx, count, T, k));
+  DSA_TRY(check_layer_args(a, n_rows));
   if (T == 0) return DSA_OK;
-  const SplitPlan sp = attend_plan(T, k);
+  DevLock L;
+  DSA_TRY(lock_device(L));
+  dsa::DevProps props;
+  DSA_TRY(device_props(L, &props));
+  const dsa::SplitPlan sp = dsa::attend_plan(props, T, k);
   void* scratch = nullptr;
+  size_t scratch_bytes = 0;
   if (sp.n_split > 1 && !sp.merge) {
     const int64_t partials = (int64_t)T * sp.n_split;
     if (partials > kNoAllocMaxPartials)
       return fail(DSA_ERR_WORKSPACE,
                   "sparse_mla_attend_noalloc: %d queries split %d ways need %lld partials; its fixed "
-                  "scratch holds %d (use sparse_mla_attend with a workspace, or fewer queries per call)",
+                  "scratch holds %d (use sparse_mla_attend with a workspace, or another batch size: "
+                  "dsa_plan_attend predicts the split)",
                   T, sp.n_split, (long long)partials, kNoAllocMaxPartials);
-    st = noalloc_scratch(&scratch);
-    if (st != DSA_OK) return st;
+    DSA_TRY(noalloc_scratch(L, &scratch));
+    scratch_bytes = kNoAllocBytes;
   }
-  return attend_impl(q_nope, q_pe, qmul, softmax_scale, cache, n_rows, ld_c, d_rope, seq_row_start, B,
-                     q_seq, idx, count, T, k, out, lse, scratch, static_cast<cudaStream_t>(stream));
+  return launch_attend(L, &a, 1, softmax_scale, n_rows, seq_row_start, B, q_seq, q_pos, idx, count, T, k,
+                       scratch, scratch_bytes, static_cast<cudaStream_t>(stream));
 }
 
-// Workspace of the fused call for a chunk of Tc queries:
-//   [idx Tc*k i32][count Tc i32][attention partials][scores Tc*ld f32]
-static size_t forward_chunk_bytes(int32_t Tc, int64_t ld, int32_t k, bool own_idx, bool own_count) {
-  size_t b = 0;
-  if (own_idx) b += round_up((size_t)Tc * k * 4, 256);
-  if (own_count) b += round_up((size_t)Tc * 4, 256);
-  b += attend_ws_bytes(Tc, k);
-  b += round_up((size_t)Tc * ld * 4, 256);
-  return b;
+size_t sparse_mla_layers_workspace_size(int32_t T, int32_t n_layers, int32_t k) {
+  if (T <= 0 || n_layers <= 0 || k <= 0) return 0;
+  dsa::DevProps d;
+  if (props_for_query(nullptr, &d) != DSA_OK) return 0;
+  return dsa::attend_ws_layers(d, T, n_layers, k);
 }
 
-size_t dsa_forward_workspace_size(int32_t T, int64_t ld, int32_t k, int32_t q_group) {
+dsa_status_t sparse_mla_attend_layers(int32_t n_layers, const dsa_layer_args* layers, float softmax_scale,
+                                      int64_t n_rows, const int64_t* seq_row_start, int32_t B,
+                                      const int32_t* q_seq, const int32_t* q_pos, const int32_t* idx,
+                                      const int32_t* count, int32_t T, int32_t k, void* workspace,
+                                      size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("sparse_mla_attend_layers");
+  DSA_REQUIRE(n_layers >= 0 && (n_layers == 0 || layers != nullptr), "bad layer list");
+  DSA_TRY(check_attend_common(n_rows, seq_row_start, B, q_seq, q_pos, idx, count, T, k));
+  for (int l = 0; l < n_layers; ++l) {
+    const dsa_status_t st = check_layer_args(layers[l], n_rows);
+    if (st != DSA_OK) return fail(st, "layer %d: %s", l, g_last_error.c_str());
+  }
+  if (T == 0 || n_layers == 0) return DSA_OK;
+  DevLock L;
+  DSA_TRY(lock_device(L));
+  return attend_layers_impl(L, layers, n_layers, softmax_scale, n_rows, seq_row_start, B, q_seq, q_pos, idx,
+                            count, T, k, 0, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_forward_workspace_size(int32_t T, int64_t ld, int32_t k, int32_t q_group, int32_t n_layers) {
   (void)q_group;
   if (T <= 0 || ld <= 0 || k <= 0) return 0;
-  return forward_chunk_bytes(T, ld, k, true, true);
+  dsa::DevProps d;
+  if (props_for_query(nullptr, &d) != DSA_OK) return 0;
+  return dsa::forward_layout_for(d, T, ld, k, std::max(0, n_layers), true, true, T).end;
 }
 
 dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const void* k_idx, int64_t n_rows,
@@ -652,69 +720,95 @@ dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const voi
                                     int32_t* count_out, void* workspace, size_t ws_bytes,
                                     void* stream) {
   NvtxRange nvtx_range("dsa_sparse_mla_forward");
-  dsa_status_t st = check_index_args(q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T,
-                                     q_group, ld);
-  if (st != DSA_OK) return st;
+  DSA_TRY(check_index_args(q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, ld));
   DSA_REQUIRE(k >= 1 && k <= kMaxK, "k must be in [1, %d]", kMaxK);
   DSA_REQUIRE(n_layers >= 0 && (n_layers == 0 || layers != nullptr), "bad layer list");
   DSA_REQUIRE(idx_out == nullptr || aligned(idx_out, 4), "misaligned idx_out");
   DSA_REQUIRE(count_out == nullptr || aligned(count_out, 4), "misaligned count_out");
   for (int l = 0; l < n_layers; ++l) {
-    const dsa_layer_args& L = layers[l];
-    st = check_attend_args(L.q_nope, L.q_pe, L.qmul, L.cache, n_rows, L.ld_c, L.d_rope, seq_row_start,
-                           B, q_seq, q_seq /* idx checked below */, q_pos, T, k, L.out);
+    const dsa_status_t st = check_layer_args(layers[l], n_rows);
     if (st != DSA_OK) return fail(st, "layer %d: %s", l, g_last_error.c_str());
-    DSA_REQUIRE(L.lse == nullptr || aligned(L.lse, 4), "layer %d: misaligned lse", l);
   }
   if (T == 0) return DSA_OK;
   DSA_REQUIRE(workspace != nullptr && aligned(workspace, 256), "workspace must be non-null and 256-byte aligned");
+  DevLock L;
+  DSA_TRY(lock_device(L));
+  dsa::DevProps props;
+  DSA_TRY(device_props(L, &props));
   const bool own_idx = idx_out == nullptr, own_count = count_out == nullptr;
-  // Largest chunk (a multiple of q_group) whose working set fits the workspace.
-  int32_t Tc = T;
-  while (Tc > q_group && forward_chunk_bytes(Tc, ld, k, own_idx, own_count) > ws_bytes)
-    Tc = std::max<int32_t>(q_group, (Tc / 2 + q_group - 1) / q_group * q_group);
-  if (forward_chunk_bytes(Tc, ld, k, own_idx, own_count) > ws_bytes)
+  const dsa::ForwardLayout f =
+      dsa::forward_layout(props, T, ld, k, q_group, n_layers, own_idx, own_count, ws_bytes);
+  if (f.chunk == 0)
     return fail(DSA_ERR_WORKSPACE, "workspace of %zu bytes is too small (need %zu for %d queries)", ws_bytes,
-                forward_chunk_bytes(Tc, ld, k, own_idx, own_count), Tc);
+                f.end, std::min(T, q_group));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int32_t* idx_ws = nullptr;
-  int32_t* cnt_ws = nullptr;
-  size_t off = 0;
-  if (own_idx) {
-    idx_ws = reinterpret_cast<int32_t*>(ws + off);
-    off += round_up((size_t)Tc * k * 4, 256);
-  }
-  if (own_count) {
-    cnt_ws = reinterpret_cast<int32_t*>(ws + off);
-    off += round_up((size_t)Tc * 4, 256);
-  }
-  void* att_ws = ws + off;
-  off += attend_ws_bytes(Tc, k);
-  float* scores = reinterpret_cast<float*>(ws + off);
+  int32_t* idx_ws = own_idx ? reinterpret_cast<int32_t*>(ws + f.idx_off) : nullptr;
+  int32_t* cnt_ws = own_count ? reinterpret_cast<int32_t*>(ws + f.cnt_off) : nullptr;
+  void* att_ws = ws + f.att_off;
+  float* scores = reinterpret_cast<float*>(ws + f.scores_off);
 
-  for (int32_t t0 = 0; t0 < T; t0 += Tc) {
-    const int32_t n = std::min(Tc, T - t0);
+  for (int32_t t0 = 0; t0 < T; t0 += f.chunk) {
+    const int32_t n = std::min(f.chunk, T - t0);
     int32_t* idx_c = own_idx ? idx_ws : idx_out + (int64_t)t0 * k;
     int32_t* cnt_c = own_count ? cnt_ws : count_out + t0;
-    st = indexer_impl(static_cast<const __nv_bfloat16*>(q_idx) + (int64_t)t0 * dsa::kIdxHeads * dsa::kIdxDim,
-                      w + (int64_t)t0 * dsa::kIdxHeads, k_idx, n_rows, seq_row_start, B, q_seq + t0,
-                      q_pos + t0, n, q_group, scores, ld, s);
-    if (st != DSA_OK) return st;
-    st = topk_impl(scores, ld, q_pos + t0, n, k, idx_c, cnt_c, s);
-    if (st != DSA_OK) return st;
-    for (int l = 0; l < n_layers; ++l) {
-      const dsa_layer_args& L = layers[l];
-      const int64_t qo = (int64_t)t0 * dsa::kHeads;
-      st = attend_impl(static_cast<const __nv_bfloat16*>(L.q_nope) + qo * dsa::kLatent,
-                       L.q_pe ? static_cast<const __nv_bfloat16*>(L.q_pe) + qo * 64 : nullptr,
-                       L.qmul + qo, softmax_scale, L.cache, n_rows, L.ld_c, L.d_rope, seq_row_start, B,
-                       q_seq + t0, idx_c, cnt_c, n, k,
-                       static_cast<__nv_bfloat16*>(L.out) + qo * dsa::kLatent,
-                       L.lse ? L.lse + qo : nullptr, att_ws, s);
-      if (st != DSA_OK) return st;
-    }
+    DSA_TRY(indexer_impl(L, static_cast<const __nv_bfloat16*>(q_idx) + (int64_t)t0 * dsa::kIdxHeads * dsa::kIdxDim,
+                         w + (int64_t)t0 * dsa::kIdxHeads, k_idx, n_rows, seq_row_start, B, q_seq + t0,
+                         q_pos + t0, n, q_group, scores, ld, s));
+    DSA_TRY(topk_impl(L, scores, ld, q_pos + t0, n, k, idx_c, cnt_c, s));
+    DSA_TRY(attend_layers_impl(L, layers, n_layers, softmax_scale, n_rows, seq_row_start, B, q_seq + t0,
+                               q_pos + t0, idx_c, cnt_c, n, k, t0, att_ws, f.att_bytes, s));
   }
+  return DSA_OK;
+}
+
+dsa_status_t dsa_get_device_props(dsa_device_props* out) {
+  DSA_REQUIRE(out != nullptr, "null pointer argument");
+  dsa::DevProps d;
+  DSA_TRY(props_for_query(nullptr, &d));
+  out->sms = d.sms;
+  for (int c = 0; c < 9; ++c) out->max_clusters[c] = d.max_clusters[c];
+  return DSA_OK;
+}
+
+dsa_status_t dsa_plan_attend(int32_t T, int32_t n_layers, int32_t k, const dsa_device_props* props,
+                             dsa_attend_plan* out) {
+  DSA_REQUIRE(out != nullptr, "null pointer argument");
+  DSA_REQUIRE(T >= 1 && n_layers >= 1 && n_layers <= dsa::kMaxAttLayers && k >= 1 && k <= kMaxK,
+              "T >= 1, 1 <= n_layers <= %d and 1 <= k <= %d required", dsa::kMaxAttLayers, kMaxK);
+  dsa::DevProps d;
+  DSA_TRY(props_for_query(props, &d));
+  fill_attend_plan(d, (int64_t)T * n_layers, k, out);
+  return DSA_OK;
+}
+
+dsa_status_t dsa_plan_forward(int32_t T, int64_t ld, int32_t k, int32_t q_group, int32_t n_layers,
+                              int32_t has_idx_out, int32_t has_count_out, size_t ws_bytes,
+                              const dsa_device_props* props, dsa_forward_plan* out) {
+  DSA_REQUIRE(out != nullptr, "null pointer argument");
+  DSA_REQUIRE(T >= 1 && ld >= 4 && k >= 1 && k <= kMaxK && (q_group == 1 || q_group == 8) && n_layers >= 0,
+              "bad sizes");
+  dsa::DevProps d;
+  DSA_TRY(props_for_query(props, &d));
+  const dsa::ForwardLayout f = dsa::forward_layout(d, T, ld, k, q_group, n_layers, !has_idx_out, !has_count_out,
+                                                   ws_bytes);
+  out->chunk = f.chunk;
+  out->n_chunks = f.chunk ? f.n_chunks : 0;
+  out->last_chunk = f.chunk ? f.last_chunk : 0;
+  out->reserved = 0;
+  out->idx_offset = f.idx_off;
+  out->count_offset = f.cnt_off;
+  out->attend_offset = f.att_off;
+  out->attend_bytes = f.att_bytes;
+  out->scores_offset = f.scores_off;
+  out->end = f.end;
+  if (f.chunk == 0) return fail(DSA_ERR_WORKSPACE, "workspace of %zu bytes is too small (need %zu)", ws_bytes, f.end);
+  return DSA_OK;
+}
+
+dsa_status_t dsa_set_fault_test(uint64_t wait_limit_ns, int32_t stall_tile) {
+  g_wait_limit_ns.store(wait_limit_ns, std::memory_order_relaxed);
+  g_stall_tile.store(stall_tile < 0 ? -1 : stall_tile, std::memory_order_relaxed);
   return DSA_OK;
 }
 
@@ -734,6 +828,6 @@ uint64_t dsa_launch_count(void) { return g_launches.load(std::memory_order_relax
 
 const char* dsa_last_error(void) { return g_last_error.c_str(); }
 
-int32_t dsa_version(void) { return 100; }
+int32_t dsa_version(void) { return 200; }
 
 }  // extern "C"

@@ -98,21 +98,22 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs of wall time, raises kErrTimeout and returns false so that the
-// caller can unwind instead of hanging the GPU.
+// `limit_ns` of wall time (default kWaitLimitNs), raises kErrTimeout and
+// returns false so that the caller can unwind instead of hanging the GPU.
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s: far above any legal wait
 
 // When `abort` is non-null the wait also gives up (without raising) as soon as
 // another role of the CTA has set *abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          const volatile int* abort = nullptr) {
+                                          const volatile int* abort = nullptr,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if ((++spins & 255u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         raise_error(kErrTimeout);
         return false;
       }

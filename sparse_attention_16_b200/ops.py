@@ -39,19 +39,48 @@ class LayerArgs(ctypes.Structure):
                 ("d_rope", _I32), ("out", _P), ("lse", _P)]
 
 
+class DeviceProps(ctypes.Structure):
+    """Mirror of ``dsa_device_props``."""
+
+    _fields_ = [("sms", _I32), ("max_clusters", _I32 * 9)]
+
+
+class AttendPlan(ctypes.Structure):
+    """Mirror of ``dsa_attend_plan``."""
+
+    _fields_ = [("n_split", _I32), ("rows_per_split", _I32), ("merge", _I32), ("reserved", _I32),
+                ("workspace_bytes", _SZ)]
+
+
+class ForwardPlan(ctypes.Structure):
+    """Mirror of ``dsa_forward_plan``."""
+
+    _fields_ = [("chunk", _I32), ("n_chunks", _I32), ("last_chunk", _I32), ("reserved", _I32),
+                ("idx_offset", _SZ), ("count_offset", _SZ), ("attend_offset", _SZ), ("attend_bytes", _SZ),
+                ("scores_offset", _SZ), ("end", _SZ)]
+
+
 SIGNATURES = {
     "dsa_index_scores": (_I32, [_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _P, _I64, _P]),
     "dsa_index_scores_fp8": (_I32, [_P, _P, _P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _P, _I64, _P]),
     "dsa_topk_workspace_size": (_SZ, [_I32, _I64, _I32]),
     "dsa_topk": (_I32, [_P, _I64, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "sparse_mla_workspace_size": (_SZ, [_I32, _I32]),
-    "sparse_mla_attend": (_I32, [_P, _P, _P, _F, _P, _I64, _I32, _I32, _P, _I32, _P, _P, _P, _I32,
+    "sparse_mla_attend": (_I32, [_P, _P, _P, _F, _P, _I64, _I32, _I32, _P, _I32, _P, _P, _P, _P, _I32,
                                  _I32, _P, _P, _P, _SZ, _P]),
-    "sparse_mla_attend_noalloc": (_I32, [_P, _P, _P, _F, _P, _I64, _I32, _I32, _P, _I32, _P, _P, _P,
+    "sparse_mla_attend_noalloc": (_I32, [_P, _P, _P, _F, _P, _I64, _I32, _I32, _P, _I32, _P, _P, _P, _P,
                                          _I32, _I32, _P, _P, _P]),
-    "dsa_forward_workspace_size": (_SZ, [_I32, _I64, _I32, _I32]),
+    "sparse_mla_layers_workspace_size": (_SZ, [_I32, _I32, _I32]),
+    "sparse_mla_attend_layers": (_I32, [_I32, ctypes.POINTER(LayerArgs), _F, _I64, _P, _I32, _P, _P, _P, _P,
+                                        _I32, _I32, _P, _SZ, _P]),
+    "dsa_forward_workspace_size": (_SZ, [_I32, _I64, _I32, _I32, _I32]),
     "dsa_sparse_mla_forward": (_I32, [_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I64, _I32,
                                       ctypes.POINTER(LayerArgs), _F, _I32, _P, _P, _P, _SZ, _P]),
+    "dsa_get_device_props": (_I32, [ctypes.POINTER(DeviceProps)]),
+    "dsa_plan_attend": (_I32, [_I32, _I32, _I32, ctypes.POINTER(DeviceProps), ctypes.POINTER(AttendPlan)]),
+    "dsa_plan_forward": (_I32, [_I32, _I64, _I32, _I32, _I32, _I32, _I32, _SZ, ctypes.POINTER(DeviceProps),
+                                ctypes.POINTER(ForwardPlan)]),
+    "dsa_set_fault_test": (_I32, [ctypes.c_uint64, _I32]),
     "dsa_check_errors": (_I32, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "dsa_launch_count": (ctypes.c_uint64, []),
     "dsa_last_error": (ctypes.c_char_p, []),
@@ -174,8 +203,47 @@ def attend_workspace_bytes(T, k):
     return int(load_library().sparse_mla_workspace_size(T, k))
 
 
-def forward_workspace_bytes(T, ld, k, q_group=1):
-    return int(load_library().dsa_forward_workspace_size(T, ld, k, q_group))
+def forward_workspace_bytes(T, ld, k, q_group=1, n_layers=1):
+    return int(load_library().dsa_forward_workspace_size(T, ld, k, q_group, n_layers))
+
+
+def device_props():
+    """SM count and attention cluster residency of the current device (dsa_get_device_props)."""
+    out = DeviceProps()
+    _check(load_library().dsa_get_device_props(ctypes.byref(out)))
+    return out
+
+
+def make_props(sms, max_clusters):
+    """A DeviceProps for planning without a GPU: max_clusters maps size c (2..8) to resident clusters."""
+    d = DeviceProps()
+    d.sms = sms
+    for c, n in dict(max_clusters).items():
+        d.max_clusters[c] = n
+    return d
+
+
+def plan_attend(T, n_layers=1, k=2048, props=None):
+    """How the attention splits T queries x n_layers layers (dsa_plan_attend)."""
+    out = AttendPlan()
+    _check(load_library().dsa_plan_attend(T, n_layers, k, ctypes.byref(props) if props is not None else None,
+                                          ctypes.byref(out)))
+    return out
+
+
+def plan_forward(T, ld, k, q_group, n_layers, has_idx_out, has_count_out, ws_bytes, props=None):
+    """Chunking and workspace layout of dsa_sparse_mla_forward (dsa_plan_forward); raises
+    DSAError(DSA_ERR_WORKSPACE) when nothing fits."""
+    out = ForwardPlan()
+    _check(load_library().dsa_plan_forward(T, ld, k, q_group, n_layers, int(bool(has_idx_out)),
+                                           int(bool(has_count_out)), ws_bytes,
+                                           ctypes.byref(props) if props is not None else None, ctypes.byref(out)))
+    return out
+
+
+def set_fault_test(wait_limit_ns=0, stall_tile=-1):
+    """Testing hook of the attention kernel's timeout path (dsa_set_fault_test); (0, -1) = off."""
+    _check(load_library().dsa_set_fault_test(int(wait_limit_ns), int(stall_tile)))
 
 
 def workspace(nbytes, device):
@@ -184,7 +252,7 @@ def workspace(nbytes, device):
 
 
 def sparse_mla_attend(q_nope, q_pe, qmul, cache, d_rope, seq_row_start, q_seq, idx, count, out,
-                      lse=None, softmax_scale=SOFTMAX_SCALE, ws=None, stream=None):
+                      lse=None, softmax_scale=SOFTMAX_SCALE, ws=None, stream=None, q_pos=None):
     """Absorbed sparse MLA into ``out`` [T, 64, 512] bf16 (see sparse_mla_attend)."""
     T = q_nope.shape[0]
     k = idx.shape[1]
@@ -202,16 +270,18 @@ def sparse_mla_attend(q_nope, q_pe, qmul, cache, d_rope, seq_row_start, q_seq, i
     need = attend_workspace_bytes(T, k)
     if ws is None and need > 0:
         ws = workspace(need, q_nope.device)
+    if q_pos is not None:
+        _need(q_pos, torch.int32, (T,), "q_pos")
     _check(lib.sparse_mla_attend(_ptr(q_nope), _ptr(q_pe) if d_rope else None, _ptr(qmul),
                                  float(softmax_scale), _ptr(cache), cache.shape[0], cache.shape[1],
-                                 d_rope, _ptr(seq_row_start), seq_row_start.shape[0], _ptr(q_seq),
+                                 d_rope, _ptr(seq_row_start), seq_row_start.shape[0], _ptr(q_seq), _ptr(q_pos),
                                  _ptr(idx), _ptr(count), T, k, _ptr(out), _ptr(lse), _ptr(ws),
                                  0 if ws is None else ws.numel(), _stream(stream)))
     return out, lse
 
 
 def sparse_mla_attend_noalloc(q_nope, q_pe, qmul, cache, d_rope, seq_row_start, q_seq, idx, count,
-                              out, lse=None, softmax_scale=SOFTMAX_SCALE, stream=None):
+                              out, lse=None, softmax_scale=SOFTMAX_SCALE, stream=None, q_pos=None):
     """Same as sparse_mla_attend without a workspace, for callers that may not
     allocate device memory: the library's fixed scratch array holds the split
     partials (see sparse_mla_attend_noalloc in include/dsa.h for the limit and
@@ -229,12 +299,61 @@ def sparse_mla_attend_noalloc(q_nope, q_pe, qmul, cache, d_rope, seq_row_start, 
     if lse is not None:
         _need(lse, torch.float32, (T, 64), "lse")
     lib = load_library()
+    if q_pos is not None:
+        _need(q_pos, torch.int32, (T,), "q_pos")
     _check(lib.sparse_mla_attend_noalloc(_ptr(q_nope), _ptr(q_pe) if d_rope else None, _ptr(qmul),
                                          float(softmax_scale), _ptr(cache), cache.shape[0], cache.shape[1],
                                          d_rope, _ptr(seq_row_start), seq_row_start.shape[0], _ptr(q_seq),
-                                         _ptr(idx), _ptr(count), T, k, _ptr(out), _ptr(lse),
+                                         _ptr(q_pos), _ptr(idx), _ptr(count), T, k, _ptr(out), _ptr(lse),
                                          _stream(stream)))
     return out, lse
+
+
+def _layer_array(layers, T):
+    arr = (LayerArgs * max(1, len(layers)))()
+    for i, L in enumerate(layers):
+        _need(L["q_nope"], torch.bfloat16, (T, 64, 512), f"layers[{i}].q_nope")
+        if L["d_rope"]:
+            _need(L["q_pe"], torch.bfloat16, (T, 64, L["d_rope"]), f"layers[{i}].q_pe")
+        _need(L["qmul"], torch.float32, (T, 64), f"layers[{i}].qmul")
+        _need(L["cache"], torch.bfloat16, None, f"layers[{i}].cache")
+        _need(L["out"], torch.bfloat16, (T, 64, 512), f"layers[{i}].out")
+        if L.get("lse") is not None:
+            _need(L["lse"], torch.float32, (T, 64), f"layers[{i}].lse")
+        arr[i] = LayerArgs(L["q_nope"].data_ptr(),
+                           L["q_pe"].data_ptr() if L.get("q_pe") is not None else None,
+                           L["qmul"].data_ptr(), L["cache"].data_ptr(), L["cache"].shape[1],
+                           L["d_rope"], L["out"].data_ptr(),
+                           L["lse"].data_ptr() if L.get("lse") is not None else None)
+    return arr
+
+
+def layers_workspace_bytes(T, n_layers, k):
+    return int(load_library().sparse_mla_layers_workspace_size(T, n_layers, k))
+
+
+def sparse_mla_attend_layers(layers, n_rows, seq_row_start, q_seq, idx, count, q_pos=None,
+                             softmax_scale=SOFTMAX_SCALE, ws=None, stream=None):
+    """Attention of several layers over one shared selection (see sparse_mla_attend_layers).
+
+    ``layers``: list of dicts with q_nope, q_pe (or None), qmul, cache, d_rope, out, lse (or None);
+    every cache has ``n_rows`` rows.
+    """
+    T, k = idx.shape
+    _need(idx, torch.int32, (T, k), "idx")
+    _need(count, torch.int32, (T,), "count")
+    _need(seq_row_start, torch.int64, None, "seq_row_start")
+    _need(q_seq, torch.int32, (T,), "q_seq")
+    if q_pos is not None:
+        _need(q_pos, torch.int32, (T,), "q_pos")
+    arr = _layer_array(layers, T)
+    lib = load_library()
+    need = layers_workspace_bytes(T, len(layers), k)
+    if ws is None and need > 0:
+        ws = workspace(need, idx.device)
+    _check(lib.sparse_mla_attend_layers(len(layers), arr, float(softmax_scale), n_rows, _ptr(seq_row_start),
+                                        seq_row_start.shape[0], _ptr(q_seq), _ptr(q_pos), _ptr(idx), _ptr(count),
+                                        T, k, _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def sparse_mla_forward(q_idx, w, k_idx, seq_row_start, q_seq, q_pos, layers, ld, k=2048, q_group=1,
@@ -247,18 +366,10 @@ def sparse_mla_forward(q_idx, w, k_idx, seq_row_start, q_seq, q_pos, layers, ld,
     T = q_idx.shape[0]
     _need(q_idx, torch.bfloat16, (T, 32, 128), "q_idx")
     _need(w, torch.float32, (T, 32), "w")
-    arr = (LayerArgs * max(1, len(layers)))()
-    for i, L in enumerate(layers):
-        _need(L["q_nope"], torch.bfloat16, (T, 64, 512), f"layers[{i}].q_nope")
-        _need(L["out"], torch.bfloat16, (T, 64, 512), f"layers[{i}].out")
-        arr[i] = LayerArgs(L["q_nope"].data_ptr(),
-                           L["q_pe"].data_ptr() if L.get("q_pe") is not None else None,
-                           L["qmul"].data_ptr(), L["cache"].data_ptr(), L["cache"].shape[1],
-                           L["d_rope"], L["out"].data_ptr(),
-                           L["lse"].data_ptr() if L.get("lse") is not None else None)
+    arr = _layer_array(layers, T)
     lib = load_library()
     if ws is None:
-        ws = workspace(forward_workspace_bytes(T, ld, k, q_group), q_idx.device)
+        ws = workspace(forward_workspace_bytes(T, ld, k, q_group, len(layers)), q_idx.device)
     _check(lib.dsa_sparse_mla_forward(_ptr(q_idx), _ptr(w), _ptr(k_idx), k_idx.shape[0],
                                       _ptr(seq_row_start), seq_row_start.shape[0], _ptr(q_seq),
                                       _ptr(q_pos), T, q_group, ld, len(layers), arr,

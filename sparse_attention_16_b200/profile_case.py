@@ -25,7 +25,8 @@ def main():
     ap.add_argument("--kernel", choices=["indexer", "topk", "attend"], required=True)
     ap.add_argument("--config", default="decode_b64_32k", choices=sorted(CONFIGS))
     ap.add_argument("--launches", type=int, default=3)
-    ap.add_argument("--layer", type=int, default=0, help="attention: which layer of the configuration")
+    ap.add_argument("--layer", type=int, default=-1,
+                    help="attention: one layer of the configuration (default: all its layers in one launch)")
     ap.add_argument("--fp8", action="store_true", help="indexer: FP8 (E4M3) keys and queries, per-row scales")
     a = ap.parse_args()
 
@@ -60,14 +61,16 @@ def main():
         topk()
     run = {"indexer": indexer, "topk": topk}.get(a.kernel)
     if a.kernel == "attend":
-        lay = wl.layers[a.layer]
-        out = torch.empty((T, 64, 512), dtype=torch.bfloat16, device=dev)
-        lse = torch.empty((T, 64), dtype=torch.float32, device=dev)
-        ws = ops.workspace(ops.attend_workspace_bytes(T, k), dev)
+        chosen = wl.layers if a.layer < 0 else [wl.layers[a.layer]]
+        outs = [torch.empty((T, 64, 512), dtype=torch.bfloat16, device=dev) for _ in chosen]
+        lses = [torch.empty((T, 64), dtype=torch.float32, device=dev) for _ in chosen]
+        layers = [dict(q_nope=L.q_nope, q_pe=L.q_pe, qmul=L.qmul, cache=L.cache, d_rope=L.d_rope, out=o, lse=l)
+                  for L, o, l in zip(chosen, outs, lses)]
+        ws = ops.workspace(ops.layers_workspace_bytes(T, len(layers), k), dev)
 
         def run():
-            ops.sparse_mla_attend(lay.q_nope, lay.q_pe, lay.qmul, lay.cache, lay.d_rope, wl.seq_row_start,
-                                  wl.q_seq, idx, cnt, out, lse, ws=ws)
+            ops.sparse_mla_attend_layers(layers, chosen[0].cache.shape[0], wl.seq_row_start, wl.q_seq, idx, cnt,
+                                         q_pos=wl.q_pos, ws=ws)
 
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -177,24 +177,65 @@ def test_attention_matches_oracle_single_split_path(d_rope):
     pu.assert_attention_close(to_numpy(o)[ts], to_numpy(lse)[ts], ref_o, ref_l)
 
 
-@pytest.mark.parametrize("T", [64, 40, 36, 27, 24, 21, 14, 10])
-def test_attention_matches_oracle_cluster_merge_path(T):
-    # With 2-8 CTAs per query (2 to 8 for these batch sizes on 148 SMs)
-    # the CTAs of a query merge their partials in distributed shared memory and
-    # no workspace is needed.  Short selections leave trailing CTAs empty.
-    if ops.attend_workspace_bytes(T, 2048) != 0:
-        pytest.skip("this GPU's split plan for this batch size uses the combine kernel")
-    rng = np.random.default_rng(T)
-    lengths = tuple(int(x) for x in rng.integers(2100, 6000, size=T))
-    case = small_case(f"attn_merge{T}", lengths, layers=(64,), seed=40 + T, mla_q_std=1.0)
+def _merge_widths():
+    """(T, n_layers) of the smallest batch for which this GPU's plan merges a
+    (layer, query)'s splits in a cluster of each width (2-8 blocks)."""
+    found = {}
+    for n_layers in (1, 2, 4):
+        for T in range(1, 149):
+            p = ops.plan_attend(T, n_layers, 2048)
+            if p.merge and p.n_split not in found:
+                found[p.n_split] = (T, n_layers)
+    return found
+
+
+def test_attention_cluster_merge_every_width_the_gpu_runs():
+    # The splits of a (layer, query) merge their partials in distributed shared
+    # memory when every cluster of that width can be resident at once.  The
+    # batch sizes come from the library's own plan for this GPU, so every width
+    # the GPU can run is exercised.  Short selections leave trailing CTAs empty.
+    found = _merge_widths()
+    assert len(found) >= 3, found
+    for width, (T, n_layers) in sorted(found.items()):
+        rng = np.random.default_rng(T * 10 + n_layers)
+        lengths = tuple(int(x) for x in rng.integers(2100, 6000, size=T))
+        rope = [64, 0, 64, 64][:n_layers]
+        case = small_case(f"merge{width}", lengths, layers=tuple(rope), seed=40 + width, mla_q_std=1.0)
+        wl = make_workload(case, DEV)
+        counts = [2048 if i % 4 else int(rng.integers(1, 700)) for i in range(T)]
+        idx, cnt = _random_selection(wl, counts, sort=(T % 2 == 0), holes=True, seed=T)
+        plan = ops.plan_attend(T, n_layers, 2048)
+        assert plan.merge and plan.n_split == width
+        outs, lses = _attend_layers(wl, idx, cnt)
+        ts = sorted(set(range(0, T, max(1, T // 4))) | {T - 1})
+        for lay, o, l in zip(wl.layers, outs, lses):
+            ref_o, ref_l = pu.oracle_attend(wl, lay, ts, idx, cnt)
+            pu.assert_attention_close(to_numpy(o)[ts], to_numpy(l)[ts], ref_o, ref_l)
+
+
+def _attend_layers(wl, idx, cnt, q_pos=None):
+    T = wl.T
+    outs = [torch.empty((T, 64, 512), dtype=torch.bfloat16, device=DEV) for _ in wl.layers]
+    lses = [torch.empty((T, 64), dtype=torch.float32, device=DEV) for _ in wl.layers]
+    layers = [dict(q_nope=L.q_nope, q_pe=L.q_pe, qmul=L.qmul, cache=L.cache, d_rope=L.d_rope, out=o, lse=l)
+              for L, o, l in zip(wl.layers, outs, lses)]
+    ops.sparse_mla_attend_layers(layers, wl.layers[0].cache.shape[0], wl.seq_row_start, wl.q_seq,
+                                 torch.as_tensor(idx, device=DEV), torch.as_tensor(cnt, device=DEV), q_pos=q_pos)
+    torch.cuda.synchronize()
+    return outs, lses
+
+
+def test_attend_layers_mixed_rope_and_nope_share_one_selection():
+    # Four layers (three RoPE, one NoPE, as the 1M-context decode configuration)
+    # in one launch over one selection: each layer against the oracle.
+    case = small_case("layers4", (5000, 3000, 2100, 900), layers=(64, 64, 64, 0), seed=26)
     wl = make_workload(case, DEV)
-    counts = [2048 if i % 4 else int(rng.integers(1, 700)) for i in range(T)]
-    idx, cnt = _random_selection(wl, counts, sort=(T % 2 == 0), holes=True, seed=T)
-    lay = wl.layers[0]
-    o, lse = pu.gpu_attend(wl, lay, torch.as_tensor(idx, device=DEV), torch.as_tensor(cnt, device=DEV))
-    ts = sorted(set(range(0, T, 3)) | {T - 1})
-    ref_o, ref_l = pu.oracle_attend(wl, lay, ts, idx, cnt)
-    pu.assert_attention_close(to_numpy(o)[ts], to_numpy(lse)[ts], ref_o, ref_l)
+    idx, cnt = _random_selection(wl, [2048, 2048, 2048, 900], seed=9, sort=False, holes=True)
+    outs, lses = _attend_layers(wl, idx, cnt, q_pos=wl.q_pos)
+    for lay, o, l in zip(wl.layers, outs, lses):
+        ref_o, ref_l = pu.oracle_attend(wl, lay, list(range(wl.T)), idx, cnt)
+        pu.assert_attention_close(to_numpy(o), to_numpy(l), ref_o, ref_l)
+    assert ops.check_errors() == 0
 
 
 def test_attention_empty_selection_gives_zero_and_minus_inf():
@@ -267,12 +308,77 @@ def test_forward_one_selection_feeds_rope_and_nope_layers_with_chunking():
                    lse=l) for L, o, l in zip(wl.layers, outs, lses)]
     idx = torch.empty((T, 2048), dtype=torch.int32, device=DEV)
     cnt = torch.empty((T,), dtype=torch.int32, device=DEV)
-    # a workspace for 16 queries forces three chunks (16 + 16 + 8)
-    ws = ops.workspace(ops.forward_workspace_bytes(16, ld, 2048, 8), DEV)
+    # a workspace for 16 queries forces several chunks; a canary after it must survive
+    ws_bytes = ops.forward_workspace_bytes(16, ld, 2048, 8, 2)
+    plan = ops.plan_forward(T, ld, 2048, 8, 2, 1, 1, ws_bytes)
+    assert plan.n_chunks > 1
+    buf = torch.full((ws_bytes + (2 << 20),), 0xA5, dtype=torch.uint8, device=DEV)
     ops.sparse_mla_forward(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, layers, ld,
-                           q_group=8, idx_out=idx, count_out=cnt, ws=ws)
+                           q_group=8, idx_out=idx, count_out=cnt, ws=buf[:ws_bytes])
     torch.cuda.synchronize()
+    assert bool((buf[ws_bytes:] == 0xA5).all()), "the fused call wrote past its workspace"
     idx_h, cnt_h = to_numpy(idx), to_numpy(cnt)
+    s_ref = pu.oracle_scores(wl, list(range(T)), ld)
+    for t in range(T):
+        n = int(to_numpy(wl.q_pos)[t]) + 1
+        pu.assert_selection_overlap(idx_h[t, :cnt_h[t]], s_ref[t, :n], 2048)
+    for L, o, l in zip(wl.layers, outs, lses):
+        ref_o, ref_l = pu.oracle_attend(wl, L, list(range(T)), idx_h, cnt_h)
+        pu.assert_attention_close(to_numpy(o), to_numpy(l), ref_o, ref_l)
+
+
+def test_forward_tail_chunk_stays_inside_the_workspace():
+    # 151 decode queries at context 4,096 with a workspace sized for 148: the
+    # last chunk is planned differently from the full ones (a small batch is
+    # split wider).  A 2 MB canary after the workspace must survive, and the
+    # results must match the oracle.
+    case = small_case("tail151", (4096,) * 151, seed=25)
+    wl = make_workload(case, DEV)
+    T, ld = wl.T, case.ld
+    lay = wl.layers[0]
+    out = torch.empty((T, 64, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((T, 64), dtype=torch.float32, device=DEV)
+    ws_bytes = ops.forward_workspace_bytes(148, ld, 2048, 1, 1)
+    plan = ops.plan_forward(T, ld, 2048, 1, 1, 0, 0, ws_bytes)
+    assert plan.n_chunks > 1 and plan.end <= ws_bytes
+    buf = torch.full((ws_bytes + (2 << 20),), 0x5A, dtype=torch.uint8, device=DEV)
+    idx = torch.empty((T, 2048), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((T,), dtype=torch.int32, device=DEV)
+    ops.sparse_mla_forward(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos,
+                           [dict(q_nope=lay.q_nope, q_pe=lay.q_pe, qmul=lay.qmul, cache=lay.cache, d_rope=64,
+                                 out=out, lse=lse)], ld, ws=buf[:ws_bytes])
+    torch.cuda.synchronize()
+    assert bool((buf[ws_bytes:] == 0x5A).all()), "the fused call wrote past its workspace"
+    assert ops.check_errors() == 0
+    # the same selection through the separate calls, for the sampled queries' parity
+    s = pu.gpu_scores(wl)
+    idx2, cnt2 = pu.gpu_topk(s, wl.q_pos, 2048)
+    ts = [0, 37, 75, 112, 147, 148, 150]
+    idx_h, cnt_h = to_numpy(idx2), to_numpy(cnt2)
+    ref_s = pu.oracle_scores(wl, ts, ld)
+    for i, t in enumerate(ts):
+        pu.assert_selection_overlap(idx_h[t, :cnt_h[t]], ref_s[i, :4096], 2048)
+    ref_o, ref_l = pu.oracle_attend(wl, lay, ts, idx_h, cnt_h)
+    pu.assert_attention_close(to_numpy(out)[ts], to_numpy(lse)[ts], ref_o, ref_l)
+
+
+def test_forward_four_layers_small_decode():
+    # The 1M-context configuration's shape of work (4 queries, one selection ->
+    # 3 RoPE + 1 NoPE layers) at small contexts, through the fused call.
+    case = small_case("fwd4", (9000, 5000, 2049, 700), layers=(64, 64, 64, 0), seed=27)
+    wl = make_workload(case, DEV)
+    T, ld = wl.T, case.ld
+    outs = [torch.empty((T, 64, 512), dtype=torch.bfloat16, device=DEV) for _ in wl.layers]
+    lses = [torch.empty((T, 64), dtype=torch.float32, device=DEV) for _ in wl.layers]
+    layers = [dict(q_nope=L.q_nope, q_pe=L.q_pe, qmul=L.qmul, cache=L.cache, d_rope=L.d_rope, out=o,
+                   lse=l) for L, o, l in zip(wl.layers, outs, lses)]
+    idx = torch.empty((T, 2048), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((T,), dtype=torch.int32, device=DEV)
+    ops.sparse_mla_forward(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, layers, ld,
+                           idx_out=idx, count_out=cnt)
+    assert ops.check_errors() == 0
+    idx_h, cnt_h = to_numpy(idx), to_numpy(cnt)
+    assert cnt_h.tolist() == [2048, 2048, 2048, 700]
     s_ref = pu.oracle_scores(wl, list(range(T)), ld)
     for t in range(T):
         n = int(to_numpy(wl.q_pos)[t]) + 1
@@ -299,6 +405,32 @@ def test_bad_indices_are_flagged_not_faulted():
     assert "0x1" in str(e.value)
     assert ops.check_errors() == 0   # cleared; the context is still usable
     assert torch.isfinite(out.float()).all()
+
+
+def test_positions_past_q_pos_are_flagged_and_skipped():
+    # A selected position past the query's own position (here: inside the cache,
+    # in the next sequence's rows) is skipped and flagged when q_pos is given.
+    case = small_case("qpos", (3000, 2500, 1000), seed=24)
+    wl = make_workload(case, DEV)
+    idx, cnt = _random_selection(wl, [500, 400, 300], seed=8)
+    bad = idx.copy()
+    bad[0, 10] = 3005          # sequence 1's rows
+    bad[1, 20] = 2600          # sequence 2's rows
+    lay = wl.layers[0]
+    out = torch.empty((3, 64, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((3, 64), dtype=torch.float32, device=DEV)
+    ops.sparse_mla_attend(lay.q_nope, lay.q_pe, lay.qmul, lay.cache, 64, wl.seq_row_start, wl.q_seq,
+                          torch.as_tensor(bad, device=DEV), torch.as_tensor(cnt, device=DEV), out, lse,
+                          q_pos=wl.q_pos)
+    with pytest.raises(ops.DSAError) as e:
+        ops.check_errors()
+    assert "0x1" in str(e.value)
+    skipped = bad.copy()
+    skipped[0, 10] = -1
+    skipped[1, 20] = -1
+    ref_o, ref_l = pu.oracle_attend(wl, lay, [0, 1, 2], skipped, cnt)
+    pu.assert_attention_close(to_numpy(out), to_numpy(lse), ref_o, ref_l)
+    assert ops.check_errors() == 0
 
 
 def test_bad_sequence_ids_are_flagged():

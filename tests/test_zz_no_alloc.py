@@ -5,9 +5,10 @@ pool and can synchronize the device).  Its split partials live in a fixed scratc
 array inside the library instead of a caller workspace.
 
 Checked through the C ABI against sparse_mla_attend (the entry point that takes a
-workspace) with the attention tolerances used everywhere else, on two calls in a
-row with different inputs, so stale scratch contents from the first call would
-show up in the second.  This file is collected last on purpose.
+workspace) and against the CPU oracle, with the attention tolerances used
+everywhere else, on two calls in a row with different inputs, so stale scratch
+contents from the first call would show up in the second.  This file is
+collected last on purpose.
 """
 
 import numpy as np
@@ -57,13 +58,23 @@ def _both(wl, lay, idx, cnt):
     return o, l, ref_o, ref_l
 
 
+def _scratch_batch():
+    """A batch size whose split partials go through the scratch on this GPU
+    (split across blocks that do not merge on chip, within the scratch limit)."""
+    for T in range(8, 0, -1):
+        p = ops.plan_attend(T, 1, 2048)
+        if p.workspace_bytes > 0 and T * p.n_split <= 128:
+            return T
+    pytest.fail("no batch of 1-8 queries uses the scratch on this GPU")
+
+
 @pytest.mark.parametrize("d_rope", [64, 0])
 def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(d_rope):
-    # 6 queries: each selection is split across several blocks, so the scratch is used.
-    assert ops.attend_workspace_bytes(6, 2048) > 0
-    wl1 = make_workload(small_case("na1", (4096, 3000, 2500, 600, 2049, 90), layers=(d_rope,), seed=31), DEV)
-    wl2 = make_workload(small_case("na2", (5000, 2048, 100, 4000, 3333, 777), layers=(d_rope,), seed=32,
-                                   mla_q_std=1.0), DEV)
+    T = _scratch_batch()
+    wl1 = make_workload(small_case("na1", (4096, 3000, 2500, 600, 2049, 90, 5000, 2100)[:T], layers=(d_rope,),
+                                   seed=31), DEV)
+    wl2 = make_workload(small_case("na2", (5000, 2048, 100, 4000, 3333, 777, 2200, 4100)[:T], layers=(d_rope,),
+                                   seed=32, mla_q_std=1.0), DEV)
     for wl, seed in ((wl1, 1), (wl2, 2)):
         idx, cnt = _selection(wl, seed)
         o, l, ref_o, ref_l = _both(wl, wl.layers[0], idx, cnt)
@@ -72,20 +83,26 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(d_rope):
         for t in range(wl.T):
             assert np.abs(g[t] - r[t]).max() <= pu.ATTN_REL * np.abs(r[t]).max() + 1e-6
         assert np.abs(to_numpy(l).astype(np.float64) - to_numpy(ref_l)).max() <= pu.LSE_ATOL
+        # and against the oracle on the same selection
+        ts = list(range(wl.T))
+        o_ref, l_ref = pu.oracle_attend(wl, wl.layers[0], ts, to_numpy(idx), to_numpy(cnt))
+        pu.assert_attention_close(to_numpy(o), to_numpy(l), o_ref, l_ref)
     assert ops.check_errors() == 0
 
 
 def test_noalloc_rejects_more_partials_than_its_scratch_holds():
-    # A workspace partial is 64 heads x (512 numerators + 4 statistics) floats.
-    per_partial = 64 * (512 + 4) * 4
-    # a batch size whose split plan needs more partials than the fixed scratch holds
-    T = next(T for T in range(1, 4096)
-             if ops.attend_workspace_bytes(T, 2048) // per_partial > 128)
+    # A batch (and selection width k) whose split plan needs more partials than
+    # the fixed scratch holds, found from the library's plan for this GPU.
+    case = next(((T, k) for k in (2048, 4096, 16384) for T in range(1, 149)
+                 if ops.plan_attend(T, 1, k).workspace_bytes > 0 and T * ops.plan_attend(T, 1, k).n_split > 128),
+                None)
+    assert case is not None, "no batch exceeds the scratch on this GPU"
+    T, k = case
     # Real buffers of the right sizes: the call must refuse before launching,
     # and nothing could read out of bounds even if it did not.
     wl = make_workload(small_case("na_rej", (2100,) * T, layers=(64,), seed=33), DEV)
     lay = wl.layers[0]
-    idx = torch.zeros((T, 2048), dtype=torch.int32, device=DEV)
+    idx = torch.zeros((T, k), dtype=torch.int32, device=DEV)
     cnt = torch.ones((T,), dtype=torch.int32, device=DEV)
     out = torch.empty((T, 64, 512), dtype=torch.bfloat16, device=DEV)
     with pytest.raises(ops.DSAError) as err:
