@@ -178,6 +178,9 @@ def measure(name, dev, steps, warmup, rank, world, local, min_seconds=0.0, sampl
               for L, o, l in zip(wl.layers, outs, lses)]
     n_rows = wl.layers[0].cache.shape[0]
     att_ws = ops.workspace(ops.layers_workspace_bytes(T, n_layers, k), dev)
+    # decode: the indexer also counts its scores into a histogram that the top-k's first pass reads
+    hist = torch.empty((T, 2048), dtype=torch.int32, device=dev) if q_group == 1 else None
+    topk_ws = ops.workspace(ops.topk_workspace_bytes(T, ld, k), dev) if q_group == 1 else None
     stream = torch.cuda.current_stream()
     if fp8:
         # E4M3 codes + per-row scales of the same seeded keys/queries (input preparation, untimed)
@@ -193,13 +196,13 @@ def measure(name, dev, steps, warmup, rank, world, local, min_seconds=0.0, sampl
             e[0].record(stream)
         if fp8:
             ops.index_scores_fp8(q8, q8_scale, wl.w, k8, k8_scale, wl.seq_row_start, wl.q_seq, wl.q_pos, scores,
-                                 q_group=q_group)
+                                 q_group=q_group, hist=hist)
         else:
             ops.index_scores(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, scores,
-                             q_group=q_group)
+                             q_group=q_group, hist=hist)
         if e:
             e[1].record(stream)
-        ops.topk(scores, wl.q_pos, k, idx, cnt)
+        ops.topk(scores, wl.q_pos, k, idx, cnt, hist=hist, ws=topk_ws)
         if e:
             e[2].record(stream)
         ops.sparse_mla_attend_layers(layers, n_rows, wl.seq_row_start, wl.q_seq, idx, cnt, q_pos=wl.q_pos,
@@ -328,6 +331,9 @@ def measure(name, dev, steps, warmup, rank, world, local, min_seconds=0.0, sampl
                            "traffic": profiled_traffic(idx_kernel, case.name),
                            "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": idx_bytes,
                            "avg_launch_ms": round(idx_ms, 4)}
+    plan = ops.plan_attend(T, min(n_layers, 8), k)
+    res["attend_plan"] = {"n_split": plan.n_split, "rows_per_split": plan.rows_per_split, "merge": bool(plan.merge),
+                          "workspace_bytes": int(plan.workspace_bytes)}
     if e2e and not fp8:
         res["e2e"] = run_e2e(wl, ld, k, q_group, dev, e2e_steps)
     del graph, graph_ev
@@ -414,8 +420,10 @@ def run_ours(args, rank, world, local):
                            "kernel_ms from a second graph of the same steps with events around each kernel")},
         "step_hbm": head["step_hbm"], "attention_hbm": head["attention_hbm"], "kernel_ms": head["kernel_ms"],
         "roofline": head["roofline"], "gpu_launches": head["launches"], "clocks": head["clocks"],
-        "e2e": head.get("e2e"),
+        "e2e": head.get("e2e"), "attend_plan": head["attend_plan"],
     }
+    props = ops.device_props()
+    line["device"] = {"sms": props.sms, "attend_max_clusters": {c: props.max_clusters[c] for c in range(2, 9)}}
     if world == 1 and not args.no_extras:
         extras = {}
         for name in EXTRAS:
@@ -425,7 +433,7 @@ def run_ours(args, rank, world, local):
                         min_seconds=0.0 if CONFIGS[name].kind == "prefill" else 0.3, fp8=args.fp8_keys)
             torch.cuda.empty_cache()
             keep = ("ms_per_step", "queries_per_s", "query_layers_per_s", "kernel_ms", "step_hbm", "attention_hbm",
-                    "roofline", "timed_steps")
+                    "roofline", "timed_steps", "attend_plan")
             extras[name] = {k_: (round(v, 4) if isinstance(v, float) else v) for k_, v in r.items() if k_ in keep}
         line["extra_configs"] = extras
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -88,13 +88,17 @@ typedef enum dsa_status {
  *           scored together, 8 queries x 32 heads per tensor-core tile.
  *   scores  f32 [T, ld]: I[t,s] for s <= q_pos[t], -inf for q_pos[t] < s < ld.
  *           ld >= max(q_pos) + 1 and ld % 4 == 0.
+ *   hist    uint32 [T, 2048] or NULL (q_group 1 only): overwritten with, for
+ *           each query, how many of its scores s <= q_pos[t] fall in each bin of
+ *           the top 11 bits of their order-preserving key (the first histogram
+ *           of dsa_topk's radix select, which then skips that pass).
  * Returns DSA_ERR_INVALID_ARG for null/misaligned pointers, T < 0, n_rows < 1,
- * n_rows >= 2^31 - 256, ld < 4 or ld % 4, q_group not 1 or 8.
+ * n_rows >= 2^31 - 256, ld < 4 or ld % 4, q_group not 1 or 8, hist with q_group 8.
  */
 dsa_status_t dsa_index_scores(const void* q_idx, const float* w, const void* k_idx,
                               int64_t n_rows, const int64_t* seq_row_start, int32_t B,
                               const int32_t* q_seq, const int32_t* q_pos, int32_t T,
-                              int32_t q_group, float* scores, int64_t ld, void* stream);
+                              int32_t q_group, float* scores, int64_t ld, uint32_t* hist, void* stream);
 
 /*
  * dsa_index_scores_fp8 - lightning-indexer scores on FP8 (E4M3) keys and queries.
@@ -112,15 +116,16 @@ dsa_status_t dsa_index_scores(const void* q_idx, const float* w, const void* k_i
  *   w       f32   [T, 32]
  *   k8      uint8 [n_rows, 128] E4M3 codes, rows located by seq_row_start
  *   k_scale f32   [n_rows]      > 0
- *   the remaining arguments, layouts, q_group and errors as dsa_index_scores;
- *   additionally DSA_ERR_INVALID_ARG for a null or misaligned q_scale / k_scale.
+ *   the remaining arguments (hist included), layouts, q_group and errors as
+ *   dsa_index_scores; additionally DSA_ERR_INVALID_ARG for a null or misaligned
+ *   q_scale / k_scale.
  * Scales must be positive (the ReLU is applied to the unscaled dot product
  * times the scales); codes must not be NaN.
  */
 dsa_status_t dsa_index_scores_fp8(const void* q8, const float* q_scale, const float* w, const void* k8,
                                   const float* k_scale, int64_t n_rows, const int64_t* seq_row_start,
                                   int32_t B, const int32_t* q_seq, const int32_t* q_pos, int32_t T,
-                                  int32_t q_group, float* scores, int64_t ld, void* stream);
+                                  int32_t q_group, float* scores, int64_t ld, uint32_t* hist, void* stream);
 
 /*
  * dsa_topk - per-query top-k of a score array.
@@ -133,11 +138,16 @@ dsa_status_t dsa_index_scores_fp8(const void* q8, const float* q_scale, const fl
  *
  *   scores f32 [T, ld] (ld % 4 == 0, 16-byte aligned), q_pos int32 [T],
  *   idx int32 [T, k] (out), count int32 [T] (out), 1 <= k <= 16384.
- *   workspace: dsa_topk_workspace_size() bytes (currently 0; may be NULL).
+ *   hist   uint32 [T, 2048] or NULL: the histogram dsa_index_scores wrote for
+ *          these scores.  With it, the first radix pass is skipped and each
+ *          query's row is filtered on every SM; it then needs a workspace of
+ *          dsa_topk_workspace_size(T, ld, k) bytes, 256-byte aligned.  The
+ *          result is the same (a histogram that does not match the scores is
+ *          detected and the row selected without it).  NULL: no workspace.
  */
 size_t dsa_topk_workspace_size(int32_t T, int64_t ld, int32_t k);
 dsa_status_t dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, int32_t T,
-                      int32_t k, int32_t* idx, int32_t* count, void* workspace,
+                      int32_t k, int32_t* idx, int32_t* count, const uint32_t* hist, void* workspace,
                       size_t ws_bytes, void* stream);
 
 /*
@@ -291,11 +301,15 @@ dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const voi
  * n_split blocks per (layer, query) of rows_per_split selected rows each;
  * merge = 1 when those blocks form a cluster and merge on chip; and
  * workspace_bytes, the split partials that otherwise go through the workspace.
+ * The plan is the split of least estimated time; allow_partials = 0 restricts
+ * it to plans without partials (what dsa_sparse_mla_forward uses when its
+ * workspace is too tight for partials: dsa_forward_plan.attend_partials = 0).
  *
  * dsa_plan_forward: how dsa_sparse_mla_forward cuts T queries into chunks for
  * a workspace of ws_bytes, and where each region sits in it (byte offsets;
  * SIZE_MAX for idx / count regions replaced by the caller's idx_out /
- * count_out, i.e. has_idx_out / has_count_out != 0).  Returns
+ * count_out, i.e. has_idx_out / has_count_out != 0; the score histogram and
+ * top-k lists exist for decode, q_group = 1).  Returns
  * DSA_ERR_WORKSPACE (chunk = 0) when even q_group queries do not fit.
  */
 typedef struct dsa_device_props {
@@ -315,18 +329,21 @@ typedef struct dsa_forward_plan {
   int32_t chunk;               /* queries per chunk (a multiple of q_group, or T) */
   int32_t n_chunks;
   int32_t last_chunk;          /* queries in the final chunk                      */
-  int32_t reserved;
+  int32_t attend_partials;     /* 0: attention plans restricted to no partials    */
   size_t idx_offset;           /* [chunk, k] int32 selection (SIZE_MAX: idx_out)  */
   size_t count_offset;         /* [chunk] int32 counts (SIZE_MAX: count_out)      */
   size_t attend_offset;        /* attention split partials                        */
   size_t attend_bytes;         /* the largest need of any chunk's launches        */
+  size_t hist_offset;          /* [chunk, 2048] score histogram (SIZE_MAX: none)  */
+  size_t topk_offset;          /* top-k candidate lists (SIZE_MAX: none)          */
+  size_t topk_bytes;
   size_t scores_offset;        /* [chunk, ld] f32 scores                          */
   size_t end;                  /* bytes used (<= ws_bytes)                        */
 } dsa_forward_plan;
 
 dsa_status_t dsa_get_device_props(dsa_device_props* out);
-dsa_status_t dsa_plan_attend(int32_t T, int32_t n_layers, int32_t k, const dsa_device_props* props,
-                             dsa_attend_plan* out);
+dsa_status_t dsa_plan_attend(int32_t T, int32_t n_layers, int32_t k, int32_t allow_partials,
+                             const dsa_device_props* props, dsa_attend_plan* out);
 dsa_status_t dsa_plan_forward(int32_t T, int64_t ld, int32_t k, int32_t q_group, int32_t n_layers,
                               int32_t has_idx_out, int32_t has_count_out, size_t ws_bytes,
                               const dsa_device_props* props, dsa_forward_plan* out);

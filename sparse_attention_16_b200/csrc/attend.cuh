@@ -41,11 +41,11 @@
 // a head's maximum grows by more than 2^8, so p <= 256 and the final
 // normalisation uses the same reference for numerator and denominator.
 // A single split writes bf16 output directly.  When a query's selection is
-// split over 2-8 CTAs, those CTAs form a thread-block cluster: each stages its
-// unnormalised O and per-head (max, sum) in its own shared memory, and rank r
-// merges columns [r 512 / n, (r + 1) 512 / n) of all heads from every CTA
-// through distributed shared memory.  Otherwise the splits write fp32 partials
-// that a small combine kernel merges.
+// split over 2-8 CTAs, those CTAs form a thread-block cluster: each pushes the
+// column slices of its unnormalised O and its per-head (max, sum) into the
+// shared memory of the rank that owns those columns, and rank r merges columns
+// [r 512 / n, (r + 1) 512 / n) of all heads locally.  Otherwise the splits
+// write fp32 partials that a small combine kernel merges.
 //
 // A selected position is used only if it lies in [0, q_pos[t]] (when q_pos is
 // given) and inside the cache; anything else except the -1 padding is skipped
@@ -195,22 +195,66 @@ __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr));
 }
 
-// Merge of a query's split partials inside its cluster (n = p.n_split CTAs,
-// rank = split).  Each CTA has staged O_j[64][512] (unnormalised, fp32, pieces
-// swizzled by h & 7) and (m_j, l_j, lx_j) per head at the start of its shared
-// memory (l: sum of the bf16 weights the products used, lx: of the fp32
-// weights); rank r produces columns [r 512 / n, (r + 1) 512 / n) of every head:
+// Merge of a (layer, query)'s split partials inside its cluster (n = p.n_split
+// CTAs, rank = split), called by every thread of the CTA once all its roles
+// are done.  Rank r produces float4 columns [c0(r), c0(r+1)) of every head,
+// c0(r) = r 128 / n.  Push model: after a cluster barrier (every CTA has left
+// its tile loop, so every tile buffer is free), each CTA reads its
+// unnormalised O from tensor memory and stores each column slice straight into
+// the owner rank's receive buffer (distributed shared memory stores, which do
+// not wait for a reply), and its per-head (m, l, lx) into every rank; after a
+// second barrier each rank merges from its own shared memory:
 //   M = max_j m_j,  w_j = 2^(m_j - M),  L = sum_j w_j l_j,
 //   o[h, c] = sum_j (w_j / L) O_j[h, c],
-//   lse[h] = (M + log2 sum_j w_j lx_j) ln 2 (rank 0).
-__device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLayer& L, uint8_t* cs,
-                                              uint8_t* ps, int t, int rank) {
+//   lse[h] = (M + log2 sum_j w_j lx_j) ln 2 (rank 0)
+// (l: sum of the bf16 weights the products used, lx: of the fp32 weights).
+__device__ __forceinline__ int merge_c0(int r, int n) { return r * (kLatent / 4) / n; }
+
+__device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLayer& L, uint8_t* cs, uint8_t* ps,
+                                              int t, int rank, bool softmax_thread, uint32_t hi_base, bool have_o,
+                                              float m_used, float Lsum, float Lx) {
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int n = p.n_split;
-  cl.sync();   // every CTA's partial is staged
-  float* wt = reinterpret_cast<float*>(ps);   // [64 heads][8]: w_j / L
+  const int W = (kLatent / 4 + n - 1) / n;                                   // float4 columns per rank, at most
+  float4* recv = reinterpret_cast<float4*>(cs);                              // [n sources][64 heads][W]
+  float* stats = reinterpret_cast<float*>(cs + (size_t)n * kHeads * W * 16); // [n sources][64 heads][4]
   const int tid = threadIdx.x;
+  cl.sync();   // every CTA has left its tile loop: all receive buffers are free
+  if (softmax_thread) {
+    const int lane = tid & 31;
+    const int hf = lane >> 4;
+    const int h = 16 * (tid >> 5) + (lane & 15);
+#pragma unroll 1
+    for (int cb = 0; cb < kLatent; cb += 64) {
+      uint32_t u[32];
+      if (have_o) {
+        tmem_ld16x2_32(hi_base + cb, u);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) u[c] = 0u;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int c4 = (cb + 32 * hf) / 4 + q;
+        const int r = (c4 * n + n - 1) / (kLatent / 4);                      // owner rank of column c4
+        float4* dst = cl.map_shared_rank(recv, r) + ((rank * kHeads + h) * W + (c4 - merge_c0(r, n)));
+        *dst = make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]), __uint_as_float(u[4 * q + 2]),
+                           __uint_as_float(u[4 * q + 3]));
+      }
+    }
+    if (hf == 0) {
+      for (int r = 0; r < n; ++r) {
+        float* dst = cl.map_shared_rank(stats, r) + (rank * kHeads + h) * 4;
+        dst[0] = have_o ? m_used : -INFINITY;
+        dst[1] = have_o ? Lsum : 0.f;
+        dst[2] = have_o ? Lx : 0.f;
+      }
+    }
+  }
+  cl.sync();   // every slice is in its owner's receive buffer; no remote access follows
+  float* wt = reinterpret_cast<float*>(ps);   // [64 heads][8]: w_j / L
   if (tid < kHeads) {
     const int h = tid;
     float m[8], l[8], lx[8];
@@ -221,42 +265,36 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLa
       l[j] = 0.f;
       lx[j] = 0.f;
       if (j < n) {
-        const float* xml = cl.map_shared_rank(reinterpret_cast<float*>(cs + kHeads * kLatent * 4), j);
-        m[j] = xml[4 * h];
-        l[j] = xml[4 * h + 1];
-        lx[j] = xml[4 * h + 2];
+        m[j] = stats[(j * kHeads + h) * 4];
+        l[j] = stats[(j * kHeads + h) * 4 + 1];
+        lx[j] = stats[(j * kHeads + h) * 4 + 2];
         M = fmaxf(M, m[j]);
       }
     }
-    float w[8], Ls = 0.f, Lx = 0.f;
+    float w[8], Ls = 0.f, Lxs = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       w[j] = (m[j] == -INFINITY) ? 0.f : ex2_approx(m[j] - M);
       Ls += w[j] * l[j];
-      Lx += w[j] * lx[j];
+      Lxs += w[j] * lx[j];
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j) wt[h * 8 + j] = (Ls > 0.f) ? w[j] / Ls : 0.f;
     if (rank == 0 && L.lse != nullptr)
-      L.lse[(int64_t)t * kHeads + h] = (Lx > 0.f) ? (M + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
+      L.lse[(int64_t)t * kHeads + h] = (Lxs > 0.f) ? (M + lg2_approx(Lxs)) * 0.69314718055994531f : -INFINITY;
   }
   __syncthreads();
-  const int c0 = rank * (kLatent / 4) / n, c1 = (rank + 1) * (kLatent / 4) / n;   // float4 columns
-  const int nc = c1 - c0;
-  const float4* xo[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    xo[j] = cl.map_shared_rank(reinterpret_cast<const float4*>(cs), j < n ? j : 0);
+  const int c0 = merge_c0(rank, n);
+  const int nc = merge_c0(rank + 1, n) - c0;
   for (int i = tid; i < kHeads * nc; i += blockDim.x) {
     const int h = i / nc;
-    const int c = c0 + (i - h * nc);
-    const int piece = h * (kLatent / 4) + (c ^ (h & 7));
+    const int c = i - h * nc;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const float wj = (j < n) ? wt[h * 8 + j] : 0.f;
       if (wj != 0.f) {
-        const float4 v = xo[j][piece];
+        const float4 v = recv[(j * kHeads + h) * W + c];
         acc.x = fmaf(wj, v.x, acc.x);
         acc.y = fmaf(wj, v.y, acc.y);
         acc.z = fmaf(wj, v.z, acc.z);
@@ -266,9 +304,8 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLa
     uint2 o;
     o.x = pack_bf16x2(acc.x, acc.y);
     o.y = pack_bf16x2(acc.z, acc.w);
-    *reinterpret_cast<uint2*>(L.out + ((int64_t)t * kHeads + h) * kLatent + 4 * c) = o;
+    *reinterpret_cast<uint2*>(L.out + ((int64_t)t * kHeads + h) * kLatent + 4 * (c0 + c)) = o;
   }
-  cl.sync();   // no CTA leaves while its staged partial may still be read
 }
 
 // The work of one CTA on one unit; KCH = 64-column chunks per row (9 RoPE, 8 NoPE).
@@ -603,12 +640,16 @@ __device__ __forceinline__ void attend_unit(const AttendParams& p, const AttLaye
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const uint32_t hi_base = tmem_base + ((uint32_t)((warp & 3) * 32 + C::O_LANE) << 16);
+  if (p.merge) {
+    cluster_merge(p, L, cs, ps, t, jsplit, warp < 4, hi_base, have_o, m_used, Lsum, Lx);
+    return;
+  }
   if (warp >= 4) return;
 
-  // ---- epilogue (softmax warps): normalised output, staged partial or workspace partial
+  // ---- epilogue (softmax warps): normalised output or workspace partial
   const int hf = lane >> 4;
   const int h = 16 * warp + (lane & 15);
-  const uint32_t hi_base = tmem_base + ((uint32_t)(warp * 32 + C::O_LANE) << 16);
   const int64_t unit = blockIdx.x;   // (pair, split)
   auto read_o = [&](int cb, uint32_t (&u)[32]) {
     if (have_o) {
@@ -639,26 +680,6 @@ __device__ __forceinline__ void attend_unit(const AttendParams& p, const AttLaye
     if (L.lse != nullptr && hf == 0)
       L.lse[(int64_t)t * kHeads + h] =
           (have_o && Lx > 0.f) ? (m_used + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
-  } else if (p.merge) {
-    // Stage unnormalised O[h, :] (fp32, 16-byte pieces XOR-swizzled by h & 7
-    // within 128-byte groups) and (max, sum) in this CTA's tile buffers.
-    const uint32_t xrow = smem_u32(cs) + h * (kLatent * 4);
-#pragma unroll 1
-    for (int cb = 0; cb < kLatent; cb += 64) {
-      uint32_t u[32];
-      read_o(cb, u);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int piece = (cb / 4 + 8 * hf + q) ^ (h & 7);
-        st_shared_v4(xrow + piece * 16, u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
-      }
-    }
-    if (hf == 0) {
-      float* xml = reinterpret_cast<float*>(cs + kHeads * kLatent * 4);
-      xml[4 * h] = have_o ? m_used : -INFINITY;
-      xml[4 * h + 1] = have_o ? Lsum : 0.f;
-      xml[4 * h + 2] = have_o ? Lx : 0.f;
-    }
   } else {
     float4* wo = reinterpret_cast<float4*>(p.ws_o + (unit * kHeads + h) * kLatent + 32 * hf);
 #pragma unroll 1
@@ -734,7 +755,6 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
-  if (p.merge) cluster_merge(p, L, cs, ps, t, jsplit);
 }
 
 // Merges the split partials of each (layer, query, head): o = sum_j 2^(m_j - M) O_j / L,

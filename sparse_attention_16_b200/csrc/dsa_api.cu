@@ -28,6 +28,8 @@
 static_assert(dsa::kPlanMaxLayers == dsa::kMaxAttLayers, "planner and kernel agree on layers per launch");
 static_assert(dsa::kPlanMaxSplits == dsa::kMaxSplits, "planner and kernel agree on the split limit");
 static_assert(dsa::kPlanTileRows == dsa::AttCfg::ROWS, "planner and kernel agree on the tile height");
+static_assert(dsa::kPlanTopkCap == dsa::kTopkCandCap && dsa::kPlanTopkBins == dsa::kTopkBins,
+              "planner and top-k kernels agree on the candidate lists");
 
 namespace {
 
@@ -99,7 +101,8 @@ uint64_t current_context_id() {
 
 // ----------------------------------------------------------------- per-device state
 enum KernelId : uint32_t {
-  kKIdx1 = 0, kKIdx8, kKIdx1F8, kKIdx8F8, kKTopk1, kKTopk2, kKTopk4, kKTopk8, kKTopk16, kKAttend, kKCount
+  kKIdx1 = 0, kKIdx8, kKIdx1F8, kKIdx8F8, kKTopk1, kKTopk2, kKTopk4, kKTopk8, kKTopk16, kKAttend, kKTopkFilter,
+  kKTopkSelect, kKCount
 };
 
 constexpr int kMaxDevices = 64;
@@ -285,7 +288,7 @@ template <int QG, bool F8>
 dsa_status_t launch_indexer(DevLock& L, const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                             const float* k_scale, int64_t n_rows, const int64_t* seq_row_start, int32_t B,
                             const int32_t* q_seq, const int32_t* q_pos, int32_t T, float* scores, int64_t ld,
-                            cudaStream_t stream) {
+                            uint32_t* hist, cudaStream_t stream) {
   using C = dsa::IdxCfg<QG, F8>;
   // One 128-byte swizzled block per box row: 64 bf16 or 128 fp8 values.  TMA
   // moves bytes, so an fp8 row (128 B) is described as 64 two-byte elements:
@@ -303,11 +306,13 @@ dsa_status_t launch_indexer(DevLock& L, const void* q_idx, const float* q_scale,
   p.q_seq = q_seq;
   p.q_pos = q_pos;
   p.scores = scores;
+  p.hist = (QG == 1) ? hist : nullptr;
   p.ld = ld;
   p.n_rows = n_rows;
   p.T = T;
   p.B = B;
   p.n_kt = (int32_t)((ld + dsa::kKeyTile - 1) / dsa::kKeyTile);
+  if (p.hist != nullptr) DSA_CUDA(cudaMemsetAsync(hist, 0, (size_t)T * dsa::kTopkBins * 4, stream));
   const int64_t n_groups = (T + QG - 1) / QG;
   p.n_units = n_groups * p.n_kt;
   dsa::DevProps props;
@@ -322,12 +327,12 @@ dsa_status_t launch_indexer(DevLock& L, const void* q_idx, const float* q_scale,
 dsa_status_t indexer_impl(DevLock& L, const void* q_idx, const float* w, const void* k_idx, int64_t n_rows,
                           const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
                           const int32_t* q_pos, int32_t T, int32_t q_group, float* scores,
-                          int64_t ld, cudaStream_t stream) {
+                          int64_t ld, uint32_t* hist, cudaStream_t stream) {
   if (q_group == 8)
     return launch_indexer<8, false>(L, q_idx, nullptr, w, k_idx, nullptr, n_rows, seq_row_start, B, q_seq, q_pos,
-                                    T, scores, ld, stream);
+                                    T, scores, ld, nullptr, stream);
   return launch_indexer<1, false>(L, q_idx, nullptr, w, k_idx, nullptr, n_rows, seq_row_start, B, q_seq, q_pos, T,
-                                  scores, ld, stream);
+                                  scores, ld, hist, stream);
 }
 
 // ----------------------------------------------------------------- top-k
@@ -351,7 +356,8 @@ int topk_cluster_size(const DevState& s, int sms, int32_t T, int64_t ld) {
 }
 
 dsa_status_t topk_impl(DevLock& L, const float* scores, int64_t ld, const int32_t* q_pos, int32_t T, int32_t k,
-                       int32_t* idx, int32_t* count, cudaStream_t stream) {
+                       int32_t* idx, int32_t* count, const uint32_t* hist, void* ws, size_t ws_bytes,
+                       cudaStream_t stream) {
   dsa::DevProps props;
   DSA_TRY(device_props(L, &props));
   dsa::TopkParams p;
@@ -362,6 +368,28 @@ dsa_status_t topk_impl(DevLock& L, const float* scores, int64_t ld, const int32_
   p.ld = ld;
   p.T = T;
   p.k = k;
+  if (hist != nullptr) {
+    // first pass from the indexer's histogram: slices on every SM, then one CTA per query
+    const int S = dsa::topk_slices(props.sms, T, ld);
+    const size_t need = dsa::topk_hist_ws_bytes(props.sms, T, ld);
+    if (ws == nullptr || ws_bytes < need || !aligned(ws, 256))
+      return fail(DSA_ERR_WORKSPACE, "top-k with a histogram needs %zu bytes of 256-byte aligned workspace (got %zu)",
+                  need, ws_bytes);
+    const size_t ts = (size_t)T * S;
+    const size_t lists = dsa::plan_round_up(ts * dsa::kTopkCandCap * 4, 256);
+    dsa::TopkHistParams hp;
+    hp.base = p;
+    hp.hist = hist;
+    hp.cand_key = static_cast<uint32_t*>(ws);
+    hp.cand_pos = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + lists);
+    hp.cand_cnt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + 2 * lists);
+    hp.S = S;
+    DSA_TRY(set_smem(*L.s, kKTopkFilter, dsa::topk_filter_kernel, dsa::kTopkSmemBytes));
+    DSA_TRY(set_smem(*L.s, kKTopkSelect, dsa::topk_select_kernel, dsa::kTopkSmemBytes));
+    DSA_TRY(launch(dsa::topk_filter_kernel, (unsigned)(T * S), dsa::kTopkThreads, dsa::kTopkSmemBytes, stream, 1,
+                   hp));
+    return launch(dsa::topk_select_kernel, (unsigned)T, dsa::kTopkThreads, dsa::kTopkSmemBytes, stream, 1, hp);
+  }
   switch (topk_cluster_size(*L.s, props.sms, T, ld)) {
     case 1: return launch_topk_cl<1>(L, kKTopk1, p, stream);
     case 2: return launch_topk_cl<2>(L, kKTopk2, p, stream);
@@ -378,12 +406,12 @@ dsa_status_t topk_impl(DevLock& L, const float* scores, int64_t ld, const int32_
 dsa_status_t launch_attend(DevLock& L, const dsa_layer_args* layers, int32_t n_layers, float scale,
                            int64_t n_rows, const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
                            const int32_t* q_pos, const int32_t* idx, const int32_t* count, int32_t T, int32_t k,
-                           void* ws, size_t ws_bytes, cudaStream_t stream) {
+                           void* ws, size_t ws_bytes, cudaStream_t stream, bool allow_partials = true) {
   using C = dsa::AttCfg;
   dsa::DevProps props;
   DSA_TRY(device_props(L, &props));
   const int64_t units = (int64_t)T * n_layers;
-  const dsa::SplitPlan sp = dsa::attend_plan(props, units, k);
+  const dsa::SplitPlan sp = dsa::attend_plan(props, units, k, allow_partials);
   dsa::AttendParams p;
   std::memset(&p, 0, sizeof(p));
   for (int l = 0; l < n_layers; ++l) {
@@ -435,7 +463,8 @@ dsa_status_t launch_attend(DevLock& L, const dsa_layer_args* layers, int32_t n_l
 dsa_status_t attend_layers_impl(DevLock& L, const dsa_layer_args* layers, int32_t n_layers, float scale,
                                 int64_t n_rows, const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
                                 const int32_t* q_pos, const int32_t* idx, const int32_t* count, int32_t T,
-                                int32_t k, int64_t q_offset, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                                int32_t k, int64_t q_offset, void* ws, size_t ws_bytes, cudaStream_t stream,
+                                bool allow_partials = true) {
   for (int l0 = 0; l0 < n_layers; l0 += dsa::kMaxAttLayers) {
     const int g = std::min(dsa::kMaxAttLayers, n_layers - l0);
     dsa_layer_args sub[dsa::kMaxAttLayers];
@@ -450,7 +479,7 @@ dsa_status_t attend_layers_impl(DevLock& L, const dsa_layer_args* layers, int32_
       sub[i].lse = a.lse ? a.lse + qo : nullptr;
     }
     DSA_TRY(launch_attend(L, sub, g, scale, n_rows, seq_row_start, B, q_seq, q_pos, idx, count, T, k, ws,
-                          ws_bytes, stream));
+                          ws_bytes, stream, allow_partials));
   }
   return DSA_OK;
 }
@@ -527,8 +556,9 @@ dsa_layer_args one_layer(const void* q_nope, const void* q_pe, const float* qmul
   return a;
 }
 
-void fill_attend_plan(const dsa::DevProps& d, int64_t units, int32_t k, dsa_attend_plan* out) {
-  const dsa::SplitPlan sp = dsa::attend_plan(d, units, k);
+void fill_attend_plan(const dsa::DevProps& d, int64_t units, int32_t k, bool allow_partials,
+                      dsa_attend_plan* out) {
+  const dsa::SplitPlan sp = dsa::attend_plan(d, units, k, allow_partials);
   out->n_split = sp.n_split;
   out->rows_per_split = sp.rows_per_split;
   out->merge = sp.merge ? 1 : 0;
@@ -573,49 +603,57 @@ extern "C" {
 dsa_status_t dsa_index_scores(const void* q_idx, const float* w, const void* k_idx, int64_t n_rows,
                               const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
                               const int32_t* q_pos, int32_t T, int32_t q_group, float* scores,
-                              int64_t ld, void* stream) {
+                              int64_t ld, uint32_t* hist, void* stream) {
   NvtxRange nvtx_range("dsa_index_scores");
   DSA_TRY(check_index_args(q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, ld));
   DSA_REQUIRE(scores && aligned(scores, 16), "scores must be non-null and 16-byte aligned");
+  DSA_REQUIRE(hist == nullptr || (q_group == 1 && aligned(hist, 16)), "hist needs q_group 1 and 16-byte alignment");
   if (T == 0) return DSA_OK;
   DevLock L;
   DSA_TRY(lock_device(L));
-  return indexer_impl(L, q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, scores, ld,
+  return indexer_impl(L, q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, scores, ld, hist,
                       static_cast<cudaStream_t>(stream));
 }
 
 dsa_status_t dsa_index_scores_fp8(const void* q8, const float* q_scale, const float* w, const void* k8,
                                   const float* k_scale, int64_t n_rows, const int64_t* seq_row_start,
                                   int32_t B, const int32_t* q_seq, const int32_t* q_pos, int32_t T,
-                                  int32_t q_group, float* scores, int64_t ld, void* stream) {
+                                  int32_t q_group, float* scores, int64_t ld, uint32_t* hist, void* stream) {
   NvtxRange nvtx_range("dsa_index_scores_fp8");
   DSA_TRY(check_index_args(q8, w, k8, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, ld));
   DSA_REQUIRE(q_scale && k_scale && aligned(q_scale, 4) && aligned(k_scale, 4),
               "q_scale and k_scale must be non-null and 4-byte aligned");
   DSA_REQUIRE(scores && aligned(scores, 16), "scores must be non-null and 16-byte aligned");
+  DSA_REQUIRE(hist == nullptr || (q_group == 1 && aligned(hist, 16)), "hist needs q_group 1 and 16-byte alignment");
   if (T == 0) return DSA_OK;
   DevLock L;
   DSA_TRY(lock_device(L));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (q_group == 8)
     return launch_indexer<8, true>(L, q8, q_scale, w, k8, k_scale, n_rows, seq_row_start, B, q_seq, q_pos, T,
-                                   scores, ld, s);
+                                   scores, ld, nullptr, s);
   return launch_indexer<1, true>(L, q8, q_scale, w, k8, k_scale, n_rows, seq_row_start, B, q_seq, q_pos, T, scores,
-                                 ld, s);
+                                 ld, hist, s);
 }
 
-size_t dsa_topk_workspace_size(int32_t, int64_t, int32_t) { return 0; }
+size_t dsa_topk_workspace_size(int32_t T, int64_t ld, int32_t k) {
+  if (T <= 0 || ld <= 0 || k <= 0) return 0;
+  dsa::DevProps d;
+  if (props_for_query(nullptr, &d) != DSA_OK) return 0;
+  return dsa::topk_hist_ws_bytes(d.sms, T, ld);
+}
 
 dsa_status_t dsa_topk(const float* scores, int64_t ld, const int32_t* q_pos, int32_t T, int32_t k,
-                      int32_t* idx, int32_t* count, void* workspace, size_t ws_bytes, void* stream) {
+                      int32_t* idx, int32_t* count, const uint32_t* hist, void* workspace, size_t ws_bytes,
+                      void* stream) {
   NvtxRange nvtx_range("dsa_topk");
-  (void)workspace;
-  (void)ws_bytes;
   DSA_TRY(check_topk_args(scores, ld, q_pos, T, k, idx, count));
+  DSA_REQUIRE(hist == nullptr || aligned(hist, 16), "hist must be 16-byte aligned");
   if (T == 0) return DSA_OK;
   DevLock L;
   DSA_TRY(lock_device(L));
-  return topk_impl(L, scores, ld, q_pos, T, k, idx, count, static_cast<cudaStream_t>(stream));
+  return topk_impl(L, scores, ld, q_pos, T, k, idx, count, hist, workspace, ws_bytes,
+                   static_cast<cudaStream_t>(stream));
 }
 
 size_t sparse_mla_workspace_size(int32_t T, int32_t k) {
@@ -709,7 +747,7 @@ size_t dsa_forward_workspace_size(int32_t T, int64_t ld, int32_t k, int32_t q_gr
   if (T <= 0 || ld <= 0 || k <= 0) return 0;
   dsa::DevProps d;
   if (props_for_query(nullptr, &d) != DSA_OK) return 0;
-  return dsa::forward_layout_for(d, T, ld, k, std::max(0, n_layers), true, true, T).end;
+  return dsa::forward_layout_for(d, T, ld, k, std::max(0, n_layers), true, true, T, true, q_group == 1).end;
 }
 
 dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const void* k_idx, int64_t n_rows,
@@ -746,6 +784,8 @@ dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const voi
   int32_t* idx_ws = own_idx ? reinterpret_cast<int32_t*>(ws + f.idx_off) : nullptr;
   int32_t* cnt_ws = own_count ? reinterpret_cast<int32_t*>(ws + f.cnt_off) : nullptr;
   void* att_ws = ws + f.att_off;
+  uint32_t* hist = (f.hist_off != SIZE_MAX) ? reinterpret_cast<uint32_t*>(ws + f.hist_off) : nullptr;
+  void* topk_ws = (f.topk_off != SIZE_MAX) ? ws + f.topk_off : nullptr;
   float* scores = reinterpret_cast<float*>(ws + f.scores_off);
 
   for (int32_t t0 = 0; t0 < T; t0 += f.chunk) {
@@ -754,10 +794,10 @@ dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const voi
     int32_t* cnt_c = own_count ? cnt_ws : count_out + t0;
     DSA_TRY(indexer_impl(L, static_cast<const __nv_bfloat16*>(q_idx) + (int64_t)t0 * dsa::kIdxHeads * dsa::kIdxDim,
                          w + (int64_t)t0 * dsa::kIdxHeads, k_idx, n_rows, seq_row_start, B, q_seq + t0,
-                         q_pos + t0, n, q_group, scores, ld, s));
-    DSA_TRY(topk_impl(L, scores, ld, q_pos + t0, n, k, idx_c, cnt_c, s));
+                         q_pos + t0, n, q_group, scores, ld, hist, s));
+    DSA_TRY(topk_impl(L, scores, ld, q_pos + t0, n, k, idx_c, cnt_c, hist, topk_ws, f.topk_bytes, s));
     DSA_TRY(attend_layers_impl(L, layers, n_layers, softmax_scale, n_rows, seq_row_start, B, q_seq + t0,
-                               q_pos + t0, idx_c, cnt_c, n, k, t0, att_ws, f.att_bytes, s));
+                               q_pos + t0, idx_c, cnt_c, n, k, t0, att_ws, f.att_bytes, s, f.partials));
   }
   return DSA_OK;
 }
@@ -771,14 +811,14 @@ dsa_status_t dsa_get_device_props(dsa_device_props* out) {
   return DSA_OK;
 }
 
-dsa_status_t dsa_plan_attend(int32_t T, int32_t n_layers, int32_t k, const dsa_device_props* props,
-                             dsa_attend_plan* out) {
+dsa_status_t dsa_plan_attend(int32_t T, int32_t n_layers, int32_t k, int32_t allow_partials,
+                             const dsa_device_props* props, dsa_attend_plan* out) {
   DSA_REQUIRE(out != nullptr, "null pointer argument");
   DSA_REQUIRE(T >= 1 && n_layers >= 1 && n_layers <= dsa::kMaxAttLayers && k >= 1 && k <= kMaxK,
               "T >= 1, 1 <= n_layers <= %d and 1 <= k <= %d required", dsa::kMaxAttLayers, kMaxK);
   dsa::DevProps d;
   DSA_TRY(props_for_query(props, &d));
-  fill_attend_plan(d, (int64_t)T * n_layers, k, out);
+  fill_attend_plan(d, (int64_t)T * n_layers, k, allow_partials != 0, out);
   return DSA_OK;
 }
 
@@ -795,11 +835,14 @@ dsa_status_t dsa_plan_forward(int32_t T, int64_t ld, int32_t k, int32_t q_group,
   out->chunk = f.chunk;
   out->n_chunks = f.chunk ? f.n_chunks : 0;
   out->last_chunk = f.chunk ? f.last_chunk : 0;
-  out->reserved = 0;
+  out->attend_partials = f.partials ? 1 : 0;
   out->idx_offset = f.idx_off;
   out->count_offset = f.cnt_off;
   out->attend_offset = f.att_off;
   out->attend_bytes = f.att_bytes;
+  out->hist_offset = f.hist_off;
+  out->topk_offset = f.topk_off;
+  out->topk_bytes = f.topk_bytes;
   out->scores_offset = f.scores_off;
   out->end = f.end;
   if (f.chunk == 0) return fail(DSA_ERR_WORKSPACE, "workspace of %zu bytes is too small (need %zu)", ws_bytes, f.end);

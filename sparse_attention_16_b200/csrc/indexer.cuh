@@ -61,7 +61,9 @@ struct IdxCfg {
   static constexpr int NACC = (F8 && QG == 1) ? 4 : 2;   // TMEM accumulators in flight (measured best)
   static constexpr int TMEM_COLS = (NACC * N < 32) ? 32 : NACC * N;
   static constexpr int SMEM_TILES = STAGES * KT_BYTES + QBUFS * Q_BYTES;
-  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024 + EPI_WARPS * ((QG == 1) ? 1 : 4) * kIdxHeads * 4;
+  static constexpr int W_BYTES = EPI_WARPS * ((QG == 1) ? 1 : 4) * kIdxHeads * 4;
+  static constexpr int HIST_BYTES = (QG == 1) ? 2048 * 4 : 0;   // decode: score histogram of the current query
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024 + W_BYTES + HIST_BYTES;
   static constexpr uint32_t IDESC = F8 ? idesc_e4m3_f32(128, N) : idesc_bf16_f32(128, N, 0, 0);
 };
 
@@ -73,6 +75,8 @@ struct IndexerParams {
   const int32_t* q_seq;           // [T]
   const int32_t* q_pos;           // [T]
   float* scores;                  // [T, ld]
+  uint32_t* hist;                 // [T, 2048] or null (q_group 1): candidates' score keys counted by their
+                                  // top 11 bits, accumulated (the caller zeroes it)
   int64_t ld;
   int64_t n_rows;
   int64_t n_units;                // n_groups * n_kt
@@ -169,6 +173,7 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* w_s = reinterpret_cast<float*>(smem + C::SMEM_TILES + 1024);
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + C::SMEM_TILES + 1024 + C::W_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -301,15 +306,40 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
     constexpr int QPW = (QG == 1) ? 1 : 4;        // queries per epilogue warp
     const int qbase = (QG == 1) ? 0 : (epi >> 2) * 4;
     float* w_my = w_s + epi * (QPW * kIdxHeads);
+    // Decode (one query per group): every candidate score is also counted in a
+    // shared-memory histogram of its key's top 11 bits, flushed to the query's
+    // global histogram when the group changes and at the end (the top-k's first
+    // pass).  The flushes are met by every epilogue warp, also after an abort.
+    const bool do_hist = (QG == 1) && p.hist != nullptr;
+    constexpr int EPI_THREADS = 32 * C::EPI_WARPS;
+    const int etid = threadIdx.x - 64;
+    auto flush_hist = [&](int g_old) {
+      named_bar_sync(1, EPI_THREADS);   // every epilogue warp has counted its scores of g_old
+      if (g_old >= 0)
+        for (int b = etid; b < 2048; b += EPI_THREADS) {
+          const uint32_t v = hist_s[b];
+          if (v) {
+            atomicAdd(&p.hist[(int64_t)g_old * 2048 + b], v);
+            hist_s[b] = 0;
+          }
+        }
+      named_bar_sync(1, EPI_THREADS);   // cleared before anyone counts the next group
+    };
+    if (do_hist) {
+      for (int b = etid; b < 2048; b += EPI_THREADS) hist_s[b] = 0;
+    }
     Ring as{0, 0};
     int cur_g = -1;
     GroupInfo gi{0, -1};
     int qpos_q[QPW];
+    bool dead = false;   // gave up after an abort: keeps walking the units only to meet the flushes
     int g = (int)(u_begin / p.n_kt), kt = (int)(u_begin % p.n_kt);   // unit u = g * n_kt + kt
     for (int64_t u = u_begin; u < u_end; ++u, kt = (kt + 1 == p.n_kt) ? 0 : kt + 1, g += (kt == 0)) {
       if constexpr (!F8) unit_of(u, p.n_kt, g, kt);
-      if (*abort_flag) break;
+      if (!dead && *abort_flag) dead = true;
+      if (dead && !do_hist) break;
       if (g != cur_g) {
+        if (do_hist) flush_hist(cur_g);
         gi = load_group<QG>(p, g, false);
         cur_g = g;
         // Weights of this warp's queries, in a warp-private slice of shared memory.
@@ -330,13 +360,18 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
           if (gi.maxpos < 0) qpos_q[qi] = -1;     // bad sequence id: nothing valid
         }
       }
+      if (dead) continue;
       const int64_t pos = (int64_t)kt * kKeyTile + row;
       float res[QPW];
       float kscale = 1.f;
       if (F8 && pos <= gi.maxpos && gi.row_base + pos < p.n_rows)
         kscale = p.k_scale[gi.row_base + pos];   // issued before the wait
       if (kt * kKeyTile <= gi.maxpos) {
-        if (!mbar_wait(&acc_full[as.idx], as.phase, abort_flag)) { *abort_flag = 1; break; }
+        if (!mbar_wait(&acc_full[as.idx], as.phase, abort_flag)) {
+          *abort_flag = 1;
+          dead = true;
+          continue;
+        }
         tc_fence_after();
         // Per query: ReLU of the 32 head dot products, weighted head sum (two
         // partial sums to halve the dependent FMA chain; weights as float4).
@@ -377,8 +412,10 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
           const int t = g * QG + qbase + qi;
           if (t < p.T) p.scores[(int64_t)t * p.ld + pos] = (pos <= qpos_q[qi]) ? res[qi] : -INFINITY;
         }
+        if (do_hist && pos <= qpos_q[0]) atomicAdd(&hist_s[score_key(res[0]) >> 21], 1u);
       }
     }
+    if (do_hist) flush_hist(cur_g);
   }
 
   tc_fence_before();

@@ -303,6 +303,15 @@ __device__ __forceinline__ float lg2_approx(float x) {
   return y;
 }
 
+// Order-preserving 32-bit key of an fp32 score (larger score, larger key); NaN
+// maps to the key of -inf and -0.0 to that of +0.0 (the selection's readings).
+__device__ __forceinline__ uint32_t score_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) u = 0xFF800000u;  // NaN ranks as -inf
+  if (u == 0x80000000u) u = 0u;                           // -0 == +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // Order-preserving map float -> signed int (its own inverse).
 __device__ __forceinline__ int f2ord(float f) {
   int i = __float_as_int(f);

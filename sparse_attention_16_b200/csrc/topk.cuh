@@ -11,13 +11,23 @@
 // (output slot of a kept element = #(> tau before it) + min(#(== tau before it),
 // need_eq)), so the result is unique and deterministic.
 //
-// One query is processed by a cluster of CL CTAs (CL in {1, 2, 4, 8, 16}); each
-// CTA owns a contiguous slice of the candidates and stages its keys in shared
-// memory: whole keys up to 32K per CTA, the top 16 bits of each key up to 64K
-// (enough for the first pass's 11-bit bins; the few candidates then read their
-// full key from the scores).  The per-CTA histograms and counts are combined through
-// distributed shared memory with cluster barriers (hardware barriers: every
-// CTA of a cluster is co-resident, so no software spin is involved).
+// Two ways to run it:
+//  * topk_kernel<CL>: one query per cluster of CL CTAs (CL in {1, 2, 4, 8, 16});
+//    each CTA owns a contiguous slice of the candidates and stages its keys in
+//    shared memory (whole keys up to 32K per CTA, their top 16 bits up to 64K,
+//    where candidates re-read their full key).  The first histogram is summed
+//    over the cluster through distributed shared memory; the keys in bins at
+//    or above the k-th one are filtered into candidate lists and gathered in
+//    rank 0, which finishes alone (or, if they overflow, the cluster runs the
+//    passes over its whole slices).
+//  * With the first histogram already made by the indexer (its epilogue counts
+//    every score it writes), the first pass is free: topk_filter_kernel spreads
+//    each query over S slices on every SM, each finding the k-th bin b1 from the
+//    histogram and keeping its keys in bins >= b1 (ordered, warp-private lists)
+//    in a workspace; topk_select_kernel (one CTA per query) gathers them and
+//    runs the last two passes and the ordered output.  If the candidates would
+//    exceed kTopkCandCap (a bin full of near-equal scores) or do not add up to
+//    the histogram's count, that CTA runs the single-CTA algorithm on the row.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -44,12 +54,6 @@ struct TopkParams {
   int32_t k;
 };
 
-__device__ __forceinline__ uint32_t score_key(float x) {
-  uint32_t u = __float_as_uint(x);
-  if ((u & 0x7FFFFFFFu) > 0x7F800000u) u = 0xFF800000u;  // NaN ranks as -inf
-  if (u == 0x80000000u) u = 0u;                           // -0 == +0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 // Exclusive scan of one uint32 per thread over the whole 1024-thread block.
 // `tmp` needs 33 words of shared memory; returns the block total in *total.
@@ -143,8 +147,10 @@ __device__ __forceinline__ void cluster_sum_hist(uint32_t* hist, uint32_t* tot) 
   }
 }
 
+// The selection of query t by the CTA of cluster rank `rank` (all CL CTAs of a
+// cluster call it for the same t).
 template <int CL>
-__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams p) {
+__device__ __forceinline__ void topk_query(const TopkParams& p, int t, int rank) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
   uint32_t* tot = hist + kTopkBins;
@@ -152,12 +158,6 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   uint32_t* res = tmp + 40;                  // threshold results
   uint32_t* cnt = res + 8;                   // this CTA's (#gt, #eq), read by peers
   uint32_t* stash = reinterpret_cast<uint32_t*>(smem_raw + 2 * kTopkBins * 4 + 1024);
-
-  griddep_wait();
-  const int t = blockIdx.x / CL;
-  int rank = 0;
-  if constexpr (CL > 1) rank = (int)cg::this_cluster().block_rank();
-  if (t >= p.T) return;  // whole clusters only: T * CL blocks are launched
 
   int qp = p.q_pos[t];
   if (qp >= p.ld) {
@@ -448,6 +448,292 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
     base_eq += total & 0xFFFFu;
   }
   if (rank == 0 && threadIdx.x == 0) p.count[t] = p.k;
+  (void)above;
+}
+
+template <int CL>
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams p) {
+  griddep_wait();
+  const int t = blockIdx.x / CL;
+  int rank = 0;
+  if constexpr (CL > 1) rank = (int)cg::this_cluster().block_rank();
+  if (t >= p.T) return;  // whole clusters only: T * CL blocks are launched
+  topk_query<CL>(p, t, rank);
+}
+
+// ------------------------------------------------------------------ selection from the indexer's histogram
+struct TopkHistParams {
+  TopkParams base;
+  const uint32_t* hist;   // [T, 2048]: the query's candidate keys counted by their top 11 bits
+  uint32_t* cand_key;     // [T, S, kTopkCandCap] candidates of each slice, in position order
+  int32_t* cand_pos;      // [T, S, kTopkCandCap]
+  uint32_t* cand_cnt;     // [T, S]: candidates of the slice (kTopkNoList: none written)
+  int32_t S;              // slices per query
+};
+constexpr uint32_t kTopkNoList = 0xFFFFFFFFu;
+
+// Query t's candidate count n (0 when q_pos < 0; clamped to ld, flagged).
+__device__ __forceinline__ int64_t topk_row_len(const TopkParams& p, int t, bool report) {
+  int qp = p.q_pos[t];
+  if (qp >= p.ld) {
+    if (report) raise_error(kErrBadSeq);
+    qp = (int)p.ld - 1;
+  }
+  return (qp < 0) ? 0 : (int64_t)qp + 1;
+}
+
+// k-th bin of the query's histogram (copied to `h` in shared memory): writes
+// (b1, keys in bins above b1, keys in bin b1) to res[0..2].
+__device__ __forceinline__ void topk_bin_from_hist(const uint32_t* g_hist, uint32_t* h, uint32_t k, uint32_t* tmp,
+                                                   uint32_t* res) {
+  for (int b = threadIdx.x; b < kTopkBins; b += kTopkThreads) h[b] = g_hist[b];
+  if (threadIdx.x == 0) {
+    res[0] = kTopkNoList;
+    res[1] = 0;
+  }
+  __syncthreads();
+  find_threshold_bin<kTopkBins>(h, k, tmp, res);
+  if (threadIdx.x == 0) res[2] = (res[0] == kTopkNoList) ? 0u : h[res[0]];
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_filter_kernel(const TopkHistParams hp) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
+  uint32_t* tmp = hist + 2 * kTopkBins;
+  uint32_t* res = tmp + 40;
+  uint32_t* wkey = reinterpret_cast<uint32_t*>(smem_raw + 2 * kTopkBins * 4 + 1024);   // warp lists
+  int32_t* wposs = reinterpret_cast<int32_t*>(wkey + kTopkCandCap);
+  griddep_wait();
+  const TopkParams& p = hp.base;
+  const int t = blockIdx.x / hp.S;
+  const int s = blockIdx.x - t * hp.S;
+  uint32_t* cnt_out = hp.cand_cnt + (int64_t)t * hp.S + s;
+  const int64_t n = topk_row_len(p, t, false);
+  if (n <= p.k) {
+    if (threadIdx.x == 0) *cnt_out = kTopkNoList;
+    return;
+  }
+  topk_bin_from_hist(hp.hist + (int64_t)t * kTopkBins, hist, (uint32_t)p.k, tmp, res);
+  const uint32_t b1 = res[0];
+  if (b1 == kTopkNoList || (uint64_t)res[1] + res[2] > (uint64_t)kTopkCandCap) {
+    if (threadIdx.x == 0) *cnt_out = kTopkNoList;   // the select kernel runs the whole row
+    return;
+  }
+  // This slice of the row; warp w owns a contiguous segment of it (multiple of 128).
+  const float* row = p.scores + (int64_t)t * p.ld;
+  const int64_t lo = ((int64_t)s * n / hp.S) & ~int64_t(3);
+  const int64_t hi = (s == hp.S - 1) ? n : (((int64_t)(s + 1) * n / hp.S) & ~int64_t(3));
+  const int64_t len = hi - lo;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kWarps = kTopkThreads / 32;
+  constexpr uint32_t WCAP = kTopkCandCap / kWarps;
+  const int64_t seg = ((len + kWarps - 1) / kWarps + 127) & ~int64_t(127);
+  const int64_t s_lo = (warp * seg < len) ? warp * seg : len;
+  const int64_t s_hi = (s_lo + seg < len) ? s_lo + seg : len;
+  const uint32_t lanes_below = (1u << lane) - 1u;
+  uint32_t* wk = wkey + warp * WCAP;
+  int32_t* wp = wposs + warp * WCAP;
+  uint32_t wcount = 0;
+  // four float4 loads in flight per lane
+  for (int64_t i0 = s_lo; i0 < s_hi; i0 += 512) {
+    uint32_t kk[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t e0 = i0 + 128 * u + 4 * lane;
+      if (e0 + 3 < s_hi) {
+        const float4 f = *reinterpret_cast<const float4*>(row + lo + e0);
+        kk[u][0] = score_key(f.x);
+        kk[u][1] = score_key(f.y);
+        kk[u][2] = score_key(f.z);
+        kk[u][3] = score_key(f.w);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) kk[u][e] = (e0 + e < s_hi) ? score_key(row[lo + e0 + e]) : 0u;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t e0 = i0 + 128 * u + 4 * lane;
+      uint32_t flags = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) flags |= ((e0 + e < s_hi) && (kk[u][e] >> 21) >= b1) ? (1u << e) : 0u;
+      if (__any_sync(0xffffffffu, flags != 0)) {
+        uint32_t before = 0, total = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t bal = __ballot_sync(0xffffffffu, (flags >> e) & 1u);
+          before += __popc(bal & lanes_below);
+          total += __popc(bal);
+        }
+        uint32_t at = wcount + before;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (flags & (1u << e)) {
+            if (at < WCAP) {
+              wk[at] = kk[u][e];
+              wp[at] = (int32_t)(lo + e0 + e);
+            }
+            ++at;
+          }
+        }
+        wcount += total;
+      }
+    }
+  }
+  // warp offsets, the slice's count, overflow
+  if (lane == 0) tmp[warp] = wcount;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t w = tmp[lane];
+    uint32_t x = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    const bool over = __any_sync(0xffffffffu, w > WCAP);
+    tmp[lane] = x - w;
+    if (lane == 31) res[3] = (over || x > (uint32_t)kTopkCandCap) ? kTopkNoList : x;
+  }
+  __syncthreads();
+  const uint32_t nc = res[3];
+  if (nc != kTopkNoList) {
+    const int64_t base = ((int64_t)t * hp.S + s) * kTopkCandCap + tmp[warp];
+    for (uint32_t i = lane; i < wcount; i += 32) {
+      hp.cand_key[base + i] = wk[i];
+      hp.cand_pos[base + i] = wp[i];
+    }
+  }
+  if (threadIdx.x == 0) *cnt_out = nc;
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_select_kernel(const TopkHistParams hp) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
+  uint32_t* tmp = hist + 2 * kTopkBins;
+  uint32_t* res = tmp + 40;
+  uint32_t* gkey = reinterpret_cast<uint32_t*>(smem_raw + 2 * kTopkBins * 4 + 1024);   // gathered candidates
+  int32_t* gpos = reinterpret_cast<int32_t*>(gkey + kTopkCandCap);
+  griddep_wait();
+  const TopkParams& p = hp.base;
+  const int t = blockIdx.x;
+  if (t >= p.T) return;
+  const int64_t n = topk_row_len(p, t, threadIdx.x == 0);
+  int32_t* out = p.idx + (int64_t)t * p.k;
+  if (n <= p.k) {  // every candidate is kept
+    for (int64_t i = threadIdx.x; i < p.k; i += kTopkThreads) out[i] = (i < n) ? (int32_t)i : -1;
+    if (threadIdx.x == 0) p.count[t] = (int32_t)n;
+    return;
+  }
+  topk_bin_from_hist(hp.hist + (int64_t)t * kTopkBins, hist, (uint32_t)p.k, tmp, res);
+  const uint32_t b1 = res[0];
+  uint32_t above = res[1];
+  const uint32_t n_cand = res[1] + res[2];
+  // Every slice's list must be there and add up to the histogram's count.
+  if (threadIdx.x == 0) {
+    bool ok = b1 != kTopkNoList && n_cand <= (uint32_t)kTopkCandCap;
+    uint32_t sum = 0;
+    for (int s = 0; ok && s < hp.S; ++s) {
+      const uint32_t c = hp.cand_cnt[(int64_t)t * hp.S + s];
+      if (c == kTopkNoList) ok = false;
+      else sum += c;
+    }
+    res[4] = (ok && sum == n_cand) ? 1u : 0u;
+  }
+  __syncthreads();
+  if (res[4] == 0u) {
+    topk_query<1>(p, t, 0);   // the single-CTA algorithm on the whole row
+    return;
+  }
+  // gather the slices' lists in slice (= position) order, recounting the keys
+  // above and in bin b1: they must be the histogram's counts, or b1 is not the
+  // row's k-th bin (a histogram that does not belong to these scores)
+  if (threadIdx.x == 0) {
+    res[5] = 0;
+    res[6] = 0;
+  }
+  __syncthreads();
+  uint32_t off = 0, my_gt = 0, my_eq = 0;
+  for (int s = 0; s < hp.S; ++s) {
+    const int64_t src = ((int64_t)t * hp.S + s) * kTopkCandCap;
+    const uint32_t c = hp.cand_cnt[(int64_t)t * hp.S + s];
+    for (uint32_t i = threadIdx.x; i < c; i += kTopkThreads) {
+      const uint32_t kk = hp.cand_key[src + i];
+      gkey[off + i] = kk;
+      gpos[off + i] = hp.cand_pos[src + i];
+      my_gt += (kk >> 21) > b1;
+      my_eq += (kk >> 21) == b1;
+    }
+    off += c;
+  }
+  if (my_gt) atomicAdd(&res[5], my_gt);
+  if (my_eq) atomicAdd(&res[6], my_eq);
+  __syncthreads();
+  if (res[5] != above || res[6] != n_cand - above || above >= (uint32_t)p.k) {
+    __syncthreads();
+    topk_query<1>(p, t, 0);
+    return;
+  }
+  const uint32_t n_items = n_cand;
+  uint32_t need = (uint32_t)p.k - above;
+
+  // ---- pass 2: next 11 bits of keys in bin b1
+  for (int b = threadIdx.x; b < kTopkBins; b += kTopkThreads) hist[b] = 0;
+  __syncthreads();
+  for (uint32_t i = threadIdx.x; i < n_items; i += kTopkThreads) {
+    const uint32_t kk = gkey[i];
+    if ((kk >> 21) == b1) atomicAdd(&hist[(kk >> 10) & 0x7FFu], 1u);
+  }
+  __syncthreads();
+  find_threshold_bin<kTopkBins>(hist, need, tmp, res);
+  const uint32_t pre2 = (b1 << 11) | res[0];
+  above += res[1];
+  need -= res[1];
+  // ---- pass 3: last 10 bits of keys with prefix pre2
+  for (int b = threadIdx.x; b < 1024; b += kTopkThreads) hist[b] = 0;
+  __syncthreads();
+  for (uint32_t i = threadIdx.x; i < n_items; i += kTopkThreads) {
+    const uint32_t kk = gkey[i];
+    if ((kk >> 10) == pre2) atomicAdd(&hist[kk & 0x3FFu], 1u);
+  }
+  __syncthreads();
+  find_threshold_bin<1024>(hist, need, tmp, res);
+  const uint32_t tau = (pre2 << 10) | res[0];
+  need -= res[1];
+  const uint32_t need_eq = need;
+  // ---- ordered output: 4 consecutive items (in position order) per thread per round
+  uint32_t base_gt = 0, base_eq = 0;
+  for (uint32_t r0 = 0; r0 < n_items; r0 += 4 * kTopkThreads) {
+    const uint32_t i0 = r0 + 4 * threadIdx.x;
+    uint32_t kk[4];
+    uint32_t c_gt = 0, c_eq = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      kk[e] = (i0 + e < n_items) ? gkey[i0 + e] : 0u;
+      c_gt += (i0 + e < n_items) && (kk[e] > tau);
+      c_eq += (i0 + e < n_items) && (kk[e] == tau);
+    }
+    uint32_t total;
+    const uint32_t ex = block_excl_scan((c_gt << 16) | c_eq, tmp, &total);
+    uint32_t g = base_gt + (ex >> 16), q = base_eq + (ex & 0xFFFFu);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (i0 + e < n_items) {
+        if (kk[e] > tau) {
+          const uint32_t slot = g + min(q, need_eq);
+          if (slot < (uint32_t)p.k) out[slot] = gpos[i0 + e];
+          ++g;
+        } else if (kk[e] == tau) {
+          if (q < need_eq && g + q < (uint32_t)p.k) out[g + q] = gpos[i0 + e];
+          ++q;
+        }
+      }
+    }
+    base_gt += total >> 16;
+    base_eq += total & 0xFFFFu;
+  }
+  if (threadIdx.x == 0) p.count[t] = p.k;
   (void)above;
 }
 

@@ -55,16 +55,17 @@ class AttendPlan(ctypes.Structure):
 class ForwardPlan(ctypes.Structure):
     """Mirror of ``dsa_forward_plan``."""
 
-    _fields_ = [("chunk", _I32), ("n_chunks", _I32), ("last_chunk", _I32), ("reserved", _I32),
+    _fields_ = [("chunk", _I32), ("n_chunks", _I32), ("last_chunk", _I32), ("attend_partials", _I32),
                 ("idx_offset", _SZ), ("count_offset", _SZ), ("attend_offset", _SZ), ("attend_bytes", _SZ),
-                ("scores_offset", _SZ), ("end", _SZ)]
+                ("hist_offset", _SZ), ("topk_offset", _SZ), ("topk_bytes", _SZ), ("scores_offset", _SZ),
+                ("end", _SZ)]
 
 
 SIGNATURES = {
-    "dsa_index_scores": (_I32, [_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _P, _I64, _P]),
-    "dsa_index_scores_fp8": (_I32, [_P, _P, _P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _P, _I64, _P]),
+    "dsa_index_scores": (_I32, [_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _P, _I64, _P, _P]),
+    "dsa_index_scores_fp8": (_I32, [_P, _P, _P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _P, _I64, _P, _P]),
     "dsa_topk_workspace_size": (_SZ, [_I32, _I64, _I32]),
-    "dsa_topk": (_I32, [_P, _I64, _P, _I32, _I32, _P, _P, _P, _SZ, _P]),
+    "dsa_topk": (_I32, [_P, _I64, _P, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
     "sparse_mla_workspace_size": (_SZ, [_I32, _I32]),
     "sparse_mla_attend": (_I32, [_P, _P, _P, _F, _P, _I64, _I32, _I32, _P, _I32, _P, _P, _P, _P, _I32,
                                  _I32, _P, _P, _P, _SZ, _P]),
@@ -77,7 +78,7 @@ SIGNATURES = {
     "dsa_sparse_mla_forward": (_I32, [_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I64, _I32,
                                       ctypes.POINTER(LayerArgs), _F, _I32, _P, _P, _P, _SZ, _P]),
     "dsa_get_device_props": (_I32, [ctypes.POINTER(DeviceProps)]),
-    "dsa_plan_attend": (_I32, [_I32, _I32, _I32, ctypes.POINTER(DeviceProps), ctypes.POINTER(AttendPlan)]),
+    "dsa_plan_attend": (_I32, [_I32, _I32, _I32, _I32, ctypes.POINTER(DeviceProps), ctypes.POINTER(AttendPlan)]),
     "dsa_plan_forward": (_I32, [_I32, _I64, _I32, _I32, _I32, _I32, _I32, _SZ, ctypes.POINTER(DeviceProps),
                                 ctypes.POINTER(ForwardPlan)]),
     "dsa_set_fault_test": (_I32, [ctypes.c_uint64, _I32]),
@@ -140,8 +141,9 @@ def _need(t, dtype, shape, name):
 
 # ----------------------------------------------------------------- calls
 
-def index_scores(q_idx, w, k_idx, seq_row_start, q_seq, q_pos, scores, q_group=1, stream=None):
-    """I[t, s] into ``scores`` [T, ld] (see dsa_index_scores)."""
+def index_scores(q_idx, w, k_idx, seq_row_start, q_seq, q_pos, scores, q_group=1, stream=None, hist=None):
+    """I[t, s] into ``scores`` [T, ld] (see dsa_index_scores); with ``hist`` (uint32 [T, 2048],
+    decode groups only) also the score histogram the top-k's histogram path uses."""
     T = q_idx.shape[0]
     _need(q_idx, torch.bfloat16, (T, 32, 128), "q_idx")
     _need(w, torch.float32, (T, 32), "w")
@@ -150,10 +152,12 @@ def index_scores(q_idx, w, k_idx, seq_row_start, q_seq, q_pos, scores, q_group=1
     _need(q_seq, torch.int32, (T,), "q_seq")
     _need(q_pos, torch.int32, (T,), "q_pos")
     _need(scores, torch.float32, None, "scores")
+    if hist is not None:
+        _need(hist, torch.int32, (T, 2048), "hist")
     lib = load_library()
     _check(lib.dsa_index_scores(_ptr(q_idx), _ptr(w), _ptr(k_idx), k_idx.shape[0], _ptr(seq_row_start),
                                 seq_row_start.shape[0], _ptr(q_seq), _ptr(q_pos), T, q_group,
-                                _ptr(scores), scores.shape[1], _stream(stream)))
+                                _ptr(scores), scores.shape[1], _ptr(hist), _stream(stream)))
     return scores
 
 
@@ -166,7 +170,7 @@ def _codes(t, shape, name):
 
 
 def index_scores_fp8(q8, q_scale, w, k8, k_scale, seq_row_start, q_seq, q_pos, scores, q_group=1,
-                     stream=None):
+                     stream=None, hist=None):
     """I[t, s] on FP8 (E4M3) keys and queries with per-row scales into ``scores``
     [T, ld] (see dsa_index_scores_fp8)."""
     T = q8.shape[0]
@@ -179,23 +183,35 @@ def index_scores_fp8(q8, q_scale, w, k8, k_scale, seq_row_start, q_seq, q_pos, s
     _need(q_seq, torch.int32, (T,), "q_seq")
     _need(q_pos, torch.int32, (T,), "q_pos")
     _need(scores, torch.float32, None, "scores")
+    if hist is not None:
+        _need(hist, torch.int32, (T, 2048), "hist")
     lib = load_library()
     _check(lib.dsa_index_scores_fp8(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), k8.shape[0],
                                     _ptr(seq_row_start), seq_row_start.shape[0], _ptr(q_seq), _ptr(q_pos), T,
-                                    q_group, _ptr(scores), scores.shape[1], _stream(stream)))
+                                    q_group, _ptr(scores), scores.shape[1], _ptr(hist), _stream(stream)))
     return scores
 
 
-def topk(scores, q_pos, k, idx, count, stream=None):
-    """Top-k positions per query into ``idx`` [T, k] and ``count`` [T] (see dsa_topk)."""
+def topk_workspace_bytes(T, ld, k):
+    return int(load_library().dsa_topk_workspace_size(T, ld, k))
+
+
+def topk(scores, q_pos, k, idx, count, stream=None, hist=None, ws=None):
+    """Top-k positions per query into ``idx`` [T, k] and ``count`` [T] (see dsa_topk); with the
+    indexer's ``hist`` the first pass is skipped (a workspace is then needed)."""
     T = scores.shape[0]
     _need(scores, torch.float32, None, "scores")
     _need(q_pos, torch.int32, (T,), "q_pos")
     _need(idx, torch.int32, (T, k), "idx")
     _need(count, torch.int32, (T,), "count")
+    if hist is not None:
+        _need(hist, torch.int32, (T, 2048), "hist")
+        if ws is None:
+            ws = workspace(topk_workspace_bytes(T, scores.shape[1], k), scores.device)
     lib = load_library()
-    _check(lib.dsa_topk(_ptr(scores), scores.shape[1], _ptr(q_pos), T, k, _ptr(idx), _ptr(count),
-                        None, 0, _stream(stream)))
+    _check(lib.dsa_topk(_ptr(scores), scores.shape[1], _ptr(q_pos), T, k, _ptr(idx), _ptr(count), _ptr(hist),
+                        _ptr(ws) if hist is not None else None, ws.numel() if hist is not None else 0,
+                        _stream(stream)))
     return idx, count
 
 
@@ -223,11 +239,11 @@ def make_props(sms, max_clusters):
     return d
 
 
-def plan_attend(T, n_layers=1, k=2048, props=None):
+def plan_attend(T, n_layers=1, k=2048, props=None, allow_partials=True):
     """How the attention splits T queries x n_layers layers (dsa_plan_attend)."""
     out = AttendPlan()
-    _check(load_library().dsa_plan_attend(T, n_layers, k, ctypes.byref(props) if props is not None else None,
-                                          ctypes.byref(out)))
+    _check(load_library().dsa_plan_attend(T, n_layers, k, int(bool(allow_partials)),
+                                          ctypes.byref(props) if props is not None else None, ctypes.byref(out)))
     return out
 
 

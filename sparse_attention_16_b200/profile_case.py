@@ -28,9 +28,15 @@ def main():
     ap.add_argument("--layer", type=int, default=-1,
                     help="attention: one layer of the configuration (default: all its layers in one launch)")
     ap.add_argument("--fp8", action="store_true", help="indexer: FP8 (E4M3) keys and queries, per-row scales")
+    ap.add_argument("--context", type=int, default=0,
+                    help="decode configurations: every sequence this long instead (a smaller capture of the same "
+                         "launch shape)")
     a = ap.parse_args()
 
     case = CONFIGS[a.config]
+    if a.context:
+        assert case.kind == "decode", "--context applies to decode configurations"
+        case = dataclasses.replace(case, lengths=(a.context,) * len(case.lengths))
     if a.kernel != "attend":
         case = dataclasses.replace(case, layers=())
     dev = torch.device("cuda", 0)
@@ -40,6 +46,9 @@ def main():
     scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     cnt = torch.empty((T,), dtype=torch.int32, device=dev)
+    # decode: the indexer's score histogram feeds the top-k's first pass (as in the fused call)
+    hist = torch.empty((T, 2048), dtype=torch.int32, device=dev) if q_group == 1 else None
+    topk_ws = ops.workspace(ops.topk_workspace_bytes(T, ld, k), dev) if q_group == 1 else None
 
     if a.fp8:
         q8, q8_scale = quantize_e4m3_rows(wl.q_idx)
@@ -48,13 +57,13 @@ def main():
     def indexer():
         if a.fp8:
             ops.index_scores_fp8(q8, q8_scale, wl.w, k8, k8_scale, wl.seq_row_start, wl.q_seq, wl.q_pos, scores,
-                                 q_group=q_group)
+                                 q_group=q_group, hist=hist)
         else:
             ops.index_scores(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, scores,
-                             q_group=q_group)
+                             q_group=q_group, hist=hist)
 
     def topk():
-        ops.topk(scores, wl.q_pos, k, idx, cnt)
+        ops.topk(scores, wl.q_pos, k, idx, cnt, hist=hist, ws=topk_ws)
 
     if a.kernel in ("topk", "attend"):
         indexer()

@@ -49,7 +49,7 @@ NULL = None
 
 def test_index_scores_rejects_bad_arguments(lib):
     fake = ctypes.c_void_p(256)  # never dereferenced: validation fails first
-    args = [fake, fake, fake, 100, fake, 1, fake, fake, 4, 1, fake, 128, NULL]
+    args = [fake, fake, fake, 100, fake, 1, fake, fake, 4, 1, fake, 128, NULL, NULL]
     bad = {
         8: -1,     # T < 0
         9: 3,      # q_group not in {1, 8}
@@ -68,16 +68,19 @@ def test_index_scores_rejects_bad_arguments(lib):
     a = list(args)
     a[0] = ctypes.c_void_p(258)  # misaligned
     assert lib.dsa_index_scores(*a) == 1
+    a = list(args)
+    a[9], a[12] = 8, fake        # a histogram needs q_group 1
+    assert lib.dsa_index_scores(*a) == 1
 
 
 def test_topk_rejects_bad_arguments(lib):
     fake = ctypes.c_void_p(256)
-    ok = [fake, 1024, fake, 3, 2048, fake, fake, NULL, 0, NULL]
-    for pos, val in [(4, 0), (4, 16385), (1, 1022), (3, -5)]:
+    ok = [fake, 1024, fake, 3, 2048, fake, fake, NULL, NULL, 0, NULL]
+    for pos, val in [(4, 0), (4, 16385), (1, 1022), (3, -5), (7, ctypes.c_void_p(260))]:
         a = list(ok)
         a[pos] = val
         assert lib.dsa_topk(*a) == 1, (pos, val)
-    assert lib.dsa_topk(fake, 1024, fake, 0, 2048, fake, fake, NULL, 0, NULL) == 0  # T == 0: no-op
+    assert lib.dsa_topk(fake, 1024, fake, 0, 2048, fake, fake, NULL, NULL, 0, NULL) == 0  # T == 0: no-op
 
 
 def test_attend_rejects_bad_arguments(lib):
@@ -169,8 +172,6 @@ def test_attend_plan_covers_every_row_and_fits_its_workspace(lib, name):
                     assert p.workspace_bytes >= units * p.n_split * PER_PARTIAL
                 else:
                     assert p.workspace_bytes == 0
-                if units >= sms:
-                    assert p.n_split == 1
 
 
 def _check_forward_layout(lib, T, ld, k, q_group, n_layers, has_idx, has_cnt, ws, props):
@@ -188,7 +189,7 @@ def _check_forward_layout(lib, T, ld, k, q_group, n_layers, has_idx, has_cnt, ws
     for n in {f.chunk, f.last_chunk}:
         for g in groups:
             if g:
-                need = ops.plan_attend(n, g, k, props).workspace_bytes
+                need = ops.plan_attend(n, g, k, props, allow_partials=bool(f.attend_partials)).workspace_bytes
                 assert need <= f.attend_bytes, (T, ws, n, g, need, f.attend_bytes)
     # regions in order, disjoint, inside the workspace
     regions = []
@@ -196,7 +197,13 @@ def _check_forward_layout(lib, T, ld, k, q_group, n_layers, has_idx, has_cnt, ws
         regions.append((f.idx_offset, f.chunk * k * 4))
     if not has_cnt:
         regions.append((f.count_offset, f.chunk * 4))
-    regions += [(f.attend_offset, f.attend_bytes), (f.scores_offset, f.chunk * ld * 4)]
+    regions.append((f.attend_offset, f.attend_bytes))
+    if q_group == 1:
+        regions += [(f.hist_offset, f.chunk * 2048 * 4), (f.topk_offset, f.topk_bytes)]
+        assert f.topk_bytes >= 2 * f.chunk * 10240 * 4     # at least one candidate list per query
+    else:
+        assert f.hist_offset == f.topk_offset == 2 ** 64 - 1
+    regions.append((f.scores_offset, f.chunk * ld * 4))
     end = 0
     for off, size in regions:
         assert off >= end and off % 256 == 0
@@ -247,3 +254,19 @@ def test_workspace_sizes_need_a_device_or_explicit_props(lib):
     assert p.n_split == 32 and not p.merge and p.workspace_bytes >= 4 * 32 * PER_PARTIAL
     f = ops.plan_forward(64, 32768, 2048, 1, 1, 0, 0, 1 << 40, _props("b200_like"))
     assert f.chunk == 64 and f.n_chunks == 1 and f.end >= 64 * 32768 * 4
+
+
+def test_tight_workspace_falls_back_to_plans_without_partials(lib):
+    # A workspace sized for 16 prefill queries (two layers) must still run 40:
+    # chunks of 8 would need split partials that do not fit, so the layout
+    # restricts the attention to plans without partials.
+    for name in ("b200_like", "no_merge", "small_gpu"):
+        props = _props(name)
+        ws = ops.plan_forward(16, 3040, 2048, 8, 2, 1, 1, 1 << 60, props).end
+        f = _check_forward_layout(lib, 40, 3040, 2048, 8, 2, 1, 1, ws, props)
+        assert f is not None, name
+        if not f.attend_partials:
+            assert f.attend_bytes == 0
+            for n in {f.chunk, f.last_chunk}:
+                p = ops.plan_attend(n, 2, 2048, props, allow_partials=False)
+                assert p.workspace_bytes == 0 and (p.n_split == 1 or p.merge)

@@ -5,6 +5,7 @@ seconds; the full-size configurations are checked on sampled queries in
 test_gpu_fullsize.py.
 """
 
+import dataclasses
 import math
 
 import numpy as np
@@ -127,6 +128,96 @@ def test_topk_special_values_and_short_rows():
     pu.assert_topk_exact(to_numpy(idx), to_numpy(cnt), to_numpy(s).astype(np.float64),
                          to_numpy(q_pos), 2048)
     assert to_numpy(cnt).tolist()[-2:] == [101, 0]
+
+
+# ------------------------------------------------------------------ top-k from the indexer's histogram
+
+def _key_bins(scores_row):
+    """Top 11 bits of the order-preserving key of fp32 scores (NaN as -inf, -0 as +0),
+    written out from the IEEE-754 bit layout."""
+    u = np.asarray(scores_row, dtype=np.float32).view(np.uint32).copy()
+    u[(u & 0x7FFFFFFF) > 0x7F800000] = 0xFF800000
+    u[u == 0x80000000] = 0
+    key = np.where(u & 0x80000000, ~u, u | 0x80000000).astype(np.uint32)
+    return key >> 21
+
+
+def _hist_of(scores, q_pos):
+    s = to_numpy(scores)
+    qp = to_numpy(q_pos)
+    h = np.zeros((s.shape[0], 2048), np.int64)
+    for t in range(s.shape[0]):
+        n = int(qp[t]) + 1
+        if n > 0:
+            h[t] = np.bincount(_key_bins(s[t, :n]), minlength=2048)
+    return h
+
+
+HIST_CASES = [
+    small_case("hist_ragged", (4096, 40000, 1500, 37, 9000, 2049, 2048, 130000), seed=51),
+    small_case("hist_many", (32768,) * 70, seed=52),
+]
+
+
+@pytest.mark.parametrize("case", HIST_CASES, ids=lambda c: c.name)
+def test_indexer_histogram_counts_its_scores(case):
+    wl = make_workload(dataclasses.replace(case, layers=()), DEV)
+    scores = torch.empty((wl.T, case.ld), dtype=torch.float32, device=DEV)
+    hist = torch.full((wl.T, 2048), 12345, dtype=torch.int32, device=DEV)   # overwritten by the call
+    ops.index_scores(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, scores, hist=hist)
+    np.testing.assert_array_equal(to_numpy(hist).astype(np.int64), _hist_of(scores, wl.q_pos))
+
+
+@pytest.mark.parametrize("case", HIST_CASES, ids=lambda c: c.name)
+def test_topk_from_the_histogram_is_bit_exact(case):
+    wl = make_workload(dataclasses.replace(case, layers=()), DEV)
+    scores = torch.empty((wl.T, case.ld), dtype=torch.float32, device=DEV)
+    hist = torch.empty((wl.T, 2048), dtype=torch.int32, device=DEV)
+    ops.index_scores(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, scores, hist=hist)
+    for k in (2048, 7, 4096):
+        idx = torch.empty((wl.T, k), dtype=torch.int32, device=DEV)
+        cnt = torch.empty((wl.T,), dtype=torch.int32, device=DEV)
+        ops.topk(scores, wl.q_pos, k, idx, cnt, hist=hist)
+        pu.assert_topk_exact(to_numpy(idx), to_numpy(cnt), to_numpy(scores).astype(np.float64),
+                             to_numpy(wl.q_pos), k)
+    assert ops.check_errors() == 0
+
+
+def test_topk_from_the_histogram_one_million_positions():
+    case = dataclasses.replace(CONFIGS["decode_b4_1m_4layers"], layers=())
+    wl = make_workload(case, DEV)
+    scores = torch.empty((wl.T, case.ld), dtype=torch.float32, device=DEV)
+    hist = torch.empty((wl.T, 2048), dtype=torch.int32, device=DEV)
+    ops.index_scores(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, scores, hist=hist)
+    idx, cnt = pu.gpu_topk(scores, wl.q_pos, 2048)
+    idx2 = torch.empty_like(idx)
+    cnt2 = torch.empty_like(cnt)
+    ops.topk(scores, wl.q_pos, 2048, idx2, cnt2, hist=hist)
+    assert torch.equal(idx, idx2) and torch.equal(cnt, cnt2)     # both paths agree bit for bit
+    s0 = to_numpy(scores[:2]).astype(np.float64)
+    pu.assert_topk_exact(to_numpy(idx2[:2]), to_numpy(cnt2[:2]), s0, to_numpy(wl.q_pos[:2]), 2048)
+
+
+def test_topk_histogram_path_ties_and_foreign_histograms():
+    # (a) Integer scores: heavy ties, bins far over the candidate cap -> the
+    #     select kernel runs the whole row; (b) a histogram of other scores, and
+    #     one with its bins shifted, must not change the result.
+    g = torch.Generator(device=DEV).manual_seed(77)
+    T, ld = 6, 300_000
+    scores = torch.randint(-3, 4, (T, ld), generator=g, device=DEV).float()
+    scores[1] = torch.randn((ld,), generator=g, device=DEV)
+    scores[2, :] = 1.0
+    q_pos = torch.tensor([ld - 1, ld - 1, 99_999, 5000, 2047, ld - 1], dtype=torch.int32, device=DEV)
+    true_hist = torch.as_tensor(_hist_of(scores, q_pos), dtype=torch.int32, device=DEV)
+    other = torch.as_tensor(_hist_of(torch.randn((T, ld), generator=g, device=DEV), q_pos), dtype=torch.int32,
+                            device=DEV)
+    shifted = torch.roll(true_hist, 3, dims=1)
+    for h in (true_hist, other, shifted):
+        idx = torch.empty((T, 2048), dtype=torch.int32, device=DEV)
+        cnt = torch.empty((T,), dtype=torch.int32, device=DEV)
+        ops.topk(scores, q_pos, 2048, idx, cnt, hist=h)
+        pu.assert_topk_exact(to_numpy(idx), to_numpy(cnt), to_numpy(scores).astype(np.float64), to_numpy(q_pos), 2048)
+    assert ops.check_errors() == 0
 
 
 # ------------------------------------------------------------------ attention
