@@ -57,7 +57,7 @@ from sparse_attention_16_b200 import replicas  # noqa: E402
 from sparse_attention_16_b200.workloads import CONFIGS, make_workload, quantize_e4m3_rows, small_case  # noqa: E402
 
 HEADLINE = "decode_b4_1m_4layers"
-EXTRAS = ("decode_b64_32k", "prefill_32k_plus_8k")
+EXTRAS = ("decode_b64_32k", "prefill_32k_plus_8k", "decode_b16_32k_4queries")
 METRIC = "sparse-MLA+DSA decode queries/s per layer; achieved HBM TB/s vs peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -155,6 +155,14 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- our arm
 
+def query_group(case):
+    """Queries scored together per key tile: 8 in chunked prefill, 4 when a
+    sequence decodes 4 queries at once, else 1."""
+    if case.kind == "prefill":
+        return 8
+    return 4 if case.per_seq % 4 == 0 else 1
+
+
 def measure(name, dev, steps, warmup, rank, world, local, min_seconds=0.0, sample_clocks=False, fp8=False,
             eager=False, e2e=False, e2e_steps=20):
     """Times `steps` steps of configuration `name` (see the module docstring).
@@ -167,7 +175,7 @@ def measure(name, dev, steps, warmup, rank, world, local, min_seconds=0.0, sampl
     wl = make_workload(case, dev)
     T, ld, k = wl.T, case.ld, case.topk
     n_layers = len(wl.layers)
-    q_group = 8 if case.kind == "prefill" else 1
+    q_group = query_group(case)
 
     scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
@@ -296,7 +304,8 @@ def measure(name, dev, steps, warmup, rank, world, local, min_seconds=0.0, sampl
     idx_name = "indexer_kernel<{},{}>".format(q_group, "fp8" if fp8 else "bf16")
     idx_kernel = "indexer_fp8" if fp8 else "indexer"
     res = {
-        "config": case.name, "T": T, "n_layers": n_layers, "ld": ld, "steps": steps, "graph_replays": replays,
+        "config": case.name, "T": T, "n_layers": n_layers, "ld": ld, "q_group": q_group, "steps": steps,
+        "graph_replays": replays,
         "timed_steps": timed_steps, "timed_region_s": round(elapsed, 4), "ms_per_step": round(step_s * 1e3, 4),
         "queries_per_s": T * world / step_s, "query_layers_per_s": T * n_layers * world / step_s,
         "launches": launches, "clocks": clocks,
@@ -433,7 +442,7 @@ def run_ours(args, rank, world, local):
                         min_seconds=0.0 if CONFIGS[name].kind == "prefill" else 0.3, fp8=args.fp8_keys)
             torch.cuda.empty_cache()
             keep = ("ms_per_step", "queries_per_s", "query_layers_per_s", "kernel_ms", "step_hbm", "attention_hbm",
-                    "roofline", "timed_steps", "attend_plan")
+                    "roofline", "timed_steps", "attend_plan", "q_group")
             extras[name] = {k_: (round(v, 4) if isinstance(v, float) else v) for k_, v in r.items() if k_ in keep}
         line["extra_configs"] = extras
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -460,7 +469,7 @@ def _oracle_sample(config, n_queries):
     case = CONFIGS[config]
     if case.kind == "decode":
         sub = small_case(config + "_sample", case.lengths[:n_queries], layers=case.layers, qmul=case.qmul,
-                         mla_q_std=case.mla_q_std, seed=case.seed, planted=case.planted)
+                         mla_q_std=case.mla_q_std, seed=case.seed, planted=case.planted, per_seq=case.per_seq)
     else:
         sub = small_case(config + "_sample", kind="prefill", cached=case.cached + case.new - n_queries,
                          new=n_queries, layers=case.layers, qmul=case.qmul, mla_q_std=case.mla_q_std,

@@ -83,9 +83,11 @@ typedef enum dsa_status {
  *   w       f32  [T, 32]        per-head weights
  *   k_idx   bf16 [n_rows, 128]  index keys, rows located by seq_row_start
  *   seq_row_start int64 [B], q_seq int32 [T], q_pos int32 [T]  (device); B >= 1
- *   q_group 1: no assumption.  8: the caller guarantees that queries
- *           [8g, 8g+8) share one sequence (chunked prefill); they are then
- *           scored together, 8 queries x 32 heads per tensor-core tile.
+ *   q_group 1: no assumption.  4 or 8: the caller guarantees that queries
+ *           [q_group g, q_group (g + 1)) share one sequence (several decode
+ *           queries of a sequence, e.g. drafted tokens being verified; chunked
+ *           prefill); they are then scored together, q_group queries x 32
+ *           heads per tensor-core tile, so each key row is read once per group.
  *   scores  f32 [T, ld]: I[t,s] for s <= q_pos[t], -inf for q_pos[t] < s < ld.
  *           ld >= max(q_pos) + 1 and ld % 4 == 0.
  *   hist    uint32 [T, 2048] or NULL (q_group 1 only): overwritten with, for
@@ -93,7 +95,7 @@ typedef enum dsa_status {
  *           the top 11 bits of their order-preserving key (the first histogram
  *           of dsa_topk's radix select, which then skips that pass).
  * Returns DSA_ERR_INVALID_ARG for null/misaligned pointers, T < 0, n_rows < 1,
- * n_rows >= 2^31 - 256, ld < 4 or ld % 4, q_group not 1 or 8, hist with q_group 8.
+ * n_rows >= 2^31 - 256, ld < 4 or ld % 4, q_group not 1, 4 or 8, hist with q_group > 1.
  */
 dsa_status_t dsa_index_scores(const void* q_idx, const float* w, const void* k_idx,
                               int64_t n_rows, const int64_t* seq_row_start, int32_t B,
@@ -234,14 +236,16 @@ dsa_status_t sparse_mla_attend_noalloc(const void* q_nope, const void* q_pe, con
 
 /* One attention layer fed by a shared selection (fields as in sparse_mla_attend). */
 typedef struct dsa_layer_args {
-  const void* q_nope;   /* bf16 [T, 64, 512]                      */
-  const void* q_pe;     /* bf16 [T, 64, 64] or NULL (NoPE)        */
-  const float* qmul;    /* f32 [T, 64]                            */
-  const void* cache;    /* bf16 [n_rows, ld_c]                    */
+  const void* q_nope;   /* bf16 [T, 64, 512]                                  */
+  const void* q_pe;     /* bf16 [T, 64, 64] or NULL (NoPE)                    */
+  const float* qmul;    /* f32 [T, 64]                                        */
+  const void* cache;    /* bf16 [n_rows, ld_c]                                */
   int32_t ld_c;
-  int32_t d_rope;       /* 64 or 0                                */
-  void* out;            /* bf16 [T, 64, 512]                      */
-  float* lse;           /* f32 [T, 64] or NULL                    */
+  int32_t d_rope;       /* 64 or 0                                            */
+  void* out;            /* bf16 [T, 64, 512], or f32 when out_f32 = 1         */
+  float* lse;           /* f32 [T, 64] or NULL                                */
+  int32_t out_f32;      /* 1: fp32 output (partials for dsa_lse_combine)      */
+  int32_t reserved;     /* 0                                                  */
 } dsa_layer_args;
 
 /*
@@ -287,6 +291,47 @@ dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const voi
                                     const dsa_layer_args* layers, float softmax_scale,
                                     int32_t k, int32_t* idx_out, int32_t* count_out,
                                     void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Context-parallel decode (report's serving section, Figures 16-17: the
+ * positions of a long sequence are split over ranks; each rank scores and
+ * selects among its own positions, the candidates are exchanged and merged
+ * into the global selection, each rank attends over the selected rows it
+ * holds, and the partial outputs are combined).  The exchanges themselves
+ * (all-gathers over NCCL) are the caller's; these calls are the steps between.
+ *
+ * dsa_topk_export: a rank's selection as exchange candidates.  For query t and
+ *   i < count[t]: out_score[t, i] = scores[t, idx[t, i]], out_pos[t, i] =
+ *   idx[t, i] + pos_offset (the global position); -inf / -1 elsewhere and for
+ *   -1 entries.  scores f32 [T, ld], idx int32 [T, k], count int32 [T],
+ *   out_score f32 [T, k], out_pos int32 [T, k]; global positions < 2^31.
+ *
+ * dsa_topk_merge: the global selection from R ranks' candidates
+ *   cand_score f32 [R, T, kr], cand_pos int32 [R, T, kr] (-1 = empty slot).
+ *   Rank r must hold a contiguous range of positions, ranges in rank order, and
+ *   list its candidates in ascending position (dsa_topk's order), so that the
+ *   concatenation is in position order.  Same ranking rule as dsa_topk (score
+ *   descending, ties to the lower position, -0 == +0, NaN as -inf); writes the
+ *   best min(k, valid candidates) positions ascending to idx_global [T, k]
+ *   (optional), their number to count [T], and (optional, together) the ones
+ *   in this rank's shard [shard_lo, shard_hi) as shard-local positions
+ *   (position - shard_lo), ascending and compacted, -1 after them, to
+ *   idx_local [T, k], with their number in count_local [T] - the selection
+ *   this rank's attention runs over.  R x kr <= 16384.
+ *
+ * dsa_lse_combine: merges R partial attentions over disjoint parts of one
+ *   selection: o_parts f32 [R, T, 64, 512] (each normalised over its part: a
+ *   layer run with out_f32 = 1), lse_parts f32 [R, T, 64] (-inf for an empty
+ *   part) -> out bf16 [T, 64, 512] = sum_r exp(lse_r - lse) o_r and lse f32
+ *   [T, 64] (optional) = log sum_r exp(lse_r).  1 <= R <= 64.
+ */
+dsa_status_t dsa_topk_export(const float* scores, int64_t ld, const int32_t* idx, const int32_t* count, int32_t T,
+                             int32_t k, int64_t pos_offset, float* out_score, int32_t* out_pos, void* stream);
+dsa_status_t dsa_topk_merge(const float* cand_score, const int32_t* cand_pos, int32_t R, int32_t T, int32_t kr,
+                            int32_t k, int64_t shard_lo, int64_t shard_hi, int32_t* idx_global, int32_t* idx_local,
+                            int32_t* count_local, int32_t* count, void* stream);
+dsa_status_t dsa_lse_combine(const float* o_parts, const float* lse_parts, int32_t R, int32_t T, void* out,
+                             float* lse, void* stream);
 
 /*
  * Launch planning queries (host only: no device work, no allocation).  They

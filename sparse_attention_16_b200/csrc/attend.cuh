@@ -102,8 +102,20 @@ struct AttLayer {
   float* lse;                     // [T, 64] or null
   int64_t ld_c;                   // row stride of the cache, elements
   int32_t d_rope;                 // 64 (RoPE) or 0 (NoPE)
-  int32_t pad_;
+  int32_t out_f32;                // 1: `out` is fp32 [T, 64, 512] (partial outputs to combine later)
 };
+
+// Stores four output values of (t, h) at column c (a multiple of 4) in the layer's output type.
+__device__ __forceinline__ void store_out4(const AttLayer& L, int64_t th, int c, float a, float b, float cc, float d) {
+  if (L.out_f32) {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(L.out) + th * kLatent + c) = make_float4(a, b, cc, d);
+  } else {
+    uint2 o;
+    o.x = pack_bf16x2(a, b);
+    o.y = pack_bf16x2(cc, d);
+    *reinterpret_cast<uint2*>(L.out + th * kLatent + c) = o;
+  }
+}
 
 struct AttendParams {
   AttLayer layer[kMaxAttLayers];
@@ -301,10 +313,7 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLa
         acc.w = fmaf(wj, v.w, acc.w);
       }
     }
-    uint2 o;
-    o.x = pack_bf16x2(acc.x, acc.y);
-    o.y = pack_bf16x2(acc.z, acc.w);
-    *reinterpret_cast<uint2*>(L.out + ((int64_t)t * kHeads + h) * kLatent + 4 * (c0 + c)) = o;
+    store_out4(L, (int64_t)t * kHeads + h, 4 * (c0 + c), acc.x, acc.y, acc.z, acc.w);
   }
 }
 
@@ -662,19 +671,28 @@ __device__ __forceinline__ void attend_unit(const AttendParams& p, const AttLaye
   };
   if (p.n_split == 1) {
     const float inv = (have_o && Lsum > 0.f) ? 1.f / Lsum : 0.f;
-    uint4* o_t = reinterpret_cast<uint4*>(L.out + ((int64_t)t * kHeads + h) * kLatent + 32 * hf);
+    const int64_t th = (int64_t)t * kHeads + h;
 #pragma unroll 1
     for (int cb = 0; cb < kLatent; cb += 64) {
       uint32_t u[32];
       read_o(cb, u);
+      if (L.out_f32) {
+        float4* o_t = reinterpret_cast<float4*>(reinterpret_cast<float*>(L.out) + th * kLatent + 32 * hf + cb);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 w;
-        w.x = pack_bf16x2(__uint_as_float(u[8 * q]) * inv, __uint_as_float(u[8 * q + 1]) * inv);
-        w.y = pack_bf16x2(__uint_as_float(u[8 * q + 2]) * inv, __uint_as_float(u[8 * q + 3]) * inv);
-        w.z = pack_bf16x2(__uint_as_float(u[8 * q + 4]) * inv, __uint_as_float(u[8 * q + 5]) * inv);
-        w.w = pack_bf16x2(__uint_as_float(u[8 * q + 6]) * inv, __uint_as_float(u[8 * q + 7]) * inv);
-        o_t[cb / 8 + q] = w;
+        for (int q = 0; q < 8; ++q)
+          o_t[q] = make_float4(__uint_as_float(u[4 * q]) * inv, __uint_as_float(u[4 * q + 1]) * inv,
+                               __uint_as_float(u[4 * q + 2]) * inv, __uint_as_float(u[4 * q + 3]) * inv);
+      } else {
+        uint4* o_t = reinterpret_cast<uint4*>(L.out + th * kLatent + 32 * hf);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(u[8 * q]) * inv, __uint_as_float(u[8 * q + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(u[8 * q + 2]) * inv, __uint_as_float(u[8 * q + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(u[8 * q + 4]) * inv, __uint_as_float(u[8 * q + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(u[8 * q + 6]) * inv, __uint_as_float(u[8 * q + 7]) * inv);
+          o_t[cb / 8 + q] = w;
+        }
       }
     }
     if (L.lse != nullptr && hf == 0)
@@ -804,13 +822,68 @@ __global__ void __launch_bounds__(128) attend_combine_kernel(const __grid_consta
     acc.z = fmaf(wj, o4.z, acc.z);
     acc.w = fmaf(wj, o4.w, acc.w);
   }
-  __nv_bfloat16* o = L.out + ((int64_t)t * kHeads + h) * kLatent + d;
-  *reinterpret_cast<__nv_bfloat162*>(o) = __floats2bfloat162_rn(acc.x, acc.y);
-  *reinterpret_cast<__nv_bfloat162*>(o + 2) = __floats2bfloat162_rn(acc.z, acc.w);
+  store_out4(L, (int64_t)t * kHeads + h, d, acc.x, acc.y, acc.z, acc.w);
   if (threadIdx.x == 0 && L.lse != nullptr) {
     const float Lx = stats[1];
     L.lse[(int64_t)t * kHeads + h] = (Lx > 0.f) ? (stats[0] + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
   }
+}
+
+// Context-parallel output combine (report's serving section): R ranks each
+// attended over their own part of one selection, giving o_r (normalised over
+// that part, fp32) and lse_r.  Over the whole selection
+//   lse = log sum_r exp(lse_r),  o = sum_r exp(lse_r - lse) o_r
+// (a part with lse_r = -inf contributes nothing; all parts empty: o = 0,
+// lse = -inf).  One block per (query, head); 128 threads x 4 columns.
+struct LseCombineParams {
+  const float* o_parts;       // [R, T, 64, 512]
+  const float* lse_parts;     // [R, T, 64]
+  __nv_bfloat16* out;         // [T, 64, 512]
+  float* lse;                 // [T, 64] or null
+  int32_t R, T;
+};
+
+__global__ void __launch_bounds__(128) lse_combine_kernel(const LseCombineParams cp) {
+  griddep_wait();
+  const int t = blockIdx.x / kHeads;
+  const int h = blockIdx.x % kHeads;
+  __shared__ float wr[64];
+  __shared__ float stat;
+  if (threadIdx.x < 32) {
+    float M = -INFINITY;
+    for (int r = threadIdx.x; r < cp.R; r += 32) M = fmaxf(M, cp.lse_parts[((int64_t)r * cp.T + t) * kHeads + h]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float S = 0.f;
+    for (int r = threadIdx.x; r < cp.R; r += 32) {
+      const float l = cp.lse_parts[((int64_t)r * cp.T + t) * kHeads + h];
+      const float w = (l == -INFINITY) ? 0.f : ex2_approx((l - M) * 1.4426950408889634f);
+      wr[r] = w;
+      S += w;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+    __syncwarp();
+    for (int r = threadIdx.x; r < cp.R; r += 32) wr[r] = (S > 0.f) ? wr[r] / S : 0.f;
+    if (threadIdx.x == 0) stat = (S > 0.f) ? M + lg2_approx(S) * 0.69314718055994531f : -INFINITY;
+  }
+  __syncthreads();
+  const int d = threadIdx.x * 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int r = 0; r < cp.R; ++r) {
+    const float w = wr[r];
+    if (w == 0.f) continue;
+    const float4 o4 = *reinterpret_cast<const float4*>(cp.o_parts + (((int64_t)r * cp.T + t) * kHeads + h) * kLatent + d);
+    acc.x = fmaf(w, o4.x, acc.x);
+    acc.y = fmaf(w, o4.y, acc.y);
+    acc.z = fmaf(w, o4.z, acc.z);
+    acc.w = fmaf(w, o4.w, acc.w);
+  }
+  uint2 o;
+  o.x = pack_bf16x2(acc.x, acc.y);
+  o.y = pack_bf16x2(acc.z, acc.w);
+  *reinterpret_cast<uint2*>(cp.out + ((int64_t)t * kHeads + h) * kLatent + d) = o;
+  if (threadIdx.x == 0 && cp.lse != nullptr) cp.lse[(int64_t)t * kHeads + h] = stat;
 }
 
 }  // namespace dsa

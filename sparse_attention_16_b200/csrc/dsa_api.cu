@@ -101,8 +101,8 @@ uint64_t current_context_id() {
 
 // ----------------------------------------------------------------- per-device state
 enum KernelId : uint32_t {
-  kKIdx1 = 0, kKIdx8, kKIdx1F8, kKIdx8F8, kKTopk1, kKTopk2, kKTopk4, kKTopk8, kKTopk16, kKAttend, kKTopkFilter,
-  kKTopkSelect, kKCount
+  kKIdx1 = 0, kKIdx4, kKIdx8, kKIdx1F8, kKIdx4F8, kKIdx8F8, kKTopk1, kKTopk2, kKTopk4, kKTopk8, kKTopk16, kKAttend, kKTopkFilter,
+  kKTopkSelect, kKTopkMerge, kKCount
 };
 
 constexpr int kMaxDevices = 64;
@@ -318,7 +318,8 @@ dsa_status_t launch_indexer(DevLock& L, const void* q_idx, const float* q_scale,
   dsa::DevProps props;
   DSA_TRY(device_props(L, &props));
   const int grid = (int)std::min<int64_t>(p.n_units, props.sms);
-  const KernelId id = F8 ? (QG == 8 ? kKIdx8F8 : kKIdx1F8) : (QG == 8 ? kKIdx8 : kKIdx1);
+  const KernelId id = F8 ? (QG == 8 ? kKIdx8F8 : (QG == 4 ? kKIdx4F8 : kKIdx1F8))
+                          : (QG == 8 ? kKIdx8 : (QG == 4 ? kKIdx4 : kKIdx1));
   DSA_TRY(set_smem(*L.s, id, dsa::indexer_kernel<QG, F8>, C::SMEM_BYTES));
   return launch(dsa::indexer_kernel<QG, F8>, (unsigned)grid, C::THREADS, C::SMEM_BYTES, stream, 1, kmap, qmap,
                 p);
@@ -330,6 +331,9 @@ dsa_status_t indexer_impl(DevLock& L, const void* q_idx, const float* w, const v
                           int64_t ld, uint32_t* hist, cudaStream_t stream) {
   if (q_group == 8)
     return launch_indexer<8, false>(L, q_idx, nullptr, w, k_idx, nullptr, n_rows, seq_row_start, B, q_seq, q_pos,
+                                    T, scores, ld, nullptr, stream);
+  if (q_group == 4)
+    return launch_indexer<4, false>(L, q_idx, nullptr, w, k_idx, nullptr, n_rows, seq_row_start, B, q_seq, q_pos,
                                     T, scores, ld, nullptr, stream);
   return launch_indexer<1, false>(L, q_idx, nullptr, w, k_idx, nullptr, n_rows, seq_row_start, B, q_seq, q_pos, T,
                                   scores, ld, hist, stream);
@@ -424,6 +428,7 @@ dsa_status_t launch_attend(DevLock& L, const dsa_layer_args* layers, int32_t n_l
     p.layer[l].lse = a.lse;
     p.layer[l].ld_c = a.ld_c;
     p.layer[l].d_rope = a.d_rope;
+    p.layer[l].out_f32 = a.out_f32 ? 1 : 0;
   }
   p.seq_row_start = seq_row_start;
   p.q_seq = q_seq;
@@ -475,7 +480,8 @@ dsa_status_t attend_layers_impl(DevLock& L, const dsa_layer_args* layers, int32_
       sub[i].q_nope = static_cast<const __nv_bfloat16*>(a.q_nope) + qo * dsa::kLatent;
       sub[i].q_pe = a.q_pe ? static_cast<const __nv_bfloat16*>(a.q_pe) + qo * 64 : nullptr;
       sub[i].qmul = a.qmul + qo;
-      sub[i].out = static_cast<__nv_bfloat16*>(a.out) + qo * dsa::kLatent;
+      sub[i].out = a.out_f32 ? static_cast<void*>(static_cast<float*>(a.out) + qo * dsa::kLatent)
+                             : static_cast<void*>(static_cast<__nv_bfloat16*>(a.out) + qo * dsa::kLatent);
       sub[i].lse = a.lse ? a.lse + qo : nullptr;
     }
     DSA_TRY(launch_attend(L, sub, g, scale, n_rows, seq_row_start, B, q_seq, q_pos, idx, count, T, k, ws,
@@ -496,7 +502,7 @@ dsa_status_t check_index_args(const void* q_idx, const float* w, const void* k_i
   DSA_REQUIRE(B >= 1, "B must be >= 1");
   DSA_REQUIRE(n_rows >= 1 && n_rows < (int64_t(1) << 31) - 256, "n_rows out of range");
   DSA_REQUIRE(ld >= 4 && ld % 4 == 0 && ld < (int64_t(1) << 31), "ld must be a multiple of 4 in [4, 2^31)");
-  DSA_REQUIRE(q_group == 1 || q_group == 8, "q_group must be 1 or 8");
+  DSA_REQUIRE(q_group == 1 || q_group == 4 || q_group == 8, "q_group must be 1, 4 or 8");
   DSA_REQUIRE((int64_t)T * dsa::kIdxHeads < (int64_t(1) << 31), "T too large");
   return DSA_OK;
 }
@@ -516,6 +522,7 @@ dsa_status_t check_topk_args(const float* scores, int64_t ld, const int32_t* q_p
 dsa_status_t check_layer_args(const dsa_layer_args& a, int64_t n_rows) {
   DSA_REQUIRE(a.d_rope == 0 || a.d_rope == 64, "d_rope must be 0 or 64 (got %d)", a.d_rope);
   DSA_REQUIRE(a.q_nope && a.qmul && a.cache && a.out, "null pointer argument");
+  DSA_REQUIRE(a.out_f32 == 0 || a.out_f32 == 1, "out_f32 must be 0 or 1");
   DSA_REQUIRE((a.q_pe != nullptr) == (a.d_rope == 64), "q_pe must be given iff d_rope == 64");
   DSA_REQUIRE(aligned(a.q_nope, 16) && aligned(a.cache, 16) && aligned(a.out, 16) &&
                   (a.q_pe == nullptr || aligned(a.q_pe, 16)),
@@ -553,6 +560,8 @@ dsa_layer_args one_layer(const void* q_nope, const void* q_pe, const float* qmul
   a.d_rope = d_rope;
   a.out = out;
   a.lse = lse;
+  a.out_f32 = 0;
+  a.reserved = 0;
   return a;
 }
 
@@ -631,6 +640,9 @@ dsa_status_t dsa_index_scores_fp8(const void* q8, const float* q_scale, const fl
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (q_group == 8)
     return launch_indexer<8, true>(L, q8, q_scale, w, k8, k_scale, n_rows, seq_row_start, B, q_seq, q_pos, T,
+                                   scores, ld, nullptr, s);
+  if (q_group == 4)
+    return launch_indexer<4, true>(L, q8, q_scale, w, k8, k_scale, n_rows, seq_row_start, B, q_seq, q_pos, T,
                                    scores, ld, nullptr, s);
   return launch_indexer<1, true>(L, q8, q_scale, w, k8, k_scale, n_rows, seq_row_start, B, q_seq, q_pos, T, scores,
                                  ld, hist, s);
@@ -802,6 +814,77 @@ dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const voi
   return DSA_OK;
 }
 
+dsa_status_t dsa_topk_export(const float* scores, int64_t ld, const int32_t* idx, const int32_t* count, int32_t T,
+                             int32_t k, int64_t pos_offset, float* out_score, int32_t* out_pos, void* stream) {
+  NvtxRange nvtx_range("dsa_topk_export");
+  DSA_REQUIRE(T >= 0 && k >= 1 && k <= kMaxK && ld >= 1, "bad sizes");
+  DSA_REQUIRE(scores && idx && count && out_score && out_pos, "null pointer argument");
+  DSA_REQUIRE(aligned(scores, 4) && aligned(idx, 4) && aligned(count, 4) && aligned(out_score, 4) &&
+                  aligned(out_pos, 4), "misaligned argument");
+  DSA_REQUIRE(pos_offset >= 0 && pos_offset + ld < (int64_t(1) << 31), "global positions must fit int32");
+  if (T == 0) return DSA_OK;
+  DevLock L;
+  DSA_TRY(lock_device(L));
+  return launch(dsa::topk_export_kernel, (unsigned)T, 256, 0, static_cast<cudaStream_t>(stream), 1, scores, ld, idx,
+                count, T, k, pos_offset, out_score, out_pos);
+}
+
+dsa_status_t dsa_topk_merge(const float* cand_score, const int32_t* cand_pos, int32_t R, int32_t T, int32_t kr,
+                            int32_t k, int64_t shard_lo, int64_t shard_hi, int32_t* idx_global, int32_t* idx_local,
+                            int32_t* count_local, int32_t* count, void* stream) {
+  NvtxRange nvtx_range("dsa_topk_merge");
+  DSA_REQUIRE(R >= 1 && T >= 0 && kr >= 1 && k >= 1 && k <= kMaxK, "bad sizes");
+  DSA_REQUIRE((int64_t)R * kr <= dsa::kMergeCap, "R x kr must be <= %d candidates per query", dsa::kMergeCap);
+  DSA_REQUIRE(cand_score && cand_pos && count, "null pointer argument");
+  DSA_REQUIRE((idx_local == nullptr) == (count_local == nullptr), "idx_local and count_local go together");
+  DSA_REQUIRE(count_local == nullptr || aligned(count_local, 4), "misaligned count_local");
+  DSA_REQUIRE(aligned(cand_score, 4) && aligned(cand_pos, 4) && aligned(count, 4) &&
+                  (idx_global == nullptr || aligned(idx_global, 4)) && (idx_local == nullptr || aligned(idx_local, 4)),
+              "misaligned argument");
+  DSA_REQUIRE(0 <= shard_lo && shard_lo <= shard_hi, "bad shard range");
+  if (T == 0) return DSA_OK;
+  DevLock L;
+  DSA_TRY(lock_device(L));
+  dsa::MergeParams mp;
+  mp.cand_score = cand_score;
+  mp.cand_pos = cand_pos;
+  mp.shard_lo = shard_lo;
+  mp.shard_hi = shard_hi;
+  mp.idx_global = idx_global;
+  mp.idx_local = idx_local;
+  mp.count_local = count_local;
+  mp.count = count;
+  mp.R = R;
+  mp.T = T;
+  mp.kr = kr;
+  mp.k = k;
+  DSA_TRY(set_smem(*L.s, kKTopkMerge, dsa::topk_merge_kernel, dsa::kTopkSmemBytes));
+  return launch(dsa::topk_merge_kernel, (unsigned)T, dsa::kTopkThreads, dsa::kTopkSmemBytes,
+                static_cast<cudaStream_t>(stream), 1, mp);
+}
+
+dsa_status_t dsa_lse_combine(const float* o_parts, const float* lse_parts, int32_t R, int32_t T, void* out,
+                             float* lse, void* stream) {
+  NvtxRange nvtx_range("dsa_lse_combine");
+  DSA_REQUIRE(R >= 1 && R <= 64 && T >= 0, "1 <= R <= 64 and T >= 0 required");
+  DSA_REQUIRE(o_parts && lse_parts && out, "null pointer argument");
+  DSA_REQUIRE(aligned(o_parts, 16) && aligned(out, 16) && aligned(lse_parts, 4) && (lse == nullptr || aligned(lse, 4)),
+              "misaligned argument");
+  DSA_REQUIRE((int64_t)T * dsa::kHeads < (int64_t(1) << 31), "T too large");
+  if (T == 0) return DSA_OK;
+  DevLock L;
+  DSA_TRY(lock_device(L));
+  dsa::LseCombineParams cp;
+  cp.o_parts = o_parts;
+  cp.lse_parts = lse_parts;
+  cp.out = static_cast<__nv_bfloat16*>(out);
+  cp.lse = lse;
+  cp.R = R;
+  cp.T = T;
+  return launch(dsa::lse_combine_kernel, (unsigned)(T * dsa::kHeads), 128, 0, static_cast<cudaStream_t>(stream), 1,
+                cp);
+}
+
 dsa_status_t dsa_get_device_props(dsa_device_props* out) {
   DSA_REQUIRE(out != nullptr, "null pointer argument");
   dsa::DevProps d;
@@ -826,7 +909,8 @@ dsa_status_t dsa_plan_forward(int32_t T, int64_t ld, int32_t k, int32_t q_group,
                               int32_t has_idx_out, int32_t has_count_out, size_t ws_bytes,
                               const dsa_device_props* props, dsa_forward_plan* out) {
   DSA_REQUIRE(out != nullptr, "null pointer argument");
-  DSA_REQUIRE(T >= 1 && ld >= 4 && k >= 1 && k <= kMaxK && (q_group == 1 || q_group == 8) && n_layers >= 0,
+  DSA_REQUIRE(T >= 1 && ld >= 4 && k >= 1 && k <= kMaxK && (q_group == 1 || q_group == 4 || q_group == 8) &&
+                  n_layers >= 0,
               "bad sizes");
   dsa::DevProps d;
   DSA_TRY(props_for_query(props, &d));

@@ -5,7 +5,8 @@
 // multiply-adds per scored position).
 //
 // One tile = 128 consecutive key rows of one sequence x QG queries (QG = 1 for
-// decode, 8 for chunked prefill).  The 128 x 128 bf16 key tile and the
+// decode, 4 for several queries of one sequence decoded together - e.g. the
+// verification of drafted tokens - and 8 for chunked prefill).  The 128 x 128 bf16 key tile and the
 // (32*QG) x 128 query block are brought into shared memory by TMA with the
 // 128-byte swizzle; one tcgen05.mma chain (M = 128 keys, N = 32*QG, K = 128)
 // leaves, in TMEM lane r, the 32 head dot products of key r for every query in
@@ -50,13 +51,13 @@ struct IdxCfg {
   static constexpr int N = 32 * QG;                     // MMA N: heads x queries
   static constexpr int KBLK = F8 ? 1 : 2;               // 128-byte column blocks per row
   static constexpr int STAGES = F8 ? ((QG == 1) ? 12 : 8) : ((QG == 1) ? 6 : 4);   // key tiles in flight
-  static constexpr int QBUFS = (QG == 1) ? 2 : 1;       // query blocks in flight
+  static constexpr int QBUFS = (QG == 8) ? 1 : 2;       // query blocks in flight
   static constexpr int KHALF = kKeyTile * 128;          // bytes of one 128-byte column block
   static constexpr int KT_BYTES = KBLK * KHALF;         // 32 KB (bf16) / 16 KB (fp8) per key tile
   static constexpr int QHALF = N * 128;
   static constexpr int Q_BYTES = KBLK * QHALF;
   static constexpr int KSTEPS = F8 ? kIdxDim / 32 : kIdxDim / 16;   // MMAs per tile (K = 32 / 16)
-  static constexpr int EPI_WARPS = (QG == 1) ? 4 : 8;
+  static constexpr int EPI_WARPS = (QG == 8) ? 8 : 4;   // QG 4: four warps x four queries
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int NACC = (F8 && QG == 1) ? 4 : 2;   // TMEM accumulators in flight (measured best)
   static constexpr int TMEM_COLS = (NACC * N < 32) ? 32 : NACC * N;

@@ -497,6 +497,70 @@ __device__ __forceinline__ void topk_bin_from_hist(const uint32_t* g_hist, uint3
   __syncthreads();
 }
 
+// The last two radix passes and the ordered output over items gathered in
+// shared memory in position order (one CTA): b1 is the k-th key's top-11-bit
+// bin and `above` the number of items in higher bins.  Writes the k selected
+// positions to out[0..k) in ascending order.
+__device__ __forceinline__ void finish_gathered(const uint32_t* gkey, const int32_t* gpos, uint32_t n_items,
+                                                uint32_t b1, uint32_t above, uint32_t k, int32_t* out,
+                                                uint32_t* hist, uint32_t* tmp, uint32_t* res) {
+  uint32_t need = k - above;
+  // ---- pass 2: next 11 bits of keys in bin b1
+  for (int b = threadIdx.x; b < kTopkBins; b += kTopkThreads) hist[b] = 0;
+  __syncthreads();
+  for (uint32_t i = threadIdx.x; i < n_items; i += kTopkThreads) {
+    const uint32_t kk = gkey[i];
+    if ((kk >> 21) == b1) atomicAdd(&hist[(kk >> 10) & 0x7FFu], 1u);
+  }
+  __syncthreads();
+  find_threshold_bin<kTopkBins>(hist, need, tmp, res);
+  const uint32_t pre2 = (b1 << 11) | res[0];
+  need -= res[1];
+  // ---- pass 3: last 10 bits of keys with prefix pre2
+  for (int b = threadIdx.x; b < 1024; b += kTopkThreads) hist[b] = 0;
+  __syncthreads();
+  for (uint32_t i = threadIdx.x; i < n_items; i += kTopkThreads) {
+    const uint32_t kk = gkey[i];
+    if ((kk >> 10) == pre2) atomicAdd(&hist[kk & 0x3FFu], 1u);
+  }
+  __syncthreads();
+  find_threshold_bin<1024>(hist, need, tmp, res);
+  const uint32_t tau = (pre2 << 10) | res[0];
+  need -= res[1];
+  const uint32_t need_eq = need;
+  // ---- ordered output: 4 consecutive items (in position order) per thread per round
+  uint32_t base_gt = 0, base_eq = 0;
+  for (uint32_t r0 = 0; r0 < n_items; r0 += 4 * kTopkThreads) {
+    const uint32_t i0 = r0 + 4 * threadIdx.x;
+    uint32_t kk[4];
+    uint32_t c_gt = 0, c_eq = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      kk[e] = (i0 + e < n_items) ? gkey[i0 + e] : 0u;
+      c_gt += (i0 + e < n_items) && (kk[e] > tau);
+      c_eq += (i0 + e < n_items) && (kk[e] == tau);
+    }
+    uint32_t total;
+    const uint32_t ex = block_excl_scan((c_gt << 16) | c_eq, tmp, &total);
+    uint32_t g = base_gt + (ex >> 16), q = base_eq + (ex & 0xFFFFu);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (i0 + e < n_items) {
+        if (kk[e] > tau) {
+          const uint32_t slot = g + min(q, need_eq);
+          if (slot < k) out[slot] = gpos[i0 + e];
+          ++g;
+        } else if (kk[e] == tau) {
+          if (q < need_eq && g + q < k) out[g + q] = gpos[i0 + e];
+          ++q;
+        }
+      }
+    }
+    base_gt += total >> 16;
+    base_eq += total & 0xFFFFu;
+  }
+}
+
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_filter_kernel(const TopkHistParams hp) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
@@ -675,66 +739,137 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_select_kernel(const Topk
     topk_query<1>(p, t, 0);
     return;
   }
-  const uint32_t n_items = n_cand;
-  uint32_t need = (uint32_t)p.k - above;
+  finish_gathered(gkey, gpos, n_cand, b1, above, (uint32_t)p.k, out, hist, tmp, res);
+  if (threadIdx.x == 0) p.count[t] = p.k;
+}
 
-  // ---- pass 2: next 11 bits of keys in bin b1
-  for (int b = threadIdx.x; b < kTopkBins; b += kTopkThreads) hist[b] = 0;
-  __syncthreads();
-  for (uint32_t i = threadIdx.x; i < n_items; i += kTopkThreads) {
-    const uint32_t kk = gkey[i];
-    if ((kk >> 21) == b1) atomicAdd(&hist[(kk >> 10) & 0x7FFu], 1u);
+// ------------------------------------------------------------------ context-parallel decode
+// Report's serving section (context-parallel decode: each rank selects among
+// its own positions, the candidates are exchanged, then merged).
+
+// A rank's selection as (score, global position) candidates: for i < count[t],
+// out_score[t, i] = scores[t, idx[t, i]] and out_pos = idx[t, i] + pos_offset;
+// -inf / -1 elsewhere (also for -1 entries).
+__global__ void __launch_bounds__(256) topk_export_kernel(const float* scores, int64_t ld, const int32_t* idx,
+                                                          const int32_t* count, int32_t T, int32_t k,
+                                                          int64_t pos_offset, float* out_score, int32_t* out_pos) {
+  griddep_wait();
+  const int t = blockIdx.x;
+  if (t >= T) return;
+  int c = count[t];
+  c = c < 0 ? 0 : (c > k ? k : c);
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    const int32_t q = (i < c) ? idx[(int64_t)t * k + i] : -1;
+    const bool ok = q >= 0 && q < ld;
+    out_score[(int64_t)t * k + i] = ok ? scores[(int64_t)t * ld + q] : -INFINITY;
+    out_pos[(int64_t)t * k + i] = ok ? (int32_t)(q + pos_offset) : -1;
   }
-  __syncthreads();
-  find_threshold_bin<kTopkBins>(hist, need, tmp, res);
-  const uint32_t pre2 = (b1 << 11) | res[0];
-  above += res[1];
-  need -= res[1];
-  // ---- pass 3: last 10 bits of keys with prefix pre2
-  for (int b = threadIdx.x; b < 1024; b += kTopkThreads) hist[b] = 0;
-  __syncthreads();
-  for (uint32_t i = threadIdx.x; i < n_items; i += kTopkThreads) {
-    const uint32_t kk = gkey[i];
-    if ((kk >> 10) == pre2) atomicAdd(&hist[kk & 0x3FFu], 1u);
-  }
-  __syncthreads();
-  find_threshold_bin<1024>(hist, need, tmp, res);
-  const uint32_t tau = (pre2 << 10) | res[0];
-  need -= res[1];
-  const uint32_t need_eq = need;
-  // ---- ordered output: 4 consecutive items (in position order) per thread per round
-  uint32_t base_gt = 0, base_eq = 0;
-  for (uint32_t r0 = 0; r0 < n_items; r0 += 4 * kTopkThreads) {
+}
+
+constexpr int kMergeCap = 16384;   // candidates per query the merge holds (in the stash region)
+
+struct MergeParams {
+  const float* cand_score;   // [R, T, kr]
+  const int32_t* cand_pos;   // [R, T, kr]: global positions, -1 = empty slot
+  int64_t shard_lo;          // this rank's positions [shard_lo, shard_hi)
+  int64_t shard_hi;
+  int32_t* idx_global;       // [T, k] or null
+  int32_t* idx_local;        // [T, k] or null: the selected positions inside the shard, as
+                             // position - shard_lo, ascending and compacted, -1 after them
+  int32_t* count_local;      // [T] (with idx_local): how many there are
+  int32_t* count;            // [T]
+  int32_t R, T, kr, k;
+};
+
+// Global top-k of one query from every rank's candidates (ranks hold disjoint
+// position ranges in rank order and list their candidates in ascending order,
+// so the concatenation is in position order).  Same rule as topk_kernel:
+// higher score first, ties to the lower position, -0 == +0, NaN as -inf.
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_merge_kernel(const MergeParams mp) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
+  uint32_t* tmp = hist + 2 * kTopkBins;
+  uint32_t* res = tmp + 40;
+  uint32_t* gkey = reinterpret_cast<uint32_t*>(smem_raw + 2 * kTopkBins * 4 + 1024);   // [kMergeCap]
+  int32_t* gpos = reinterpret_cast<int32_t*>(gkey + kMergeCap);                       // [kMergeCap]
+  int32_t* sel = gpos + kMergeCap;                                                     // [k]
+  griddep_wait();
+  const int t = blockIdx.x;
+  if (t >= mp.T) return;
+  // ordered compaction of the valid candidates: 4 consecutive slots per thread per round
+  const uint32_t n_in = (uint32_t)mp.R * (uint32_t)mp.kr;
+  uint32_t n_items = 0;
+  for (uint32_t r0 = 0; r0 < n_in; r0 += 4 * kTopkThreads) {
     const uint32_t i0 = r0 + 4 * threadIdx.x;
     uint32_t kk[4];
-    uint32_t c_gt = 0, c_eq = 0;
+    int32_t pp[4];
+    uint32_t c = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      kk[e] = (i0 + e < n_items) ? gkey[i0 + e] : 0u;
-      c_gt += (i0 + e < n_items) && (kk[e] > tau);
-      c_eq += (i0 + e < n_items) && (kk[e] == tau);
+      pp[e] = -1;
+      kk[e] = 0;
+      const uint32_t i = i0 + e;
+      if (i < n_in) {
+        const uint32_t r = i / (uint32_t)mp.kr, j = i - r * (uint32_t)mp.kr;
+        const int64_t src = ((int64_t)r * mp.T + t) * mp.kr + j;
+        pp[e] = mp.cand_pos[src];
+        if (pp[e] >= 0) kk[e] = score_key(mp.cand_score[src]);
+      }
+      c += pp[e] >= 0;
     }
     uint32_t total;
-    const uint32_t ex = block_excl_scan((c_gt << 16) | c_eq, tmp, &total);
-    uint32_t g = base_gt + (ex >> 16), q = base_eq + (ex & 0xFFFFu);
+    uint32_t at = n_items + block_excl_scan(c, tmp, &total);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (i0 + e < n_items) {
-        if (kk[e] > tau) {
-          const uint32_t slot = g + min(q, need_eq);
-          if (slot < (uint32_t)p.k) out[slot] = gpos[i0 + e];
-          ++g;
-        } else if (kk[e] == tau) {
-          if (q < need_eq && g + q < (uint32_t)p.k) out[g + q] = gpos[i0 + e];
-          ++q;
-        }
+    for (int e = 0; e < 4; ++e)
+      if (pp[e] >= 0) {
+        gkey[at] = kk[e];
+        gpos[at] = pp[e];
+        ++at;
       }
-    }
-    base_gt += total >> 16;
-    base_eq += total & 0xFFFFu;
+    n_items += total;
   }
-  if (threadIdx.x == 0) p.count[t] = p.k;
-  (void)above;
+  __syncthreads();
+  const uint32_t k = (uint32_t)mp.k;
+  const uint32_t k_eff = n_items < k ? n_items : k;
+  if (n_items <= k) {
+    for (uint32_t i = threadIdx.x; i < k; i += kTopkThreads) sel[i] = (i < n_items) ? gpos[i] : -1;
+  } else {
+    // first pass on the items, then the last two and the ordered output
+    for (int b = threadIdx.x; b < kTopkBins; b += kTopkThreads) hist[b] = 0;
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < n_items; i += kTopkThreads) atomicAdd(&hist[gkey[i] >> 21], 1u);
+    __syncthreads();
+    find_threshold_bin<kTopkBins>(hist, k, tmp, res);
+    finish_gathered(gkey, gpos, n_items, res[0], res[1], k, sel, hist, tmp, res);
+  }
+  __syncthreads();
+  if (mp.idx_global)
+    for (uint32_t i = threadIdx.x; i < k; i += kTopkThreads) mp.idx_global[(int64_t)t * k + i] = sel[i];
+  if (mp.idx_local) {
+    // this shard's positions, compacted in order (4 consecutive slots per thread per round)
+    uint32_t n_loc = 0;
+    for (uint32_t r0 = 0; r0 < k; r0 += 4 * kTopkThreads) {
+      const uint32_t i0 = r0 + 4 * threadIdx.x;
+      int32_t q[4];
+      uint32_t c = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        q[e] = (i0 + e < k) ? sel[i0 + e] : -1;
+        const bool mine = q[e] >= 0 && q[e] >= mp.shard_lo && q[e] < mp.shard_hi;
+        if (!mine) q[e] = -1;
+        c += mine;
+      }
+      uint32_t total;
+      uint32_t at = n_loc + block_excl_scan(c, tmp, &total);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (q[e] >= 0) mp.idx_local[(int64_t)t * k + at++] = (int32_t)(q[e] - mp.shard_lo);
+      n_loc += total;
+    }
+    for (uint32_t i = n_loc + threadIdx.x; i < k; i += kTopkThreads) mp.idx_local[(int64_t)t * k + i] = -1;
+    if (threadIdx.x == 0) mp.count_local[t] = (int32_t)n_loc;
+  }
+  if (threadIdx.x == 0) mp.count[t] = (int32_t)k_eff;
 }
 
 }  // namespace dsa

@@ -36,7 +36,7 @@ class LayerArgs(ctypes.Structure):
     """Mirror of ``dsa_layer_args``."""
 
     _fields_ = [("q_nope", _P), ("q_pe", _P), ("qmul", _P), ("cache", _P), ("ld_c", _I32),
-                ("d_rope", _I32), ("out", _P), ("lse", _P)]
+                ("d_rope", _I32), ("out", _P), ("lse", _P), ("out_f32", _I32), ("reserved", _I32)]
 
 
 class DeviceProps(ctypes.Structure):
@@ -77,6 +77,9 @@ SIGNATURES = {
     "dsa_forward_workspace_size": (_SZ, [_I32, _I64, _I32, _I32, _I32]),
     "dsa_sparse_mla_forward": (_I32, [_P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I64, _I32,
                                       ctypes.POINTER(LayerArgs), _F, _I32, _P, _P, _P, _SZ, _P]),
+    "dsa_topk_export": (_I32, [_P, _I64, _P, _P, _I32, _I32, _I64, _P, _P, _P]),
+    "dsa_topk_merge": (_I32, [_P, _P, _I32, _I32, _I32, _I32, _I64, _I64, _P, _P, _P, _P, _P]),
+    "dsa_lse_combine": (_I32, [_P, _P, _I32, _I32, _P, _P, _P]),
     "dsa_get_device_props": (_I32, [ctypes.POINTER(DeviceProps)]),
     "dsa_plan_attend": (_I32, [_I32, _I32, _I32, _I32, ctypes.POINTER(DeviceProps), ctypes.POINTER(AttendPlan)]),
     "dsa_plan_forward": (_I32, [_I32, _I64, _I32, _I32, _I32, _I32, _I32, _SZ, ctypes.POINTER(DeviceProps),
@@ -333,14 +336,15 @@ def _layer_array(layers, T):
             _need(L["q_pe"], torch.bfloat16, (T, 64, L["d_rope"]), f"layers[{i}].q_pe")
         _need(L["qmul"], torch.float32, (T, 64), f"layers[{i}].qmul")
         _need(L["cache"], torch.bfloat16, None, f"layers[{i}].cache")
-        _need(L["out"], torch.bfloat16, (T, 64, 512), f"layers[{i}].out")
+        f32 = L["out"].dtype == torch.float32
+        _need(L["out"], torch.float32 if f32 else torch.bfloat16, (T, 64, 512), f"layers[{i}].out")
         if L.get("lse") is not None:
             _need(L["lse"], torch.float32, (T, 64), f"layers[{i}].lse")
         arr[i] = LayerArgs(L["q_nope"].data_ptr(),
                            L["q_pe"].data_ptr() if L.get("q_pe") is not None else None,
                            L["qmul"].data_ptr(), L["cache"].data_ptr(), L["cache"].shape[1],
                            L["d_rope"], L["out"].data_ptr(),
-                           L["lse"].data_ptr() if L.get("lse") is not None else None)
+                           L["lse"].data_ptr() if L.get("lse") is not None else None, int(f32), 0)
     return arr
 
 
@@ -391,6 +395,49 @@ def sparse_mla_forward(q_idx, w, k_idx, seq_row_start, q_seq, q_pos, layers, ld,
                                       _ptr(q_pos), T, q_group, ld, len(layers), arr,
                                       float(softmax_scale), k, _ptr(idx_out), _ptr(count_out),
                                       _ptr(ws), ws.numel(), _stream(stream)))
+
+
+# ----------------------------------------------------------------- context-parallel decode steps
+
+def topk_export(scores, idx, count, pos_offset, out_score, out_pos, stream=None):
+    """A rank's selection as (score, global position) exchange candidates (see dsa_topk_export)."""
+    T, k = idx.shape
+    _need(scores, torch.float32, None, "scores")
+    _need(idx, torch.int32, (T, k), "idx")
+    _need(count, torch.int32, (T,), "count")
+    _need(out_score, torch.float32, (T, k), "out_score")
+    _need(out_pos, torch.int32, (T, k), "out_pos")
+    _check(load_library().dsa_topk_export(_ptr(scores), scores.shape[1], _ptr(idx), _ptr(count), T, k,
+                                          int(pos_offset), _ptr(out_score), _ptr(out_pos), _stream(stream)))
+
+
+def topk_merge(cand_score, cand_pos, k, count, idx_global=None, idx_local=None, count_local=None, shard=(0, 0),
+               stream=None):
+    """Global top-k from every rank's candidates [R, T, kr] (see dsa_topk_merge)."""
+    R, T, kr = cand_pos.shape
+    _need(cand_score, torch.float32, (R, T, kr), "cand_score")
+    _need(cand_pos, torch.int32, (R, T, kr), "cand_pos")
+    _need(count, torch.int32, (T,), "count")
+    if idx_global is not None:
+        _need(idx_global, torch.int32, (T, k), "idx_global")
+    if idx_local is not None:
+        _need(idx_local, torch.int32, (T, k), "idx_local")
+        _need(count_local, torch.int32, (T,), "count_local")
+    _check(load_library().dsa_topk_merge(_ptr(cand_score), _ptr(cand_pos), R, T, kr, k, int(shard[0]),
+                                         int(shard[1]), _ptr(idx_global), _ptr(idx_local), _ptr(count_local),
+                                         _ptr(count), _stream(stream)))
+
+
+def lse_combine(o_parts, lse_parts, out, lse=None, stream=None):
+    """Merge R partial attentions over disjoint parts of a selection (see dsa_lse_combine)."""
+    R, T = lse_parts.shape[:2]
+    _need(o_parts, torch.float32, (R, T, 64, 512), "o_parts")
+    _need(lse_parts, torch.float32, (R, T, 64), "lse_parts")
+    _need(out, torch.bfloat16, (T, 64, 512), "out")
+    if lse is not None:
+        _need(lse, torch.float32, (T, 64), "lse")
+    _check(load_library().dsa_lse_combine(_ptr(o_parts), _ptr(lse_parts), R, T, _ptr(out), _ptr(lse),
+                                          _stream(stream)))
 
 
 def launch_count():

@@ -46,6 +46,7 @@ class Case:
     kind: str
     seed: int
     lengths: tuple = ()           # decode: context length per sequence
+    per_seq: int = 1              # decode: queries per sequence, at its last per_seq positions
     cached: int = 0               # prefill
     new: int = 0                  # prefill
     layers: tuple = (64,)         # d_rope per layer (64 = RoPE, 0 = NoPE)
@@ -56,7 +57,7 @@ class Case:
 
     @property
     def n_queries(self) -> int:
-        return len(self.lengths) if self.kind == "decode" else self.new
+        return len(self.lengths) * self.per_seq if self.kind == "decode" else self.new
 
     @property
     def seq_lengths(self) -> tuple:
@@ -88,6 +89,11 @@ CONFIGS = {
     "decode_b4_1m_4layers": Case(
         name="decode_b4_1m_4layers", kind="decode", seed=4,
         lengths=(1 << 20,) * 4, layers=(64, 64, 64, 0), qmul="uniform"),
+    # several queries per sequence decoded together (the last 4 positions of each
+    # sequence: one token plus 3 drafted ones being verified)
+    "decode_b16_32k_4queries": Case(
+        name="decode_b16_32k_4queries", kind="decode", seed=5,
+        lengths=(32768,) * 16, per_seq=4, layers=(64,), qmul="uniform"),
 }
 
 
@@ -147,9 +153,10 @@ def make_workload(case: Case, device="cpu") -> Workload:
     seq_row_start = torch.tensor(starts, dtype=torch.int64, device=device)
     rows = case.total_rows
     if case.kind == "decode":
-        T = len(lens)
-        q_seq = torch.arange(T, dtype=torch.int32, device=device)
-        q_pos = torch.tensor([L - 1 for L in lens], dtype=torch.int32, device=device)
+        m = case.per_seq
+        T = len(lens) * m
+        q_seq = torch.arange(len(lens), dtype=torch.int32, device=device).repeat_interleave(m)
+        q_pos = torch.tensor([L - m + i for L in lens for i in range(m)], dtype=torch.int32, device=device)
     elif case.kind == "prefill":
         T = case.new
         q_seq = torch.zeros(T, dtype=torch.int32, device=device)
@@ -167,7 +174,7 @@ def make_workload(case: Case, device="cpu") -> Workload:
     if case.planted:
         # Push ``planted`` random positions of each sequence along the direction
         # d = sum_j w_j q_j of that sequence's query by 3 standard deviations.
-        assert case.kind == "decode"
+        assert case.kind == "decode" and case.per_seq == 1
         planted = torch.empty((len(lens), case.planted), dtype=torch.int64, device=device)
         for b, L in enumerate(lens):
             pos = torch.randperm(L, generator=gen, device=device)[:case.planted]
@@ -209,11 +216,11 @@ def quantize_e4m3_rows(x: torch.Tensor):
 
 def small_case(name, lengths=None, *, kind="decode", cached=0, new=0, layers=(64,),
                qmul="uniform", mla_q_std=1.0 / math.sqrt(192.0), seed=7, topk=2048,
-               planted=0) -> Case:
+               planted=0, per_seq=1) -> Case:
     """A parity-test recipe with custom sizes (same distributions as above)."""
     return Case(name=name, kind=kind, seed=seed, lengths=tuple(lengths or ()),
                 cached=cached, new=new, layers=tuple(layers), qmul=qmul,
-                mla_q_std=mla_q_std, planted=planted, topk=topk)
+                mla_q_std=mla_q_std, planted=planted, topk=topk, per_seq=per_seq)
 
 
 def to_numpy(x: torch.Tensor):

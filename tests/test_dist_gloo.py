@@ -89,35 +89,36 @@ def _cp_worker(rank, world, port, out):
         import oracle
         from sparse_attention_16_b200.workloads import SOFTMAX_SCALE, make_workload, small_case, to_numpy
 
+        from sparse_attention_16_b200 import context_parallel as cp
+
         k = 256
         wl = make_workload(small_case("cp", (5000,), layers=(64,), seed=4), "cpu")
         lay = wl.layers[0]
-        L = 5000
-        lo, hi = rank * L // world, (rank + 1) * L // world
+        lo, hi = cp.shard_range(5000, rank, world)
+        qp = int(cp.local_q_pos(wl.q_pos, lo, hi)[0])      # the query sits at 4999: the shard's last position
+        assert qp == hi - lo - 1
+        exchange = cp.dist_exchange()
         keys = to_numpy(wl.k_idx[lo:hi])
         s = oracle.index_scores(to_numpy(wl.q_idx), to_numpy(wl.w), keys, np.array([0]), np.array([0]),
-                                np.array([hi - lo - 1]), hi - lo)
-        sel, cnt = oracle.topk_select(s, np.array([hi - lo - 1]), k)
+                                np.array([qp]), hi - lo)
+        sel, cnt = oracle.topk_select(s, np.array([qp]), k)
         pos = np.full(k, -1, np.int64)
         sc = np.full(k, -np.inf)
         pos[:cnt[0]] = sel[0, :cnt[0]] + lo
         sc[:cnt[0]] = s[0, sel[0, :cnt[0]]]
-        all_pos = [torch.empty(k, dtype=torch.int64) for _ in range(world)]
-        all_sc = [torch.empty(k, dtype=torch.float64) for _ in range(world)]
-        dist.all_gather(all_pos, torch.from_numpy(pos))
-        dist.all_gather(all_sc, torch.from_numpy(sc))
-        chosen = oracle.topk_merge(torch.cat(all_sc).numpy(), torch.cat(all_pos).numpy(), k)
+        all_pos = exchange(torch.from_numpy(pos))
+        all_sc = exchange(torch.from_numpy(sc))
+        assert tuple(all_pos.shape) == (world, k)
+        chosen = oracle.topk_merge(all_sc.reshape(-1).numpy(), all_pos.reshape(-1).numpy(), k)
         mine = chosen[(chosen >= lo) & (chosen < hi)] - lo
         idx = np.full((1, 2048), -1, np.int32)
         idx[0, :mine.size] = mine
         o, lse = oracle.sparse_mla(to_numpy(lay.q_nope), to_numpy(lay.q_pe), to_numpy(lay.qmul), SOFTMAX_SCALE,
                                    to_numpy(lay.cache[lo:hi]), 64, np.array([0]), np.array([0]), idx,
                                    np.array([mine.size]))
-        all_o = [torch.empty(o[0].shape, dtype=torch.float64) for _ in range(world)]
-        all_l = [torch.empty(lse[0].shape, dtype=torch.float64) for _ in range(world)]
-        dist.all_gather(all_o, torch.from_numpy(o[0]))
-        dist.all_gather(all_l, torch.from_numpy(lse[0]))
-        oc, lc = oracle.lse_combine(torch.stack(all_o).numpy(), torch.stack(all_l).numpy())
+        all_o = exchange(torch.from_numpy(o[0]))
+        all_l = exchange(torch.from_numpy(lse[0]))
+        oc, lc = oracle.lse_combine(all_o.numpy(), all_l.numpy())
         out[rank] = {"chosen": chosen.tolist(), "o": oc, "lse": lc}
     finally:
         dist.destroy_process_group()
@@ -142,6 +143,20 @@ def test_context_parallel_exchange_world_size_2():
         assert out[r]["chosen"] == idx[0, :cnt[0]].tolist()
         np.testing.assert_allclose(out[r]["o"], o[0], rtol=1e-12, atol=1e-14)
         np.testing.assert_allclose(out[r]["lse"], lse[0], rtol=1e-12)
+
+
+def test_context_parallel_shards_cover_the_sequence_in_order():
+    from sparse_attention_16_b200 import context_parallel as cp
+
+    for length in (1, 127, 128, 5000, 1 << 20):
+        for world in (1, 2, 3, 8):
+            parts = [cp.shard_range(length, r, world) for r in range(world)]
+            assert parts[0][0] == 0 and parts[-1][1] == length
+            for (a, b), (c, d) in zip(parts, parts[1:]):
+                assert b == c and a <= b
+            assert all(lo % 128 == 0 for lo, _ in parts)
+    q_pos = torch.tensor([0, 99, 100, 250, 5000], dtype=torch.int32)
+    assert cp.local_q_pos(q_pos, 100, 200).tolist() == [-1, -1, 0, 99, 99]
 
 
 def test_shards_cover_and_balance():

@@ -60,6 +60,28 @@ def test_indexer_matches_oracle_prefill_groups(new):
         pu.assert_scores_close(to_numpy(s), ref, to_numpy(wl.q_pos))
 
 
+def test_indexer_groups_of_four_queries_of_one_sequence():
+    # Several queries of a sequence decoded together (its last 4 positions):
+    # scored in groups of 4 per key tile, against the oracle; and the same
+    # queries scored one by one.
+    case = small_case("mq4", (5000, 3000, 2100, 700, 131), per_seq=4, seed=28)
+    wl = make_workload(case, DEV)
+    ref = pu.oracle_scores(wl, list(range(wl.T)), case.ld)
+    for qg in (4, 1):
+        s = pu.gpu_scores(wl, q_group=qg)
+        pu.assert_scores_close(to_numpy(s), ref, to_numpy(wl.q_pos))
+
+
+def test_query_group_mixing_sequences_is_flagged():
+    case = small_case("mq_bad", (3000, 3000), per_seq=2, seed=29)   # groups of 4 would span two sequences
+    wl = make_workload(case, DEV)
+    s = torch.empty((wl.T, case.ld), dtype=torch.float32, device=DEV)
+    ops.index_scores(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, s, q_group=4)
+    with pytest.raises(ops.DSAError) as e:
+        ops.check_errors()
+    assert "0x4" in str(e.value)
+
+
 def test_indexer_integer_inputs_are_bit_exact():
     # Small-integer q, k and dyadic w make every product and partial sum exact in fp32.
     case = small_case("int_exact", (3000, 700, 130), seed=15)
@@ -477,6 +499,31 @@ def test_forward_four_layers_small_decode():
     for L, o, l in zip(wl.layers, outs, lses):
         ref_o, ref_l = pu.oracle_attend(wl, L, list(range(T)), idx_h, cnt_h)
         pu.assert_attention_close(to_numpy(o), to_numpy(l), ref_o, ref_l)
+
+
+def test_forward_four_queries_per_sequence():
+    # One token plus three drafted tokens per sequence verified in one pass:
+    # the fused call with q_group 4, against the oracle.
+    case = small_case("fwd_mq", (6000, 2500, 2051), per_seq=4, layers=(64,), seed=30)
+    wl = make_workload(case, DEV)
+    T, ld = wl.T, case.ld
+    lay = wl.layers[0]
+    out = torch.empty((T, 64, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((T, 64), dtype=torch.float32, device=DEV)
+    idx = torch.empty((T, 2048), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((T,), dtype=torch.int32, device=DEV)
+    ops.sparse_mla_forward(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos,
+                           [dict(q_nope=lay.q_nope, q_pe=lay.q_pe, qmul=lay.qmul, cache=lay.cache, d_rope=64,
+                                 out=out, lse=lse)], ld, q_group=4, idx_out=idx, count_out=cnt)
+    assert ops.check_errors() == 0
+    idx_h, cnt_h = to_numpy(idx), to_numpy(cnt)
+    q_pos = to_numpy(wl.q_pos)
+    assert cnt_h.tolist() == [min(2048, int(p) + 1) for p in q_pos]
+    s_ref = pu.oracle_scores(wl, list(range(T)), ld)
+    for t in range(T):
+        pu.assert_selection_overlap(idx_h[t, :cnt_h[t]], s_ref[t, :int(q_pos[t]) + 1], 2048)
+    ref_o, ref_l = pu.oracle_attend(wl, lay, list(range(T)), idx_h, cnt_h)
+    pu.assert_attention_close(to_numpy(out), to_numpy(lse), ref_o, ref_l)
 
 
 # ------------------------------------------------------------------ device-side checks
