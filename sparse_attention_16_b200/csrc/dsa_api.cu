@@ -253,8 +253,8 @@ bool pdl_enabled() {
 }
 
 template <typename... KArgs, typename... Args>
-dsa_status_t launch(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
-                    unsigned cl, Args&&... args) {
+dsa_status_t launch_ex(bool pdl, void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t stream, unsigned cl, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(block);
@@ -262,7 +262,7 @@ dsa_status_t launch(void (*kernel)(KArgs...), unsigned grid, unsigned block, siz
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   unsigned n = 0;
-  if (pdl_enabled()) {
+  if (pdl) {
     attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[n].val.programmaticStreamSerializationAllowed = 1;
     ++n;
@@ -279,6 +279,12 @@ dsa_status_t launch(void (*kernel)(KArgs...), unsigned grid, unsigned block, siz
   DSA_CUDA(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return DSA_OK;
+}
+
+template <typename... KArgs, typename... Args>
+dsa_status_t launch(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                    unsigned cl, Args&&... args) {
+  return launch_ex(pdl_enabled(), kernel, grid, block, smem, stream, cl, std::forward<Args>(args)...);
 }
 
 // ----------------------------------------------------------------- indexer
@@ -387,12 +393,16 @@ dsa_status_t topk_impl(DevLock& L, const float* scores, int64_t ld, const int32_
     hp.cand_key = static_cast<uint32_t*>(ws);
     hp.cand_pos = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + lists);
     hp.cand_cnt = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + 2 * lists);
+    hp.bin_info = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + 2 * lists + dsa::plan_round_up(ts * 4, 256));
     hp.S = S;
     DSA_TRY(set_smem(*L.s, kKTopkFilter, dsa::topk_filter_kernel, dsa::kTopkSmemBytes));
     DSA_TRY(set_smem(*L.s, kKTopkSelect, dsa::topk_select_kernel, dsa::kTopkSmemBytes));
     DSA_TRY(launch(dsa::topk_filter_kernel, (unsigned)(T * S), dsa::kTopkThreads, dsa::kTopkSmemBytes, stream, 1,
                    hp));
-    return launch(dsa::topk_select_kernel, (unsigned)T, dsa::kTopkThreads, dsa::kTopkSmemBytes, stream, 1, hp);
+    // programmatic dependent launch: the select CTAs are scheduled as the filter's
+    // blocks retire and wait (griddepcontrol.wait) for all of its writes
+    return launch_ex(true, dsa::topk_select_kernel, (unsigned)T, dsa::kTopkThreads, dsa::kTopkSmemBytes, stream, 1,
+                     hp);
   }
   switch (topk_cluster_size(*L.s, props.sms, T, ld)) {
     case 1: return launch_topk_cl<1>(L, kKTopk1, p, stream);

@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
     // ------------------------------------------------------------- producer
     if (lane == 0) {
       prefetch_tmap(&kmap);
+      const uint64_t key_policy = make_policy_evict_first();
       prefetch_tmap(&qmap);
       Ring ks{0, 0}, qs{C::QBUFS - 1, 1u};
       int cur_g = -1;
@@ -242,8 +243,13 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
         mbar_arrive_expect_tx(&k_full[ks.idx], C::KT_BYTES);
         uint8_t* kb = ktiles + ks.idx * C::KT_BYTES;
         const int32_t row0 = (int32_t)(gi.row_base + (int64_t)kt * kKeyTile);
-        for (int blk = 0; blk < C::KBLK; ++blk)
-          tma_load_2d(kb + blk * C::KHALF, &kmap, blk * 64, row0, &k_full[ks.idx]);
+        for (int blk = 0; blk < C::KBLK; ++blk) {
+          // decode streams each key once: evict it first, so that the scores this
+          // kernel writes stay in L2 for the top-k that reads them next (prefill
+          // groups re-read the keys, which then keep the normal policy)
+          if constexpr (QG == 1) tma_load_2d_hint(kb + blk * C::KHALF, &kmap, blk * 64, row0, &k_full[ks.idx], key_policy);
+          else tma_load_2d(kb + blk * C::KHALF, &kmap, blk * 64, row0, &k_full[ks.idx]);
+        }
         kused[ks.idx] = true;
         klast[ks.idx] = ks.phase;
         ks.next(C::STAGES);

@@ -128,10 +128,12 @@ inline int topk_slices(int sms, int32_t T, int64_t ld) {
   const int64_t by_len = std::max<int64_t>(1, (ld + 8191) / 8192);
   return (int)std::min<int64_t>(64, std::min(by_sms, by_len));
 }
-// Workspace of that path: per (query, slice) kPlanTopkCap keys and positions, then the counts.
+// Workspace of that path: per (query, slice) kPlanTopkCap keys and positions,
+// then the slices' counts, then per query the k-th bin as the filter read it.
 inline size_t topk_hist_ws_bytes(int sms, int32_t T, int64_t ld) {
   const size_t ts = (size_t)T * topk_slices(sms, T, ld);
-  return 2 * plan_round_up(ts * kPlanTopkCap * 4, 256) + plan_round_up(ts * 4, 256);
+  return 2 * plan_round_up(ts * kPlanTopkCap * 4, 256) + plan_round_up(ts * 4, 256) +
+         plan_round_up((size_t)T * 16, 256);
 }
 inline size_t hist_bytes(int32_t T) { return plan_round_up((size_t)T * kPlanTopkBins * 4, 256); }
 

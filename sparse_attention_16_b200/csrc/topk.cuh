@@ -468,6 +468,7 @@ struct TopkHistParams {
   uint32_t* cand_key;     // [T, S, kTopkCandCap] candidates of each slice, in position order
   int32_t* cand_pos;      // [T, S, kTopkCandCap]
   uint32_t* cand_cnt;     // [T, S]: candidates of the slice (kTopkNoList: none written)
+  uint32_t* bin_info;     // [T, 4]: (b1, keys above bin b1, keys in bin b1) as the filter read them
   int32_t S;              // slices per query
 };
 constexpr uint32_t kTopkNoList = 0xFFFFFFFFu;
@@ -561,89 +562,121 @@ __device__ __forceinline__ void finish_gathered(const uint32_t* gkey, const int3
   }
 }
 
+// Keys of one slice with their top 11 bits >= b1, in position order, into
+// warp-private lists.  The slice streams into shared memory by bulk copies of
+// up to kTopkStashCap scores (issued before the k-th bin is read from the
+// histogram, so the copy overlaps it); the last < 4 scores come by plain loads.
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_filter_kernel(const TopkHistParams hp) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem_raw);
   uint32_t* tmp = hist + 2 * kTopkBins;
   uint32_t* res = tmp + 40;
-  uint32_t* wkey = reinterpret_cast<uint32_t*>(smem_raw + 2 * kTopkBins * 4 + 1024);   // warp lists
+  uint64_t* bar = reinterpret_cast<uint64_t*>(res + 8);
+  float* chunk = reinterpret_cast<float*>(smem_raw + 2 * kTopkBins * 4 + 1024);     // [kTopkStashCap]
+  uint32_t* wkey = reinterpret_cast<uint32_t*>(chunk + kTopkStashCap);                  // warp lists
   int32_t* wposs = reinterpret_cast<int32_t*>(wkey + kTopkCandCap);
-  griddep_wait();
   const TopkParams& p = hp.base;
   const int t = blockIdx.x / hp.S;
   const int s = blockIdx.x - t * hp.S;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();
   uint32_t* cnt_out = hp.cand_cnt + (int64_t)t * hp.S + s;
   const int64_t n = topk_row_len(p, t, false);
   if (n <= p.k) {
     if (threadIdx.x == 0) *cnt_out = kTopkNoList;
     return;
   }
-  topk_bin_from_hist(hp.hist + (int64_t)t * kTopkBins, hist, (uint32_t)p.k, tmp, res);
-  const uint32_t b1 = res[0];
-  if (b1 == kTopkNoList || (uint64_t)res[1] + res[2] > (uint64_t)kTopkCandCap) {
-    if (threadIdx.x == 0) *cnt_out = kTopkNoList;   // the select kernel runs the whole row
-    return;
-  }
-  // This slice of the row; warp w owns a contiguous segment of it (multiple of 128).
+  // this slice of the row
   const float* row = p.scores + (int64_t)t * p.ld;
   const int64_t lo = ((int64_t)s * n / hp.S) & ~int64_t(3);
   const int64_t hi = (s == hp.S - 1) ? n : (((int64_t)(s + 1) * n / hp.S) & ~int64_t(3));
   const int64_t len = hi - lo;
+  const int64_t len4 = len & ~int64_t(3);                // the part the bulk copies take
+  auto issue = [&](int64_t c0) {
+    const int64_t c = min((int64_t)kTopkStashCap, len4 - c0);
+    if (threadIdx.x == 0 && c > 0) {
+      mbar_arrive_expect_tx(bar, (uint32_t)(c * 4));
+      bulk_load_g2s(chunk, row + lo + c0, (uint32_t)(c * 4), bar);
+    }
+  };
+  issue(0);
+  topk_bin_from_hist(hp.hist + (int64_t)t * kTopkBins, hist, (uint32_t)p.k, tmp, res);
+  const uint32_t b1 = res[0];
+  const bool give_up = b1 == kTopkNoList || (uint64_t)res[1] + res[2] > (uint64_t)kTopkCandCap;
+  if (s == 0 && threadIdx.x < 3) hp.bin_info[(int64_t)t * 4 + threadIdx.x] = res[threadIdx.x];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kWarps = kTopkThreads / 32;
   constexpr uint32_t WCAP = kTopkCandCap / kWarps;
-  const int64_t seg = ((len + kWarps - 1) / kWarps + 127) & ~int64_t(127);
-  const int64_t s_lo = (warp * seg < len) ? warp * seg : len;
-  const int64_t s_hi = (s_lo + seg < len) ? s_lo + seg : len;
   const uint32_t lanes_below = (1u << lane) - 1u;
   uint32_t* wk = wkey + warp * WCAP;
   int32_t* wp = wposs + warp * WCAP;
   uint32_t wcount = 0;
-  // four float4 loads in flight per lane
-  for (int64_t i0 = s_lo; i0 < s_hi; i0 += 512) {
-    uint32_t kk[4][4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t e0 = i0 + 128 * u + 4 * lane;
-      if (e0 + 3 < s_hi) {
-        const float4 f = *reinterpret_cast<const float4*>(row + lo + e0);
-        kk[u][0] = score_key(f.x);
-        kk[u][1] = score_key(f.y);
-        kk[u][2] = score_key(f.z);
-        kk[u][3] = score_key(f.w);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) kk[u][e] = (e0 + e < s_hi) ? score_key(row[lo + e0 + e]) : 0u;
-      }
+  bool ok = true;
+  uint32_t phase = 0;
+  for (int64_t c0 = 0; c0 < len; c0 += kTopkStashCap) {
+    const int64_t c_len = min((int64_t)kTopkStashCap, len - c0);     // scores of this chunk
+    const int64_t c_bulk = max((int64_t)0, min(c_len, len4 - c0));   // of which came by bulk copy
+    if (c_bulk > 0) {
+      const bool got = ok && mbar_wait(bar, phase, nullptr);   // every thread waits (bounded)
+      ok = __syncthreads_and(got) != 0;                         // the same verdict in every thread
+      phase ^= 1u;
     }
+    // Warp w owns a contiguous segment of the chunk (a multiple of 128 scores).
+    const int64_t seg = ((c_len + kWarps - 1) / kWarps + 127) & ~int64_t(127);
+    const int64_t s_lo = min((int64_t)warp * seg, c_len);
+    const int64_t s_hi = min(s_lo + seg, c_len);
+    if (!give_up && ok) {
+      for (int64_t e0 = s_lo + 4 * lane; e0 - 4 * lane < s_hi; e0 += 128) {
+        uint32_t kk[4];
+        if (e0 + 3 < c_bulk) {
+          const float4 f = *reinterpret_cast<const float4*>(chunk + e0);
+          kk[0] = score_key(f.x);
+          kk[1] = score_key(f.y);
+          kk[2] = score_key(f.z);
+          kk[3] = score_key(f.w);
+        } else {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t e0 = i0 + 128 * u + 4 * lane;
-      uint32_t flags = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) flags |= ((e0 + e < s_hi) && (kk[u][e] >> 21) >= b1) ? (1u << e) : 0u;
-      if (__any_sync(0xffffffffu, flags != 0)) {
-        uint32_t before = 0, total = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t bal = __ballot_sync(0xffffffffu, (flags >> e) & 1u);
-          before += __popc(bal & lanes_below);
-          total += __popc(bal);
-        }
-        uint32_t at = wcount + before;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (flags & (1u << e)) {
-            if (at < WCAP) {
-              wk[at] = kk[u][e];
-              wp[at] = (int32_t)(lo + e0 + e);
-            }
-            ++at;
+          for (int e = 0; e < 4; ++e) {
+            const int64_t i = e0 + e;
+            kk[e] = (i < s_hi) ? score_key(i < c_bulk ? chunk[i] : row[lo + c0 + i]) : 0u;
           }
         }
-        wcount += total;
+        uint32_t flags = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) flags |= ((e0 + e < s_hi) && (kk[e] >> 21) >= b1) ? (1u << e) : 0u;
+        if (__any_sync(0xffffffffu, flags != 0)) {
+          uint32_t before = 0, total = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t bal = __ballot_sync(0xffffffffu, (flags >> e) & 1u);
+            before += __popc(bal & lanes_below);
+            total += __popc(bal);
+          }
+          uint32_t at = wcount + before;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (flags & (1u << e)) {
+              if (at < WCAP) {
+                wk[at] = kk[e];
+                wp[at] = (int32_t)(lo + c0 + e0 + e);
+              }
+              ++at;
+            }
+          }
+          wcount += total;
+        }
       }
     }
+    __syncthreads();                     // the chunk is no longer read
+    if (ok) issue(c0 + kTopkStashCap);   // the next one (none past the bulk part, none after a failed wait)
+  }
+  if (give_up || !ok) {
+    if (threadIdx.x == 0) *cnt_out = kTopkNoList;   // the select kernel runs the whole row
+    return;
   }
   // warp offsets, the slice's count, overflow
   if (lane == 0) tmp[warp] = wcount;
@@ -690,49 +723,67 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_select_kernel(const Topk
     if (threadIdx.x == 0) p.count[t] = (int32_t)n;
     return;
   }
-  topk_bin_from_hist(hp.hist + (int64_t)t * kTopkBins, hist, (uint32_t)p.k, tmp, res);
-  const uint32_t b1 = res[0];
-  uint32_t above = res[1];
-  const uint32_t n_cand = res[1] + res[2];
-  // Every slice's list must be there and add up to the histogram's count.
-  if (threadIdx.x == 0) {
-    bool ok = b1 != kTopkNoList && n_cand <= (uint32_t)kTopkCandCap;
-    uint32_t sum = 0;
-    for (int s = 0; ok && s < hp.S; ++s) {
-      const uint32_t c = hp.cand_cnt[(int64_t)t * hp.S + s];
-      if (c == kTopkNoList) ok = false;
-      else sum += c;
+  // the k-th bin as the filter read it from the histogram
+  const uint32_t b1 = hp.bin_info[(int64_t)t * 4];
+  uint32_t above = hp.bin_info[(int64_t)t * 4 + 1];
+  const uint32_t n_cand = above + hp.bin_info[(int64_t)t * 4 + 2];
+  // Every slice's list must be there and add up to the histogram's count
+  // (warp 0: counts, their prefix in `offs`, the verdict in res[4]).
+  uint32_t* offs = hist + kTopkBins;   // [S + 1]
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    bool bad = b1 == kTopkNoList || n_cand > (uint32_t)kTopkCandCap;
+    uint32_t run = 0;
+    for (int s0 = 0; s0 < hp.S; s0 += 32) {
+      const int s = s0 + lane;
+      const uint32_t c = (s < hp.S) ? hp.cand_cnt[(int64_t)t * hp.S + s] : 0u;
+      bad |= __any_sync(0xffffffffu, c == kTopkNoList);
+      const uint32_t cc = (c == kTopkNoList) ? 0u : c;
+      uint32_t x = cc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (s < hp.S) offs[s] = run + x - cc;
+      run += __shfl_sync(0xffffffffu, x, 31);
     }
-    res[4] = (ok && sum == n_cand) ? 1u : 0u;
+    if (lane == 0) {
+      offs[hp.S] = run;
+      res[4] = (!bad && run == n_cand) ? 1u : 0u;
+      res[5] = 0;
+      res[6] = 0;
+    }
   }
   __syncthreads();
   if (res[4] == 0u) {
     topk_query<1>(p, t, 0);   // the single-CTA algorithm on the whole row
     return;
   }
-  // gather the slices' lists in slice (= position) order, recounting the keys
-  // above and in bin b1: they must be the histogram's counts, or b1 is not the
-  // row's k-th bin (a histogram that does not belong to these scores)
-  if (threadIdx.x == 0) {
-    res[5] = 0;
-    res[6] = 0;
-  }
-  __syncthreads();
-  uint32_t off = 0, my_gt = 0, my_eq = 0;
-  for (int s = 0; s < hp.S; ++s) {
-    const int64_t src = ((int64_t)t * hp.S + s) * kTopkCandCap;
-    const uint32_t c = hp.cand_cnt[(int64_t)t * hp.S + s];
-    for (uint32_t i = threadIdx.x; i < c; i += kTopkThreads) {
-      const uint32_t kk = hp.cand_key[src + i];
-      gkey[off + i] = kk;
-      gpos[off + i] = hp.cand_pos[src + i];
+  // gather the slices' lists in slice (= position) order: item i of the query
+  // lies in the slice s with offs[s] <= i < offs[s + 1] (binary search); the
+  // keys above and in bin b1 are recounted: they must be the histogram's
+  // counts, or b1 is not the row's k-th bin (a histogram that does not belong
+  // to these scores)
+  {
+    uint32_t my_gt = 0, my_eq = 0;
+    for (uint32_t i = threadIdx.x; i < n_cand; i += kTopkThreads) {
+      int s_lo = 0, s_hi = hp.S;   // offs[s_lo] <= i < offs[s_hi]
+      while (s_hi - s_lo > 1) {
+        const int mid = (s_lo + s_hi) >> 1;
+        if (offs[mid] <= i) s_lo = mid;
+        else s_hi = mid;
+      }
+      const int64_t src = ((int64_t)t * hp.S + s_lo) * kTopkCandCap + (i - offs[s_lo]);
+      const uint32_t kk = hp.cand_key[src];
+      gkey[i] = kk;
+      gpos[i] = hp.cand_pos[src];
       my_gt += (kk >> 21) > b1;
       my_eq += (kk >> 21) == b1;
     }
-    off += c;
+    if (my_gt) atomicAdd(&res[5], my_gt);
+    if (my_eq) atomicAdd(&res[6], my_eq);
   }
-  if (my_gt) atomicAdd(&res[5], my_gt);
-  if (my_eq) atomicAdd(&res[6], my_eq);
   __syncthreads();
   if (res[5] != above || res[6] != n_cand - above || above >= (uint32_t)p.k) {
     __syncthreads();
