@@ -343,20 +343,25 @@ def measure(name, dev, steps, warmup, rank, world, local, min_seconds=0.0, sampl
     plan = ops.plan_attend(T, min(n_layers, 8), k)
     res["attend_plan"] = {"n_split": plan.n_split, "rows_per_split": plan.rows_per_split, "merge": bool(plan.merge),
                           "workspace_bytes": int(plan.workspace_bytes)}
-    if e2e and not fp8:
-        res["e2e"] = run_e2e(wl, ld, k, q_group, dev, e2e_steps)
+    if e2e:
+        res["e2e"] = run_e2e(wl, ld, k, q_group, dev, e2e_steps,
+                             fp8=(q8, q8_scale, k8, k8_scale) if fp8 else None)
     del graph, graph_ev
     return res
 
 
-def run_e2e(wl, ld, k, q_group, dev, steps):
-    """Same metric through dsa_sparse_mla_forward with pinned host inputs/outputs:
-    each step copies the step's queries host->device and the outputs back."""
+def run_e2e(wl, ld, k, q_group, dev, steps, fp8=None):
+    """Same metric through dsa_sparse_mla_forward (dsa_sparse_mla_forward_fp8 with
+    `fp8` = (q8, q_scale, k8, k_scale)) with pinned host inputs/outputs: each step
+    copies the step's queries host->device and the outputs back."""
     from sparse_attention_16_b200 import ops
 
     T = wl.T
     n_layers = len(wl.layers)
-    host_in = {"q_idx": wl.q_idx, "w": wl.w, "q_seq": wl.q_seq, "q_pos": wl.q_pos}
+    if fp8 is None:
+        host_in = {"q_idx": wl.q_idx, "w": wl.w, "q_seq": wl.q_seq, "q_pos": wl.q_pos}
+    else:
+        host_in = {"q8": fp8[0], "q_scale": fp8[1], "w": wl.w, "q_seq": wl.q_seq, "q_pos": wl.q_pos}
     for i, L in enumerate(wl.layers):
         host_in[f"q_nope{i}"] = L.q_nope
         if L.q_pe is not None:
@@ -375,8 +380,12 @@ def run_e2e(wl, ld, k, q_group, dev, steps):
             dev_in[n].copy_(pinned[n], non_blocking=True)
         layers = [dict(q_nope=dev_in[f"q_nope{i}"], q_pe=dev_in.get(f"q_pe{i}"), qmul=dev_in[f"qmul{i}"],
                        cache=L.cache, d_rope=L.d_rope, out=outs[i], lse=None) for i, L in enumerate(wl.layers)]
-        ops.sparse_mla_forward(dev_in["q_idx"], dev_in["w"], wl.k_idx, wl.seq_row_start, dev_in["q_seq"],
-                               dev_in["q_pos"], layers, ld, k=k, q_group=q_group, ws=ws)
+        if fp8 is None:
+            ops.sparse_mla_forward(dev_in["q_idx"], dev_in["w"], wl.k_idx, wl.seq_row_start, dev_in["q_seq"],
+                                   dev_in["q_pos"], layers, ld, k=k, q_group=q_group, ws=ws)
+        else:
+            ops.sparse_mla_forward_fp8(dev_in["q8"], dev_in["q_scale"], dev_in["w"], fp8[2], fp8[3], wl.seq_row_start,
+                                       dev_in["q_seq"], dev_in["q_pos"], layers, ld, k=k, q_group=q_group, ws=ws)
         for o, h in zip(outs, host_out):
             h.copy_(o, non_blocking=True)
 
@@ -394,7 +403,7 @@ def run_e2e(wl, ld, k, q_group, dev, steps):
     el = t0.elapsed_time(t1) / 1e3
     return {"value": round(T * n_layers * steps / el, 1), "unit": "query-layers/s", "queries_per_s": round(T * steps / el, 1),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(el / steps * 1e3, 4),
-            "steps": steps, "api": "dsa_sparse_mla_forward"}
+            "steps": steps, "api": "dsa_sparse_mla_forward" + ("_fp8" if fp8 is not None else "")}
 
 
 def run_ours(args, rank, world, local):

@@ -293,6 +293,23 @@ dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const voi
                                     void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * dsa_sparse_mla_forward_fp8 - dsa_sparse_mla_forward with FP8 (E4M3) index keys.
+ * Concept page, 1M-token serving scenario (indexer keys kept in FP8): the
+ * indexer scores E4M3 keys and queries with per-row / per-head scales exactly
+ * as dsa_index_scores_fp8 does; the selection and every layer's attention are
+ * those of dsa_sparse_mla_forward.  q8 uint8 [T, 32, 128], q_scale f32 [T, 32],
+ * k8 uint8 [n_rows, 128], k_scale f32 [n_rows]; everything else, the workspace
+ * size included, as dsa_sparse_mla_forward.
+ */
+dsa_status_t dsa_sparse_mla_forward_fp8(const void* q8, const float* q_scale, const float* w, const void* k8,
+                                        const float* k_scale, int64_t n_rows, const int64_t* seq_row_start,
+                                        int32_t B, const int32_t* q_seq, const int32_t* q_pos, int32_t T,
+                                        int32_t q_group, int64_t ld, int32_t n_layers,
+                                        const dsa_layer_args* layers, float softmax_scale, int32_t k,
+                                        int32_t* idx_out, int32_t* count_out, void* workspace, size_t ws_bytes,
+                                        void* stream);
+
+/*
  * Context-parallel decode (report's serving section, Figures 16-17: the
  * positions of a long sequence are split over ranks; each rank scores and
  * selects among its own positions, the candidates are exchanged and merged

@@ -59,9 +59,9 @@ dsa_status_t fail(dsa_status_t st, const char* fmt, ...) {
     if (e_ != cudaSuccess) return fail(DSA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
   } while (0)
 
-#define DSA_TRY(expr)                      \
+#define DSA_TRY(...)                       \
   do {                                     \
-    dsa_status_t st_ = (expr);             \
+    dsa_status_t st_ = (__VA_ARGS__);      \
     if (st_ != DSA_OK) return st_;         \
   } while (0)
 
@@ -772,15 +772,27 @@ size_t dsa_forward_workspace_size(int32_t T, int64_t ld, int32_t k, int32_t q_gr
   return dsa::forward_layout_for(d, T, ld, k, std::max(0, n_layers), true, true, T, true, q_group == 1).end;
 }
 
-dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const void* k_idx, int64_t n_rows,
-                                    const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
-                                    const int32_t* q_pos, int32_t T, int32_t q_group, int64_t ld,
-                                    int32_t n_layers, const dsa_layer_args* layers,
-                                    float softmax_scale, int32_t k, int32_t* idx_out,
-                                    int32_t* count_out, void* workspace, size_t ws_bytes,
-                                    void* stream) {
-  NvtxRange nvtx_range("dsa_sparse_mla_forward");
-  DSA_TRY(check_index_args(q_idx, w, k_idx, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, ld));
+}  // extern "C"
+
+namespace {
+
+// Index keys of the fused call: bf16 (q_idx, k_idx) or E4M3 codes with scales.
+struct IndexKeys {
+  const void* q;
+  const float* q_scale;   // FP8 only
+  const void* k;
+  const float* k_scale;   // FP8 only
+  bool fp8;
+};
+
+dsa_status_t forward_impl(const IndexKeys& ik, const float* w, int64_t n_rows, const int64_t* seq_row_start,
+                          int32_t B, const int32_t* q_seq, const int32_t* q_pos, int32_t T, int32_t q_group,
+                          int64_t ld, int32_t n_layers, const dsa_layer_args* layers, float softmax_scale, int32_t k,
+                          int32_t* idx_out, int32_t* count_out, void* workspace, size_t ws_bytes, void* stream) {
+  DSA_TRY(check_index_args(ik.q, w, ik.k, n_rows, seq_row_start, B, q_seq, q_pos, T, q_group, ld));
+  if (ik.fp8)
+    DSA_REQUIRE(ik.q_scale && ik.k_scale && aligned(ik.q_scale, 4) && aligned(ik.k_scale, 4),
+                "q_scale and k_scale must be non-null and 4-byte aligned");
   DSA_REQUIRE(k >= 1 && k <= kMaxK, "k must be in [1, %d]", kMaxK);
   DSA_REQUIRE(n_layers >= 0 && (n_layers == 0 || layers != nullptr), "bad layer list");
   DSA_REQUIRE(idx_out == nullptr || aligned(idx_out, 4), "misaligned idx_out");
@@ -809,19 +821,64 @@ dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const voi
   uint32_t* hist = (f.hist_off != SIZE_MAX) ? reinterpret_cast<uint32_t*>(ws + f.hist_off) : nullptr;
   void* topk_ws = (f.topk_off != SIZE_MAX) ? ws + f.topk_off : nullptr;
   float* scores = reinterpret_cast<float*>(ws + f.scores_off);
+  const int64_t q_row = (int64_t)dsa::kIdxHeads * dsa::kIdxDim;   // values (bytes for FP8, elements for bf16)
 
   for (int32_t t0 = 0; t0 < T; t0 += f.chunk) {
     const int32_t n = std::min(f.chunk, T - t0);
     int32_t* idx_c = own_idx ? idx_ws : idx_out + (int64_t)t0 * k;
     int32_t* cnt_c = own_count ? cnt_ws : count_out + t0;
-    DSA_TRY(indexer_impl(L, static_cast<const __nv_bfloat16*>(q_idx) + (int64_t)t0 * dsa::kIdxHeads * dsa::kIdxDim,
-                         w + (int64_t)t0 * dsa::kIdxHeads, k_idx, n_rows, seq_row_start, B, q_seq + t0,
-                         q_pos + t0, n, q_group, scores, ld, hist, s));
+    const float* w_c = w + (int64_t)t0 * dsa::kIdxHeads;
+    if (ik.fp8) {
+      const uint8_t* q8 = static_cast<const uint8_t*>(ik.q) + (int64_t)t0 * q_row;
+      const float* qs = ik.q_scale + (int64_t)t0 * dsa::kIdxHeads;
+      if (q_group == 8)
+        DSA_TRY(launch_indexer<8, true>(L, q8, qs, w_c, ik.k, ik.k_scale, n_rows, seq_row_start, B, q_seq + t0,
+                                        q_pos + t0, n, scores, ld, nullptr, s));
+      else if (q_group == 4)
+        DSA_TRY(launch_indexer<4, true>(L, q8, qs, w_c, ik.k, ik.k_scale, n_rows, seq_row_start, B, q_seq + t0,
+                                        q_pos + t0, n, scores, ld, nullptr, s));
+      else
+        DSA_TRY(launch_indexer<1, true>(L, q8, qs, w_c, ik.k, ik.k_scale, n_rows, seq_row_start, B, q_seq + t0,
+                                        q_pos + t0, n, scores, ld, hist, s));
+    } else {
+      DSA_TRY(indexer_impl(L, static_cast<const __nv_bfloat16*>(ik.q) + (int64_t)t0 * q_row, w_c, ik.k, n_rows,
+                           seq_row_start, B, q_seq + t0, q_pos + t0, n, q_group, scores, ld, hist, s));
+    }
     DSA_TRY(topk_impl(L, scores, ld, q_pos + t0, n, k, idx_c, cnt_c, hist, topk_ws, f.topk_bytes, s));
     DSA_TRY(attend_layers_impl(L, layers, n_layers, softmax_scale, n_rows, seq_row_start, B, q_seq + t0,
                                q_pos + t0, idx_c, cnt_c, n, k, t0, att_ws, f.att_bytes, s, f.partials));
   }
   return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dsa_status_t dsa_sparse_mla_forward(const void* q_idx, const float* w, const void* k_idx, int64_t n_rows,
+                                    const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
+                                    const int32_t* q_pos, int32_t T, int32_t q_group, int64_t ld,
+                                    int32_t n_layers, const dsa_layer_args* layers,
+                                    float softmax_scale, int32_t k, int32_t* idx_out,
+                                    int32_t* count_out, void* workspace, size_t ws_bytes,
+                                    void* stream) {
+  NvtxRange nvtx_range("dsa_sparse_mla_forward");
+  return forward_impl(IndexKeys{q_idx, nullptr, k_idx, nullptr, false}, w, n_rows, seq_row_start, B, q_seq, q_pos, T,
+                      q_group, ld, n_layers, layers, softmax_scale, k, idx_out, count_out, workspace, ws_bytes,
+                      stream);
+}
+
+dsa_status_t dsa_sparse_mla_forward_fp8(const void* q8, const float* q_scale, const float* w, const void* k8,
+                                        const float* k_scale, int64_t n_rows, const int64_t* seq_row_start,
+                                        int32_t B, const int32_t* q_seq, const int32_t* q_pos, int32_t T,
+                                        int32_t q_group, int64_t ld, int32_t n_layers,
+                                        const dsa_layer_args* layers, float softmax_scale, int32_t k,
+                                        int32_t* idx_out, int32_t* count_out, void* workspace, size_t ws_bytes,
+                                        void* stream) {
+  NvtxRange nvtx_range("dsa_sparse_mla_forward_fp8");
+  return forward_impl(IndexKeys{q8, q_scale, k8, k_scale, true}, w, n_rows, seq_row_start, B, q_seq, q_pos, T,
+                      q_group, ld, n_layers, layers, softmax_scale, k, idx_out, count_out, workspace, ws_bytes,
+                      stream);
 }
 
 dsa_status_t dsa_topk_export(const float* scores, int64_t ld, const int32_t* idx, const int32_t* count, int32_t T,

@@ -85,6 +85,8 @@ SIGNATURES = {
     "dsa_plan_forward": (_I32, [_I32, _I64, _I32, _I32, _I32, _I32, _I32, _SZ, ctypes.POINTER(DeviceProps),
                                 ctypes.POINTER(ForwardPlan)]),
     "dsa_set_fault_test": (_I32, [ctypes.c_uint64, _I32]),
+    "dsa_sparse_mla_forward_fp8": (_I32, [_P, _P, _P, _P, _P, _I64, _P, _I32, _P, _P, _I32, _I32, _I64, _I32,
+                                          ctypes.POINTER(LayerArgs), _F, _I32, _P, _P, _P, _SZ, _P]),
     "dsa_check_errors": (_I32, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "dsa_launch_count": (ctypes.c_uint64, []),
     "dsa_last_error": (ctypes.c_char_p, []),
@@ -395,6 +397,26 @@ def sparse_mla_forward(q_idx, w, k_idx, seq_row_start, q_seq, q_pos, layers, ld,
                                       _ptr(q_pos), T, q_group, ld, len(layers), arr,
                                       float(softmax_scale), k, _ptr(idx_out), _ptr(count_out),
                                       _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def sparse_mla_forward_fp8(q8, q_scale, w, k8, k_scale, seq_row_start, q_seq, q_pos, layers, ld, k=2048,
+                           q_group=1, idx_out=None, count_out=None, softmax_scale=SOFTMAX_SCALE, ws=None,
+                           stream=None):
+    """sparse_mla_forward with FP8 (E4M3) index keys and queries (see dsa_sparse_mla_forward_fp8)."""
+    T = q8.shape[0]
+    q8 = _codes(q8, (T, 32, 128), "q8")
+    k8 = _codes(k8, None, "k8")
+    _need(q_scale, torch.float32, (T, 32), "q_scale")
+    _need(k_scale, torch.float32, (k8.shape[0],), "k_scale")
+    _need(w, torch.float32, (T, 32), "w")
+    arr = _layer_array(layers, T)
+    lib = load_library()
+    if ws is None:
+        ws = workspace(forward_workspace_bytes(T, ld, k, q_group, len(layers)), q8.device)
+    _check(lib.dsa_sparse_mla_forward_fp8(_ptr(q8), _ptr(q_scale), _ptr(w), _ptr(k8), _ptr(k_scale), k8.shape[0],
+                                          _ptr(seq_row_start), seq_row_start.shape[0], _ptr(q_seq), _ptr(q_pos), T,
+                                          q_group, ld, len(layers), arr, float(softmax_scale), k, _ptr(idx_out),
+                                          _ptr(count_out), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 # ----------------------------------------------------------------- context-parallel decode steps

@@ -88,3 +88,35 @@ def test_fp8_selection_overlaps_bf16_selection():
     i16, _ = pu.gpu_topk(s16, wl.q_pos, 2048)
     a, b = set(to_numpy(i8)[0].tolist()), set(to_numpy(i16)[0].tolist())
     assert len(a & b) / 2048 > 0.8
+
+
+@pytest.mark.parametrize("per_seq,q_group", [(1, 1), (4, 4)])
+def test_fused_forward_with_fp8_keys(per_seq, q_group):
+    # The fused call on FP8 (E4M3) index keys: the selection is the top-k of the
+    # FP8 indexer's own scores (bit-exact against the separate calls), overlaps
+    # the oracle's fp64 FP8 ranking, and the attention matches the oracle.
+    lengths = (7000, 4096, 2500, 900) if per_seq == 1 else (6000, 3000)
+    case = small_case("fwd_fp8", lengths, layers=(64, 0), seed=36, per_seq=per_seq)
+    wl = make_workload(case, DEV)
+    T, ld = wl.T, case.ld
+    q8, qs, k8, ks = pu.fp8_inputs(wl)
+    outs = [torch.empty((T, 64, 512), dtype=torch.bfloat16, device=DEV) for _ in wl.layers]
+    lses = [torch.empty((T, 64), dtype=torch.float32, device=DEV) for _ in wl.layers]
+    layers = [dict(q_nope=L.q_nope, q_pe=L.q_pe, qmul=L.qmul, cache=L.cache, d_rope=L.d_rope, out=o, lse=l)
+              for L, o, l in zip(wl.layers, outs, lses)]
+    idx = torch.empty((T, 2048), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((T,), dtype=torch.int32, device=DEV)
+    ops.sparse_mla_forward_fp8(q8, qs, wl.w, k8, ks, wl.seq_row_start, wl.q_seq, wl.q_pos, layers, ld,
+                               q_group=q_group, idx_out=idx, count_out=cnt)
+    assert ops.check_errors() == 0
+    s = pu.gpu_scores_fp8(wl, q8, qs, k8, ks, q_group=q_group)
+    idx2, cnt2 = pu.gpu_topk(s, wl.q_pos, 2048)
+    assert torch.equal(idx, idx2) and torch.equal(cnt, cnt2)
+    idx_h, cnt_h = to_numpy(idx), to_numpy(cnt)
+    q_pos = to_numpy(wl.q_pos)
+    ref_s = pu.oracle_scores_fp8(wl, q8, qs, k8, ks, list(range(T)), ld)
+    for t in range(T):
+        pu.assert_selection_overlap(idx_h[t, :cnt_h[t]], ref_s[t, :int(q_pos[t]) + 1], 2048)
+    for L, o, l in zip(wl.layers, outs, lses):
+        ref_o, ref_l = pu.oracle_attend(wl, L, list(range(T)), idx_h, cnt_h)
+        pu.assert_attention_close(to_numpy(o), to_numpy(l), ref_o, ref_l)
