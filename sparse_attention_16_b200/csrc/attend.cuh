@@ -228,7 +228,9 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLa
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int n = p.n_split;
-  const int W = (kLatent / 4 + n - 1) / n;                                   // float4 columns per rank, at most
+  // float4 columns per rank (at most), padded to an odd stride so that the 16
+  // heads a half-warp pushes at once fall in different shared-memory banks
+  const int W = ((kLatent / 4 + n - 1) / n) | 1;
   float4* recv = reinterpret_cast<float4*>(cs);                              // [n sources][64 heads][W]
   float* stats = reinterpret_cast<float*>(cs + (size_t)n * kHeads * W * 16); // [n sources][64 heads][4]
   const int tid = threadIdx.x;

@@ -470,7 +470,8 @@ dsa_status_t launch_attend(DevLock& L, const dsa_layer_args* layers, int32_t n_l
   DSA_TRY(launch(dsa::attend_kernel, (unsigned)(units * sp.n_split), C::THREADS, C::SMEM_BYTES, stream,
                  sp.merge ? (unsigned)sp.n_split : 1u, p));
   if (!partials) return DSA_OK;
-  return launch(dsa::attend_combine_kernel, (unsigned)(units * dsa::kHeads), 128, 0, stream, 1, p);
+  // programmatic dependent launch: scheduled while the attention drains, waits for its writes
+  return launch_ex(true, dsa::attend_combine_kernel, (unsigned)(units * dsa::kHeads), 128, 0, stream, 1, p);
 }
 
 // Several layers over one selection: launches of up to kMaxAttLayers layers

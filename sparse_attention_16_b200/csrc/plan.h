@@ -54,11 +54,13 @@ inline bool merge_fits(const DevProps& d, int64_t units, int n_split) {
 // blocks run in waves; each block pays a fixed start (query gather, first-tile
 // latency) plus its tiles; splits then merge on chip (cluster) or through the
 // combine kernel (an extra launch and the partials' round trip through L2).
-// The constants are per-tile and per-launch times measured on B200 at 64 heads.
+// The constants are per-tile and per-launch times measured on B200 at 64 heads
+// (the combine path: ~5 us to write the fp32 partials, ~5-7 us for the combine
+// kernel; the on-chip merge: a few us).
 constexpr double kCostStartUs = 3.0;
 constexpr double kCostTileUs = 2.3;
-constexpr double kCostMergeUs = 1.5;
-constexpr double kCostCombineUs = 4.0;
+constexpr double kCostMergeUs = 10.0;
+constexpr double kCostCombineUs = 10.0;
 
 inline double plan_cost(const DevProps& d, int64_t units, int32_t k, const SplitPlan& sp) {
   const int max_tiles = (int)((k + kPlanTileRows - 1) / kPlanTileRows);

@@ -60,7 +60,7 @@ def test_replicas_world_size_2():
     from sparse_attention_16_b200.workloads import SOFTMAX_SCALE, make_workload, small_case, to_numpy
 
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
     r0, r1 = out[0], out[1]
@@ -129,7 +129,7 @@ def test_context_parallel_exchange_world_size_2():
     from sparse_attention_16_b200.workloads import SOFTMAX_SCALE, make_workload, small_case, to_numpy
 
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.start_processes(_cp_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
     wl = make_workload(small_case("cp", (5000,), layers=(64,), seed=4), "cpu")

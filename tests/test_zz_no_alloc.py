@@ -31,14 +31,14 @@ def _lib():
     yield
 
 
-def _selection(wl, seed):
+def _selection(wl, seed, k=2048):
     rng = np.random.default_rng(seed)
     q_pos = to_numpy(wl.q_pos)
-    idx = np.full((wl.T, 2048), -1, np.int32)
+    idx = np.full((wl.T, k), -1, np.int32)
     cnt = np.zeros(wl.T, np.int32)
     for t in range(wl.T):
         n = int(q_pos[t]) + 1
-        c = min(2048, n)
+        c = min(k, n)
         idx[t, :c] = np.sort(rng.choice(n, c, replace=False))
         cnt[t] = c
     return torch.as_tensor(idx, device=DEV), torch.as_tensor(cnt, device=DEV)
@@ -59,24 +59,26 @@ def _both(wl, lay, idx, cnt):
 
 
 def _scratch_batch():
-    """A batch size whose split partials go through the scratch on this GPU
-    (split across blocks that do not merge on chip, within the scratch limit)."""
-    for T in range(8, 0, -1):
-        p = ops.plan_attend(T, 1, 2048)
-        if p.workspace_bytes > 0 and T * p.n_split <= 128:
-            return T
+    """A batch size and selection width whose split partials go through the
+    scratch on this GPU (split across blocks that do not merge on chip, within
+    the scratch limit)."""
+    for k in (2048, 4096, 8192):
+        for T in range(8, 0, -1):
+            p = ops.plan_attend(T, 1, k)
+            if p.workspace_bytes > 0 and T * p.n_split <= 128:
+                return T, k
     pytest.fail("no batch of 1-8 queries uses the scratch on this GPU")
 
 
 @pytest.mark.parametrize("d_rope", [64, 0])
 def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(d_rope):
-    T = _scratch_batch()
-    wl1 = make_workload(small_case("na1", (4096, 3000, 2500, 600, 2049, 90, 5000, 2100)[:T], layers=(d_rope,),
+    T, k = _scratch_batch()
+    wl1 = make_workload(small_case("na1", (9000, 3000, 2500, 600, 4097, 90, 5000, 2100)[:T], layers=(d_rope,),
                                    seed=31), DEV)
-    wl2 = make_workload(small_case("na2", (5000, 2048, 100, 4000, 3333, 777, 2200, 4100)[:T], layers=(d_rope,),
+    wl2 = make_workload(small_case("na2", (5000, 2048, 100, 8000, 3333, 777, 2200, 4100)[:T], layers=(d_rope,),
                                    seed=32, mla_q_std=1.0), DEV)
     for wl, seed in ((wl1, 1), (wl2, 2)):
-        idx, cnt = _selection(wl, seed)
+        idx, cnt = _selection(wl, seed, k)
         o, l, ref_o, ref_l = _both(wl, wl.layers[0], idx, cnt)
         g, r = to_numpy(o).astype(np.float64), to_numpy(ref_o).astype(np.float64)
         assert np.abs(g - r).max() <= pu.ATTN_ATOL
