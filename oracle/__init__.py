@@ -36,6 +36,13 @@ Parity status per function (what pins it, see tests/test_oracle_pins.py):
   index_scores_fp8  pinned: hand-worked example with integer codes, positive
                     homogeneity in each key scale and in each query's scales, zero
                     scale gives zero scores, causal/offset checks.
+  latent_fp8_decode pinned: hand-worked row (landmark codes, subnormal, per-block
+                    scales, the rotary block's own scale, padding ignored).
+  sparse_mla_fp8    pinned: with unit scales it is sparse_mla on the codes' values;
+                    doubling one block's scale while halving that block of the query
+                    doubles exactly that block of the output and leaves lse alone;
+                    the rotary scale trades against q_pe; a zero rotary scale equals
+                    a zero rotary query.
 """
 
 from .dsa_oracle import (  # noqa: F401
@@ -49,4 +56,6 @@ from .dsa_oracle import (  # noqa: F401
     dense_causal_mla,
     explicit_mla,
     forward,
+    latent_fp8_decode,
+    sparse_mla_fp8,
 )

@@ -42,6 +42,8 @@ __all__ = [
     "dense_causal_mla",
     "explicit_mla",
     "forward",
+    "latent_fp8_decode",
+    "sparse_mla_fp8",
 ]
 
 
@@ -230,6 +232,58 @@ def sparse_mla(q_nope, q_pe, qmul, scale, cache, d_rope, seq_row_start, q_seq,
         sel = sel[sel >= 0]
         base = int(seq_row_start[int(q_seq[t])])
         rows = _f64(cache_np[base + sel, :d_c + int(d_rope)])
+        o[t], lse[t] = _attend_rows(qn_all[t], None if qp_all is None else qp_all[t],
+                                    mult_all[t], scale, rows, d_c)
+    return o, lse
+
+
+LATENT_BLOCK = 128   # latent values per FP8 scale (the report's blockwise scales)
+
+
+def latent_fp8_decode(rows8, d_c, d_rope):
+    """Values of latent-cache rows kept in FP8 (E4M3) with blockwise scales.
+
+    The report's serving section keeps the KV cache in FP8 natively, and its
+    training section runs FP8 with blockwise scales; neither gives a layout.
+    The reading taken, for one position (one row of bytes):
+      bytes [0, d_c + d_rope)                E4M3 codes of [c_s | kR_s]
+      bytes [d_c + d_rope, + 4 * n_blocks)   fp32 scales (little-endian): one per
+                                             128 latent values (d_c / 128 of them)
+                                             and, when d_rope > 0, one more for kR_s
+    so that column i < d_c is scale[i // 128] * e4m3(code[i]) and column d_c + j
+    is scale[d_c // 128] * e4m3(code[d_c + j]).  Bytes after the scales are
+    padding.  rows8: uint8 [n, >= d_c + d_rope + 4 * n_blocks].
+    Returns float64 [n, d_c + d_rope].
+    """
+    r = np.asarray(rows8, dtype=np.uint8)
+    n_codes = d_c + d_rope
+    n_blk = d_c // LATENT_BLOCK + (1 if d_rope > 0 else 0)
+    values = e4m3_decode(r[:, :n_codes])
+    scales = np.ascontiguousarray(r[:, n_codes:n_codes + 4 * n_blk]).view("<f4").astype(np.float64)
+    block_of_col = np.concatenate([np.arange(d_c) // LATENT_BLOCK,
+                                   np.full(d_rope, d_c // LATENT_BLOCK, dtype=np.int64)])
+    return values * scales[:, block_of_col]
+
+
+def sparse_mla_fp8(q_nope, q_pe, qmul, scale, cache8, d_rope, seq_row_start, q_seq,
+                   idx, count):
+    """sparse_mla over a latent cache kept in FP8 (rows as latent_fp8_decode
+    reads them; the report's serving section, native FP8 KV cache): the
+    attention of the decoded values, everything else as sparse_mla.
+    Returns (o float64 [T, H, d_c], lse float64 [T, H]).
+    """
+    qn_all = _f64(q_nope)
+    T, H, d_c = qn_all.shape
+    qp_all = _f64(q_pe) if (q_pe is not None and d_rope > 0) else None
+    mult_all = _f64(qmul)
+    cache_np = np.asarray(cache8, dtype=np.uint8)
+    o = np.zeros((T, H, d_c))
+    lse = np.full((T, H), -np.inf)
+    for t in range(T):
+        sel = np.asarray(idx[t, :int(count[t])], dtype=np.int64)
+        sel = sel[sel >= 0]
+        base = int(seq_row_start[int(q_seq[t])])
+        rows = latent_fp8_decode(cache_np[base + sel], d_c, int(d_rope))
         o[t], lse[t] = _attend_rows(qn_all[t], None if qp_all is None else qp_all[t],
                                     mult_all[t], scale, rows, d_c)
     return o, lse

@@ -214,6 +214,41 @@ def quantize_e4m3_rows(x: torch.Tensor):
     return codes.contiguous(), scale.contiguous()
 
 
+LATENT_FP8_BLOCK = 128
+
+
+def latent_fp8_row_bytes(d_rope: int, d_c: int = 512) -> int:
+    """Bytes per position of an FP8 latent-cache row: the E4M3 codes of
+    [c_s | kR_s], one fp32 scale per 128 latent values and one for kR_s (RoPE
+    layers), rounded up to a multiple of 16 (608 for RoPE, 528 for NoPE)."""
+    n_blk = d_c // LATENT_FP8_BLOCK + (1 if d_rope else 0)
+    return (d_c + d_rope + 4 * n_blk + 15) // 16 * 16
+
+
+def quantize_latent_fp8(cache: torch.Tensor, d_rope: int) -> torch.Tensor:
+    """FP8 latent-cache rows from a bf16 cache [rows, >= 512 + d_rope]: per
+    128-value block of c_s (and for kR_s as one block) scale = max |x| / 448
+    (1 for an all-zero block), codes = e4m3(x / scale) with torch's
+    float8_e4m3fn conversion; layout [codes | fp32 scales | zero padding].
+    Input preparation only: both the library and the oracle receive these bytes."""
+    d_c = 512
+    rows = cache.shape[0]
+    x = cache[:, :d_c + d_rope].float()
+    parts = [x[:, :d_c].reshape(rows, d_c // LATENT_FP8_BLOCK, LATENT_FP8_BLOCK)]
+    amax = parts[0].abs().amax(dim=-1)
+    if d_rope:
+        amax = torch.cat([amax, x[:, d_c:].abs().amax(dim=-1, keepdim=True)], dim=1)
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    blk_scale = torch.cat([scale[:, :d_c // LATENT_FP8_BLOCK].repeat_interleave(LATENT_FP8_BLOCK, dim=1)] +
+                          ([scale[:, -1:].expand(rows, d_rope)] if d_rope else []), dim=1)
+    codes = (x / blk_scale).to(torch.float8_e4m3fn).view(torch.uint8)
+    out = torch.zeros((rows, latent_fp8_row_bytes(d_rope, d_c)), dtype=torch.uint8, device=cache.device)
+    out[:, :d_c + d_rope] = codes
+    n_blk = scale.shape[1]
+    out[:, d_c + d_rope:d_c + d_rope + 4 * n_blk] = scale.contiguous().view(torch.uint8).reshape(rows, 4 * n_blk)
+    return out
+
+
 def small_case(name, lengths=None, *, kind="decode", cached=0, new=0, layers=(64,),
                qmul="uniform", mla_q_std=1.0 / math.sqrt(192.0), seed=7, topk=2048,
                planted=0, per_seq=1) -> Case:

@@ -55,6 +55,14 @@ MUTATIONS = {
     "forward_every_layer_reads_first_cache": ('lay["cache"], lay["d_rope"], seq_row_start',
                                               'layers[0]["cache"], lay["d_rope"], seq_row_start'),
     "forward_drops_last_layer": ("    for lay in layers:\n", "    for lay in layers[:-1]:\n"),
+    "fp8_latent_blocks_of_64": ("np.concatenate([np.arange(d_c) // LATENT_BLOCK,",
+                                "np.concatenate([np.arange(d_c) // 64 % 4,"),
+    "fp8_latent_rotary_takes_last_latent_scale": ("np.full(d_rope, d_c // LATENT_BLOCK, dtype=np.int64)",
+                                                  "np.full(d_rope, d_c // LATENT_BLOCK - 1, dtype=np.int64)"),
+    "fp8_latent_scales_ignored": ("    return values * scales[:, block_of_col]", "    return values"),
+    "fp8_latent_scales_read_after_latent": ("r[:, n_codes:n_codes + 4 * n_blk]", "r[:, d_c:d_c + 4 * n_blk]"),
+    "fp8_latent_reads_first_rows": ("rows = latent_fp8_decode(cache_np[base + sel], d_c, int(d_rope))",
+                                    "rows = latent_fp8_decode(cache_np[sel], d_c, int(d_rope))"),
     "fp8_indexer_relu_after_weighting": ("out[t, :n] = np.maximum(k_rows @ q.T, 0.0) @ wt[t]",
                                          "out[t, :n] = np.maximum(k_rows @ q.T @ wt[t], 0.0)"),
 }
@@ -70,7 +78,8 @@ def _mutant(name):
 
 def _run_pins(mod, golden_dir, monkeypatch):
     for fn in ("index_scores", "topk_select", "sparse_mla", "dense_causal_mla", "explicit_mla",
-               "forward", "e4m3_decode", "index_scores_fp8", "topk_merge", "lse_combine"):
+               "forward", "e4m3_decode", "index_scores_fp8", "topk_merge", "lse_combine",
+               "latent_fp8_decode", "sparse_mla_fp8"):
         monkeypatch.setattr(pins, fn, getattr(mod, fn))
     failures = 0
     for tname, test in inspect.getmembers(pins, inspect.isfunction):
@@ -82,6 +91,8 @@ def _run_pins(mod, golden_dir, monkeypatch):
             variants = [{"trial": i} for i in range(40)]
         if "d_r" in params:
             variants = [{"d_r": 64}, {"d_r": 0}]
+        if "blk" in params:
+            variants = [{"blk": b} for b in range(4)]
         for kw in variants:
             if "golden_dir" in params:
                 kw = dict(kw, golden_dir=golden_dir)

@@ -15,7 +15,8 @@ import numpy as np
 import pytest
 
 from oracle import (dense_causal_mla, e4m3_decode, explicit_mla, forward, index_scores,
-                    index_scores_fp8, lse_combine, sparse_mla, topk_merge, topk_select)
+                    index_scores_fp8, latent_fp8_decode, lse_combine, sparse_mla, sparse_mla_fp8,
+                    topk_merge, topk_select)
 
 RNG = np.random.default_rng(1234)
 
@@ -454,6 +455,109 @@ def test_empty_selection():
     idx = np.full((1, 2048), -1, np.int32)
     o, lse = sparse_mla(qn, qp, m, 0.2, cache, 64, starts, q_seq, idx, np.array([0]))
     assert np.all(o == 0) and np.all(np.isneginf(lse))
+
+
+# --------------------------------------------------------------------------- FP8 latent cache
+
+def _fp8_rows(codes, scales, row_bytes, pad=0):
+    """Byte rows of the FP8 latent layout: codes, then little-endian fp32 scales, then padding."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    scales = np.asarray(scales, dtype="<f4")
+    n, nc = codes.shape
+    out = np.full((n, row_bytes), pad, dtype=np.uint8)
+    out[:, :nc] = codes
+    out[:, nc:nc + 4 * scales.shape[1]] = scales.view(np.uint8).reshape(n, -1)
+    return out
+
+
+def test_latent_fp8_hand_worked_rows(golden_dir):
+    g = _toy(golden_dir)["latent_fp8"]
+    d_c, d_r = g["d_c"], g["d_rope"]
+    codes, scales = [], []
+    for r in g["rows"]:
+        c = np.full(d_c + d_r, r["fill_code"], dtype=np.uint8)
+        for col, code in r["codes_at"].items():
+            c[int(col)] = code
+        codes.append(c)
+        scales.append(r["scales"])
+    rows = _fp8_rows(np.stack(codes), np.array(scales), g["row_bytes"], pad=g["pad_byte"])
+    got = latent_fp8_decode(rows, d_c, d_r)
+    assert got.shape == (len(g["rows"]), d_c + d_r)
+    for i, e in enumerate(g["expected"]):
+        want = np.concatenate([np.full(128, e["fill_by_block"][0]), np.full(d_c - 128, e["fill_by_block"][1]),
+                               np.full(d_r, e["fill_by_block"][2])])
+        for col, v in e["at"].items():
+            want[int(col)] = v
+        np.testing.assert_array_equal(got[i], want)
+
+
+def _rand_fp8_attn_case(T=2, lens=(40, 70), d_r=64):
+    qn, qp, m, _, starts, q_seq, q_pos = _rand_attn_case(T=T, lens=lens, d_r=d_r, std=0.3)
+    rows = sum(lens)
+    codes = RNG.integers(0, 256, size=(rows, 512 + d_r)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x38                  # no NaN codes
+    n_blk = 4 + (1 if d_r else 0)
+    scales = np.exp2(RNG.integers(-3, 2, size=(rows, n_blk))) * (1.0 + RNG.random((rows, n_blk)))
+    scales = (scales / 64.0).astype(np.float32)           # values up to ~448 * 4 / 64
+    row_bytes = (512 + d_r + 4 * n_blk + 15) // 16 * 16
+    idx = np.full((T, 64), -1, np.int32)
+    cnt = np.zeros(T, np.int32)
+    for t in range(T):
+        n = min(64, q_pos[t] + 1)
+        idx[t, :n] = np.sort(RNG.choice(q_pos[t] + 1, size=n, replace=False))
+        cnt[t] = n
+    return qn, qp, m, codes, scales, row_bytes, starts, q_seq, idx, cnt
+
+
+@pytest.mark.parametrize("d_r", [64, 0])
+def test_sparse_mla_fp8_with_unit_scales_is_attention_on_the_code_values(d_r):
+    # all scales 1: the decoded cache is the E4M3 values themselves (e4m3_decode is pinned on
+    # every code), so the FP8 attention is sparse_mla on those values.
+    qn, qp, m, codes, scales, rb, starts, q_seq, idx, cnt = _rand_fp8_attn_case(d_r=d_r)
+    rows8 = _fp8_rows(codes, np.ones_like(scales), rb, pad=0x7F)
+    o8, l8 = sparse_mla_fp8(qn, qp, m, 0.1, rows8, d_r, starts, q_seq, idx, cnt)
+    o, l = sparse_mla(qn, qp, m, 0.1, e4m3_decode(codes), d_r, starts, q_seq, idx, cnt)
+    np.testing.assert_allclose(o8, o, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(l8, l, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("blk", [0, 1, 2, 3])
+def test_sparse_mla_fp8_block_scale_trades_against_that_block_of_the_query(blk):
+    # Doubling the scale of latent block b in every row while halving columns
+    # [128 b, 128 b + 128) of every query leaves every logit unchanged, so the
+    # weights and lse are unchanged and exactly that block of the output doubles.
+    qn, qp, m, codes, scales, rb, starts, q_seq, idx, cnt = _rand_fp8_attn_case()
+    o, l = sparse_mla_fp8(qn, qp, m, 0.1, _fp8_rows(codes, scales, rb), 64, starts, q_seq, idx, cnt)
+    s2 = scales.copy()
+    s2[:, blk] *= 2
+    qn2 = qn.astype(np.float64).copy()
+    qn2[:, :, 128 * blk:128 * blk + 128] /= 2
+    o2, l2 = sparse_mla_fp8(qn2, qp, m, 0.1, _fp8_rows(codes, s2, rb), 64, starts, q_seq, idx, cnt)
+    np.testing.assert_allclose(l2, l, rtol=1e-12, atol=1e-12)
+    want = o.copy()
+    want[:, :, 128 * blk:128 * blk + 128] *= 2
+    np.testing.assert_allclose(o2, want, rtol=1e-11, atol=1e-14)
+
+
+def test_sparse_mla_fp8_rotary_scale_trades_against_q_pe_and_zero_equals_no_rotary_query():
+    qn, qp, m, codes, scales, rb, starts, q_seq, idx, cnt = _rand_fp8_attn_case()
+    o, l = sparse_mla_fp8(qn, qp, m, 0.1, _fp8_rows(codes, scales, rb), 64, starts, q_seq, idx, cnt)
+    s2 = scales.copy()
+    s2[:, 4] *= 4
+    o2, l2 = sparse_mla_fp8(qn, qp.astype(np.float64) / 4, m, 0.1, _fp8_rows(codes, s2, rb), 64, starts, q_seq,
+                            idx, cnt)
+    np.testing.assert_allclose(o2, o, rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(l2, l, rtol=1e-12, atol=1e-12)
+    # the rotary part really takes part ...
+    s3 = scales.copy()
+    s3[:, 4] = 0.0
+    o3, l3 = sparse_mla_fp8(qn, qp, m, 0.1, _fp8_rows(codes, s3, rb), 64, starts, q_seq, idx, cnt)
+    assert np.abs(l3 - l).max() > 1e-3
+    # ... and a zero rotary scale is a zero rotary query
+    o4, l4 = sparse_mla_fp8(qn, np.zeros_like(qp), m, 0.1, _fp8_rows(codes, scales, rb), 64, starts, q_seq,
+                            idx, cnt)
+    np.testing.assert_allclose(o3, o4, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(l3, l4, rtol=1e-12, atol=1e-12)
 
 
 # --------------------------------------------------------------------------- composition
