@@ -54,7 +54,8 @@ sys.path.insert(0, ROOT)
 
 from sparse_attention_16_b200 import accounting as acc  # noqa: E402
 from sparse_attention_16_b200 import replicas  # noqa: E402
-from sparse_attention_16_b200.workloads import CONFIGS, make_workload, quantize_e4m3_rows, small_case  # noqa: E402
+from sparse_attention_16_b200.workloads import (CONFIGS, make_workload, quantize_e4m3_rows, quantize_latent_fp8,  # noqa: E402
+                                                small_case)
 
 HEADLINE = "decode_b4_1m_4layers"
 EXTRAS = ("decode_b64_32k", "prefill_32k_plus_8k", "decode_b16_32k_4queries")
@@ -164,7 +165,7 @@ def query_group(case):
 
 
 def measure(name, dev, steps, warmup, rank, world, local, min_seconds=0.0, sample_clocks=False, fp8=False,
-            eager=False, e2e=False, e2e_steps=20):
+            eager=False, e2e=False, e2e_steps=20, fp8_cache=False):
     """Times `steps` steps of configuration `name` (see the module docstring).
     Returns a dict with the timing, the per-kernel breakdown and the rooflines."""
     from sparse_attention_16_b200 import ops
@@ -182,9 +183,17 @@ def measure(name, dev, steps, warmup, rank, world, local, min_seconds=0.0, sampl
     cnt = torch.empty((T,), dtype=torch.int32, device=dev)
     outs = [torch.empty((T, 64, 512), dtype=torch.bfloat16, device=dev) for _ in wl.layers]
     lses = [torch.empty((T, 64), dtype=torch.float32, device=dev) for _ in wl.layers]
-    layers = [dict(q_nope=L.q_nope, q_pe=L.q_pe, qmul=L.qmul, cache=L.cache, d_rope=L.d_rope, out=o, lse=l)
-              for L, o, l in zip(wl.layers, outs, lses)]
-    n_rows = wl.layers[0].cache.shape[0]
+    if fp8_cache:
+        # FP8 latent rows (E4M3 codes + block scales) of the same seeded caches (input preparation, untimed)
+        caches = [quantize_latent_fp8(L.cache, L.d_rope) for L in wl.layers]
+        for L in wl.layers:
+            L.cache = None
+        torch.cuda.empty_cache()
+    else:
+        caches = [L.cache for L in wl.layers]
+    layers = [dict(q_nope=L.q_nope, q_pe=L.q_pe, qmul=L.qmul, cache=c, d_rope=L.d_rope, out=o, lse=l)
+              for L, c, o, l in zip(wl.layers, caches, outs, lses)]
+    n_rows = caches[0].shape[0]
     att_ws = ops.workspace(ops.layers_workspace_bytes(T, n_layers, k), dev)
     # decode: the indexer also counts its scores into a histogram that the top-k's first pass reads
     hist = torch.empty((T, 2048), dtype=torch.int32, device=dev) if q_group == 1 else None
@@ -297,7 +306,8 @@ def measure(name, dev, steps, warmup, rank, world, local, min_seconds=0.0, sampl
     n_scored = int((q_pos + 1).sum())
     idx_bytes = acc.indexer_bytes(n_scored, T, T * ld, fp8=fp8)
     n_rows_att = int(np.minimum(q_pos + 1, k).sum())
-    att_bytes = sum(acc.attend_bytes(n_rows_att, T, L.d_rope) for L in wl.layers)
+    att_bytes = sum(acc.attend_bytes(n_rows_att, T, L.d_rope, row_bytes=c.shape[1] if fp8_cache else None)
+                    for L, c in zip(wl.layers, caches))
     step_bytes = idx_bytes + acc.topk_bytes(n_scored, T, k) + att_bytes
     timed_steps = steps * replays
     step_s = elapsed / timed_steps
@@ -345,12 +355,12 @@ def measure(name, dev, steps, warmup, rank, world, local, min_seconds=0.0, sampl
                           "workspace_bytes": int(plan.workspace_bytes)}
     if e2e:
         res["e2e"] = run_e2e(wl, ld, k, q_group, dev, e2e_steps,
-                             fp8=(q8, q8_scale, k8, k8_scale) if fp8 else None)
+                             fp8=(q8, q8_scale, k8, k8_scale) if fp8 else None, caches=caches)
     del graph, graph_ev
     return res
 
 
-def run_e2e(wl, ld, k, q_group, dev, steps, fp8=None):
+def run_e2e(wl, ld, k, q_group, dev, steps, fp8=None, caches=None):
     """Same metric through dsa_sparse_mla_forward (dsa_sparse_mla_forward_fp8 with
     `fp8` = (q8, q_scale, k8, k_scale)) with pinned host inputs/outputs: each step
     copies the step's queries host->device and the outputs back."""
@@ -379,7 +389,8 @@ def run_e2e(wl, ld, k, q_group, dev, steps, fp8=None):
         for n in pinned:
             dev_in[n].copy_(pinned[n], non_blocking=True)
         layers = [dict(q_nope=dev_in[f"q_nope{i}"], q_pe=dev_in.get(f"q_pe{i}"), qmul=dev_in[f"qmul{i}"],
-                       cache=L.cache, d_rope=L.d_rope, out=outs[i], lse=None) for i, L in enumerate(wl.layers)]
+                       cache=caches[i] if caches is not None else L.cache, d_rope=L.d_rope, out=outs[i], lse=None)
+                  for i, L in enumerate(wl.layers)]
         if fp8 is None:
             ops.sparse_mla_forward(dev_in["q_idx"], dev_in["w"], wl.k_idx, wl.seq_row_start, dev_in["q_seq"],
                                    dev_in["q_pos"], layers, ld, k=k, q_group=q_group, ws=ws)
@@ -417,7 +428,8 @@ def run_ours(args, rank, world, local):
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     ops.load_library()
     head = measure(args.config, dev, args.steps, args.warmup, rank, world, local, min_seconds=args.min_seconds,
-                   sample_clocks=True, fp8=args.fp8_keys, eager=args.eager, e2e=not args.no_e2e)
+                   sample_clocks=True, fp8=args.fp8_keys, eager=args.eager, e2e=not args.no_e2e,
+                   fp8_cache=args.fp8_cache)
     torch.cuda.empty_cache()
     case = CONFIGS[args.config]
     wl_T = head["T"]
@@ -426,7 +438,8 @@ def run_ours(args, rank, world, local):
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": head["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded, shapes/distributions of the configuration)",
-        "config": {"workload": args.config + ("+fp8_index_keys" if args.fp8_keys else ""),
+        "config": {"workload": args.config + ("+fp8_index_keys" if args.fp8_keys else "")
+                   + ("+fp8_latent_cache" if args.fp8_cache else ""),
                    "queries_per_gpu": wl_T, "context": list(case.seq_lengths)[:1],
                    "layers": [("rope" if d else "nope") for d in case.layers], "topk": case.topk,
                    "parallelism": f"replicas{world}" if world > 1 else "1gpu",
@@ -448,7 +461,8 @@ def run_ours(args, rank, world, local):
             if name == args.config:
                 continue
             r = measure(name, dev, 3 if CONFIGS[name].kind == "prefill" else args.steps, 3, rank, world, local,
-                        min_seconds=0.0 if CONFIGS[name].kind == "prefill" else 0.3, fp8=args.fp8_keys)
+                        min_seconds=0.0 if CONFIGS[name].kind == "prefill" else 0.3, fp8=args.fp8_keys,
+                        fp8_cache=args.fp8_cache)
             torch.cuda.empty_cache()
             keep = ("ms_per_step", "queries_per_s", "query_layers_per_s", "kernel_ms", "step_hbm", "attention_hbm",
                     "roofline", "timed_steps", "attend_plan", "q_group")
@@ -609,6 +623,9 @@ def main():
     ap.add_argument("--fp8-keys", action="store_true",
                     help="score with FP8 (E4M3) index keys and queries, per-row scales (dsa_index_scores_fp8); "
                          "the selection and attention are unchanged")
+    ap.add_argument("--fp8-cache", action="store_true",
+                    help="keep every layer's latent cache as FP8 rows (E4M3 codes, one fp32 scale per 128 values "
+                         "and one for the rotary key); the attention widens the selected rows on chip")
     args = ap.parse_args()
     rank, world, local = dist_env()
     if args.gpus > 1 and "RANK" not in os.environ:

@@ -239,14 +239,31 @@ typedef struct dsa_layer_args {
   const void* q_nope;   /* bf16 [T, 64, 512]                                  */
   const void* q_pe;     /* bf16 [T, 64, 64] or NULL (NoPE)                    */
   const float* qmul;    /* f32 [T, 64]                                        */
-  const void* cache;    /* bf16 [n_rows, ld_c]                                */
-  int32_t ld_c;
+  const void* cache;    /* bf16 [n_rows, ld_c], or FP8 rows when cache_fp8 = 1 */
+  int32_t ld_c;         /* row stride: elements (bf16) or bytes (FP8 rows)    */
   int32_t d_rope;       /* 64 or 0                                            */
   void* out;            /* bf16 [T, 64, 512], or f32 when out_f32 = 1         */
   float* lse;           /* f32 [T, 64] or NULL                                */
   int32_t out_f32;      /* 1: fp32 output (partials for dsa_lse_combine)      */
-  int32_t reserved;     /* 0                                                  */
+  int32_t cache_fp8;    /* 1: the cache holds FP8 latent rows (below)         */
 } dsa_layer_args;
+
+/*
+ * FP8 latent-cache rows (cache_fp8 = 1).  The report's serving section keeps
+ * the KV cache in FP8 natively and its training section runs FP8 with
+ * blockwise scales; the pages give no layout.  This library's layout, one row
+ * of ld_c bytes per position (ld_c % 16 == 0, the cache 16-byte aligned):
+ *   bytes [0, 512 + d_rope)            E4M3 codes (OCP FP8 E4M3) of [c_s | kR_s]
+ *   bytes [512 + d_rope, + 4 * nb)     little-endian fp32 scales: one per 128
+ *                                      latent values (4) and, on RoPE layers, one
+ *                                      for kR_s (nb = 5; NoPE: nb = 4)
+ *   then padding (ignored)             minimum ld_c: 608 (RoPE), 528 (NoPE)
+ * Column i < 512 is scale[i / 128] * e4m3(code[i]); column 512 + j is
+ * scale[4] * e4m3(code[512 + j]).  The attention widens each selected row to
+ * bf16 on chip (one rounding of scale * value to bf16) and then computes
+ * exactly as on a bf16 cache.  Codes must not be NaN.  Every layer of one call
+ * must use the same cache format (DSA_ERR_INVALID_ARG otherwise).
+ */
 
 /*
  * sparse_mla_attend_layers - sparse_mla_attend for several layers that share
@@ -442,7 +459,7 @@ uint64_t dsa_launch_count(void);
 /* Text of the last failure reported on the calling thread ("" if none). */
 const char* dsa_last_error(void);
 
-/* ABI version of this library (major * 100 + minor): 200. */
+/* ABI version of this library (major * 100 + minor): 201. */
 int32_t dsa_version(void);
 
 #ifdef __cplusplus

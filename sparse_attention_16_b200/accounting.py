@@ -143,9 +143,11 @@ def topk_bytes(n_candidates_total: int, n_queries: int, k: int = TOPK) -> int:
     return n_candidates_total * F32 + n_queries * (k * I32 + I32)
 
 
-def attend_bytes(n_rows_total: int, n_queries: int, d_rope: int, with_lse: bool = True) -> int:
-    """Selected cache rows gathered once, query/multiplier read, output written."""
-    row = (D_LATENT + d_rope) * BF16
+def attend_bytes(n_rows_total: int, n_queries: int, d_rope: int, with_lse: bool = True,
+                 row_bytes: int | None = None) -> int:
+    """Selected cache rows gathered once, query/multiplier read, output written.
+    ``row_bytes``: bytes per cache row when it is not bf16 (FP8 latent rows)."""
+    row = (D_LATENT + d_rope) * BF16 if row_bytes is None else row_bytes
     q = N_HEADS * (D_LATENT + d_rope) * BF16 + N_HEADS * F32
     out = N_HEADS * D_LATENT * BF16 + (N_HEADS * F32 if with_lse else 0)
     idx = TOPK * I32 + I32

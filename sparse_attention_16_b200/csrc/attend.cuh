@@ -97,10 +97,10 @@ struct AttLayer {
   const __nv_bfloat16* q_nope;    // [T, 64, 512]
   const __nv_bfloat16* q_pe;      // [T, 64, 64] (RoPE layers) or null
   const float* qmul;              // [T, 64]
-  const __nv_bfloat16* cache;     // [n_rows, ld_c]
+  const __nv_bfloat16* cache;     // [n_rows, ld_c] bf16, or FP8 rows of ld_c bytes (attend_kernel<true>)
   __nv_bfloat16* out;             // [T, 64, 512]
   float* lse;                     // [T, 64] or null
-  int64_t ld_c;                   // row stride of the cache, elements
+  int64_t ld_c;                   // row stride of the cache: elements (bf16) or bytes (FP8 rows)
   int32_t d_rope;                 // 64 (RoPE) or 0 (NoPE)
   int32_t out_f32;                // 1: `out` is fp32 [T, 64, 512] (partial outputs to combine later)
 };
@@ -165,6 +165,27 @@ __device__ __forceinline__ void unit_rows(const AttendParams& p, int t, int j, i
   r_begin = j * p.rows_per_split;
   r_end = min(cnt, r_begin + p.rows_per_split);
   if (r_end < r_begin) r_end = r_begin;
+}
+
+// Two E4M3 codes (bits 0-7: the first, bits 8-15: the second) to two floats;
+// every E4M3 value is exact in f16 and in f32.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t codes) {
+  float lo, hi;
+  asm("{\n\t.reg .b16 c, l, h;\n\t.reg .b32 x;\n\t"
+      "cvt.u16.u32 c, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 x, c;\n\t"
+      "mov.b32 {l, h}, x;\n\t"
+      "cvt.f32.f16 %0, l;\n\t"
+      "cvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(codes));
+  return make_float2(lo, hi);
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // tcgen05.st over the 16 lanes [taddr.lane, +16): threads 0-15 write columns
@@ -319,8 +340,10 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLa
   }
 }
 
-// The work of one CTA on one unit; KCH = 64-column chunks per row (9 RoPE, 8 NoPE).
-template <int KCH>
+// The work of one CTA on one unit; KCH = 64-column chunks per row (9 RoPE, 8 NoPE);
+// F8: the cache rows are FP8 (E4M3 codes + block scales) and are widened to bf16
+// in shared memory.
+template <int KCH, bool F8>
 __device__ __forceinline__ void attend_unit(const AttendParams& p, const AttLayer& L, uint8_t* cs, uint8_t* ps,
                                             AttScratch* sc, uint32_t tmem_base, int t, int jsplit,
                                             bool smem_ok) {
@@ -392,41 +415,174 @@ __device__ __forceinline__ void attend_unit(const AttendParams& p, const AttLaye
     };
     int32_t cur = load_idx(0);
     bool ok = true;
-    for (int i = 0; i < n_tiles; ++i) {
-      const int buf = i % C::NBUF;
-      if (i >= C::NBUF &&
-          !mbar_wait(&sc->free_[buf], (uint32_t)((i / C::NBUF - 1) & 1), abort_flag, limit)) {
-        ok = false;
-        break;
-      }
-      // Buffer 2 holds Q until the softmax warps have moved it to TMEM.
-      if (i == 2 && !mbar_wait(&sc->q_full, 0, abort_flag, limit)) {
-        ok = false;
-        break;
-      }
-      int32_t row = -1;   // row of the cache, or -1: the copy zero-fills
-      if (cur >= 0 && cur <= qpos && base + cur < p.n_rows) row = (int32_t)(base + cur);
-      else if (cur != -1) raise_error(kErrBadIndex);
-      cur = load_idx(i + 1);
-      if (i == p.stall_tile) continue;   // testing hook: this tile never arrives
-      const uint32_t tb = cs0 + buf * C::TILE_BYTES;
-#pragma unroll 1
-      for (int kq = 0; kq < QPW; ++kq) {
-        const int quad = pw + 3 * kq;
-        if (quad >= NQ) break;
-#pragma unroll
-        for (int j = 0; j < KCH; ++j) {
-          const int g = 32 * j + lane;
-          const int riq = g / PPR;
-          const int pr = g - riq * PPR;
-          const int32_t src_row = __shfl_sync(0xffffffffu, row, 4 * kq + riq);
-          const int r = 4 * quad + riq;
-          const uint32_t dst = tb + (pr >> 3) * C::CHUNK_BYTES + r * 128 + (((pr & 7) ^ (r & 7)) << 4);
-          const char* src = src_row >= 0 ? cache_bytes + (int64_t)src_row * L.ld_c * 2 + pr * 16 : cache_bytes;
-          cp_async_16(dst, src, src_row >= 0 ? 16u : 0u);
+    if constexpr (!F8) {
+      for (int i = 0; i < n_tiles; ++i) {
+        const int buf = i % C::NBUF;
+        if (i >= C::NBUF &&
+            !mbar_wait(&sc->free_[buf], (uint32_t)((i / C::NBUF - 1) & 1), abort_flag, limit)) {
+          ok = false;
+          break;
         }
+        // Buffer 2 holds Q until the softmax warps have moved it to TMEM.
+        if (i == 2 && !mbar_wait(&sc->q_full, 0, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        int32_t row = -1;   // row of the cache, or -1: the copy zero-fills
+        if (cur >= 0 && cur <= qpos && base + cur < p.n_rows) row = (int32_t)(base + cur);
+        else if (cur != -1) raise_error(kErrBadIndex);
+        cur = load_idx(i + 1);
+        if (i == p.stall_tile) continue;   // testing hook: this tile never arrives
+        const uint32_t tb = cs0 + buf * C::TILE_BYTES;
+#pragma unroll 1
+        for (int kq = 0; kq < QPW; ++kq) {
+          const int quad = pw + 3 * kq;
+          if (quad >= NQ) break;
+#pragma unroll
+          for (int j = 0; j < KCH; ++j) {
+            const int g = 32 * j + lane;
+            const int riq = g / PPR;
+            const int pr = g - riq * PPR;
+            const int32_t src_row = __shfl_sync(0xffffffffu, row, 4 * kq + riq);
+            const int r = 4 * quad + riq;
+            const uint32_t dst = tb + (pr >> 3) * C::CHUNK_BYTES + r * 128 + (((pr & 7) ^ (r & 7)) << 4);
+            const char* src = src_row >= 0 ? cache_bytes + (int64_t)src_row * L.ld_c * 2 + pr * 16 : cache_bytes;
+            cp_async_16(dst, src, src_row >= 0 ? 16u : 0u);
+          }
+        }
+        cp_async_arrive_noinc(&sc->full[buf]);   // lands once this thread's copies so far have
       }
-      cp_async_arrive_noinc(&sc->full[buf]);   // lands once this thread's copies so far have
+    } else {
+      // FP8 rows: the 64 E4M3 codes of a row's 64-column chunk c land in the
+      // upper half of that row's 128-byte line of chunk c (pieces 4-7, swizzled
+      // like the bf16 pieces) and the row's block scales in registers of the
+      // lane that owns the row.  Once a tile's copies have landed, the warp
+      // widens every line in place: a lane reads the line's 64 codes, then
+      // writes the 64 bf16 values scale * e4m3(code) over the whole line, so the
+      // products see the bf16 tile layout.  The copies of tile i are issued
+      // before tile i - 1 is widened, so they are in flight meanwhile.
+      constexpr int CPR = 4 * KCH;               // 16-byte code pieces per row
+      constexpr int NBLK = (KCH == 9) ? 5 : 4;   // fp32 scales per row
+      constexpr int SCALE_OFF = 64 * KCH;        // byte offset of the scales in a row
+      constexpr int CPI = (4 * CPR + 31) / 32;   // warp-wide copy instructions per quad
+      const int rows_w = 4 * ((NQ - pw + 2) / 3);   // rows this warp gathers; local row l = lane l's row
+      const int lines_w = rows_w * KCH;
+      float sc_next[NBLK], sc_pend[NBLK];
+#pragma unroll
+      for (int b = 0; b < NBLK; ++b) sc_next[b] = sc_pend[b] = 0.f;
+      // Widens the lines of this warp's rows in buffer `buf`; line lane + 32 m
+      // is (local row rl, chunk c), rows fastest.
+      auto widen = [&](int buf) {
+        const uint32_t tb = cs0 + buf * C::TILE_BYTES;
+        int rl = lane, c = 0;
+        while (rl >= rows_w) {
+          rl -= rows_w;
+          ++c;
+        }
+        const int n_it = (lines_w + 31) / 32;
+#pragma unroll 1
+        for (int it = 0; it < n_it; ++it) {
+          const bool active = c < KCH;
+          const int blk = (c < 8) ? (c >> 1) : 4;
+          float s = 0.f;
+#pragma unroll
+          for (int b = 0; b < NBLK; ++b) {
+            const float v = __shfl_sync(0xffffffffu, sc_pend[b], active ? rl : 0);
+            if (b == blk) s = v;
+          }
+          if (active) {
+            const int r = 4 * (pw + 3 * (rl >> 2)) + (rl & 3);
+            const uint32_t line = tb + c * C::CHUNK_BYTES + r * 128;
+            uint32_t w[16];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+              ld_shared_v4(line + (((4 + jj) ^ (r & 7)) << 4), w[4 * jj], w[4 * jj + 1], w[4 * jj + 2], w[4 * jj + 3]);
+#pragma unroll
+            for (int pp = 0; pp < 8; ++pp) {
+              const float2 a = e4m3x2_to_float2(w[2 * pp]);
+              const float2 b = e4m3x2_to_float2(w[2 * pp] >> 16);
+              const float2 cc = e4m3x2_to_float2(w[2 * pp + 1]);
+              const float2 d = e4m3x2_to_float2(w[2 * pp + 1] >> 16);
+              st_shared_v4(line + ((pp ^ (r & 7)) << 4), pack_bf16x2(a.x * s, a.y * s), pack_bf16x2(b.x * s, b.y * s),
+                           pack_bf16x2(cc.x * s, cc.y * s), pack_bf16x2(d.x * s, d.y * s));
+            }
+          }
+          rl += 32;
+          while (rl >= rows_w) {
+            rl -= rows_w;
+            ++c;
+          }
+        }
+      };
+      int pend_buf = -1;   // buffer whose copies are in flight and not yet widened
+      for (int i = 0; i < n_tiles; ++i) {
+        const int buf = i % C::NBUF;
+        if (i >= C::NBUF &&
+            !mbar_wait(&sc->free_[buf], (uint32_t)((i / C::NBUF - 1) & 1), abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        if (i == 2 && !mbar_wait(&sc->q_full, 0, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        int32_t row = -1;
+        if (cur >= 0 && cur <= qpos && base + cur < p.n_rows) row = (int32_t)(base + cur);
+        else if (cur != -1) raise_error(kErrBadIndex);
+        cur = load_idx(i + 1);
+        const bool live = i != p.stall_tile;   // testing hook: that tile never arrives
+        if (live) {
+          const uint32_t tb = cs0 + buf * C::TILE_BYTES;
+#pragma unroll 1
+          for (int kq = 0; kq < QPW; ++kq) {
+            const int quad = pw + 3 * kq;
+            if (quad >= NQ) break;
+#pragma unroll
+            for (int j = 0; j < CPI; ++j) {
+              const int g = 32 * j + lane;
+              const int riq = min(g / CPR, 3);
+              const int32_t src_row = __shfl_sync(0xffffffffu, row, 4 * kq + riq);
+              if (g < 4 * CPR) {
+                const int pr = g - riq * CPR;
+                const int r = 4 * quad + riq;
+                const uint32_t dst = tb + (pr >> 2) * C::CHUNK_BYTES + r * 128 + (((4 + (pr & 3)) ^ (r & 7)) << 4);
+                const char* src = src_row >= 0 ? cache_bytes + (int64_t)src_row * L.ld_c + pr * 16 : cache_bytes;
+                cp_async_16(dst, src, src_row >= 0 ? 16u : 0u);
+              }
+            }
+          }
+          if (lane < rows_w && row >= 0) {
+            const float* sr = reinterpret_cast<const float*>(cache_bytes + (int64_t)row * L.ld_c + SCALE_OFF);
+            const float4 v = __ldg(reinterpret_cast<const float4*>(sr));
+            sc_next[0] = v.x;
+            sc_next[1] = v.y;
+            sc_next[2] = v.z;
+            sc_next[3] = v.w;
+            if constexpr (NBLK == 5) sc_next[4] = __ldg(sr + 4);
+          } else {
+#pragma unroll
+            for (int b = 0; b < NBLK; ++b) sc_next[b] = 0.f;
+          }
+        }
+        cp_async_commit();
+        if (pend_buf >= 0) {
+          cp_async_wait_group<1>();   // this lane's copies of the previous tile have landed
+          __syncwarp();               // ... and every lane's
+          widen(pend_buf);
+          fence_proxy_async_smem();   // generic-proxy writes, read by the tensor core
+          mbar_arrive(&sc->full[pend_buf]);
+        }
+        pend_buf = live ? buf : -1;
+#pragma unroll
+        for (int b = 0; b < NBLK; ++b) sc_pend[b] = sc_next[b];
+      }
+      if (ok && pend_buf >= 0) {
+        cp_async_wait_group<0>();
+        __syncwarp();
+        widen(pend_buf);
+        fence_proxy_async_smem();
+        mbar_arrive(&sc->full[pend_buf]);
+      }
     }
     if (!ok) *abort_flag = 1;
     cp_async_wait_all();   // nothing may still be landing in shared memory at the barrier below
@@ -720,6 +876,8 @@ __device__ __forceinline__ void attend_unit(const AttendParams& p, const AttLaye
   }
 }
 
+// F8: every layer of the launch keeps its latent cache in FP8 rows.
+template <bool F8>
 __global__ void __launch_bounds__(AttCfg::THREADS, 1)
     attend_kernel(const __grid_constant__ AttendParams p) {
   using C = AttCfg;
@@ -766,8 +924,8 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = sc->tmem_slot;
 
-  if (L.d_rope == 64) attend_unit<9>(p, L, cs, ps, sc, tmem_base, t, jsplit, smem_ok);
-  else attend_unit<8>(p, L, cs, ps, sc, tmem_base, t, jsplit, smem_ok);
+  if (L.d_rope == 64) attend_unit<9, F8>(p, L, cs, ps, sc, tmem_base, t, jsplit, smem_ok);
+  else attend_unit<8, F8>(p, L, cs, ps, sc, tmem_base, t, jsplit, smem_ok);
 
   tc_fence_before();
   __syncthreads();

@@ -101,7 +101,7 @@ uint64_t current_context_id() {
 
 // ----------------------------------------------------------------- per-device state
 enum KernelId : uint32_t {
-  kKIdx1 = 0, kKIdx4, kKIdx8, kKIdx1F8, kKIdx4F8, kKIdx8F8, kKTopk1, kKTopk2, kKTopk4, kKTopk8, kKTopk16, kKAttend, kKTopkFilter,
+  kKIdx1 = 0, kKIdx4, kKIdx8, kKIdx1F8, kKIdx4F8, kKIdx8F8, kKTopk1, kKTopk2, kKTopk4, kKTopk8, kKTopk16, kKAttend, kKAttend8, kKTopkFilter,
   kKTopkSelect, kKTopkMerge, kKCount
 };
 
@@ -179,9 +179,11 @@ dsa_status_t device_props(DevLock& L, dsa::DevProps* out) {
     int n = 0;
     DSA_CUDA(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, L.dev));
     d.sms = n > 0 ? n : 1;
-    DSA_TRY(set_smem(s, kKAttend, dsa::attend_kernel, dsa::AttCfg::SMEM_BYTES));
+    // (the FP8-cache variant has the same block size and shared memory, so the same residency)
+    DSA_TRY(set_smem(s, kKAttend, dsa::attend_kernel<false>, dsa::AttCfg::SMEM_BYTES));
     for (int c = 2; c <= dsa::kPlanMaxMerge; ++c)
-      d.max_clusters[c] = max_active_clusters(dsa::attend_kernel, dsa::AttCfg::THREADS, dsa::AttCfg::SMEM_BYTES, c);
+      d.max_clusters[c] =
+          max_active_clusters(dsa::attend_kernel<false>, dsa::AttCfg::THREADS, dsa::AttCfg::SMEM_BYTES, c);
     DSA_TRY(set_smem(s, kKTopk2, dsa::topk_kernel<2>, dsa::kTopkSmemBytes));
     DSA_TRY(set_smem(s, kKTopk4, dsa::topk_kernel<4>, dsa::kTopkSmemBytes));
     DSA_TRY(set_smem(s, kKTopk8, dsa::topk_kernel<8>, dsa::kTopkSmemBytes));
@@ -466,9 +468,15 @@ dsa_status_t launch_attend(DevLock& L, const dsa_layer_args* layers, int32_t n_l
     p.ws_o = static_cast<float*>(ws);
     p.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + dsa::partial_stats_offset(units, sp.n_split));
   }
-  DSA_TRY(set_smem(*L.s, kKAttend, dsa::attend_kernel, C::SMEM_BYTES));
-  DSA_TRY(launch(dsa::attend_kernel, (unsigned)(units * sp.n_split), C::THREADS, C::SMEM_BYTES, stream,
-                 sp.merge ? (unsigned)sp.n_split : 1u, p));
+  const unsigned grid = (unsigned)(units * sp.n_split);
+  const unsigned cluster = sp.merge ? (unsigned)sp.n_split : 1u;
+  if (layers[0].cache_fp8) {   // every layer of a call has the same cache format (checked)
+    DSA_TRY(set_smem(*L.s, kKAttend8, dsa::attend_kernel<true>, C::SMEM_BYTES));
+    DSA_TRY(launch(dsa::attend_kernel<true>, grid, C::THREADS, C::SMEM_BYTES, stream, cluster, p));
+  } else {
+    DSA_TRY(set_smem(*L.s, kKAttend, dsa::attend_kernel<false>, C::SMEM_BYTES));
+    DSA_TRY(launch(dsa::attend_kernel<false>, grid, C::THREADS, C::SMEM_BYTES, stream, cluster, p));
+  }
   if (!partials) return DSA_OK;
   // programmatic dependent launch: scheduled while the attention drains, waits for its writes
   return launch_ex(true, dsa::attend_combine_kernel, (unsigned)(units * dsa::kHeads), 128, 0, stream, 1, p);
@@ -539,8 +547,15 @@ dsa_status_t check_layer_args(const dsa_layer_args& a, int64_t n_rows) {
                   (a.q_pe == nullptr || aligned(a.q_pe, 16)),
               "q_nope, q_pe, cache and out must be 16-byte aligned");
   DSA_REQUIRE(aligned(a.qmul, 4) && (a.lse == nullptr || aligned(a.lse, 4)), "misaligned qmul / lse");
-  DSA_REQUIRE(a.ld_c >= dsa::kLatent + a.d_rope && a.ld_c % 8 == 0,
-              "ld_c must be >= 512 + d_rope and a multiple of 8");
+  DSA_REQUIRE(a.cache_fp8 == 0 || a.cache_fp8 == 1, "cache_fp8 must be 0 or 1");
+  if (a.cache_fp8) {
+    const int32_t need = dsa::kLatent + a.d_rope + 4 * (dsa::kLatent / 128 + (a.d_rope ? 1 : 0));
+    DSA_REQUIRE(a.ld_c >= need && a.ld_c % 16 == 0,
+                "FP8 cache rows: ld_c (bytes) must be >= %d and a multiple of 16 (got %d)", need, a.ld_c);
+  } else {
+    DSA_REQUIRE(a.ld_c >= dsa::kLatent + a.d_rope && a.ld_c % 8 == 0,
+                "ld_c must be >= 512 + d_rope and a multiple of 8");
+  }
   DSA_REQUIRE(n_rows * (int64_t)a.ld_c < (int64_t(1) << 62), "cache too large");
   return DSA_OK;
 }
@@ -572,7 +587,7 @@ dsa_layer_args one_layer(const void* q_nope, const void* q_pe, const float* qmul
   a.out = out;
   a.lse = lse;
   a.out_f32 = 0;
-  a.reserved = 0;
+  a.cache_fp8 = 0;
   return a;
 }
 
@@ -757,6 +772,7 @@ dsa_status_t sparse_mla_attend_layers(int32_t n_layers, const dsa_layer_args* la
   for (int l = 0; l < n_layers; ++l) {
     const dsa_status_t st = check_layer_args(layers[l], n_rows);
     if (st != DSA_OK) return fail(st, "layer %d: %s", l, g_last_error.c_str());
+    DSA_REQUIRE(layers[l].cache_fp8 == layers[0].cache_fp8, "every layer of a call must use the same cache format");
   }
   if (T == 0 || n_layers == 0) return DSA_OK;
   DevLock L;
@@ -801,6 +817,7 @@ dsa_status_t forward_impl(const IndexKeys& ik, const float* w, int64_t n_rows, c
   for (int l = 0; l < n_layers; ++l) {
     const dsa_status_t st = check_layer_args(layers[l], n_rows);
     if (st != DSA_OK) return fail(st, "layer %d: %s", l, g_last_error.c_str());
+    DSA_REQUIRE(layers[l].cache_fp8 == layers[0].cache_fp8, "every layer of a call must use the same cache format");
   }
   if (T == 0) return DSA_OK;
   DSA_REQUIRE(workspace != nullptr && aligned(workspace, 256), "workspace must be non-null and 256-byte aligned");
@@ -1023,6 +1040,6 @@ uint64_t dsa_launch_count(void) { return g_launches.load(std::memory_order_relax
 
 const char* dsa_last_error(void) { return g_last_error.c_str(); }
 
-int32_t dsa_version(void) { return 200; }
+int32_t dsa_version(void) { return 201; }
 
 }  // extern "C"

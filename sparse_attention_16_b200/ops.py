@@ -36,7 +36,7 @@ class LayerArgs(ctypes.Structure):
     """Mirror of ``dsa_layer_args``."""
 
     _fields_ = [("q_nope", _P), ("q_pe", _P), ("qmul", _P), ("cache", _P), ("ld_c", _I32),
-                ("d_rope", _I32), ("out", _P), ("lse", _P), ("out_f32", _I32), ("reserved", _I32)]
+                ("d_rope", _I32), ("out", _P), ("lse", _P), ("out_f32", _I32), ("cache_fp8", _I32)]
 
 
 class DeviceProps(ctypes.Structure):
@@ -337,7 +337,8 @@ def _layer_array(layers, T):
         if L["d_rope"]:
             _need(L["q_pe"], torch.bfloat16, (T, 64, L["d_rope"]), f"layers[{i}].q_pe")
         _need(L["qmul"], torch.float32, (T, 64), f"layers[{i}].qmul")
-        _need(L["cache"], torch.bfloat16, None, f"layers[{i}].cache")
+        fp8 = L["cache"].dtype == torch.uint8   # FP8 latent rows (E4M3 codes + block scales)
+        _need(L["cache"], torch.uint8 if fp8 else torch.bfloat16, None, f"layers[{i}].cache")
         f32 = L["out"].dtype == torch.float32
         _need(L["out"], torch.float32 if f32 else torch.bfloat16, (T, 64, 512), f"layers[{i}].out")
         if L.get("lse") is not None:
@@ -346,7 +347,7 @@ def _layer_array(layers, T):
                            L["q_pe"].data_ptr() if L.get("q_pe") is not None else None,
                            L["qmul"].data_ptr(), L["cache"].data_ptr(), L["cache"].shape[1],
                            L["d_rope"], L["out"].data_ptr(),
-                           L["lse"].data_ptr() if L.get("lse") is not None else None, int(f32), 0)
+                           L["lse"].data_ptr() if L.get("lse") is not None else None, int(f32), int(fp8))
     return arr
 
 

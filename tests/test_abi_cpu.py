@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version(lib):
-    assert lib.dsa_version() == 200
+    assert lib.dsa_version() == 201
 
 
 NULL = None
@@ -120,6 +120,31 @@ def test_attend_layers_rejects_bad_arguments(lib):
         assert st == want
     assert lib.sparse_mla_attend_layers(2, None, 0.07, 1000, fake, 1, fake, NULL, fake, fake, 4, 2048, NULL, 0,
                                         NULL) == 1
+
+
+def test_fp8_cache_rows_are_validated(lib):
+    # FP8 latent rows: ld_c in bytes, a multiple of 16, at least codes + scales
+    # (608 RoPE, 528 NoPE); every layer of a call uses one cache format.
+    fake = ctypes.c_void_p(256)
+
+    def layer(q_pe, ld_c, d_rope, fp8):
+        return ops.LayerArgs(256, q_pe, 256, 256, ld_c, d_rope, 256, None, 0, fp8)
+
+    cases = (
+        ((layer(256, 608, 64, 1),), 0),
+        ((layer(None, 528, 0, 1),), 0),
+        ((layer(256, 592, 64, 1),), 1),        # scales do not fit
+        ((layer(256, 600, 64, 1),), 1),        # not a multiple of 16
+        ((layer(None, 512, 0, 1),), 1),
+        ((layer(256, 608, 64, 2),), 1),        # unknown format
+        ((layer(256, 608, 64, 1), layer(256, 576, 64, 0)), 1),   # mixed formats
+        ((layer(256, 576, 64, 0), layer(None, 512, 0, 0)), 0),
+    )
+    for layers, want in cases:
+        arr = (ops.LayerArgs * len(layers))(*layers)
+        st = lib.sparse_mla_attend_layers(len(layers), arr, 0.07, 1000, fake, 1, fake, NULL, fake, fake, 0, 2048,
+                                          NULL, 0, NULL)
+        assert st == want, (layers, want)
 
 
 def test_forward_rejects_missing_workspace(lib):
