@@ -64,7 +64,9 @@ struct IdxCfg {
   static constexpr int SMEM_TILES = STAGES * KT_BYTES + QBUFS * Q_BYTES;
   static constexpr int W_BYTES = EPI_WARPS * ((QG == 1) ? 1 : 4) * kIdxHeads * 4;
   static constexpr int HIST_BYTES = (QG == 1) ? 2048 * 4 : 0;   // decode: score histogram of the current query
-  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024 + W_BYTES + HIST_BYTES;
+  static constexpr int KS_AHEAD = F8 ? 4 : 0;                    // key-scale loads issued this many tiles ahead
+  static constexpr int KS_BYTES = F8 ? EPI_WARPS * (KS_AHEAD + 1) * 32 * 4 : 0;
+  static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024 + W_BYTES + HIST_BYTES + KS_BYTES;
   static constexpr uint32_t IDESC = F8 ? idesc_e4m3_f32(128, N) : idesc_bf16_f32(128, N, 0, 0);
 };
 
@@ -175,6 +177,7 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* w_s = reinterpret_cast<float*>(smem + C::SMEM_TILES + 1024);
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + C::SMEM_TILES + 1024 + C::W_BYTES);
+  float* ks_s = reinterpret_cast<float*>(smem + C::SMEM_TILES + 1024 + C::W_BYTES + C::HIST_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -340,6 +343,23 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
     GroupInfo gi{0, -1};
     int qpos_q[QPW];
     bool dead = false;   // gave up after an abort: keeps walking the units only to meet the flushes
+    // FP8: this thread's key scale of tile kt + KS_AHEAD is copied (cp.async,
+    // 4 bytes) into a warp-private ring slot while tile kt is processed, so the
+    // global round trip is never on a tile's critical path.  Each thread reads
+    // only the slots it wrote itself, after waiting for its own copy group.
+    constexpr int KSA = C::KS_AHEAD;
+    const uint32_t ks_lane = smem_u32(ks_s) + (uint32_t)((epi * (KSA + 1) * 32 + lane) * 4);
+    int ks_head = 0;
+    bool ks_reset = true;
+    auto issue_ks = [&](int kt2, int slot) {
+      const int64_t pos2 = (int64_t)kt2 * kKeyTile + row;
+      const bool v = kt2 < p.n_kt && pos2 <= gi.maxpos && gi.row_base + pos2 < p.n_rows;
+      const float* src = v ? p.k_scale + gi.row_base + pos2 : p.k_scale;
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(ks_lane + (uint32_t)(slot * 128)),
+                   "l"(src), "r"(v ? 4 : 0)
+                   : "memory");
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
     int g = (int)(u_begin / p.n_kt), kt = (int)(u_begin % p.n_kt);   // unit u = g * n_kt + kt
     for (int64_t u = u_begin; u < u_end; ++u, kt = (kt + 1 == p.n_kt) ? 0 : kt + 1, g += (kt == 0)) {
       if constexpr (!F8) unit_of(u, p.n_kt, g, kt);
@@ -349,6 +369,7 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
         if (do_hist) flush_hist(cur_g);
         gi = load_group<QG>(p, g, false);
         cur_g = g;
+        ks_reset = true;
         // Weights of this warp's queries, in a warp-private slice of shared memory.
         __syncwarp();
 #pragma unroll
@@ -371,8 +392,20 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
       const int64_t pos = (int64_t)kt * kKeyTile + row;
       float res[QPW];
       float kscale = 1.f;
-      if (F8 && pos <= gi.maxpos && gi.row_base + pos < p.n_rows)
-        kscale = p.k_scale[gi.row_base + pos];   // issued before the wait
+      if constexpr (F8) {
+        if (ks_reset) {   // new group: drop what is in flight, fill the ring from this tile on
+          asm volatile("cp.async.wait_all;" ::: "memory");
+          for (int i = 0; i < KSA; ++i) issue_ks(kt + i, i);
+          ks_head = 0;
+          ks_reset = false;
+        }
+        int tail = ks_head + KSA;
+        if (tail > KSA) tail -= KSA + 1;
+        issue_ks(kt + KSA, tail);
+        asm volatile("cp.async.wait_group %0;" ::"n"(KSA) : "memory");   // this tile's copy has landed
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(kscale) : "r"(ks_lane + (uint32_t)(ks_head * 128)) : "memory");
+        if (++ks_head == KSA + 1) ks_head = 0;
+      }
       if (kt * kKeyTile <= gi.maxpos) {
         if (!mbar_wait(&acc_full[as.idx], as.phase, abort_flag)) {
           *abort_flag = 1;
@@ -423,6 +456,7 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
       }
     }
     if (do_hist) flush_hist(cur_g);
+    if constexpr (F8) asm volatile("cp.async.wait_all;" ::: "memory");   // no copy lands after the CTA ends
   }
 
   tc_fence_before();
