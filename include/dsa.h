@@ -141,8 +141,10 @@ dsa_status_t dsa_index_scores_fp8(const void* q8, const float* q_scale, const fl
  *   scores f32 [T, ld] (ld % 4 == 0, 16-byte aligned), q_pos int32 [T],
  *   idx int32 [T, k] (out), count int32 [T] (out), 1 <= k <= 16384.
  *   hist   uint32 [T, 2048] or NULL: the histogram dsa_index_scores wrote for
- *          these scores.  With it, the first radix pass is skipped and each
- *          query's row is filtered on every SM; it then needs a workspace of
+ *          these scores.  With it, the first radix pass is skipped: rows of at
+ *          most 40,960 scores (ld <= 40960) are selected by one thread block
+ *          per query from shared memory (no workspace); longer rows are
+ *          filtered on every SM and need a workspace of
  *          dsa_topk_workspace_size(T, ld, k) bytes, 256-byte aligned.  The
  *          result is the same (a histogram that does not match the scores is
  *          detected and the row selected without it).  NULL: no workspace.

@@ -100,8 +100,10 @@ uint64_t current_context_id() {
 }
 
 // ----------------------------------------------------------------- per-device state
+static_assert(dsa::kTopkRowCap == dsa::kPlanTopkRowCap, "planner and kernel agree on the shared-memory row path");
+
 enum KernelId : uint32_t {
-  kKIdx1 = 0, kKIdx4, kKIdx8, kKIdx1F8, kKIdx4F8, kKIdx8F8, kKTopk1, kKTopk2, kKTopk4, kKTopk8, kKTopk16, kKAttend, kKAttend8, kKTopkFilter,
+  kKIdx1 = 0, kKIdx4, kKIdx8, kKIdx1F8, kKIdx4F8, kKIdx8F8, kKTopk1, kKTopk2, kKTopk4, kKTopk8, kKTopk16, kKAttend, kKAttend8, kKTopkRow, kKTopkFilter,
   kKTopkSelect, kKTopkMerge, kKCount
 };
 
@@ -380,6 +382,15 @@ dsa_status_t topk_impl(DevLock& L, const float* scores, int64_t ld, const int32_
   p.ld = ld;
   p.T = T;
   p.k = k;
+  if (hist != nullptr && ld <= dsa::kTopkRowCap) {
+    // first pass from the indexer's histogram; the whole row in one CTA's shared memory
+    dsa::TopkHistParams hp;
+    std::memset(&hp, 0, sizeof(hp));
+    hp.base = p;
+    hp.hist = hist;
+    DSA_TRY(set_smem(*L.s, kKTopkRow, dsa::topk_row_kernel, dsa::kTopkRowSmemBytes));
+    return launch(dsa::topk_row_kernel, (unsigned)T, dsa::kTopkThreads, dsa::kTopkRowSmemBytes, stream, 1, hp);
+  }
   if (hist != nullptr) {
     // first pass from the indexer's histogram: slices on every SM, then one CTA per query
     const int S = dsa::topk_slices(props.sms, T, ld);

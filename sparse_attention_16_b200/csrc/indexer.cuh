@@ -24,8 +24,9 @@
 //
 // Warp roles (persistent CTA, one per SM, contiguous range of tiles):
 //   warp 0        TMA producer (key tiles ring, query block buffers)
-//   warp 1        TMEM owner + single-thread MMA issuer
-//   warps 2..     epilogue (4 or 8 warps), two TMEM accumulators in flight
+//   warp 1        TMEM owner + single-thread MMA issuer (FP8 decode: a second
+//                 issuer warp after the epilogue warps takes every other tile)
+//   warps 2..     epilogue (4 or 8 warps), two or four TMEM accumulators in flight
 #pragma once
 
 #include <cuda.h>
@@ -57,8 +58,19 @@ struct IdxCfg {
   static constexpr int QHALF = N * 128;
   static constexpr int Q_BYTES = KBLK * QHALF;
   static constexpr int KSTEPS = F8 ? kIdxDim / 32 : kIdxDim / 16;   // MMAs per tile (K = 32 / 16)
-  static constexpr int EPI_WARPS = (QG == 8) ? 8 : 4;   // QG 4: four warps x four queries
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  // QG 4: four warps x four queries; QG 8: two halves of four warps, four queries each; FP8
+  // decode: two sets of four warps that take alternate accumulators (tiles)
+  static constexpr int EPI_WARPS = (QG == 8 || (F8 && QG == 1)) ? 8 : 4;
+  static constexpr int EPI_SETS = (QG == 1 && EPI_WARPS == 8) ? 2 : 1;
+  // MMA-issuing threads: FP8 decode tiles are small (4 MMAs of M128 N32 K32), so two
+  // issuers (warp 1 and the warp after the epilogue) take the tiles in turn.  The
+  // issuer count must divide the accumulator and stage counts: every accumulator
+  // and stage then always has the same issuer, whose parity waits on it stay in
+  // order (an issuer may otherwise wait on a phase two ahead of the barrier and
+  // pass at once).  Measured: a third issuer adds nothing.
+  static constexpr int ISSUERS = (F8 && QG == 1) ? 2 : 1;
+  static constexpr int ISSUER2_WARP = 2 + EPI_WARPS;   // first of the extra issuer warps
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS + 32 * (ISSUERS - 1);
   static constexpr int NACC = (F8 && QG == 1) ? 4 : 2;   // TMEM accumulators in flight (measured best)
   static constexpr int TMEM_COLS = (NACC * N < 32) ? 32 : NACC * N;
   static constexpr int SMEM_TILES = STAGES * KT_BYTES + QBUFS * Q_BYTES;
@@ -68,6 +80,8 @@ struct IdxCfg {
   static constexpr int KS_BYTES = F8 ? EPI_WARPS * (KS_AHEAD + 1) * 32 * 4 : 0;
   static constexpr int SMEM_BYTES = 1024 + SMEM_TILES + 1024 + W_BYTES + HIST_BYTES + KS_BYTES;
   static constexpr uint32_t IDESC = F8 ? idesc_e4m3_f32(128, N) : idesc_bf16_f32(128, N, 0, 0);
+  static_assert(NACC % ISSUERS == 0 && STAGES % ISSUERS == 0, "each accumulator and stage has one issuer");
+  static_assert(NACC % EPI_SETS == 0, "each accumulator has one epilogue set");
 };
 
 struct IndexerParams {
@@ -172,8 +186,8 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
   uint64_t* q_empty = q_full + C::QBUFS;
   uint64_t* acc_full = q_empty + C::QBUFS;
   uint64_t* acc_empty = acc_full + C::NACC;
-  uint64_t* mma_done = acc_empty + C::NACC;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* mma_done = acc_empty + C::NACC;   // [ISSUERS]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + C::ISSUERS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* w_s = reinterpret_cast<float*>(smem + C::SMEM_TILES + 1024);
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + C::SMEM_TILES + 1024 + C::W_BYTES);
@@ -189,13 +203,13 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
     }
     for (int i = 0; i < C::QBUFS; ++i) {
       mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1);
+      mbar_init(&q_empty[i], C::ISSUERS);
     }
     for (int i = 0; i < C::NACC; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], C::EPI_WARPS);
+      mbar_init(&acc_empty[i], C::EPI_WARPS / C::EPI_SETS);
     }
-    mbar_init(mma_done, 1);
+    for (int i = 0; i < C::ISSUERS; ++i) mbar_init(&mma_done[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -264,13 +278,17 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
       for (int i = 0; i < C::QBUFS; ++i)
         if (qused[i]) mbar_wait(&q_full[i], qlast[i], nullptr);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || (C::ISSUERS > 1 && warp >= C::ISSUER2_WARP)) {
+    // ------------------------------------------------------------- MMA issuer(s)
+    // Issuer j issues the tiles with (work tile number) % ISSUERS == j and only
+    // steps the stage / accumulator rings over the others.
+    const int issuer = (warp == 1) ? 0 : 1 + warp - C::ISSUER2_WARP;
     if (lane == 0) {
       Ring ks{0, 0}, qs{C::QBUFS - 1, 1u}, as{0, 0};
       int cur_g = -1;
       GroupInfo gi{0, -1};
       bool ok = true;
+      uint32_t n_work = 0;
       int g = (int)(u_begin / p.n_kt), kt = (int)(u_begin % p.n_kt);   // unit u = g * n_kt + kt
       for (int64_t u = u_begin; u < u_end && ok; ++u, kt = (kt + 1 == p.n_kt) ? 0 : kt + 1, g += (kt == 0)) {
         if constexpr (!F8) unit_of(u, p.n_kt, g, kt);
@@ -283,6 +301,11 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
           if (!mbar_wait(&q_full[qs.idx], qs.phase, abort_flag)) { ok = false; break; }
         }
         if (kt * kKeyTile > gi.maxpos) continue;
+        if (C::ISSUERS > 1 && (int)(n_work++ % C::ISSUERS) != issuer) {   // another issuer's tile
+          ks.next(C::STAGES);
+          as.next(C::NACC);
+          continue;
+        }
         if (!mbar_wait(&acc_empty[as.idx], as.phase ^ 1u, abort_flag)) { ok = false; break; }
         if (!mbar_wait(&k_full[ks.idx], ks.phase, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -305,8 +328,8 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
       }
       if (!ok) *abort_flag = 1;
       // Drain: every MMA issued by this thread has finished before TMEM is freed.
-      mma_commit(mma_done);
-      mbar_wait(mma_done, 0, nullptr);
+      mma_commit(&mma_done[issuer]);
+      mbar_wait(&mma_done[issuer], 0, nullptr);
     }
   } else {
     // ------------------------------------------------------------- epilogue
@@ -315,6 +338,7 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
     const int row = quarter * 32 + lane;          // key row within the tile
     constexpr int QPW = (QG == 1) ? 1 : 4;        // queries per epilogue warp
     const int qbase = (QG == 1) ? 0 : (epi >> 2) * 4;
+    const int set = (C::EPI_SETS == 2) ? (epi >> 2) : 0;   // this warp's tiles: accumulators with idx % 2 == set
     float* w_my = w_s + epi * (QPW * kIdxHeads);
     // Decode (one query per group): every candidate score is also counted in a
     // shared-memory histogram of its key's top 11 bits, flushed to the query's
@@ -407,6 +431,10 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
         if (++ks_head == KSA + 1) ks_head = 0;
       }
       if (kt * kKeyTile <= gi.maxpos) {
+        if (C::EPI_SETS == 2 && (as.idx & 1) != set) {   // the other set's tile: it writes the scores
+          as.next(C::NACC);
+          continue;
+        }
         if (!mbar_wait(&acc_full[as.idx], as.phase, abort_flag)) {
           *abort_flag = 1;
           dead = true;
@@ -443,6 +471,7 @@ __global__ void __launch_bounds__(IdxCfg<QG, F8>::THREADS, 1)
         if (lane == 0) mbar_arrive(&acc_empty[as.idx]);
         as.next(C::NACC);
       } else {
+        if (C::EPI_SETS == 2 && set != 0) continue;   // past the causal range: the first set fills it
 #pragma unroll
         for (int qi = 0; qi < QPW; ++qi) res[qi] = -INFINITY;
       }

@@ -20,6 +20,7 @@ constexpr int kPlanMaxMerge = 8;      // largest cluster that merges on chip
 constexpr int kPlanMaxLayers = 8;     // layers per attention launch
 constexpr int kPlanTopkCap = 10240;   // top-k candidates per query (histogram path)
 constexpr int kPlanTopkBins = 2048;   // bins of the indexer's score histogram
+constexpr int kPlanTopkRowCap = 40960;   // rows up to this long are selected from shared memory (no workspace)
 
 inline size_t plan_round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -132,7 +133,10 @@ inline int topk_slices(int sms, int32_t T, int64_t ld) {
 }
 // Workspace of that path: per (query, slice) kPlanTopkCap keys and positions,
 // then the slices' counts, then per query the k-th bin as the filter read it.
+// Rows of at most kPlanTopkRowCap scores are selected by one CTA per query from
+// shared memory and need none.
 inline size_t topk_hist_ws_bytes(int sms, int32_t T, int64_t ld) {
+  if (ld <= kPlanTopkRowCap) return 0;
   const size_t ts = (size_t)T * topk_slices(sms, T, ld);
   return 2 * plan_round_up(ts * kPlanTopkCap * 4, 256) + plan_round_up(ts * 4, 256) +
          plan_round_up((size_t)T * 16, 256);

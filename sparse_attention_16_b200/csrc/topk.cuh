@@ -11,7 +11,7 @@
 // (output slot of a kept element = #(> tau before it) + min(#(== tau before it),
 // need_eq)), so the result is unique and deterministic.
 //
-// Two ways to run it:
+// Three ways to run it:
 //  * topk_kernel<CL>: one query per cluster of CL CTAs (CL in {1, 2, 4, 8, 16});
 //    each CTA owns a contiguous slice of the candidates and stages its keys in
 //    shared memory (whole keys up to 32K per CTA, their top 16 bits up to 64K,
@@ -28,6 +28,9 @@
 //    runs the last two passes and the ordered output.  If the candidates would
 //    exceed kTopkCandCap (a bin full of near-equal scores) or do not add up to
 //    the histogram's count, that CTA runs the single-CTA algorithm on the row.
+//  * With the histogram and rows of at most kTopkRowCap scores:
+//    topk_row_kernel, one CTA per query with the whole row in shared memory
+//    (position bitmaps instead of ordered lists; see there).
 #pragma once
 
 #include <cooperative_groups.h>
@@ -792,6 +795,221 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_select_kernel(const Topk
   }
   finish_gathered(gkey, gpos, n_cand, b1, above, (uint32_t)p.k, out, hist, tmp, res);
   if (threadIdx.x == 0) p.count[t] = p.k;
+}
+
+// ---------------------------------------------------------------------------
+// Rows that fit in shared memory (at most kTopkRowCap candidates), with the
+// indexer's histogram: one CTA per query stages its whole row once (bulk
+// copies, overlapping the read of the histogram) and finishes alone:
+//   A  every staged score is replaced by its key; keys above the k-th bin b1
+//      are marked in a position bitmap (one warp ballot per 32 positions);
+//      keys in b1 are counted by their next 11 bits and their positions listed;
+//   B  over that list: keys above the second threshold bin are marked; keys on
+//      it (the prefix of the final threshold) are counted by their last 10 bits
+//      and listed again; the short list then gives tau, the keys above it and
+//      the ties, of which the lowest-positioned need_eq are kept (a block scan
+//      over the tie bitmap's words in position order).
+// A last block scan over the bitmap words writes the positions in ascending
+// order.  A histogram that does not match the staged keys is replaced by one
+// counted from them; lists that overflow fall back to passes over the row.
+constexpr int kTopkRowCap = 40960;
+constexpr int kTopkRowListCap = 10240;
+constexpr int kTopkRowList2Cap = kTopkBins;   // the second list reuses the second histogram
+constexpr int kTopkRowWords = kTopkRowCap / 32;
+constexpr int kTopkRowSmemBytes =
+    kTopkRowCap * 4 + 2 * kTopkRowWords * 4 + 2 * kTopkBins * 4 + kTopkRowListCap * 4 + 1024;
+static_assert(kTopkRowWords <= 2 * kTopkThreads, "two bitmap words per thread");
+static_assert(kTopkRowSmemBytes <= 232448, "shared memory per block");
+
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHistParams hp) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  float* row = reinterpret_cast<float*>(smem_raw);                               // [kTopkRowCap] scores, then keys
+  uint32_t* keys = reinterpret_cast<uint32_t*>(row);
+  uint32_t* sel = reinterpret_cast<uint32_t*>(row + kTopkRowCap);                // selected positions
+  uint32_t* tie = sel + kTopkRowWords;                                           // keys equal to tau
+  uint32_t* h = tie + kTopkRowWords;                                             // [2048] first / third pass
+  uint32_t* h2 = h + kTopkBins;                                                  // [2048] second pass, then list 2
+  int32_t* list = reinterpret_cast<int32_t*>(h2 + kTopkBins);                    // positions in bin b1
+  uint32_t* tmp = reinterpret_cast<uint32_t*>(list + kTopkRowListCap);           // scan scratch (40)
+  uint32_t* res = tmp + 40;                                                      // [8]
+  uint32_t* cnt = res + 8;                                                       // [4]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(cnt + 4);
+  const TopkParams& p = hp.base;
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();
+  const int n = (int)topk_row_len(p, t, tid == 0);   // <= kTopkRowCap
+  const uint32_t k = (uint32_t)p.k;
+  int32_t* out = p.idx + (int64_t)t * p.k;
+  if (n <= (int)k) {   // every candidate is selected
+    for (int i = tid; i < (int)k; i += kTopkThreads) out[i] = (i < n) ? i : -1;
+    if (tid == 0) p.count[t] = n;
+    return;
+  }
+  const float* grow = p.scores + (int64_t)t * p.ld;
+  const int n4 = (n + 3) & ~3;   // <= ld: whole 16-byte pieces of the row
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar, (uint32_t)(n4 * 4));
+    for (int c0 = 0; c0 < n4; c0 += 8192) bulk_load_g2s(row + c0, grow + c0, (uint32_t)(min(8192, n4 - c0) * 4), bar);
+  }
+  const int nw = (n + 31) >> 5;
+  for (int w = tid; w < nw; w += kTopkThreads) tie[w] = 0u;
+  topk_bin_from_hist(hp.hist + (int64_t)t * kTopkBins, h, k, tmp, res);
+  uint32_t b1 = res[0], above = res[1], in_b1 = res[2];
+  const bool got = mbar_wait(bar, 0, nullptr);
+  if (!__syncthreads_and(got)) return;   // timed out (flagged)
+  const uint32_t lanes_below = (1u << lane) - 1u;
+  // scores -> keys, in place (each position is read and written by one thread)
+  for (int pos = tid; pos < n; pos += kTopkThreads) keys[pos] = score_key(row[pos]);
+  // ---- pass A
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    for (int b = tid; b < kTopkBins; b += kTopkThreads) h2[b] = 0u;
+    if (tid == 0) {
+      cnt[0] = 0;
+      cnt[1] = 0;
+    }
+    __syncthreads();
+    uint32_t my_gt = 0;
+#pragma unroll 2
+    for (int base = 0; base < n; base += kTopkThreads) {
+      const int pos = base + tid;
+      const bool valid = pos < n;
+      const uint32_t key = valid ? keys[pos] : 0u;
+      const uint32_t bin = key >> 21;
+      const bool gt = valid && bin > b1;
+      const bool eq = valid && bin == b1;
+      const uint32_t bg = __ballot_sync(0xffffffffu, gt);
+      if (lane == 0) sel[(base >> 5) + warp] = bg;
+      my_gt += __popc(bg);
+      const uint32_t be = __ballot_sync(0xffffffffu, eq);
+      if (be) {
+        uint32_t at = 0;
+        if (lane == 0) at = atomicAdd(&cnt[0], (uint32_t)__popc(be));
+        at = __shfl_sync(0xffffffffu, at, 0) + __popc(be & lanes_below);
+        if (eq) {
+          atomicAdd(&h2[(key >> 10) & 0x7FFu], 1u);
+          if (at < (uint32_t)kTopkRowListCap) list[at] = pos;
+        }
+      }
+    }
+    if (lane == 0 && my_gt) atomicAdd(&cnt[1], my_gt);
+    __syncthreads();
+    if (b1 != kTopkNoList && cnt[1] == above && cnt[0] == in_b1) break;
+    // The histogram does not describe these keys: count them here and redo the pass.
+    for (int b = tid; b < kTopkBins; b += kTopkThreads) h[b] = 0u;
+    __syncthreads();
+    for (int pos = tid; pos < n; pos += kTopkThreads) atomicAdd(&h[keys[pos] >> 21], 1u);
+    if (tid == 0) {
+      res[0] = kTopkNoList;
+      res[1] = 0;
+    }
+    __syncthreads();
+    find_threshold_bin<kTopkBins>(h, k, tmp, res);
+    b1 = res[0];
+    above = res[1];
+    in_b1 = (b1 == kTopkNoList) ? 0u : h[b1];
+    __syncthreads();
+  }
+  const uint32_t n_list = cnt[0];
+  const bool use_list = n_list <= (uint32_t)kTopkRowListCap;
+  uint32_t need = k - above;
+  find_threshold_bin<kTopkBins>(h2, need, tmp, res);
+  const uint32_t b2 = res[0];
+  need -= res[1];
+  const uint32_t pre2 = (b1 << 11) | b2;
+  // ---- pass B over the keys of bin b1
+  int32_t* list2 = reinterpret_cast<int32_t*>(h2);   // h2 is no longer needed
+  for (int b = tid; b < 1024; b += kTopkThreads) h[b] = 0u;
+  if (tid == 0) cnt[2] = 0;
+  __syncthreads();
+  auto visit_b = [&](int pos, uint32_t key) {
+    const uint32_t sub = (key >> 10) & 0x7FFu;
+    if (sub > b2) {
+      atomicOr(&sel[pos >> 5], 1u << (pos & 31));
+    } else if (sub == b2) {
+      atomicAdd(&h[key & 0x3FFu], 1u);
+      const uint32_t at = atomicAdd(&cnt[2], 1u);
+      if (at < (uint32_t)kTopkRowList2Cap) list2[at] = pos;
+    }
+  };
+  if (use_list) {
+    for (uint32_t i = tid; i < n_list; i += kTopkThreads) {
+      const int pos = list[i];
+      visit_b(pos, keys[pos]);
+    }
+  } else {
+    for (int pos = tid; pos < n; pos += kTopkThreads) {
+      const uint32_t key = keys[pos];
+      if ((key >> 21) == b1) visit_b(pos, key);
+    }
+  }
+  __syncthreads();
+  find_threshold_bin<1024>(h, need, tmp, res);
+  const uint32_t tau = (pre2 << 10) | res[0];
+  const uint32_t need_eq = need - res[1];
+  const uint32_t n_list2 = cnt[2];
+  // keys with prefix pre2 above tau are selected; keys equal to tau are ties
+  auto mark = [&](int pos, uint32_t key) {
+    if (key > tau) atomicOr(&sel[pos >> 5], 1u << (pos & 31));
+    else if (key == tau) atomicOr(&tie[pos >> 5], 1u << (pos & 31));
+  };
+  if (n_list2 <= (uint32_t)kTopkRowList2Cap) {
+    for (uint32_t i = tid; i < n_list2; i += kTopkThreads) {
+      const int pos = list2[i];
+      mark(pos, keys[pos]);
+    }
+  } else {
+    for (int pos = tid; pos < n; pos += kTopkThreads) {
+      const uint32_t key = keys[pos];
+      if ((key >> 10) == pre2) mark(pos, key);
+    }
+  }
+  __syncthreads();
+  // ---- ties: the need_eq lowest positions (thread i owns bitmap words 2i, 2i + 1)
+  const int w0 = 2 * tid, w1 = w0 + 1;
+  {
+    const uint32_t t0 = (w0 < nw) ? tie[w0] : 0u, t1 = (w1 < nw) ? tie[w1] : 0u;
+    uint32_t total;
+    uint32_t before = block_excl_scan((uint32_t)(__popc(t0) + __popc(t1)), tmp, &total);
+    uint32_t tw[2] = {t0, t1};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      uint32_t x = tw[e], keep = 0u;
+      while (x && before < need_eq) {
+        const uint32_t low = x & (0u - x);
+        keep |= low;
+        x ^= low;
+        ++before;
+      }
+      if (keep) sel[w0 + e] |= keep;   // each word has one owner: no race
+    }
+  }
+  __syncthreads();
+  // ---- ordered output
+  {
+    const uint32_t s0 = (w0 < nw) ? sel[w0] : 0u, s1 = (w1 < nw) ? sel[w1] : 0u;
+    uint32_t total;
+    uint32_t at = block_excl_scan((uint32_t)(__popc(s0) + __popc(s1)), tmp, &total);
+    uint32_t sw[2] = {s0, s1};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      uint32_t x = sw[e];
+      while (x) {
+        const int b = __ffs(x) - 1;
+        x &= x - 1u;
+        if (at < k) out[at] = 32 * (w0 + e) + b;
+        ++at;
+      }
+    }
+    if (total != k && tid == 0) raise_error(kErrBadIndex);   // cannot happen: the passes count exactly k
+    for (uint32_t i = total + tid; i < k; i += kTopkThreads) out[i] = -1;
+    if (tid == 0) p.count[t] = (int32_t)min(total, k);
+  }
 }
 
 // ------------------------------------------------------------------ context-parallel decode

@@ -225,7 +225,10 @@ def _check_forward_layout(lib, T, ld, k, q_group, n_layers, has_idx, has_cnt, ws
     regions.append((f.attend_offset, f.attend_bytes))
     if q_group == 1:
         regions += [(f.hist_offset, f.chunk * 2048 * 4), (f.topk_offset, f.topk_bytes)]
-        assert f.topk_bytes >= 2 * f.chunk * 10240 * 4     # at least one candidate list per query
+        if ld <= 40960:
+            assert f.topk_bytes == 0                       # rows selected from shared memory
+        else:
+            assert f.topk_bytes >= 2 * f.chunk * 10240 * 4     # at least one candidate list per query
     else:
         assert f.hist_offset == f.topk_offset == 2 ** 64 - 1
     regions.append((f.scores_offset, f.chunk * ld * 4))

@@ -175,9 +175,13 @@ def _hist_of(scores, q_pos):
     return h
 
 
+# Rows of at most 40,960 scores are selected from one CTA's shared memory, longer ones
+# by slices on every SM; the first and last cases take the slices, the others the rows.
 HIST_CASES = [
     small_case("hist_ragged", (4096, 40000, 1500, 37, 9000, 2049, 2048, 130000), seed=51),
     small_case("hist_many", (32768,) * 70, seed=52),
+    small_case("hist_ragged_rows", (4096, 40960, 1500, 37, 9000, 2049, 2048, 31), seed=53),
+    small_case("hist_one_past_rows", (40961, 2050), seed=54),
 ]
 
 
@@ -220,16 +224,19 @@ def test_topk_from_the_histogram_one_million_positions():
     pu.assert_topk_exact(to_numpy(idx2[:2]), to_numpy(cnt2[:2]), s0, to_numpy(wl.q_pos[:2]), 2048)
 
 
-def test_topk_histogram_path_ties_and_foreign_histograms():
-    # (a) Integer scores: heavy ties, bins far over the candidate cap -> the
-    #     select kernel runs the whole row; (b) a histogram of other scores, and
-    #     one with its bins shifted, must not change the result.
+@pytest.mark.parametrize("ld", [300_000, 40_960])
+def test_topk_histogram_path_ties_and_foreign_histograms(ld):
+    # (a) Integer scores: heavy ties, bins far over the candidate caps -> the
+    #     kernels fall back to the whole row; (b) a histogram of other scores, and
+    #     one with its bins shifted, must not change the result.  ld 40,960: the
+    #     shared-memory row path; 300,000: the slice path.
     g = torch.Generator(device=DEV).manual_seed(77)
-    T, ld = 6, 300_000
+    T = 6
     scores = torch.randint(-3, 4, (T, ld), generator=g, device=DEV).float()
     scores[1] = torch.randn((ld,), generator=g, device=DEV)
     scores[2, :] = 1.0
-    q_pos = torch.tensor([ld - 1, ld - 1, 99_999, 5000, 2047, ld - 1], dtype=torch.int32, device=DEV)
+    q_pos = torch.tensor([ld - 1, ld - 1, min(99_999, ld // 2), 5000, 2047, ld - 1], dtype=torch.int32,
+                         device=DEV)
     true_hist = torch.as_tensor(_hist_of(scores, q_pos), dtype=torch.int32, device=DEV)
     other = torch.as_tensor(_hist_of(torch.randn((T, ld), generator=g, device=DEV), q_pos), dtype=torch.int32,
                             device=DEV)
