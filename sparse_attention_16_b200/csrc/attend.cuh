@@ -274,14 +274,15 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLa
       for (int q = 0; q < 8; ++q) {
         const int c4 = (cb + 32 * hf) / 4 + q;
         const int r = (c4 * n + n - 1) / (kLatent / 4);                      // owner rank of column c4
-        float4* dst = cl.map_shared_rank(recv, r) + ((rank * kHeads + h) * W + (c4 - merge_c0(r, n)));
+        // this CTA's own columns by plain shared-memory stores, the others' through the cluster window
+        float4* dst = (r == rank ? recv : cl.map_shared_rank(recv, r)) + ((rank * kHeads + h) * W + (c4 - merge_c0(r, n)));
         *dst = make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]), __uint_as_float(u[4 * q + 2]),
                            __uint_as_float(u[4 * q + 3]));
       }
     }
     if (hf == 0) {
       for (int r = 0; r < n; ++r) {
-        float* dst = cl.map_shared_rank(stats, r) + (rank * kHeads + h) * 4;
+        float* dst = (r == rank ? stats : cl.map_shared_rank(stats, r)) + (rank * kHeads + h) * 4;
         dst[0] = have_o ? m_used : -INFINITY;
         dst[1] = have_o ? Lsum : 0.f;
         dst[2] = have_o ? Lx : 0.f;
@@ -319,24 +320,29 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLa
       L.lse[(int64_t)t * kHeads + h] = (Lxs > 0.f) ? (M + lg2_approx(Lxs)) * 0.69314718055994531f : -INFINITY;
   }
   __syncthreads();
+  // Four threads per head (thread 4 h + s takes float4 columns s, s + 4, ... of the
+  // slice); the head's weights are read once.
   const int c0 = merge_c0(rank, n);
   const int nc = merge_c0(rank + 1, n) - c0;
-  for (int i = tid; i < kHeads * nc; i += blockDim.x) {
-    const int h = i / nc;
-    const int c = i - h * nc;
+  const int h = tid >> 2, sub = tid & 3;
+  float wj[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) wj[j] = (j < n) ? wt[h * 8 + j] : 0.f;
+  const int64_t th = (int64_t)t * kHeads + h;
+#pragma unroll 4
+  for (int c = sub; c < nc; c += 4) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const float wj = (j < n) ? wt[h * 8 + j] : 0.f;
-      if (wj != 0.f) {
+      if (j < n) {
         const float4 v = recv[(j * kHeads + h) * W + c];
-        acc.x = fmaf(wj, v.x, acc.x);
-        acc.y = fmaf(wj, v.y, acc.y);
-        acc.z = fmaf(wj, v.z, acc.z);
-        acc.w = fmaf(wj, v.w, acc.w);
+        acc.x = fmaf(wj[j], v.x, acc.x);
+        acc.y = fmaf(wj[j], v.y, acc.y);
+        acc.z = fmaf(wj[j], v.z, acc.z);
+        acc.w = fmaf(wj[j], v.w, acc.w);
       }
     }
-    store_out4(L, (int64_t)t * kHeads + h, 4 * (c0 + c), acc.x, acc.y, acc.z, acc.w);
+    store_out4(L, th, 4 * (c0 + c), acc.x, acc.y, acc.z, acc.w);
   }
 }
 
