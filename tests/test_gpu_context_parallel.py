@@ -92,3 +92,41 @@ def test_context_parallel_decode_matches_the_single_gpu_path(world):
     for i, L in enumerate(wl.layers):
         ref_o, ref_l = pu.oracle_attend(wl, L, list(range(T)), idx_h, cnt_h)
         pu.assert_attention_close(to_numpy(out[i]), to_numpy(lse[i]), ref_o, ref_l)
+
+
+def test_context_parallel_decode_over_fp8_latent_caches():
+    # The same sharded decode with every rank's latent caches kept as FP8 rows:
+    # the combined output matches the oracle's FP8 attention over the merged
+    # selection (the global rows, decoded from the same bytes).
+    from sparse_attention_16_b200.workloads import quantize_latent_fp8
+
+    world = 2
+    lengths = (20_000, 9_000, 3_000, 1_500)
+    case = small_case("cp_gpu_fp8", lengths, layers=(64, 0), seed=81)
+    wl = make_workload(case, DEV)
+    T, k = wl.T, 2048
+    full8 = [quantize_latent_fp8(L.cache, L.d_rope) for L in wl.layers]
+    for L, c8 in zip(wl.layers, full8):
+        L.cache = c8   # the shards take their rows of the FP8 caches
+    shards = [_shard(wl, r, world, max(lengths)) for r in range(world)]
+    cands = [cp.select_local(sh, wl.q_idx, wl.w, k) for sh in shards]
+    all_score = cp.stack_exchange([c[0] for c in cands])
+    all_pos = cp.stack_exchange([c[1] for c in cands])
+    layers = [dict(q_nope=L.q_nope, q_pe=L.q_pe, qmul=L.qmul, d_rope=L.d_rope) for L in wl.layers]
+    parts = [cp.attend_local(sh, all_score, all_pos, layers, k) for sh in shards]
+    out, lse = cp.combine(cp.stack_exchange([p[2] for p in parts]), cp.stack_exchange([p[3] for p in parts]))
+    torch.cuda.synchronize()
+    assert ops.check_errors() == 0
+    idx_h, cnt_h = to_numpy(parts[0][0]), to_numpy(parts[0][1])
+    starts, q_seq, _ = pu.host_meta(wl)
+    for i, L in enumerate(wl.layers):
+        c8 = full8[i].cpu().numpy()
+        for t in range(T):
+            sel = idx_h[t, :cnt_h[t]]
+            o_ref, l_ref = oracle.sparse_mla_fp8(to_numpy(L.q_nope[t:t + 1]),
+                                                 to_numpy(L.q_pe[t:t + 1]) if L.q_pe is not None else None,
+                                                 to_numpy(L.qmul[t:t + 1]), pu.SOFTMAX_SCALE,
+                                                 c8[int(starts[q_seq[t]]) + sel], L.d_rope, np.array([0]),
+                                                 np.array([0]), np.arange(len(sel), dtype=np.int32)[None, :],
+                                                 np.array([len(sel)]))
+            pu.assert_attention_close(to_numpy(out[i][t:t + 1]), to_numpy(lse[i][t:t + 1]), o_ref, l_ref)

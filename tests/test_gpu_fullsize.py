@@ -76,3 +76,36 @@ def test_fullsize_config_sampled_parity(name):
     for L, o, l in zip(wl.layers, outs, lses):
         ref_o, ref_l = pu.oracle_attend(wl, L, ts, idx_h, cnt_h)
         pu.assert_attention_close(to_numpy(o)[ts], to_numpy(l)[ts], ref_o, ref_l)
+
+
+def test_fullsize_one_million_decode_with_fp8_latent_caches():
+    # The 1M x 4-layer decode with every latent cache kept as FP8 rows (the
+    # report's native FP8 KV cache), in the fused launch: the selection is the
+    # bf16 index path's, and each layer's attention on sampled queries matches
+    # the oracle's FP8 attention over the same bytes.
+    from sparse_attention_16_b200.workloads import quantize_latent_fp8
+    from tests.test_gpu_fp8_cache import _oracle_fp8
+
+    case = CONFIGS["decode_b4_1m_4layers"]
+    wl = make_workload(case, DEV)
+    T, ld = wl.T, case.ld
+    caches = []
+    for L in wl.layers:
+        caches.append(quantize_latent_fp8(L.cache, L.d_rope))
+        L.cache = None
+    torch.cuda.empty_cache()
+    outs = [torch.empty((T, 64, 512), dtype=torch.bfloat16, device=DEV) for _ in wl.layers]
+    lses = [torch.empty((T, 64), dtype=torch.float32, device=DEV) for _ in wl.layers]
+    layers = [dict(q_nope=L.q_nope, q_pe=L.q_pe, qmul=L.qmul, cache=c, d_rope=L.d_rope, out=o, lse=l)
+              for L, c, o, l in zip(wl.layers, caches, outs, lses)]
+    idx = torch.empty((T, 2048), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((T,), dtype=torch.int32, device=DEV)
+    ops.sparse_mla_forward(wl.q_idx, wl.w, wl.k_idx, wl.seq_row_start, wl.q_seq, wl.q_pos, layers, ld,
+                           idx_out=idx, count_out=cnt)
+    assert ops.check_errors() == 0
+    ts = [0, 3]
+    idx_h, cnt_h = to_numpy(idx), to_numpy(cnt)
+    assert (cnt_h == 2048).all()
+    for L, c, o, l in zip(wl.layers, caches, outs, lses):
+        ref_o, ref_l = _oracle_fp8(wl, L, c, ts, idx_h, cnt_h)
+        pu.assert_attention_close(to_numpy(o)[ts], to_numpy(l)[ts], ref_o, ref_l)
