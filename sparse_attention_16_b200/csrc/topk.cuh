@@ -769,20 +769,49 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_select_kernel(const Topk
   // counts, or b1 is not the row's k-th bin (a histogram that does not belong
   // to these scores)
   {
+    // Warp w copies items [w n / 32, (w + 1) n / 32): its first slice is found
+    // once, later ones by stepping forward; four items per lane are in flight.
     uint32_t my_gt = 0, my_eq = 0;
-    for (uint32_t i = threadIdx.x; i < n_cand; i += kTopkThreads) {
-      int s_lo = 0, s_hi = hp.S;   // offs[s_lo] <= i < offs[s_hi]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int kWarps = kTopkThreads / 32;
+    const uint32_t w_lo = (uint32_t)((uint64_t)warp * n_cand / kWarps);
+    const uint32_t w_hi = (uint32_t)((uint64_t)(warp + 1) * n_cand / kWarps);
+    int s = 0;   // offs[s] <= i < offs[s + 1] for the lane's current item i
+    {
+      int s_lo = 0, s_hi = hp.S;
       while (s_hi - s_lo > 1) {
         const int mid = (s_lo + s_hi) >> 1;
-        if (offs[mid] <= i) s_lo = mid;
+        if (offs[mid] <= w_lo) s_lo = mid;
         else s_hi = mid;
       }
-      const int64_t src = ((int64_t)t * hp.S + s_lo) * kTopkCandCap + (i - offs[s_lo]);
-      const uint32_t kk = hp.cand_key[src];
-      gkey[i] = kk;
-      gpos[i] = hp.cand_pos[src];
-      my_gt += (kk >> 21) > b1;
-      my_eq += (kk >> 21) == b1;
+      s = s_lo;
+    }
+    const int64_t lists = (int64_t)t * hp.S * kTopkCandCap;
+    for (uint32_t i0 = w_lo; i0 < w_hi; i0 += 4 * 32) {
+      uint32_t kk[4];
+      int32_t pp[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t i = i0 + 32 * e + lane;
+        kk[e] = 0u;
+        pp[e] = -1;
+        if (i < w_hi) {
+          while (offs[s + 1] <= i) ++s;
+          const int64_t src = lists + (int64_t)s * kTopkCandCap + (i - offs[s]);
+          kk[e] = hp.cand_key[src];
+          pp[e] = hp.cand_pos[src];
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t i = i0 + 32 * e + lane;
+        if (i < w_hi) {
+          gkey[i] = kk[e];
+          gpos[i] = pp[e];
+          my_gt += (kk[e] >> 21) > b1;
+          my_eq += (kk[e] >> 21) == b1;
+        }
+      }
     }
     if (my_gt) atomicAdd(&res[5], my_gt);
     if (my_eq) atomicAdd(&res[6], my_eq);
