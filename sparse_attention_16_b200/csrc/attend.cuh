@@ -920,11 +920,14 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
     sc->abort_flag = 0;
     fence_mbar_init();
   }
-  griddep_wait();
+  // Tensor memory before the dependency wait (a launch as a programmatic
+  // dependent sets up while the previous kernel finishes; only this library's
+  // attention uses tensor memory, and its blocks never share an SM).
   if (warp == 4) {
     tmem_alloc(&sc->tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  griddep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -481,12 +481,14 @@ dsa_status_t launch_attend(DevLock& L, const dsa_layer_args* layers, int32_t n_l
   }
   const unsigned grid = (unsigned)(units * sp.n_split);
   const unsigned cluster = sp.merge ? (unsigned)sp.n_split : 1u;
+  // programmatic dependent launch: the CTAs may be scheduled while the previous kernel (the top-k)
+  // still runs on other SMs; they set up and then wait (griddepcontrol.wait) before reading memory
   if (layers[0].cache_fp8) {   // every layer of a call has the same cache format (checked)
     DSA_TRY(set_smem(*L.s, kKAttend8, dsa::attend_kernel<true>, C::SMEM_BYTES));
-    DSA_TRY(launch(dsa::attend_kernel<true>, grid, C::THREADS, C::SMEM_BYTES, stream, cluster, p));
+    DSA_TRY(launch_ex(true, dsa::attend_kernel<true>, grid, C::THREADS, C::SMEM_BYTES, stream, cluster, p));
   } else {
     DSA_TRY(set_smem(*L.s, kKAttend, dsa::attend_kernel<false>, C::SMEM_BYTES));
-    DSA_TRY(launch(dsa::attend_kernel<false>, grid, C::THREADS, C::SMEM_BYTES, stream, cluster, p));
+    DSA_TRY(launch_ex(true, dsa::attend_kernel<false>, grid, C::THREADS, C::SMEM_BYTES, stream, cluster, p));
   }
   if (!partials) return DSA_OK;
   // programmatic dependent launch: scheduled while the attention drains, waits for its writes

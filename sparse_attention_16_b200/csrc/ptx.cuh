@@ -130,6 +130,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 // completed and its writes are visible, whatever that kernel was.  Without
 // the launch attribute the wait returns at once.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel of the stream (launched as a programmatic dependent) be
+// scheduled now: it may set itself up on idle SMs, and still waits in
+// griddep_wait() for this kernel's completion before it reads global memory.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // ------------------------------------------------------------------ proxies / fences
 __device__ __forceinline__ void fence_proxy_async_smem() {

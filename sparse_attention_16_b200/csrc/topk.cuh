@@ -715,6 +715,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_select_kernel(const Topk
   uint32_t* res = tmp + 40;
   uint32_t* gkey = reinterpret_cast<uint32_t*>(smem_raw + 2 * kTopkBins * 4 + 1024);   // gathered candidates
   int32_t* gpos = reinterpret_cast<int32_t*>(gkey + kTopkCandCap);
+  griddep_launch_dependents();   // one CTA per query: the attention may set up on the idle SMs meanwhile
   griddep_wait();
   const TopkParams& p = hp.base;
   const int t = blockIdx.x;
@@ -871,6 +872,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHis
     fence_mbar_init();
   }
   __syncthreads();
+  griddep_launch_dependents();   // the attention may set up on the SMs this launch leaves idle
   griddep_wait();
   const int n = (int)topk_row_len(p, t, tid == 0);   // <= kTopkRowCap
   const uint32_t k = (uint32_t)p.k;
