@@ -148,10 +148,12 @@ struct AttScratch {
   uint64_t p_full;                // P of a tile is in shared memory (128 arrivals)
   uint64_t o_done;                // the output product of a tile has completed
   uint64_t mma_done;
+  uint64_t merge_bar;             // cluster merge: the other ranks' blocks have landed (transaction bytes)
   uint64_t full[3];               // tile buffer b loaded
   uint64_t free_[3];              // tile buffer b no longer read
   uint32_t tmem_slot;
   int abort_flag;
+  int merge_have_o;               // cluster merge: O of this CTA is complete
 };
 static_assert(sizeof(AttScratch) <= 1024, "scratch overflow");
 
@@ -231,40 +233,86 @@ __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_
 // Merge of a (layer, query)'s split partials inside its cluster (n = p.n_split
 // CTAs, rank = split), called by every thread of the CTA once all its roles
 // are done.  Rank r produces float4 columns [c0(r), c0(r+1)) of every head,
-// c0(r) = r 128 / n.  Push model: after a cluster barrier (every CTA has left
-// its tile loop, so every tile buffer is free), each CTA reads its
-// unnormalised O from tensor memory and stores each column slice straight into
-// the owner rank's receive buffer (distributed shared memory stores, which do
-// not wait for a reply), and its per-head (m, l, lx) into every rank; after a
-// second barrier each rank merges from its own shared memory:
+// c0(r) = r 128 / n.  Every CTA holds a receive region of n blocks, one per
+// source rank j: [64 heads][nc(r) + 1] float4, the column slice r of O_j
+// (unnormalised) and, in the last column, j's per-head (m, l, lx).  A CTA
+// writes its own block with plain stores; for every other rank r it stages
+// that rank's block in its shared memory (all eight warps read O from tensor
+// memory) and moves it with one bulk copy into rank r's region, counted in
+// bytes on rank r's barrier.  After the cluster barrier at the start (every
+// CTA has left its tile loop, so every tile buffer is free, and every barrier
+// is armed with the bytes it will receive) no CTA waits for another except on
+// that barrier.  Rank r then merges its slice, consecutive threads on
+// consecutive columns:
 //   M = max_j m_j,  w_j = 2^(m_j - M),  L = sum_j w_j l_j,
 //   o[h, c] = sum_j (w_j / L) O_j[h, c],
 //   lse[h] = (M + log2 sum_j w_j lx_j) ln 2 (rank 0)
 // (l: sum of the bf16 weights the products used, lx: of the fp32 weights).
 __device__ __forceinline__ int merge_c0(int r, int n) { return r * (kLatent / 4) / n; }
 
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// Bulk copy from this CTA's shared memory to (another CTA's) shared memory in
+// the cluster; `bytes` land on the destination CTA's barrier `bar`.  Both
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_s2c(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                              uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster),
+      "r"(src), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLayer& L, uint8_t* cs, uint8_t* ps,
-                                              int t, int rank, bool softmax_thread, uint32_t hi_base, bool have_o,
+                                              AttScratch* sc, uint32_t tmem_base, int t, int rank, bool have_o,
                                               float m_used, float Lsum, float Lx) {
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
   const int n = p.n_split;
-  // float4 columns per rank (at most), padded to an odd stride so that the 16
-  // heads a half-warp pushes at once fall in different shared-memory banks
-  const int W = ((kLatent / 4 + n - 1) / n) | 1;
-  float4* recv = reinterpret_cast<float4*>(cs);                              // [n sources][64 heads][W]
-  float* stats = reinterpret_cast<float*>(cs + (size_t)n * kHeads * W * 16); // [n sources][64 heads][4]
   const int tid = threadIdx.x;
-  cl.sync();   // every CTA has left its tile loop: all receive buffers are free
-  if (softmax_thread) {
-    const int lane = tid & 31;
-    const int hf = lane >> 4;
-    const int h = 16 * (tid >> 5) + (lane & 15);
+  const int warp = tid >> 5, lane = tid & 31;
+  const int half_w = warp >> 2;   // warps w and w + 4 share the lanes of quarter w & 3
+  const int hf = lane >> 4;
+  const int h = 16 * (warp & 3) + (lane & 15);
+  const uint32_t hi_base = tmem_base + ((uint32_t)((warp & 3) * 32 + AttCfg::O_LANE) << 16);
+  const bool stats_thread = warp < 4 && hf == 0;   // holds (m, l, lx) of head h
+  auto wrow = [&](int r) { return merge_c0(r + 1, n) - merge_c0(r, n) + 1; };
+  const int w_own = wrow(rank);
+  const int w_max = (kLatent / 4 + n - 1) / n + 1;
+  float4* recv = reinterpret_cast<float4*>(cs);                                        // [n sources][64][w_own]
+  float4* stage = reinterpret_cast<float4*>(cs + (size_t)n * kHeads * w_max * 16);    // [64][w_max]
+  float* wtab = reinterpret_cast<float*>(ps);                                          // [8 warps][8]: w_j / L
+  static_assert(kHeads * 8 * 4 <= AttCfg::P_BYTES, "weight table");
+
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&sc->merge_bar, (uint32_t)((n - 1) * kHeads * w_own * 16));
+    sc->merge_have_o = have_o ? 1 : 0;
+  }
+  const float4 my_stats = make_float4(have_o ? m_used : -INFINITY, have_o ? Lsum : 0.f, have_o ? Lx : 0.f, 0.f);
+  cl.sync();   // every CTA has left its tile loop (receive regions free) and armed its barrier
+  const bool ho = sc->merge_have_o != 0;
+
+  // Block for rank r into `dst` ([64][wrow(r)]): O columns [lo, hi) (floats) of
+  // head h, read in 64-column tensor-memory blocks (a thread holds columns
+  // 64 k + 32 hf + [0, 32) of block k; blocks alternate between the two warps
+  // of a quarter), and the stats column.
+  auto stage_block = [&](int r, float4* dst) {
+    const int W = wrow(r), lo = 4 * merge_c0(r, n), hi = 4 * merge_c0(r + 1, n);
 #pragma unroll 1
-    for (int cb = 0; cb < kLatent; cb += 64) {
+    for (int k = lo / 64 + half_w; 64 * k < hi; k += 2) {
       uint32_t u[32];
-      if (have_o) {
-        tmem_ld16x2_32(hi_base + cb, u);
+      if (ho) {
+        tmem_ld16x2_32(hi_base + 64 * k, u);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -272,78 +320,78 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLa
       }
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        const int c4 = (cb + 32 * hf) / 4 + q;
-        const int r = (c4 * n + n - 1) / (kLatent / 4);                      // owner rank of column c4
-        // this CTA's own columns by plain shared-memory stores, the others' through the cluster window
-        float4* dst = (r == rank ? recv : cl.map_shared_rank(recv, r)) + ((rank * kHeads + h) * W + (c4 - merge_c0(r, n)));
-        *dst = make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]), __uint_as_float(u[4 * q + 2]),
-                           __uint_as_float(u[4 * q + 3]));
+        const int f = 64 * k + 32 * hf + 4 * q;
+        if (f >= lo && f < hi)
+          dst[h * W + (f - lo) / 4] = make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
+                                                  __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
       }
     }
-    if (hf == 0) {
-      for (int r = 0; r < n; ++r) {
-        float* dst = (r == rank ? stats : cl.map_shared_rank(stats, r)) + (rank * kHeads + h) * 4;
-        dst[0] = have_o ? m_used : -INFINITY;
-        dst[1] = have_o ? Lsum : 0.f;
-        dst[2] = have_o ? Lx : 0.f;
-      }
+    if (stats_thread) dst[h * W + W - 1] = my_stats;
+  };
+  stage_block(rank, recv + (size_t)rank * kHeads * w_own);   // own block, plain stores
+  for (int d = 1; d < n; ++d) {
+    const int r = (rank + d) % n;
+    if (d >= 2) {   // the staging buffer was read by the previous copy
+      if (tid == 0) bulk_wait_group_read<0>();
+      __syncthreads();
+    }
+    stage_block(r, stage);
+    fence_proxy_async_smem();   // the staged block is read by the bulk copy (async proxy)
+    __syncthreads();
+    if (tid == 0) {
+      const int W = wrow(r);
+      const uint32_t dst = mapa_shared(smem_u32(recv + (size_t)rank * kHeads * W), r);
+      bulk_copy_s2c(dst, smem_u32(stage), (uint32_t)(kHeads * W * 16), mapa_shared(smem_u32(&sc->merge_bar), r));
+      bulk_commit_group();
     }
   }
-  cl.sync();   // every slice is in its owner's receive buffer; no remote access follows
-  float* wt = reinterpret_cast<float*>(ps);   // [64 heads][8]: w_j / L
-  if (tid < kHeads) {
-    const int h = tid;
-    float m[8], l[8], lx[8];
-    float M = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      m[j] = -INFINITY;
-      l[j] = 0.f;
-      lx[j] = 0.f;
-      if (j < n) {
-        m[j] = stats[(j * kHeads + h) * 4];
-        l[j] = stats[(j * kHeads + h) * 4 + 1];
-        lx[j] = stats[(j * kHeads + h) * 4 + 2];
-        M = fmaxf(M, m[j]);
-      }
-    }
-    float w[8], Ls = 0.f, Lxs = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      w[j] = (m[j] == -INFINITY) ? 0.f : ex2_approx(m[j] - M);
-      Ls += w[j] * l[j];
-      Lxs += w[j] * lx[j];
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) wt[h * 8 + j] = (Ls > 0.f) ? w[j] / Ls : 0.f;
-    if (rank == 0 && L.lse != nullptr)
-      L.lse[(int64_t)t * kHeads + h] = (Lxs > 0.f) ? (M + lg2_approx(Lxs)) * 0.69314718055994531f : -INFINITY;
-  }
-  __syncthreads();
-  // Four threads per head (thread 4 h + s takes float4 columns s, s + 4, ... of the
-  // slice); the head's weights are read once.
+
+  // Every other rank's block has landed (counted on this CTA's barrier).
+  mbar_wait(&sc->merge_bar, 0, nullptr, p.wait_limit_ns);
+  // Warp w merges heads w, w + 8, ...: lane j < n takes source j's stats, the
+  // warp reduces them, and the lanes then walk the slice's columns.  Compact
+  // loops: this code runs once per block, so its instruction fetch is part of
+  // its cost.
+  const int64_t t64 = (int64_t)t * kHeads;
   const int c0 = merge_c0(rank, n);
-  const int nc = merge_c0(rank + 1, n) - c0;
-  const int h = tid >> 2, sub = tid & 3;
-  float wj[8];
+  const int nc = w_own - 1;
+  float* wsrc = wtab + warp * 8;   // [8 warps][8 sources]
+#pragma unroll 1
+  for (int hh = warp; hh < kHeads; hh += AttCfg::THREADS / 32) {
+    float4 st = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+    if (lane < n) st = recv[((size_t)lane * kHeads + hh) * w_own + w_own - 1];
+    float M = st.x;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) wj[j] = (j < n) ? wt[h * 8 + j] : 0.f;
-  const int64_t th = (int64_t)t * kHeads + h;
-#pragma unroll 4
-  for (int c = sub; c < nc; c += 4) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w = (st.x == -INFINITY) ? 0.f : ex2_approx(st.x - M);
+    float Ls = w * st.y, Lxs = w * st.z;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j < n) {
-        const float4 v = recv[(j * kHeads + h) * W + c];
-        acc.x = fmaf(wj[j], v.x, acc.x);
-        acc.y = fmaf(wj[j], v.y, acc.y);
-        acc.z = fmaf(wj[j], v.z, acc.z);
-        acc.w = fmaf(wj[j], v.w, acc.w);
-      }
+    for (int o = 16; o > 0; o >>= 1) {
+      Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+      Lxs += __shfl_xor_sync(0xffffffffu, Lxs, o);
     }
-    store_out4(L, th, 4 * (c0 + c), acc.x, acc.y, acc.z, acc.w);
+    __syncwarp();   // the previous head's weights have been read
+    if (lane < n) wsrc[lane] = (Ls > 0.f) ? w / Ls : 0.f;
+    if (rank == 0 && lane == 0 && L.lse != nullptr)
+      L.lse[t64 + hh] = (Lxs > 0.f) ? (M + lg2_approx(Lxs)) * 0.69314718055994531f : -INFINITY;
+    __syncwarp();
+    const float4* src = recv + (size_t)hh * w_own;
+#pragma unroll 1
+    for (int c = lane; c < nc; c += 32) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+      for (int j = 0; j < n; ++j) {
+        const float wj = wsrc[j];
+        const float4 v = src[(size_t)j * kHeads * w_own + c];
+        acc.x = fmaf(wj, v.x, acc.x);
+        acc.y = fmaf(wj, v.y, acc.y);
+        acc.z = fmaf(wj, v.z, acc.z);
+        acc.w = fmaf(wj, v.w, acc.w);
+      }
+      store_out4(L, t64 + hh, 4 * (c0 + c), acc.x, acc.y, acc.z, acc.w);
+    }
   }
+  if (tid == 0) bulk_wait_group_all();   // this CTA's outgoing copies are complete
 }
 
 // The work of one CTA on one unit; KCH = 64-column chunks per row (9 RoPE, 8 NoPE);
@@ -815,7 +863,7 @@ __device__ __forceinline__ void attend_unit(const AttendParams& p, const AttLaye
   tc_fence_after();
   const uint32_t hi_base = tmem_base + ((uint32_t)((warp & 3) * 32 + C::O_LANE) << 16);
   if (p.merge) {
-    cluster_merge(p, L, cs, ps, t, jsplit, warp < 4, hi_base, have_o, m_used, Lsum, Lx);
+    cluster_merge(p, L, cs, ps, sc, tmem_base, t, jsplit, have_o, m_used, Lsum, Lx);
     return;
   }
   if (warp >= 4) return;
@@ -913,6 +961,7 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
     mbar_init(&sc->p_full, 128);
     mbar_init(&sc->o_done, 1);
     mbar_init(&sc->mma_done, 1);
+    mbar_init(&sc->merge_bar, 1);
     for (int b = 0; b < C::NBUF; ++b) {
       mbar_init(&sc->full[b], C::PRODUCERS);
       mbar_init(&sc->free_[b], 1);
