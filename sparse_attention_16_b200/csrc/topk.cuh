@@ -833,7 +833,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_select_kernel(const Topk
 // copies, overlapping the read of the histogram) and finishes alone:
 //   A  every staged score is replaced by its key; keys above the k-th bin b1
 //      are marked in a position bitmap (one warp ballot per 32 positions);
-//      keys in b1 are counted by their next 11 bits and their positions listed;
+//      keys in b1 are counted by their next 11 bits and their positions listed
+//      (each warp appends to its own segment of the list, so no counter is
+//      shared);
 //   B  over that list: keys above the second threshold bin are marked; keys on
 //      it (the prefix of the final threshold) are counted by their last 10 bits
 //      and listed again; the short list then gives tau, the keys above it and
@@ -844,6 +846,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_select_kernel(const Topk
 // counted from them; lists that overflow fall back to passes over the row.
 constexpr int kTopkRowCap = 40960;
 constexpr int kTopkRowListCap = 10240;
+constexpr int kTopkRowSegCap = kTopkRowListCap / (kTopkThreads / 32);   // list entries per warp
 constexpr int kTopkRowList2Cap = kTopkBins;   // the second list reuses the second histogram
 constexpr int kTopkRowWords = kTopkRowCap / 32;
 constexpr int kTopkRowSmemBytes =
@@ -863,7 +866,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHis
   uint32_t* tmp = reinterpret_cast<uint32_t*>(list + kTopkRowListCap);           // scan scratch (40)
   uint32_t* res = tmp + 40;                                                      // [8]
   uint32_t* cnt = res + 8;                                                       // [4]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(cnt + 4);
+  uint32_t* seg_n = cnt + 4;                                                     // [32] list entries per warp
+  uint64_t* bar = reinterpret_cast<uint64_t*>(seg_n + kTopkThreads / 32);
   const TopkParams& p = hp.base;
   const int t = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -895,9 +899,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHis
   const bool got = mbar_wait(bar, 0, nullptr);
   if (!__syncthreads_and(got)) return;   // timed out (flagged)
   const uint32_t lanes_below = (1u << lane) - 1u;
-  // scores -> keys, in place (each position is read and written by one thread)
-  for (int pos = tid; pos < n; pos += kTopkThreads) keys[pos] = score_key(row[pos]);
-  // ---- pass A
+  // ---- pass A; its first attempt also turns the staged scores into keys in
+  // place (each position is read and written by one thread)
   for (int attempt = 0; attempt < 2; ++attempt) {
     for (int b = tid; b < kTopkBins; b += kTopkThreads) h2[b] = 0u;
     if (tid == 0) {
@@ -906,11 +909,21 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHis
     }
     __syncthreads();
     uint32_t my_gt = 0;
+    uint32_t my_eq = 0;   // entries of this warp's list segment (the same in every lane)
+    int32_t* seg = list + warp * kTopkRowSegCap;
 #pragma unroll 2
     for (int base = 0; base < n; base += kTopkThreads) {
       const int pos = base + tid;
       const bool valid = pos < n;
-      const uint32_t key = valid ? keys[pos] : 0u;
+      uint32_t key = 0u;
+      if (valid) {
+        if (attempt == 0) {
+          key = score_key(row[pos]);
+          keys[pos] = key;
+        } else {
+          key = keys[pos];
+        }
+      }
       const uint32_t bin = key >> 21;
       const bool gt = valid && bin > b1;
       const bool eq = valid && bin == b1;
@@ -918,17 +931,18 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHis
       if (lane == 0) sel[(base >> 5) + warp] = bg;
       my_gt += __popc(bg);
       const uint32_t be = __ballot_sync(0xffffffffu, eq);
-      if (be) {
-        uint32_t at = 0;
-        if (lane == 0) at = atomicAdd(&cnt[0], (uint32_t)__popc(be));
-        at = __shfl_sync(0xffffffffu, at, 0) + __popc(be & lanes_below);
-        if (eq) {
-          atomicAdd(&h2[(key >> 10) & 0x7FFu], 1u);
-          if (at < (uint32_t)kTopkRowListCap) list[at] = pos;
-        }
+      if (eq) {
+        atomicAdd(&h2[(key >> 10) & 0x7FFu], 1u);
+        const uint32_t at = my_eq + __popc(be & lanes_below);
+        if (at < (uint32_t)kTopkRowSegCap) seg[at] = pos;
       }
+      my_eq += __popc(be);
     }
-    if (lane == 0 && my_gt) atomicAdd(&cnt[1], my_gt);
+    if (lane == 0) {
+      seg_n[warp] = my_eq;
+      if (my_gt) atomicAdd(&cnt[1], my_gt);
+      if (my_eq) atomicAdd(&cnt[0], my_eq);
+    }
     __syncthreads();
     if (b1 != kTopkNoList && cnt[1] == above && cnt[0] == in_b1) break;
     // The histogram does not describe these keys: count them here and redo the pass.
@@ -946,8 +960,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHis
     in_b1 = (b1 == kTopkNoList) ? 0u : h[b1];
     __syncthreads();
   }
-  const uint32_t n_list = cnt[0];
-  const bool use_list = n_list <= (uint32_t)kTopkRowListCap;
+  bool use_list = true;   // every warp's segment held its entries
+#pragma unroll
+  for (int w = 0; w < kTopkThreads / 32; ++w) use_list &= seg_n[w] <= (uint32_t)kTopkRowSegCap;
   uint32_t need = k - above;
   find_threshold_bin<kTopkBins>(h2, need, tmp, res);
   const uint32_t b2 = res[0];
@@ -969,8 +984,11 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHis
     }
   };
   if (use_list) {
-    for (uint32_t i = tid; i < n_list; i += kTopkThreads) {
-      const int pos = list[i];
+    // warp w walks segment w
+    const uint32_t nseg = seg_n[warp];
+    const int32_t* seg = list + warp * kTopkRowSegCap;
+    for (uint32_t i = lane; i < nseg; i += 32) {
+      const int pos = seg[i];
       visit_b(pos, keys[pos]);
     }
   } else {

@@ -249,6 +249,30 @@ def test_topk_histogram_path_ties_and_foreign_histograms(ld):
     assert ops.check_errors() == 0
 
 
+def test_topk_row_path_list_segment_overflow():
+    # The shared-memory row path lists the keys of the k-th bin in per-warp
+    # segments (320 entries each).  Here the 1,280 keys of that bin all sit at
+    # the positions one warp reads (p mod 1024 in one 32-wide band), more than
+    # its segment holds although the whole bin would fit the list: the kernel
+    # must take its pass over the whole row, and stay exact.
+    g = torch.Generator(device=DEV).manual_seed(78)
+    T, ld = 3, 40_960
+    pos = torch.arange(ld, device=DEV)
+    scores = -torch.rand((T, ld), generator=g, device=DEV)
+    for t, lo in enumerate((0, 992, 480)):
+        band = ((pos % 1024) >= lo) & ((pos % 1024) < lo + 32)
+        scores[t, band] = 1.0 + 0.001 * torch.rand((int(band.sum()),), generator=g, device=DEV)
+        top = pos[~band & (pos % 7 == 0)][:1500]
+        scores[t, top] = 100.0 + torch.rand((1500,), generator=g, device=DEV)
+    q_pos = torch.full((T,), ld - 1, dtype=torch.int32, device=DEV)
+    hist = torch.as_tensor(_hist_of(scores, q_pos), dtype=torch.int32, device=DEV)
+    idx = torch.empty((T, 2048), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((T,), dtype=torch.int32, device=DEV)
+    ops.topk(scores, q_pos, 2048, idx, cnt, hist=hist)
+    pu.assert_topk_exact(to_numpy(idx), to_numpy(cnt), to_numpy(scores).astype(np.float64), to_numpy(q_pos), 2048)
+    assert ops.check_errors() == 0
+
+
 # ------------------------------------------------------------------ attention
 
 def _random_selection(wl, counts, sort=True, holes=False, seed=0):
