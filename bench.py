@@ -592,9 +592,7 @@ def _threads_used():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(config, budget_s=20.0, n_queries=1):
-    sample = _oracle_sample(config, n_queries)
-    n_layers = len(CONFIGS[config].layers)
+def _time_oracle(sample, budget_s):
     t = time.perf_counter()
     reps = 0
     while True:
@@ -602,12 +600,28 @@ def cpu_baseline(config, budget_s=20.0, n_queries=1):
         reps += 1
         if time.perf_counter() - t > budget_s or reps >= 50:
             break
-    el = time.perf_counter() - t
+    return reps, time.perf_counter() - t
+
+
+def cpu_baseline(config, budget_s=20.0, n_queries=1):
+    """The oracle on the host cores (numpy's default thread pool), then on one thread."""
+    sample = _oracle_sample(config, n_queries)
+    n_layers = len(CONFIGS[config].layers)
     T = sample[0].T
+    reps, el = _time_oracle(sample, budget_s)
     how = "attention rows drawn at the selected positions only" if sample[1] is not None else "full caches"
-    return {"value": round(reps * T * n_layers / el, 4), "unit": "query-layers/s",
-            "queries_per_s": round(reps * T / el, 4), "cores": _threads_used(), "kind": "oracle",
-            "sample": f"{reps} x {T} queries of {config} (same shape, CPU-drawn, {how}), fp64 numpy oracle"}
+    res = {"value": round(reps * T * n_layers / el, 4), "unit": "query-layers/s",
+           "queries_per_s": round(reps * T / el, 4), "cores": _threads_used(), "kind": "oracle",
+           "sample": f"{reps} x {T} queries of {config} (same shape, CPU-drawn, {how}), fp64 numpy oracle"}
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        return res
+    with threadpool_limits(limits=1):
+        reps1, el1 = _time_oracle(sample, budget_s / 2)
+    res["single_thread"] = {"value": round(reps1 * T * n_layers / el1, 4), "unit": "query-layers/s", "cores": 1,
+                            "sample": f"{reps1} x {T} queries, the same sample"}
+    return res
 
 
 def run_reference(args, rank, world):
