@@ -1006,6 +1006,17 @@ __global__ void __launch_bounds__(128) attend_combine_kernel(const __grid_consta
   const int ns = p.n_split;
   __shared__ float wsc[kMaxSplits];
   __shared__ float stats[2];   // M, sum_j 2^(m_j - M) lx_j
+  // The first PF partials of this thread's 4 columns are loaded before the
+  // weights are known, so their L2 round trips overlap each other and the
+  // statistics' round trip.
+  constexpr int PF = 8;
+  const int d = threadIdx.x * 4;
+  const float* po = p.ws_o + ((int64_t)pair * ns * kHeads + h) * kLatent + d;   // split j at + j 64 512
+  float4 pre[PF];
+#pragma unroll
+  for (int j = 0; j < PF; ++j)
+    pre[j] = (j < ns) ? *reinterpret_cast<const float4*>(po + (int64_t)j * kHeads * kLatent)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
   if (threadIdx.x < 32) {
     const int j = threadIdx.x;
     const int64_t u = (int64_t)pair * ns + j;
@@ -1029,12 +1040,18 @@ __global__ void __launch_bounds__(128) attend_combine_kernel(const __grid_consta
     }
   }
   __syncthreads();
-  const int d = threadIdx.x * 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < ns; ++j) {
+#pragma unroll
+  for (int j = 0; j < PF; ++j) {
+    const float wj = (j < ns) ? wsc[j] : 0.f;
+    acc.x = fmaf(wj, pre[j].x, acc.x);
+    acc.y = fmaf(wj, pre[j].y, acc.y);
+    acc.z = fmaf(wj, pre[j].z, acc.z);
+    acc.w = fmaf(wj, pre[j].w, acc.w);
+  }
+  for (int j = PF; j < ns; ++j) {
     const float wj = wsc[j];
-    const float4 o4 =
-        *reinterpret_cast<const float4*>(p.ws_o + (((int64_t)pair * ns + j) * kHeads + h) * kLatent + d);
+    const float4 o4 = *reinterpret_cast<const float4*>(po + (int64_t)j * kHeads * kLatent);
     acc.x = fmaf(wj, o4.x, acc.x);
     acc.y = fmaf(wj, o4.y, acc.y);
     acc.z = fmaf(wj, o4.z, acc.z);
