@@ -476,6 +476,17 @@ struct TopkHistParams {
 };
 constexpr uint32_t kTopkNoList = 0xFFFFFFFFu;
 
+// The float whose order-preserving key is `key` (score_key's inverse on keys
+// of non-NaN floats).  For a bin b with 4 <= b: a non-NaN score x has
+// score_key(x) >= b << 21 exactly when x >= bin_floor(b), and a NaN score (key
+// of -inf, in bin 3) has neither; for b >= 2045 the floor is a NaN, so the
+// comparison is false for every score, as no key lies that high.  Bins 0-3
+// (every key qualifies, NaN included) need the key itself.
+__device__ __forceinline__ float bin_floor(uint32_t b) {
+  const uint32_t key = b << 21;
+  return __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
+}
+
 // Query t's candidate count n (0 when q_pos < 0; clamped to ld, flagged).
 __device__ __forceinline__ int64_t topk_row_len(const TopkParams& p, int t, bool report) {
   int qp = p.q_pos[t];
@@ -620,38 +631,46 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_filter_kernel(const Topk
   uint32_t wcount = 0;
   bool ok = true;
   uint32_t phase = 0;
+  // A score is kept when its key's top 11 bits are >= b1: a float comparison
+  // against the bin's floor (keys are made only for the kept scores).
+  const bool keep_all = b1 <= 3u;
+  const float floor_b1 = bin_floor(b1 & 0x7FFu);
   for (int64_t c0 = 0; c0 < len; c0 += kTopkStashCap) {
-    const int64_t c_len = min((int64_t)kTopkStashCap, len - c0);     // scores of this chunk
-    const int64_t c_bulk = max((int64_t)0, min(c_len, len4 - c0));   // of which came by bulk copy
+    const int c_len = (int)min((int64_t)kTopkStashCap, len - c0);     // scores of this chunk
+    const int c_bulk = (int)max((int64_t)0, min((int64_t)c_len, len4 - c0));   // of which came by bulk copy
     if (c_bulk > 0) {
       const bool got = ok && mbar_wait(bar, phase, nullptr);   // every thread waits (bounded)
       ok = __syncthreads_and(got) != 0;                         // the same verdict in every thread
       phase ^= 1u;
     }
     // Warp w owns a contiguous segment of the chunk (a multiple of 128 scores).
-    const int64_t seg = ((c_len + kWarps - 1) / kWarps + 127) & ~int64_t(127);
-    const int64_t s_lo = min((int64_t)warp * seg, c_len);
-    const int64_t s_hi = min(s_lo + seg, c_len);
+    const int seg = ((c_len + kWarps - 1) / kWarps + 127) & ~127;
+    const int s_lo = min(warp * seg, c_len);
+    const int s_hi = min(s_lo + seg, c_len);
+    const float* tail = row + lo + c0;   // scores past the bulk-copied part
     if (!give_up && ok) {
-      for (int64_t e0 = s_lo + 4 * lane; e0 - 4 * lane < s_hi; e0 += 128) {
-        uint32_t kk[4];
+      for (int e0 = s_lo + 4 * lane; e0 - 4 * lane < s_hi; e0 += 128) {
+        float f[4];
         if (e0 + 3 < c_bulk) {
-          const float4 f = *reinterpret_cast<const float4*>(chunk + e0);
-          kk[0] = score_key(f.x);
-          kk[1] = score_key(f.y);
-          kk[2] = score_key(f.z);
-          kk[3] = score_key(f.w);
+          const float4 v = *reinterpret_cast<const float4*>(chunk + e0);
+          f[0] = v.x;
+          f[1] = v.y;
+          f[2] = v.z;
+          f[3] = v.w;
         } else {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int64_t i = e0 + e;
-            kk[e] = (i < s_hi) ? score_key(i < c_bulk ? chunk[i] : row[lo + c0 + i]) : 0u;
+            const int i = e0 + e;
+            f[e] = (i < s_hi) ? (i < c_bulk ? chunk[i] : tail[i]) : 0.f;
           }
         }
         uint32_t flags = 0;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) flags |= ((e0 + e < s_hi) && (kk[e] >> 21) >= b1) ? (1u << e) : 0u;
+        for (int e = 0; e < 4; ++e) flags |= ((e0 + e < s_hi) && (keep_all || f[e] >= floor_b1)) ? (1u << e) : 0u;
         if (__any_sync(0xffffffffu, flags != 0)) {
+          uint32_t kk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) kk[e] = score_key(f[e]);
           uint32_t before = 0, total = 0;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -831,8 +850,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_select_kernel(const Topk
 // Rows that fit in shared memory (at most kTopkRowCap candidates), with the
 // indexer's histogram: one CTA per query stages its whole row once (bulk
 // copies, overlapping the read of the histogram) and finishes alone:
-//   A  every staged score is replaced by its key; keys above the k-th bin b1
-//      are marked in a position bitmap (one warp ballot per 32 positions);
+//   A  scores above the k-th bin b1 (a float comparison against the bin's
+//      floor) are marked in a position bitmap (one warp ballot per 32 positions);
 //      keys in b1 are counted by their next 11 bits and their positions listed
 //      (each warp appends to its own segment of the list, so no counter is
 //      shared);
@@ -856,8 +875,7 @@ static_assert(kTopkRowSmemBytes <= 232448, "shared memory per block");
 
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHistParams hp) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  float* row = reinterpret_cast<float*>(smem_raw);                               // [kTopkRowCap] scores, then keys
-  uint32_t* keys = reinterpret_cast<uint32_t*>(row);
+  float* row = reinterpret_cast<float*>(smem_raw);                               // [kTopkRowCap] scores
   uint32_t* sel = reinterpret_cast<uint32_t*>(row + kTopkRowCap);                // selected positions
   uint32_t* tie = sel + kTopkRowWords;                                           // keys equal to tau
   uint32_t* h = tie + kTopkRowWords;                                             // [2048] first / third pass
@@ -899,9 +917,12 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHis
   const bool got = mbar_wait(bar, 0, nullptr);
   if (!__syncthreads_and(got)) return;   // timed out (flagged)
   const uint32_t lanes_below = (1u << lane) - 1u;
-  // ---- pass A; its first attempt also turns the staged scores into keys in
-  // place (each position is read and written by one thread)
+  auto key_at = [&](int pos) -> uint32_t { return score_key(row[pos]); };
+  // ---- pass A.  For 4 <= b1 <= 2043 the bin test is a float comparison
+  // against the floors of bins b1 and b1 + 1 (keys only for the scores in b1).
   for (int attempt = 0; attempt < 2; ++attempt) {
+    const bool by_floor = b1 >= 4u && b1 <= 2043u;
+    const float f_b1 = bin_floor(by_floor ? b1 : 4u), f_b2 = bin_floor(by_floor ? b1 + 1u : 5u);
     for (int b = tid; b < kTopkBins; b += kTopkThreads) h2[b] = 0u;
     if (tid == 0) {
       cnt[0] = 0;
@@ -915,24 +936,22 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHis
     for (int base = 0; base < n; base += kTopkThreads) {
       const int pos = base + tid;
       const bool valid = pos < n;
-      uint32_t key = 0u;
-      if (valid) {
-        if (attempt == 0) {
-          key = score_key(row[pos]);
-          keys[pos] = key;
-        } else {
-          key = keys[pos];
-        }
+      const float x = valid ? row[pos] : 0.f;
+      bool gt, eq;
+      if (by_floor) {
+        gt = valid && x >= f_b2;
+        eq = valid && !gt && x >= f_b1;
+      } else {
+        const uint32_t bin = score_key(x) >> 21;
+        gt = valid && bin > b1;
+        eq = valid && bin == b1;
       }
-      const uint32_t bin = key >> 21;
-      const bool gt = valid && bin > b1;
-      const bool eq = valid && bin == b1;
       const uint32_t bg = __ballot_sync(0xffffffffu, gt);
       if (lane == 0) sel[(base >> 5) + warp] = bg;
       my_gt += __popc(bg);
       const uint32_t be = __ballot_sync(0xffffffffu, eq);
       if (eq) {
-        atomicAdd(&h2[(key >> 10) & 0x7FFu], 1u);
+        atomicAdd(&h2[(score_key(x) >> 10) & 0x7FFu], 1u);
         const uint32_t at = my_eq + __popc(be & lanes_below);
         if (at < (uint32_t)kTopkRowSegCap) seg[at] = pos;
       }
@@ -948,7 +967,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHis
     // The histogram does not describe these keys: count them here and redo the pass.
     for (int b = tid; b < kTopkBins; b += kTopkThreads) h[b] = 0u;
     __syncthreads();
-    for (int pos = tid; pos < n; pos += kTopkThreads) atomicAdd(&h[keys[pos] >> 21], 1u);
+    for (int pos = tid; pos < n; pos += kTopkThreads) atomicAdd(&h[key_at(pos) >> 21], 1u);
     if (tid == 0) {
       res[0] = kTopkNoList;
       res[1] = 0;
@@ -989,11 +1008,11 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHis
     const int32_t* seg = list + warp * kTopkRowSegCap;
     for (uint32_t i = lane; i < nseg; i += 32) {
       const int pos = seg[i];
-      visit_b(pos, keys[pos]);
+      visit_b(pos, key_at(pos));
     }
   } else {
     for (int pos = tid; pos < n; pos += kTopkThreads) {
-      const uint32_t key = keys[pos];
+      const uint32_t key = key_at(pos);
       if ((key >> 21) == b1) visit_b(pos, key);
     }
   }
@@ -1010,11 +1029,11 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_row_kernel(const TopkHis
   if (n_list2 <= (uint32_t)kTopkRowList2Cap) {
     for (uint32_t i = tid; i < n_list2; i += kTopkThreads) {
       const int pos = list2[i];
-      mark(pos, keys[pos]);
+      mark(pos, key_at(pos));
     }
   } else {
     for (int pos = tid; pos < n; pos += kTopkThreads) {
-      const uint32_t key = keys[pos];
+      const uint32_t key = key_at(pos);
       if ((key >> 10) == pre2) mark(pos, key);
     }
   }
