@@ -853,6 +853,7 @@ __device__ __forceinline__ void attend_unit(const AttendParams& p, const AttLaye
     }
     Lsum = l_sum + __shfl_xor_sync(0xffffffffu, l_sum, 16);
     Lx = l_ex + __shfl_xor_sync(0xffffffffu, l_ex, 16);
+    if (threadIdx.x == 0) sc->merge_have_o = have_o ? 1 : 0;   // for the warps that did not compute it
   }
 
   // Every role is done: the producers' copies have landed (cp.async.wait_all),
@@ -866,12 +867,54 @@ __device__ __forceinline__ void attend_unit(const AttendParams& p, const AttLaye
     cluster_merge(p, L, cs, ps, sc, tmem_base, t, jsplit, have_o, m_used, Lsum, Lx);
     return;
   }
+  const int64_t unit = blockIdx.x;   // (pair, split)
+  if (p.n_split > 1) {
+    // ---- fp32 partial of this split, [64 heads][512] in the workspace.  All
+    // eight warps stage O in shared memory (rows padded by 16 bytes, so the
+    // 16 heads a half-warp writes at once fall in different banks; warps w and
+    // w + 4 read the same TMEM lanes and take alternate 64-column blocks), then
+    // the CTA copies the rows out with whole-line stores.
+    constexpr int SROW = kLatent + 4;
+    float* stg = reinterpret_cast<float*>(cs);
+    const bool ho = sc->merge_have_o != 0;
+    const int hf = lane >> 4;
+    const int h = 16 * (warp & 3) + (lane & 15);
+#pragma unroll 1
+    for (int cb = 64 * (warp >> 2); cb < kLatent; cb += 128) {
+      uint32_t u[32];
+      if (ho) {
+        tmem_ld16x2_32(hi_base + cb, u);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) u[c] = 0u;
+      }
+      float4* dst = reinterpret_cast<float4*>(stg + h * SROW + cb + 32 * hf);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        dst[q] = make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]), __uint_as_float(u[4 * q + 2]),
+                             __uint_as_float(u[4 * q + 3]));
+    }
+    if (warp < 4 && hf == 0) {
+      float* ml = p.ws_ml + (unit * kHeads + h) * 4;
+      ml[0] = have_o ? m_used : -INFINITY;
+      ml[1] = have_o ? Lsum : 0.f;
+      ml[2] = have_o ? Lx : 0.f;
+    }
+    __syncthreads();
+    float4* wo = reinterpret_cast<float4*>(p.ws_o + unit * kHeads * kLatent);
+#pragma unroll 4
+    for (int i = threadIdx.x; i < kHeads * kLatent / 4; i += C::THREADS) {
+      const int hh = i / (kLatent / 4), c4 = i % (kLatent / 4);
+      wo[i] = reinterpret_cast<const float4*>(stg + hh * SROW)[c4];
+    }
+    return;
+  }
   if (warp >= 4) return;
 
-  // ---- epilogue (softmax warps): normalised output or workspace partial
+  // ---- epilogue (softmax warps): normalised output
   const int hf = lane >> 4;
   const int h = 16 * warp + (lane & 15);
-  const int64_t unit = blockIdx.x;   // (pair, split)
   auto read_o = [&](int cb, uint32_t (&u)[32]) {
     if (have_o) {
       tmem_ld16x2_32(hi_base + cb, u);
@@ -910,23 +953,6 @@ __device__ __forceinline__ void attend_unit(const AttendParams& p, const AttLaye
     if (L.lse != nullptr && hf == 0)
       L.lse[(int64_t)t * kHeads + h] =
           (have_o && Lx > 0.f) ? (m_used + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
-  } else {
-    float4* wo = reinterpret_cast<float4*>(p.ws_o + (unit * kHeads + h) * kLatent + 32 * hf);
-#pragma unroll 1
-    for (int cb = 0; cb < kLatent; cb += 64) {
-      uint32_t u[32];
-      read_o(cb, u);
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        wo[cb / 4 + q] = make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
-                                     __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
-    }
-    if (hf == 0) {
-      float* ml = p.ws_ml + (unit * kHeads + h) * 4;
-      ml[0] = have_o ? m_used : -INFINITY;
-      ml[1] = have_o ? Lsum : 0.f;
-      ml[2] = have_o ? Lx : 0.f;
-    }
   }
 }
 
