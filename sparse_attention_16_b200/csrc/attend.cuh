@@ -137,6 +137,8 @@ struct AttendParams {
   int32_t n_split;
   int32_t rows_per_split;         // multiple of 64
   int32_t merge;                  // 1: the n_split CTAs of a (layer, query) are a cluster and merge in DSMEM
+  int32_t q_early;                // 1: Q may be read before the dependency wait (no earlier kernel of the
+                                  //    stream that can still be running writes Q)
   int32_t stall_tile;             // testing hook: >= 0 -> that tile is never gathered, so its wait runs out
 };
 
@@ -394,6 +396,36 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLa
   if (tid == 0) bulk_wait_group_all();   // this CTA's outgoing copies are complete
 }
 
+// Q [64 heads x (512 + 64)] of query t into tile buffer 2 in the tile layout
+// (heads as rows), by producer warp pw (0-2): 16-byte cp.async copies, then an
+// arrival on q_smem once this thread's copies have landed.
+template <int KCH>
+__device__ __forceinline__ void issue_q(const AttLayer& L, int t, uint32_t cs0, AttScratch* sc, int pw, int lane) {
+  using C = AttCfg;
+  constexpr int PPR = 8 * KCH;             // 16-byte pieces per row
+  constexpr int NQ = C::ROWS / 4;          // row quads per tile
+  constexpr int QPW = (NQ + 2) / 3;        // quads per warp, at most
+  const char* qn = reinterpret_cast<const char*>(L.q_nope + (int64_t)t * kHeads * kLatent);
+  const char* qp = (KCH == 9) ? reinterpret_cast<const char*>(L.q_pe + (int64_t)t * kHeads * 64) : qn;
+  const uint32_t qb = cs0 + 2 * C::TILE_BYTES;
+#pragma unroll 1
+  for (int kq = 0; kq < QPW; ++kq) {
+    const int quad = pw + 3 * kq;
+    if (quad >= NQ) break;
+#pragma unroll
+    for (int j = 0; j < KCH; ++j) {
+      const int g = 32 * j + lane;
+      const int riq = g / PPR;
+      const int pr = g - riq * PPR;
+      const int h = 4 * quad + riq;
+      const uint32_t dst = qb + (pr >> 3) * C::CHUNK_BYTES + h * 128 + (((pr & 7) ^ (h & 7)) << 4);
+      const char* src = (pr < 64) ? qn + h * (kLatent * 2) + pr * 16 : qp + h * 128 + (pr - 64) * 16;
+      cp_async_16(dst, src, 16u);
+    }
+  }
+  cp_async_arrive_noinc(&sc->q_smem);   // completes once this thread's Q copies have landed
+}
+
 // The work of one CTA on one unit; KCH = 64-column chunks per row (9 RoPE, 8 NoPE);
 // F8: the cache rows are FP8 (E4M3 codes + block scales) and are widened to bf16
 // in shared memory.
@@ -435,28 +467,8 @@ __device__ __forceinline__ void attend_unit(const AttendParams& p, const AttLaye
     static_assert(4 * QPW <= 32, "one index per lane");
     if (!seq_ok && threadIdx.x == 160 && n_tiles > 0) raise_error(kErrBadSeq);
     const uint32_t cs0 = smem_u32(cs);
-    if (n_tiles > 0) {
-      // Q [64 heads x (512 + 64)] into tile buffer 2 in the tile layout (heads as rows).
-      const char* qn = reinterpret_cast<const char*>(L.q_nope + (int64_t)t * kHeads * kLatent);
-      const char* qp = (KCH == 9) ? reinterpret_cast<const char*>(L.q_pe + (int64_t)t * kHeads * 64) : qn;
-      const uint32_t qb = cs0 + 2 * C::TILE_BYTES;
-#pragma unroll 1
-      for (int kq = 0; kq < QPW; ++kq) {
-        const int quad = pw + 3 * kq;
-        if (quad >= NQ) break;
-#pragma unroll
-        for (int j = 0; j < KCH; ++j) {
-          const int g = 32 * j + lane;
-          const int riq = g / PPR;
-          const int pr = g - riq * PPR;
-          const int h = 4 * quad + riq;
-          const uint32_t dst = qb + (pr >> 3) * C::CHUNK_BYTES + h * 128 + (((pr & 7) ^ (h & 7)) << 4);
-          const char* src = (pr < 64) ? qn + h * (kLatent * 2) + pr * 16 : qp + h * 128 + (pr - 64) * 16;
-          cp_async_16(dst, src, 16u);
-        }
-      }
-      cp_async_arrive_noinc(&sc->q_smem);   // completes once this thread's Q copies have landed
-    }
+    // Q into tile buffer 2 (already issued before the dependency wait when p.q_early).
+    if (n_tiles > 0 && !p.q_early) issue_q<KCH>(L, t, cs0, sc, pw, lane);
     const int my_quad = pw + 3 * (lane >> 2);
     const int my_row = 4 * my_quad + (lane & 3);
     const char* cache_bytes = reinterpret_cast<const char*>(L.cache);
@@ -994,6 +1006,15 @@ __global__ void __launch_bounds__(AttCfg::THREADS, 1)
     }
     sc->abort_flag = 0;
     fence_mbar_init();
+  }
+  if (p.q_early) {
+    // Q is not written by the kernels this launch may overlap: its copies start
+    // now, while the previous kernel finishes.
+    __syncthreads();   // the barriers are initialised
+    if (warp >= 5 && smem_ok) {
+      if (L.d_rope == 64) issue_q<9>(L, t, smem_u32(cs), sc, warp - 5, threadIdx.x & 31);
+      else issue_q<8>(L, t, smem_u32(cs), sc, warp - 5, threadIdx.x & 31);
+    }
   }
   // Tensor memory before the dependency wait (a launch as a programmatic
   // dependent sets up while the previous kernel finishes; only this library's

@@ -433,7 +433,8 @@ dsa_status_t topk_impl(DevLock& L, const float* scores, int64_t ld, const int32_
 dsa_status_t launch_attend(DevLock& L, const dsa_layer_args* layers, int32_t n_layers, float scale,
                            int64_t n_rows, const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
                            const int32_t* q_pos, const int32_t* idx, const int32_t* count, int32_t T, int32_t k,
-                           void* ws, size_t ws_bytes, cudaStream_t stream, bool allow_partials = true) {
+                           void* ws, size_t ws_bytes, cudaStream_t stream, bool allow_partials = true,
+                           bool q_early = false) {
   using C = dsa::AttCfg;
   dsa::DevProps props;
   DSA_TRY(device_props(L, &props));
@@ -470,6 +471,7 @@ dsa_status_t launch_attend(DevLock& L, const dsa_layer_args* layers, int32_t n_l
   p.n_split = sp.n_split;
   p.rows_per_split = sp.rows_per_split;
   p.merge = sp.merge ? 1 : 0;
+  p.q_early = q_early ? 1 : 0;
   const bool partials = sp.n_split > 1 && !sp.merge;
   if (partials) {
     const size_t need = dsa::partial_bytes(units, sp.n_split);
@@ -501,7 +503,7 @@ dsa_status_t attend_layers_impl(DevLock& L, const dsa_layer_args* layers, int32_
                                 int64_t n_rows, const int64_t* seq_row_start, int32_t B, const int32_t* q_seq,
                                 const int32_t* q_pos, const int32_t* idx, const int32_t* count, int32_t T,
                                 int32_t k, int64_t q_offset, void* ws, size_t ws_bytes, cudaStream_t stream,
-                                bool allow_partials = true) {
+                                bool allow_partials = true, bool q_early = false) {
   for (int l0 = 0; l0 < n_layers; l0 += dsa::kMaxAttLayers) {
     const int g = std::min(dsa::kMaxAttLayers, n_layers - l0);
     dsa_layer_args sub[dsa::kMaxAttLayers];
@@ -517,7 +519,7 @@ dsa_status_t attend_layers_impl(DevLock& L, const dsa_layer_args* layers, int32_
       sub[i].lse = a.lse ? a.lse + qo : nullptr;
     }
     DSA_TRY(launch_attend(L, sub, g, scale, n_rows, seq_row_start, B, q_seq, q_pos, idx, count, T, k, ws,
-                          ws_bytes, stream, allow_partials));
+                          ws_bytes, stream, allow_partials, q_early));
   }
   return DSA_OK;
 }
@@ -876,8 +878,11 @@ dsa_status_t forward_impl(const IndexKeys& ik, const float* w, int64_t n_rows, c
                            seq_row_start, B, q_seq + t0, q_pos + t0, n, q_group, scores, ld, hist, s));
     }
     DSA_TRY(topk_impl(L, scores, ld, q_pos + t0, n, k, idx_c, cnt_c, hist, topk_ws, f.topk_bytes, s));
+    // The kernels before the attention in this call (indexer, top-k, earlier
+    // attention groups) do not write the queries, so the attention may start
+    // copying them while the top-k finishes.
     DSA_TRY(attend_layers_impl(L, layers, n_layers, softmax_scale, n_rows, seq_row_start, B, q_seq + t0,
-                               q_pos + t0, idx_c, cnt_c, n, k, t0, att_ws, f.att_bytes, s, f.partials));
+                               q_pos + t0, idx_c, cnt_c, n, k, t0, att_ws, f.att_bytes, s, f.partials, true));
   }
   return DSA_OK;
 }
