@@ -293,7 +293,7 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLa
   const int w_max = (kLatent / 4 + n - 1) / n + 1;
   float4* recv = reinterpret_cast<float4*>(cs);                                        // [n sources][64][w_own]
   float4* stage = reinterpret_cast<float4*>(cs + (size_t)n * kHeads * w_max * 16);    // [64][w_max]
-  float* wtab = reinterpret_cast<float*>(ps);                                          // [8 warps][8]: w_j / L
+  float* wtab = reinterpret_cast<float*>(ps);                                          // [64 heads][8]: w_j / L
   static_assert(kHeads * 8 * 4 <= AttCfg::P_BYTES, "weight table");
 
   if (tid == 0) {
@@ -350,48 +350,81 @@ __device__ __forceinline__ void cluster_merge(const AttendParams& p, const AttLa
 
   // Every other rank's block has landed (counted on this CTA's barrier).
   mbar_wait(&sc->merge_bar, 0, nullptr, p.wait_limit_ns);
-  // Warp w merges heads w, w + 8, ...: lane j < n takes source j's stats, the
-  // warp reduces them, and the lanes then walk the slice's columns.  Compact
-  // loops: this code runs once per block, so its instruction fetch is part of
-  // its cost.
+  // Per-head weights (one thread per head), then the slice's float4 columns,
+  // consecutive threads on consecutive columns, four outputs per thread at a
+  // time with all their loads issued before the arithmetic.
   const int64_t t64 = (int64_t)t * kHeads;
+  if (tid < kHeads) {
+    const int hh = tid;
+    float m[8], l[8], lx[8];
+    float M = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      m[j] = -INFINITY;
+      l[j] = lx[j] = 0.f;
+      if (j < n) {
+        const float4 st = recv[((size_t)j * kHeads + hh) * w_own + w_own - 1];
+        m[j] = st.x;
+        l[j] = st.y;
+        lx[j] = st.z;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) M = fmaxf(M, m[j]);
+    float w[8], Ls = 0.f, Lxs = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      w[j] = (m[j] == -INFINITY) ? 0.f : ex2_approx(m[j] - M);
+      Ls += w[j] * l[j];
+      Lxs += w[j] * lx[j];
+    }
+    const float inv = (Ls > 0.f) ? 1.f / Ls : 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wtab[hh * 8 + j] = w[j] * inv;
+    if (rank == 0 && L.lse != nullptr)
+      L.lse[t64 + hh] = (Lxs > 0.f) ? (M + lg2_approx(Lxs)) * 0.69314718055994531f : -INFINITY;
+  }
+  __syncthreads();
   const int c0 = merge_c0(rank, n);
   const int nc = w_own - 1;
-  float* wsrc = wtab + warp * 8;   // [8 warps][8 sources]
+  const int total = kHeads * nc;
+  const bool pow2 = (nc & (nc - 1)) == 0;
+  const int sh = __ffs(nc) - 1;
+  constexpr int U = 4;
 #pragma unroll 1
-  for (int hh = warp; hh < kHeads; hh += AttCfg::THREADS / 32) {
-    float4 st = make_float4(-INFINITY, 0.f, 0.f, 0.f);
-    if (lane < n) st = recv[((size_t)lane * kHeads + hh) * w_own + w_own - 1];
-    float M = st.x;
+  for (int o0 = tid; o0 < total; o0 += U * AttCfg::THREADS) {
+    int hh[U], cc[U];
+    float4 acc[U];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float w = (st.x == -INFINITY) ? 0.f : ex2_approx(st.x - M);
-    float Ls = w * st.y, Lxs = w * st.z;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
-      Lxs += __shfl_xor_sync(0xffffffffu, Lxs, o);
+    for (int u = 0; u < U; ++u) {
+      const int o = min(o0 + u * AttCfg::THREADS, total - 1);
+      hh[u] = pow2 ? (o >> sh) : (o / nc);
+      cc[u] = o - hh[u] * nc;
+      acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    __syncwarp();   // the previous head's weights have been read
-    if (lane < n) wsrc[lane] = (Ls > 0.f) ? w / Ls : 0.f;
-    if (rank == 0 && lane == 0 && L.lse != nullptr)
-      L.lse[t64 + hh] = (Lxs > 0.f) ? (M + lg2_approx(Lxs)) * 0.69314718055994531f : -INFINITY;
-    __syncwarp();
-    const float4* src = recv + (size_t)hh * w_own;
-#pragma unroll 1
-    for (int c = lane; c < nc; c += 32) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-      for (int j = 0; j < n; ++j) {
-        const float wj = wsrc[j];
-        const float4 v = src[(size_t)j * kHeads * w_own + c];
-        acc.x = fmaf(wj, v.x, acc.x);
-        acc.y = fmaf(wj, v.y, acc.y);
-        acc.z = fmaf(wj, v.z, acc.z);
-        acc.w = fmaf(wj, v.w, acc.w);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j < n) {
+        float4 v[U];
+        float wj[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          v[u] = recv[((size_t)j * kHeads + hh[u]) * w_own + cc[u]];
+          wj[u] = wtab[hh[u] * 8 + j];
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          acc[u].x = fmaf(wj[u], v[u].x, acc[u].x);
+          acc[u].y = fmaf(wj[u], v[u].y, acc[u].y);
+          acc[u].z = fmaf(wj[u], v[u].z, acc[u].z);
+          acc[u].w = fmaf(wj[u], v[u].w, acc[u].w);
+        }
       }
-      store_out4(L, t64 + hh, 4 * (c0 + c), acc.x, acc.y, acc.z, acc.w);
     }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (o0 + u * AttCfg::THREADS < total)
+        store_out4(L, t64 + hh[u], 4 * (c0 + cc[u]), acc[u].x, acc[u].y, acc[u].z, acc[u].w);
   }
   if (tid == 0) bulk_wait_group_all();   // this CTA's outgoing copies are complete
 }
