@@ -90,24 +90,46 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, u
 
 // Finds bin b (scanning from the top) with above(b) < need <= above(b) + h[b],
 // where above(b) counts elements in bins above b.  Writes (b, above(b)) to res.
+// Thread i sums positions [i PER, (i + 1) PER) of the top-down order; a warp
+// scan gives the counts above each lane inside its warp, and every warp scans
+// the 32 warp totals itself (two barriers in all).
 template <int NB>
 __device__ __forceinline__ void find_threshold_bin(const uint32_t* h, uint32_t need, uint32_t* tmp,
                                                    uint32_t* res) {
+  static_assert(kTopkThreads == 32 * 32, "one warp total per lane of a warp");
   constexpr int PER = NB / kTopkThreads;  // 2 or 1 bins per thread, descending
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t c[PER];
   uint32_t mine = 0;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) mine += h[NB - 1 - (threadIdx.x * PER + i)];
-  uint32_t total;
-  uint32_t above = block_excl_scan(mine, tmp, &total);
+  for (int i = 0; i < PER; ++i) {
+    c[i] = h[NB - 1 - (threadIdx.x * PER + i)];
+    mine += c[i];
+  }
+  uint32_t x = mine;   // inclusive prefix inside the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[warp] = x;
+  __syncthreads();
+  const uint32_t wt = tmp[lane];
+  uint32_t ws = wt;   // inclusive prefix of the warp totals
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, ws, o);
+    if (lane >= o) ws += y;
+  }
+  uint32_t above = __shfl_sync(0xffffffffu, ws - wt, warp) + x - mine;
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int b = NB - 1 - (threadIdx.x * PER + i);
-    const uint32_t c = h[b];
-    if (above < need && need <= above + c) {
+    if (above < need && need <= above + c[i]) {
       res[0] = (uint32_t)b;
       res[1] = above;
     }
-    above += c;
+    above += c[i];
   }
   __syncthreads();
 }
