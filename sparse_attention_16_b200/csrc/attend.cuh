@@ -1084,12 +1084,12 @@ __global__ void __launch_bounds__(128) attend_combine_kernel(const __grid_consta
   const int t = pair - lyr * p.T;
   const AttLayer& L = p.layer[lyr];
   const int ns = p.n_split;
-  __shared__ float wsc[kMaxSplits];
-  __shared__ float stats[2];   // M, sum_j 2^(m_j - M) lx_j
   // The first PF partials of this thread's 4 columns are loaded before the
   // weights are known, so their L2 round trips overlap each other and the
-  // statistics' round trip.
+  // statistics' round trip.  Every warp computes the weights itself (lane j:
+  // split j), so no barrier separates them from the sums.
   constexpr int PF = 8;
+  static_assert(kMaxSplits <= 32, "one split per lane");
   const int d = threadIdx.x * 4;
   const float* po = p.ws_o + ((int64_t)pair * ns * kHeads + h) * kLatent + d;   // split j at + j 64 512
   float4 pre[PF];
@@ -1097,40 +1097,33 @@ __global__ void __launch_bounds__(128) attend_combine_kernel(const __grid_consta
   for (int j = 0; j < PF; ++j)
     pre[j] = (j < ns) ? *reinterpret_cast<const float4*>(po + (int64_t)j * kHeads * kLatent)
                       : make_float4(0.f, 0.f, 0.f, 0.f);
-  if (threadIdx.x < 32) {
-    const int j = threadIdx.x;
-    const int64_t u = (int64_t)pair * ns + j;
-    const float m = (j < ns) ? p.ws_ml[(u * kHeads + h) * 4] : -INFINITY;
-    const float l = (j < ns) ? p.ws_ml[(u * kHeads + h) * 4 + 1] : 0.f;
-    const float lx = (j < ns) ? p.ws_ml[(u * kHeads + h) * 4 + 2] : 0.f;
-    float M = m;
+  const int lane = threadIdx.x & 31;
+  const int64_t u = (int64_t)pair * ns + lane;
+  const float m = (lane < ns) ? p.ws_ml[(u * kHeads + h) * 4] : -INFINITY;
+  const float l = (lane < ns) ? p.ws_ml[(u * kHeads + h) * 4 + 1] : 0.f;
+  const float lx = (lane < ns) ? p.ws_ml[(u * kHeads + h) * 4 + 2] : 0.f;
+  float M = m;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float sc = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
-    float Ls = sc * l, Lx = sc * lx;
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float sc = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
+  float Ls = sc * l, Lx = sc * lx;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
-      Lx += __shfl_xor_sync(0xffffffffu, Lx, o);
-    }
-    wsc[j] = (Ls > 0.f) ? sc / Ls : 0.f;
-    if (j == 0) {
-      stats[0] = M;
-      stats[1] = Lx;
-    }
+  for (int o = 16; o > 0; o >>= 1) {
+    Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+    Lx += __shfl_xor_sync(0xffffffffu, Lx, o);
   }
-  __syncthreads();
+  const float w_lane = (Ls > 0.f) ? sc / Ls : 0.f;   // weight of split `lane`
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < PF; ++j) {
-    const float wj = (j < ns) ? wsc[j] : 0.f;
+    const float wj = __shfl_sync(0xffffffffu, w_lane, j);   // 0 for j >= ns
     acc.x = fmaf(wj, pre[j].x, acc.x);
     acc.y = fmaf(wj, pre[j].y, acc.y);
     acc.z = fmaf(wj, pre[j].z, acc.z);
     acc.w = fmaf(wj, pre[j].w, acc.w);
   }
   for (int j = PF; j < ns; ++j) {
-    const float wj = wsc[j];
+    const float wj = __shfl_sync(0xffffffffu, w_lane, j);
     const float4 o4 = *reinterpret_cast<const float4*>(po + (int64_t)j * kHeads * kLatent);
     acc.x = fmaf(wj, o4.x, acc.x);
     acc.y = fmaf(wj, o4.y, acc.y);
@@ -1138,10 +1131,8 @@ __global__ void __launch_bounds__(128) attend_combine_kernel(const __grid_consta
     acc.w = fmaf(wj, o4.w, acc.w);
   }
   store_out4(L, (int64_t)t * kHeads + h, d, acc.x, acc.y, acc.z, acc.w);
-  if (threadIdx.x == 0 && L.lse != nullptr) {
-    const float Lx = stats[1];
-    L.lse[(int64_t)t * kHeads + h] = (Lx > 0.f) ? (stats[0] + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
-  }
+  if (threadIdx.x == 0 && L.lse != nullptr)
+    L.lse[(int64_t)t * kHeads + h] = (Lx > 0.f) ? (M + lg2_approx(Lx)) * 0.69314718055994531f : -INFINITY;
 }
 
 // Context-parallel output combine (report's serving section): R ranks each
