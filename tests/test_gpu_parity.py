@@ -249,6 +249,38 @@ def test_topk_histogram_path_ties_and_foreign_histograms(ld):
     assert ops.check_errors() == 0
 
 
+@pytest.mark.parametrize("ld", [6_000, 300_000])
+def test_topk_histogram_path_special_values(ld):
+    # The histogram paths decide "at or above the k-th bin" by a float
+    # comparison against the bin's first value; rows whose k-th bin holds NaN
+    # (ranked as -inf), +-inf, signed zeros or values on a bin boundary.
+    # ld 6,000: the shared-memory row kernel; 300,000: the slice filter + select.
+    g = torch.Generator(device=DEV).manual_seed(ld + 5)
+    T = 7
+    s = torch.randn((T, ld), generator=g, device=DEV)
+    s[0, 100:ld - 500] = float("nan")              # k-th among the few finite ones, then NaN = -inf
+    s[1, :] = float("-inf")
+    s[1, ::997] = 3.0                              # k-th bin is that of -inf (every key qualifies)
+    s[2, :] = float("nan")                         # all NaN: ties at -inf, lowest positions win
+    s[3, :] = -0.0
+    s[3, ::3] = 0.0                                # signed zeros, all equal
+    s[3, ::701] = -1.0
+    s[4, 1000:1000 + 3000] = float("inf")          # more +inf than k
+    s[5, :] = 1.25                                 # first value of its bin
+    s[5, ::2] = 1.0                                # first value of the bin below
+    s[5, ::7] = 1.2499999                          # last value of the bin below 1.25
+    s[6, :] = -1.0                                 # negative: first value of its bin from the top
+    s[6, ::5] = -0.9999999
+    q_pos = torch.full((T,), ld - 1, dtype=torch.int32, device=DEV)
+    hist = torch.as_tensor(_hist_of(s, q_pos), dtype=torch.int32, device=DEV)
+    for k in (2048, 7):
+        idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+        cnt = torch.empty((T,), dtype=torch.int32, device=DEV)
+        ops.topk(s, q_pos, k, idx, cnt, hist=hist)
+        pu.assert_topk_exact(to_numpy(idx), to_numpy(cnt), to_numpy(s).astype(np.float64), to_numpy(q_pos), k)
+    assert ops.check_errors() == 0
+
+
 def test_topk_row_path_list_segment_overflow():
     # The shared-memory row path lists the keys of the k-th bin in per-warp
     # segments (320 entries each).  Here the 1,280 keys of that bin all sit at
