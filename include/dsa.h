@@ -294,7 +294,10 @@ dsa_status_t sparse_mla_attend_layers(int32_t n_layers, const dsa_layer_args* la
  * (work units = layers x queries x splits), so a small decode batch still
  * fills the GPU; RoPE and NoPE layers may be mixed.  Queries are processed in
  * chunks so that the fp32 score rows fit the workspace (chunked prefill);
- * every chunk, the last one included, stays inside the workspace.
+ * every chunk, the last one included, stays inside the workspace.  The
+ * attention launches start copying the layers' queries (q_nope, q_pe) while
+ * the call's top-k still runs: like every input, they must be complete before
+ * the call in stream order and must not be written while it runs.
  *
  *   idx_out / count_out: optional [T, k] / [T] copies of the selection (NULL = not needed).
  *   workspace: at least dsa_forward_workspace_size(T, ld, k, q_group, n_layers)
